@@ -1,0 +1,230 @@
+"""CPU oracle of the product-key memory (PKM) layer, forward and backward, in fp64.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the benchmark's CPU
+baseline leg may import this module.  The CUDA library never calls it, and it
+shares no code, header, table or helper with the CUDA library.
+
+What it computes (sources: "Large Memory Layers with Product Keys", method-details
+list and abstract; "Meta AI 可扩展内存层" sections 3.2, 4.3, 4.5, 5.2, 5.3):
+
+  1. query network      q = gamma * (x Wq^T - mean) / sqrt(var + eps) + beta
+                        (Linear followed by BatchNorm with running statistics)
+  2. split per head     q1 = q[h*dk : h*dk + dk/2], q2 = q[h*dk + dk/2 : (h+1)*dk]
+  3. sub-key scores     s1[i] = q1 . C[h][i],  s2[j] = q2 . C'[h][j]
+  4. key selection      the k best product keys (i, j) by s1[i] + s2[j] over ALL
+                        C1*C2 keys (brute force: the exact nearest-neighbour result
+                        the product keys are built to reach)
+  5. weights            w = softmax(score_scale * (s1[i] + s2[j])) over the k winners
+  6. output             y[t] = sum_h sum_winners w * V[i*C2 + j]
+
+Readings taken where the pages are silent (each is listed in the design notes):
+  * total order of keys: (s1+s2 desc, s1 desc, s2 desc, flat index asc); per
+    half: (score desc, index asc).  With this order the product-key search returns
+    exactly the brute-force set even with rounding ties.
+  * heads each own their sub-key sets, share the value table, and their outputs
+    are summed; the softmax is per head.
+  * the temperature is a positive ``score_scale`` applied to the softmax only;
+    selection uses the unscaled sums (a positive scale keeps the order).
+  * the backward holds the selected set fixed (top-k is piecewise constant).
+
+Every function here is pinned by a CPU test against something other than itself:
+brute force vs the product-key search (exactness), a hand-derived worked example
+(tests/golden), one-hot value tables, permutation and linearity invariants, the
+library batch_norm, autograd of an independent forward, and central finite
+differences in fp64.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+# ----------------------------------------------------------------------------- 1
+def query_network(x, Wq, bn, eps):
+    """q = gamma * (x Wq^T - mean) / sqrt(var + eps) + beta, fp64.
+
+    x [N][d_in], Wq [h*dk][d_in] (Linear weight, out x in), bn [4][h*dk] =
+    (running mean, running var, gamma, beta).  BatchNorm in eval mode on the
+    query ("Large Memory Layers with Product Keys", key results, BatchNorm remark).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    Wq = np.asarray(Wq, dtype=np.float64)
+    mean, var, gamma, beta = (np.asarray(r, dtype=np.float64) for r in bn)
+    pre = x @ Wq.T
+    qhat = (pre - mean) / np.sqrt(var + eps)
+    return gamma * qhat + beta, qhat
+
+
+# ----------------------------------------------------------------------------- 2, 3
+def split_halves(q, h, dk):
+    """q [N][h*dk] -> (q1, q2), each [N][h][dk/2]."""
+    q = q.reshape(q.shape[0], h, dk)
+    return q[:, :, : dk // 2], q[:, :, dk // 2:]
+
+
+def subkey_scores(q, subkeys, h, dk, C1):
+    """s1[t][h][i] = q1[t][h] . C[h][i];  s2[t][h][j] = q2[t][h] . C'[h][j]  (fp64)."""
+    sub = np.asarray(subkeys, dtype=np.float64)
+    q1, q2 = split_halves(q, h, dk)
+    s1 = np.einsum("thd,hid->thi", q1, sub[:, :C1, :])
+    s2 = np.einsum("thd,hjd->thj", q2, sub[:, C1:, :])
+    return s1, s2
+
+
+# ----------------------------------------------------------------------------- 4
+def half_topk(s, k):
+    """Top-k of one half's scores s [C] by (score desc, index asc) -> (index, score)."""
+    order = np.lexsort((np.arange(s.shape[0]), -s))[:k]
+    return order, s[order]
+
+
+def _order_candidates(S, a, b, flat):
+    """Indices sorting candidates by (S desc, a desc, b desc, flat asc)."""
+    return np.lexsort((flat, -b, -a, -S))
+
+
+def brute_force_topk(s1, s2, k):
+    """The k best keys over ALL C1*C2 product keys of one (token, head).
+
+    The sum s1[i] + s2[j] is formed for every key; the first k under the total
+    order (sum desc, s1 desc, s2 desc, flat asc) win.  Returns (i, j) of the
+    winners, best first.
+
+    Only keys whose sum reaches the k-th largest sum can be among the first k under
+    an order whose first key is the sum, so the order is taken over those (all of
+    them, ties included).
+    """
+    C1, C2 = s1.shape[0], s2.shape[0]
+    S = (s1[:, None] + s2[None, :]).reshape(-1)
+    flat = np.arange(C1 * C2)
+    if S.shape[0] > 4 * k:
+        kth = np.partition(S, S.shape[0] - k)[S.shape[0] - k]
+        keep = np.nonzero(S >= kth)[0]
+    else:
+        keep = flat
+    ii, jj = keep // C2, keep % C2
+    order = _order_candidates(S[keep], s1[ii], s2[jj], keep)[:k]
+    sel = keep[order]
+    return sel // C2, sel % C2
+
+
+def product_key_topk(s1, s2, k):
+    """The product-key search for one (token, head): the top-k of each half, then the
+    best k of the k x k Cartesian candidates by the same total order as
+    ``brute_force_topk`` ("Large Memory Layers with Product Keys", method details;
+    "Meta AI 可扩展内存层" section 4.3).  Returns (i, j), best first."""
+    C2 = s2.shape[0]
+    ia, va = half_topk(s1, k)
+    jb, vb = half_topk(s2, k)
+    S = (va[:, None] + vb[None, :]).reshape(-1)
+    A = np.repeat(va, k)
+    B = np.tile(vb, k)
+    I = np.repeat(ia, k)
+    J = np.tile(jb, k)
+    order = _order_candidates(S, A, B, I * C2 + J)[:k]
+    return I[order], J[order]
+
+
+# ----------------------------------------------------------------------------- 5
+def softmax(S):
+    """Softmax over the last axis, fp64."""
+    m = S.max(axis=-1, keepdims=True)
+    e = np.exp(S - m)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+# ----------------------------------------------------------------------------- 1..6
+def forward(inp, cfg, select="brute"):
+    """The layer forward for every token of ``inp['x']``.
+
+    Returns a dict with q [N][h*dk], qhat, s1 [N][h][C1], s2 [N][h][C2],
+    sub_i/sub_s [N][h][2][k] (per-half top-k, best first), idx [N][h][k]
+    (flat value rows i*C2 + j, best first), S [N][h][k] (scaled winner scores),
+    w [N][h][k] (softmax weights) and y [N][d_v].
+    """
+    h, dk, C1, C2, k = cfg.h, cfg.dk, cfg.C1, cfg.C2, cfg.k
+    q, qhat = query_network(inp["x"], inp["Wq"], inp["bn"], cfg.bn_eps)
+    s1, s2 = subkey_scores(q, inp["subkeys"], h, dk, C1)
+    N = q.shape[0]
+    pick = brute_force_topk if select == "brute" else product_key_topk
+    idx = np.zeros((N, h, k), dtype=np.int64)
+    S = np.zeros((N, h, k))
+    sub_i = np.zeros((N, h, 2, k), dtype=np.int64)
+    sub_s = np.zeros((N, h, 2, k))
+    for t in range(N):
+        for hh in range(h):
+            ii, jj = pick(s1[t, hh], s2[t, hh], k)
+            idx[t, hh] = ii * C2 + jj
+            S[t, hh] = cfg.score_scale * (s1[t, hh, ii] + s2[t, hh, jj])
+            sub_i[t, hh, 0], sub_s[t, hh, 0] = half_topk(s1[t, hh], k)
+            sub_i[t, hh, 1], sub_s[t, hh, 1] = half_topk(s2[t, hh], k)
+    w = softmax(S)
+    y = bag(w, idx, inp["values"])
+    return dict(q=q, qhat=qhat, s1=s1, s2=s2, sub_i=sub_i, sub_s=sub_s, idx=idx,
+                S=S, w=w, y=y)
+
+
+def bag(w, idx, values):
+    """y[t] = sum_h sum_j w[t][h][j] * V[idx[t][h][j]]  ("Meta AI 可扩展内存层" 5.3)."""
+    N, h, k = idx.shape
+    rows = np.asarray(values[idx.reshape(-1)], dtype=np.float64).reshape(N, h * k, -1)
+    return np.einsum("tr,trd->td", w.reshape(N, h * k), rows)
+
+
+# ----------------------------------------------------------------------------- backward
+def backward(inp, cfg, fwd, dy):
+    """Gradients of L = sum_t dy[t] . y[t] with the selected keys held fixed.
+
+    Returns dict:
+      dw   [N][h][k]   dL/dw            = dy[t] . V[row]
+      dS   [N][h][k]   dL/d(scaled score) (softmax backward)
+      g1, g2 [N][h][C1|C2]  dL/ds1, dL/ds2 (nonzero only on selected sub-keys)
+      dq   [N][h*dk], dx [N][d_in], dWq [h*dk][d_in], dgamma, dbeta [h*dk]
+      dsub [h][C1+C2][dk/2]
+      dV_rows (sorted unique rows), dV_vals [len][d_v]  (all other rows are zero)
+    """
+    h, dk, C1, C2, k = cfg.h, cfg.dk, cfg.C1, cfg.C2, cfg.k
+    dy = np.asarray(dy, dtype=np.float64)
+    idx, w = fwd["idx"], fwd["w"]
+    N = idx.shape[0]
+    V = inp["values"]
+    rows = np.asarray(V[idx.reshape(-1)], dtype=np.float64).reshape(N, h, k, -1)
+    dw = np.einsum("td,thjd->thj", dy, rows)
+    # softmax backward: dS_j = w_j (dw_j - sum_l w_l dw_l)
+    dS = w * (dw - (w * dw).sum(axis=-1, keepdims=True))
+    dsum = cfg.score_scale * dS
+    g1 = np.zeros((N, h, C1))
+    g2 = np.zeros((N, h, C2))
+    tt = np.repeat(np.arange(N), h * k)
+    hh = np.tile(np.repeat(np.arange(h), k), N)
+    np.add.at(g1, (tt, hh, (idx // C2).reshape(-1)), dsum.reshape(-1))
+    np.add.at(g2, (tt, hh, (idx % C2).reshape(-1)), dsum.reshape(-1))
+    sub = np.asarray(inp["subkeys"], dtype=np.float64)
+    q1, q2 = split_halves(fwd["q"], h, dk)
+    dq1 = np.einsum("thi,hid->thd", g1, sub[:, :C1, :])
+    dq2 = np.einsum("thj,hjd->thd", g2, sub[:, C1:, :])
+    dsub = np.zeros_like(sub)
+    dsub[:, :C1, :] = np.einsum("thi,thd->hid", g1, q1)
+    dsub[:, C1:, :] = np.einsum("thj,thd->hjd", g2, q2)
+    dq = np.concatenate([dq1, dq2], axis=2).reshape(N, h * dk)
+    mean, var, gamma, beta = (np.asarray(r, dtype=np.float64) for r in inp["bn"])
+    dq_pre = dq * gamma / np.sqrt(var + cfg.bn_eps)
+    dgamma = (dq * fwd["qhat"]).sum(axis=0)
+    dbeta = dq.sum(axis=0)
+    x = np.asarray(inp["x"], dtype=np.float64)
+    Wq = np.asarray(inp["Wq"], dtype=np.float64)
+    dWq = dq_pre.T @ x
+    dx = dq_pre @ Wq
+    # value gradient: dV[row] += w * dy[t], summed over every (t, h, j) choosing row
+    flat = idx.reshape(-1)
+    contrib = (w[..., None] * dy[:, None, None, :]).reshape(N * h * k, -1)
+    dV_rows, inv = np.unique(flat, return_inverse=True)
+    dV_vals = np.zeros((dV_rows.shape[0], dy.shape[1]))
+    np.add.at(dV_vals, inv, contrib)
+    return dict(dw=dw, dS=dS, g1=g1, g2=g2, dq=dq, dq_pre=dq_pre, dx=dx, dWq=dWq,
+                dgamma=dgamma, dbeta=dbeta, dsub=dsub, dV_rows=dV_rows, dV_vals=dV_vals)
+
+
+def loss(inp, cfg, dy, select="brute"):
+    """L = sum_t dy[t] . y[t] (the scalar whose gradient ``backward`` returns)."""
+    f = forward(inp, cfg, select=select)
+    return float((np.asarray(dy, dtype=np.float64) * f["y"]).sum()), f

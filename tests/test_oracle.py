@@ -1,0 +1,311 @@
+"""Pins of the CPU oracle against things other than itself (no GPU needed).
+
+Each test is chosen so that a plausible slip in the oracle (a dropped term, a wrong
+sign or index, a transposed operand, a wrong tie-break) fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import pkm_oracle as O
+from product_key_memory_pkm_b200.inputs import PKMConfig, TINY_FP32, make_inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _cfg(**kw):
+    base = dict(name="t", N=8, d_in=16, h=2, dk=8, C1=12, C2=9, k=4, d_v=6, dtype="f32")
+    base.update(kw)
+    return PKMConfig(**base)
+
+
+# --------------------------------------------------------------------------- golden
+def test_golden_worked_example():
+    """Hand-derived case (tests/golden/worked_example_k3.json): every forward and
+    backward quantity is a closed-form number."""
+    g = json.load(open(os.path.join(GOLDEN, "worked_example_k3.json")))
+    cfg = PKMConfig(name="golden", dtype="f32", **g["cfg"])
+    inp = {k: np.array(g[k], dtype=np.float64) for k in ("x", "Wq", "bn", "subkeys", "values")}
+    f = O.forward(inp, cfg)
+    e = g["expect"]
+    np.testing.assert_allclose(f["q"], e["q"], atol=1e-15)
+    np.testing.assert_allclose(f["s1"][0, 0], e["s1"], atol=1e-15)
+    np.testing.assert_allclose(f["s2"][0, 0], e["s2"], atol=1e-15)
+    assert f["idx"][0, 0].tolist() == e["idx"]
+    np.testing.assert_allclose(f["w"][0, 0], e["w"], atol=1e-14)
+    np.testing.assert_allclose(f["y"], e["y"], atol=1e-13)
+    # the product-key search reaches the same winners
+    f2 = O.forward(inp, cfg, select="product")
+    assert f2["idx"][0, 0].tolist() == e["idx"]
+    b = O.backward(inp, cfg, f, np.array(g["dy"], dtype=np.float64))
+    np.testing.assert_allclose(b["dw"][0, 0], e["dw"], atol=1e-13)
+    np.testing.assert_allclose(b["dS"][0, 0], e["dS"], atol=1e-13)
+    assert b["dV_rows"].tolist() == e["dV_rows"]
+    np.testing.assert_allclose(b["dV_vals"], e["dV_vals"], atol=1e-14)
+    ln2 = math.log(2.0)
+    u = e["ln2_units"]
+    np.testing.assert_allclose(b["g1"][0, 0], np.array(u["g1"]) * ln2, atol=1e-13)
+    np.testing.assert_allclose(b["g2"][0, 0], np.array(u["g2"]) * ln2, atol=1e-13)
+    for key in ("dq", "dsub", "dgamma", "dbeta", "dx", "dWq"):
+        np.testing.assert_allclose(b[key], np.array(u[key]) * ln2, atol=1e-13, err_msg=key)
+
+
+# --------------------------------------------------------------------------- selection
+def _tie_heavy_scores(rng, C1, C2):
+    # small integers: many equal sums and equal sub-scores
+    return (rng.integers(-3, 4, C1).astype(np.float64),
+            rng.integers(-3, 4, C2).astype(np.float64))
+
+
+@pytest.mark.parametrize("C1,C2,k", [(8, 8, 3), (16, 9, 4), (32, 32, 8), (7, 13, 7), (64, 40, 32)])
+def test_exactness_product_key_equals_brute_force(C1, C2, k):
+    """The k best of s1[i]+s2[j] over all C1*C2 keys lie inside top-k(s1) x top-k(s2),
+    and the product-key search returns them in the same order ("Large Memory Layers
+    with Product Keys", abstract: exact search)."""
+    rng = np.random.default_rng(C1 * 1000 + C2 * 10 + k)
+    for trial in range(60):
+        if trial % 2:
+            s1, s2 = rng.standard_normal(C1), rng.standard_normal(C2)
+        else:
+            s1, s2 = _tie_heavy_scores(rng, C1, C2)
+        bi, bj = O.brute_force_topk(s1, s2, k)
+        pi, pj = O.product_key_topk(s1, s2, k)
+        assert bi.tolist() == pi.tolist() and bj.tolist() == pj.tolist()
+
+
+def test_brute_force_is_full_sort_prefix():
+    """brute_force_topk equals the first k of a full sort of every key by the total
+    order written out with Python's sort (different code, same definition)."""
+    rng = np.random.default_rng(7)
+    for trial in range(40):
+        C1, C2, k = 40, 30, int(rng.integers(1, 31))
+        s1, s2 = _tie_heavy_scores(rng, C1, C2) if trial % 2 else (
+            rng.standard_normal(C1), rng.standard_normal(C2))
+        keys = sorted(((-(s1[i] + s2[j]), -s1[i], -s2[j], i * C2 + j)
+                       for i in range(C1) for j in range(C2)))
+        want = [kk[3] for kk in keys[:k]]
+        bi, bj = O.brute_force_topk(s1, s2, k)
+        assert (bi * C2 + bj).tolist() == want
+
+
+def test_k_equals_C_all_keys_are_candidates():
+    """k = C1 = C2: the Cartesian candidate set is the whole keyspace, so the
+    product-key path is brute force over all keys by construction."""
+    rng = np.random.default_rng(3)
+    s1, s2 = rng.standard_normal(6), rng.standard_normal(6)
+    pi, pj = O.product_key_topk(s1, s2, 6)
+    bi, bj = O.brute_force_topk(s1, s2, 6)
+    assert (pi * 6 + pj).tolist() == (bi * 6 + bj).tolist()
+    S = s1[:, None] + s2[None, :]
+    assert np.allclose(np.sort(S.ravel())[::-1][:6], s1[pi] + s2[pj])
+
+
+def test_k1_is_argmax_of_each_half():
+    rng = np.random.default_rng(4)
+    for _ in range(30):
+        s1, s2 = rng.standard_normal(20), rng.standard_normal(11)
+        i, j = O.brute_force_topk(s1, s2, 1)
+        assert i[0] == int(np.argmax(s1)) and j[0] == int(np.argmax(s2))
+
+
+def test_half_topk_order_and_ties():
+    s = np.array([1.0, 3.0, 3.0, -1.0, 2.0, 3.0])
+    i, v = O.half_topk(s, 4)
+    assert i.tolist() == [1, 2, 5, 4] and v.tolist() == [3, 3, 3, 2]
+
+
+# --------------------------------------------------------------------------- weights, bag
+def test_softmax_sums_to_one_and_monotone():
+    cfg = _cfg(score_scale=0.7)
+    inp = make_inputs(cfg, seed=1, with_dy=False)
+    f = O.forward(inp, cfg)
+    np.testing.assert_allclose(f["w"].sum(-1), 1.0, atol=1e-12)
+    # winners are listed best first, so the weights are non-increasing
+    assert np.all(np.diff(f["w"], axis=-1) <= 1e-15)
+    # ratio of weights equals exp of the score difference (closed form of softmax)
+    r = f["w"][..., 0] / f["w"][..., 1]
+    np.testing.assert_allclose(np.log(r), f["S"][..., 0] - f["S"][..., 1], rtol=1e-9, atol=1e-12)
+
+
+def test_one_hot_value_table_reads_back_the_weights():
+    """V = identity (d_v = K): y[t] is the vector of weights scattered to the chosen
+    rows and summed over heads, so indices and weights are checked at once."""
+    cfg = _cfg(C1=8, C2=6, d_v=48, h=2, k=5)
+    inp = make_inputs(cfg, seed=2, with_dy=False)
+    inp["values"] = np.eye(cfg.K)
+    f = O.forward(inp, cfg)
+    for t in range(cfg.N):
+        want = np.zeros(cfg.K)
+        for hh in range(cfg.h):
+            for j in range(cfg.k):
+                want[f["idx"][t, hh, j]] += f["w"][t, hh, j]
+        np.testing.assert_allclose(f["y"][t], want, atol=1e-14)
+        assert abs(f["y"][t].sum() - cfg.h) < 1e-12
+
+
+def test_output_is_linear_in_values():
+    cfg = _cfg()
+    inp = make_inputs(cfg, seed=3, with_dy=False)
+    rng = np.random.default_rng(0)
+    V1, V2 = rng.standard_normal((cfg.K, cfg.d_v)), rng.standard_normal((cfg.K, cfg.d_v))
+    ys = []
+    for V in (V1, V2, 2.0 * V1 - 3.0 * V2):
+        inp["values"] = V
+        ys.append(O.forward(inp, cfg)["y"])
+    np.testing.assert_allclose(ys[2], 2.0 * ys[0] - 3.0 * ys[1], atol=1e-12)
+
+
+def test_permuting_subkeys_with_values_leaves_output_unchanged():
+    """Relabel the sub-keys of each half (with the value rows moved to match): the
+    layer's output must not change (no ties in continuous random data)."""
+    cfg = _cfg(h=1)
+    inp = make_inputs(cfg, seed=4, with_dy=False)
+    y0 = O.forward(inp, cfg)["y"]
+    rng = np.random.default_rng(9)
+    p1, p2 = rng.permutation(cfg.C1), rng.permutation(cfg.C2)
+    sub = inp["subkeys"].copy()
+    sub[0, :cfg.C1] = inp["subkeys"][0, :cfg.C1][p1]
+    sub[0, cfg.C1:] = inp["subkeys"][0, cfg.C1:][p2]
+    # new sub-key a = old p1[a]; new row a*C2+b must hold old row p1[a]*C2+p2[b]
+    V = inp["values"].reshape(cfg.C1, cfg.C2, -1)[p1][:, p2].reshape(cfg.K, -1)
+    y1 = O.forward(dict(inp, subkeys=sub, values=V), cfg)["y"]
+    np.testing.assert_allclose(y1, y0, atol=1e-13)
+
+
+# --------------------------------------------------------------------------- query, scores
+def test_query_network_matches_library_batch_norm():
+    cfg = _cfg()
+    inp = make_inputs(cfg, seed=5, with_dy=False, random_bn=True)
+    q, _ = O.query_network(inp["x"], inp["Wq"], inp["bn"], cfg.bn_eps)
+    t = lambda a: torch.from_numpy(np.asarray(a, dtype=np.float64))
+    lin = torch.nn.functional.linear(t(inp["x"]), t(inp["Wq"]))
+    bn = [t(r) for r in inp["bn"]]
+    ref = torch.nn.functional.batch_norm(lin, bn[0], bn[1], bn[2], bn[3], training=False,
+                                         eps=cfg.bn_eps)
+    np.testing.assert_allclose(q, ref.numpy(), rtol=1e-13, atol=1e-13)
+
+
+def test_subkey_scores_of_one_hot_queries_are_subkey_columns():
+    cfg = _cfg(h=2, dk=8)
+    rng = np.random.default_rng(6)
+    sub = rng.standard_normal((cfg.h, cfg.C1 + cfg.C2, cfg.dk // 2))
+    q = np.zeros((cfg.h * cfg.dk, cfg.h * cfg.dk))
+    np.fill_diagonal(q, 1.0)          # token t has q = e_t
+    s1, s2 = O.subkey_scores(q, sub, cfg.h, cfg.dk, cfg.C1)
+    half = cfg.dk // 2
+    for t in range(q.shape[0]):
+        hh, r = divmod(t, cfg.dk)
+        for h2 in range(cfg.h):
+            if h2 != hh:
+                assert not s1[t, h2].any() and not s2[t, h2].any()
+        if r < half:
+            np.testing.assert_array_equal(s1[t, hh], sub[hh, :cfg.C1, r])
+            assert not s2[t, hh].any()
+        else:
+            np.testing.assert_array_equal(s2[t, hh], sub[hh, cfg.C1:, r - half])
+            assert not s1[t, hh].any()
+
+
+# --------------------------------------------------------------------------- backward
+def _torch_loss_fixed_selection(inp, cfg, idx, dy):
+    """An independent forward in torch fp64 that touches only the selected keys."""
+    t = lambda a: torch.tensor(np.asarray(a, dtype=np.float64), requires_grad=True)
+    x, Wq, sub, V = t(inp["x"]), t(inp["Wq"]), t(inp["subkeys"]), t(inp["values"])
+    mean, var = (torch.tensor(np.asarray(r, dtype=np.float64)) for r in inp["bn"][:2])
+    gamma, beta = t(inp["bn"][2]), t(inp["bn"][3])
+    q = (x @ Wq.T - mean) / torch.sqrt(var + cfg.bn_eps) * gamma + beta
+    N = q.shape[0]
+    qh = q.reshape(N, cfg.h, cfg.dk)
+    half = cfg.dk // 2
+    idx_t = torch.from_numpy(np.asarray(idx))
+    ii, jj = idx_t // cfg.C2, idx_t % cfg.C2
+    y = torch.zeros(N, V.shape[1], dtype=torch.float64)
+    for hh in range(cfg.h):
+        Ca = sub[hh, ii[:, hh]]                      # [N][k][half]
+        Cb = sub[hh, cfg.C1 + jj[:, hh]]
+        sa = (Ca * qh[:, hh, None, :half]).sum(-1)
+        sb = (Cb * qh[:, hh, None, half:]).sum(-1)
+        w = torch.softmax(cfg.score_scale * (sa + sb), dim=-1)
+        y = y + (w[..., None] * V[idx_t[:, hh]]).sum(1)
+    L = (torch.from_numpy(np.asarray(dy, dtype=np.float64)) * y).sum()
+    L.backward()
+    return dict(dx=x.grad.numpy(), dWq=Wq.grad.numpy(), dsub=sub.grad.numpy(),
+                dV=V.grad.numpy(), dgamma=gamma.grad.numpy(), dbeta=beta.grad.numpy())
+
+
+@pytest.mark.parametrize("scale", [1.0, 0.37])
+def test_backward_matches_autograd_of_independent_forward(scale):
+    cfg = _cfg(score_scale=scale, N=10, h=2)
+    inp = make_inputs(cfg, seed=8, random_bn=True)
+    f = O.forward(inp, cfg)
+    b = O.backward(inp, cfg, f, inp["dy"])
+    ref = _torch_loss_fixed_selection(inp, cfg, f["idx"], inp["dy"])
+    for key in ("dx", "dWq", "dsub", "dgamma", "dbeta"):
+        np.testing.assert_allclose(b[key], ref[key], rtol=1e-10, atol=1e-12, err_msg=key)
+    dV = np.zeros_like(ref["dV"])
+    dV[b["dV_rows"]] = b["dV_vals"]
+    np.testing.assert_allclose(dV, ref["dV"], rtol=1e-10, atol=1e-12)
+
+
+def test_value_gradient_row_sum_closed_form():
+    """sum_r dV[r] = sum_t sum_h (sum_j w) dy[t] = h * sum_t dy[t]."""
+    cfg = _cfg(h=3, N=12)
+    inp = make_inputs(cfg, seed=10)
+    f = O.forward(inp, cfg)
+    b = O.backward(inp, cfg, f, inp["dy"])
+    np.testing.assert_allclose(b["dV_vals"].sum(0), cfg.h * inp["dy"].astype(np.float64).sum(0),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_backward_central_finite_differences_tiny_config():
+    """Central differences in fp64 on the tiny workload's shapes (sampled entries),
+    skipping perturbations that change the selected keys."""
+    cfg = TINY_FP32.with_(N=16)
+    inp = make_inputs(cfg, seed=0, random_bn=True)
+    inp = {k: np.asarray(v, dtype=np.float64) for k, v in inp.items()}
+    dy = inp["dy"]
+    L0, f0 = O.loss(inp, cfg, dy)
+    b = O.backward(inp, cfg, f0, dy)
+    dV = {int(r): v for r, v in zip(b["dV_rows"], b["dV_vals"])}
+    rng = np.random.default_rng(11)
+    eps = 1e-6
+    checks = []
+    for name, shape in (("x", inp["x"].shape), ("Wq", inp["Wq"].shape),
+                        ("subkeys", inp["subkeys"].shape), ("bn", inp["bn"].shape)):
+        for _ in range(25):
+            checks.append((name, tuple(int(rng.integers(0, s)) for s in shape)))
+    for r in list(dV)[:10]:
+        checks.append(("values", (r, int(rng.integers(0, cfg.d_v)))))
+    checks.append(("values", (int(np.setdiff1d(np.arange(cfg.K), b["dV_rows"])[0]), 0)))
+    tested = 0
+    for name, ix in checks:
+        if name == "bn" and ix[0] < 2:
+            ix = (ix[0] + 2,) + ix[1:]           # running stats are not parameters
+        vals = []
+        ok = True
+        for sgn in (1, -1):
+            p = {k: v.copy() for k, v in inp.items()}
+            p[name][ix] += sgn * eps
+            L, f = O.loss(p, cfg, dy)
+            ok &= np.array_equal(f["idx"], f0["idx"])
+            vals.append(L)
+        if not ok:
+            continue
+        fd = (vals[0] - vals[1]) / (2 * eps)
+        if name == "x":
+            an = b["dx"][ix]
+        elif name == "Wq":
+            an = b["dWq"][ix]
+        elif name == "subkeys":
+            an = b["dsub"][ix]
+        elif name == "bn":
+            an = (b["dgamma"] if ix[0] == 2 else b["dbeta"])[ix[1]]
+        else:
+            an = dV.get(ix[0], np.zeros(cfg.d_v))[ix[1]]
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, ix, fd, an)
+        tested += 1
+    assert tested >= 90
