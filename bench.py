@@ -1,0 +1,422 @@
+"""Benchmark of the product-key memory layer (forward + sparse backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+                    [--workload NAME] [--no-e2e] [--no-cpu-baseline]
+
+One step = one pass of the whole layer over one batch of synthetic tokens: query
+network, sub-key scoring with per-half top-k, candidate top-k with softmax, value
+bag (forward), then the value-gradient stage and the query-gradient stage
+(backward).  Inputs are resident in HBM when the timed region starts; the L2 is
+flushed (a 256 MiB write) before every timed step, outside the step's events.
+Timing: CUDA events on the launching stream, W warm-up steps, K timed steps
+bracketed by barrier + synchronize, max over ranks.  With N > 1 (torchrun), every
+rank processes its own batch against its own replica of the tables (tokens are
+independent, so there is no data-path collective): weak scaling.
+
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from product_key_memory_pkm_b200.inputs import CONFIGS, FULL_K1024, make_inputs  # noqa: E402
+
+METRIC = "PKM layer tokens/s (fwd, fwd+bwd) at |K|=1024²,h=4,k=32; gather HBM GB/s vs peak"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return dict(hbm=float(j["hbm_gbs"]), bf16=float(j["bf16_tflops"]),
+                    bf16_sus=float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def _cfg_json(cfg):
+    return {"workload": cfg.name, "N_tokens": cfg.N, "d_in": cfg.d_in, "h": cfg.h, "dk": cfg.dk,
+            "C1": cfg.C1, "C2": cfg.C2, "K": cfg.K, "k": cfg.k, "d_v": cfg.d_v,
+            "value_dtype": cfg.dtype, "l2": "flushed before every timed step (256 MiB write)"}
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid: str | None):
+        self.uuid = gpu_uuid
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "200"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+def time_oracle(cfg, inp, seconds: float, batch: int = 8):
+    """Oracle forward (brute force over all keys) + backward on successive token batches
+    until ``seconds`` of host time have passed.  Returns (tokens/s, tokens, threads)."""
+    from oracle import pkm_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    done, t0 = 0, time.perf_counter()
+    while True:
+        sl = slice(done % cfg.N, done % cfg.N + batch)
+        sub = dict(inp, x=inp["x"][sl], dy=inp["dy"][sl])
+        f = O.forward(sub, cfg)
+        O.backward(sub, cfg, f, sub["dy"])
+        done += sub["x"].shape[0]
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            return done / el, done, threads
+
+
+# ---------------------------------------------------------------- the B200 arm
+def run_b200(args, cfg, rank, world, dist):
+    import torch
+
+    from product_key_memory_pkm_b200 import build as B
+    from product_key_memory_pkm_b200 import pkm as P
+
+    if not os.path.exists(B.LIB):
+        if rank == 0:
+            print("building libpkm_b200.so", file=sys.stderr)
+        B.build()
+    P.load()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    st = torch.cuda.current_stream()
+
+    t_gen = time.perf_counter()
+    inp = make_inputs(cfg, seed=0)
+    if world > 1:   # each rank its own batch of tokens; the tables are the same
+        other = make_inputs(cfg.with_(N=cfg.N), seed=1000 + rank)
+        inp["x"], inp["dy"] = other["x"], other["dy"]
+    bf = torch.bfloat16
+    x = torch.from_numpy(inp["x"]).to(bf).to(dev)
+    Wq = torch.from_numpy(inp["Wq"]).to(bf).to(dev)
+    bn = torch.from_numpy(inp["bn"]).to(dev)
+    sub = torch.from_numpy(inp["subkeys"]).to(bf).to(dev)
+    V = torch.from_numpy(inp["values"]).to(bf).to(dev)
+    dy = torch.from_numpy(inp["dy"]).to(dev)
+    gen_s = time.perf_counter() - t_gen
+
+    dims = P.Dims.from_config(cfg)
+    saved = P.alloc_saved(dims, with_qhat=True)
+    y = torch.empty(cfg.N, cfg.d_v, device=dev)
+    dx = torch.empty(cfg.N, cfg.d_in, device=dev)
+    dWq = torch.zeros(cfg.h * cfg.dk, cfg.d_in, device=dev)
+    dbn = torch.zeros(2, cfg.h * cfg.dk, device=dev)
+    dsub = torch.zeros(cfg.h, cfg.C1 + cfg.C2, cfg.dk // 2, device=dev)
+    dV = torch.zeros(cfg.K, cfg.d_v, device=dev)
+    dw = torch.empty(cfg.N, cfg.h, cfg.k, device=dev)
+    ws = P.alloc_workspace(dims, P.PKM_BWD, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    names = ["query", "subkey_scores", "candidate_topk", "gather_bag", "value_grad", "query_grad"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(st)
+        mark(0)
+        P.pkm_query(dims, x, Wq, bn, saved, stream=st)
+        mark(1)
+        P.pkm_subkey_scores(dims, sub, saved, stream=st)
+        mark(2)
+        P.pkm_candidate_topk(dims, saved, stream=st)
+        mark(3)
+        P.pkm_gather_bag(dims, V, saved["idx"], saved["w"], y, stream=st)
+        mark(4)
+        P.pkm_value_grad(dims, V, saved, dy, dw, dvalues=dV, workspace=ws, stream=st)
+        mark(5)
+        P.pkm_query_grad(dims, x, Wq, bn, sub, saved, dw, dx=dx, dWq=dWq, dbn=dbn, dsubkeys=dsub,
+                         workspace=ws, stream=st)
+        mark(6)
+
+    clocks = ClockSampler(torch.cuda.get_device_properties(dev).uuid and
+                          "GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    clocks.start()
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if P.pkm_check_status(st) != P.PKM_OK:
+        raise RuntimeError("device status after warm-up is not OK")
+    # algorithmic bytes of the value stage need the number of distinct rows
+    U = int(torch.unique(saved["idx"]).numel())
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = P.pkm_launch_count()
+    for s in range(args.steps):
+        flush.zero_()
+        step(evs[s])
+    torch.cuda.synchronize()
+    launches = P.pkm_launch_count() - launches0
+    if dist is not None:
+        dist.barrier()
+    stage_ms = np.array([[evs[s][i].elapsed_time(evs[s][i + 1]) for i in range(6)]
+                         for s in range(args.steps)])
+    step_ms = float(stage_ms.sum(1).mean())
+    fwd_ms = float(stage_ms[:, :4].sum(1).mean())
+    if P.pkm_check_status(st) != P.PKM_OK:
+        raise RuntimeError("device status after the timed steps is not OK")
+
+    # e2e through the public API with host buffers: H2D of x and dy, D2H of y and dx
+    e2e = None
+    if not args.no_e2e:
+        xh = torch.from_numpy(inp["x"]).to(bf).pin_memory()
+        dyh = torch.from_numpy(inp["dy"]).pin_memory()
+        yh = torch.empty(cfg.N, cfg.d_v).pin_memory()
+        dxh = torch.empty(cfg.N, cfg.d_in).pin_memory()
+        e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
+
+        def e2e_step(pair):
+            pair[0].record(st)
+            x.copy_(xh, non_blocking=True)
+            dy.copy_(dyh, non_blocking=True)
+            P.pkm_forward(dims, x, Wq, bn, sub, V, y, saved, stream=st)
+            P.pkm_backward(dims, x, Wq, bn, sub, V, saved, dy, dx=dx, dWq=dWq, dbn=dbn,
+                           dsubkeys=dsub, dvalues=dV, dw_out=dw, workspace=ws, stream=st)
+            yh.copy_(y, non_blocking=True)
+            dxh.copy_(dx, non_blocking=True)
+            pair[1].record(st)
+        for _ in range(max(1, args.warmup)):
+            e2e_step(e_ev[0])
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        for s in range(args.steps):
+            flush.zero_()
+            e2e_step(e_ev[s])
+        torch.cuda.synchronize()
+        e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in e_ev]))
+        e2e = dict(ms=e2e_ms,
+                   h2d=x.numel() * x.element_size() + dy.numel() * dy.element_size(),
+                   d2h=y.numel() * 4 + dx.numel() * 4)
+    clk = clocks.stop()
+
+    # max over ranks
+    vals = torch.tensor([step_ms, fwd_ms, e2e["ms"] if e2e else 0.0], device=dev,
+                        dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    step_ms, fwd_ms, e2e_ms = (float(v) for v in vals.tolist())
+    if rank != 0:
+        return None
+
+    pk = _peaks()
+    st_mean = stage_ms.mean(0)
+    hk = cfg.h * cfg.k
+    sel = cfg.N * hk
+    bytes_gather = sel * cfg.d_v * 2 + cfg.N * cfg.d_v * 4 + sel * 8
+    bytes_value = U * cfg.d_v * (2 + 8) + cfg.N * cfg.d_v * 4 + sel * 12
+    rl = {
+        "gather_bag": dict(bytes=bytes_gather, ms=float(st_mean[3])),
+        "value_grad": dict(bytes=bytes_value, ms=float(st_mean[4])),
+    }
+    dom = max(rl, key=lambda k: rl[k]["ms"])
+    traffic = _ncu_traffic(dom)
+
+    def roof(name):
+        r = rl[name]
+        ach = r["bytes"] / (r["ms"] * 1e-3) / 1e9
+        return {"kernel": name, "bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm"],
+                "unit": "GB/s", "frac": round(ach / pk["hbm"], 4),
+                "traffic": traffic if name == dom else _ncu_traffic(name),
+                "algorithmic_bytes": int(r["bytes"]), "peak_source": pk["src"]}
+
+    out = {
+        "metric": METRIC,
+        "value": round(cfg.N * world / (step_ms * 1e-3), 1),
+        "unit": "tokens/s (fwd+bwd)",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded; tables random-init, no trained weights)",
+        "config": dict(_cfg_json(cfg), parallelism=f"replicas{world}" if world > 1 else "single"),
+        "fwd": {"value": round(cfg.N * world / (fwd_ms * 1e-3), 1), "unit": "tokens/s (fwd)",
+                "ms": round(fwd_ms, 4)},
+        "stage_ms": {n: round(float(v), 4) for n, v in zip(names, st_mean)},
+        "roofline": roof(dom),
+        "roofline_other": [roof(n) for n in rl if n != dom],
+        "clocks": clk,
+        "gpu_launches": int(launches),
+        "input_gen_s": round(gen_s, 1),
+    }
+    if e2e:
+        out["e2e"] = {"value": round(cfg.N * world / (e2e_ms * 1e-3), 1),
+                      "unit": "tokens/s (fwd+bwd, host buffers in/out)",
+                      "h2d_bytes_per_step": int(e2e["h2d"]), "d2h_bytes_per_step": int(e2e["d2h"]),
+                      "ms": round(e2e_ms, 4)}
+    if world == 1 and not args.no_cpu_baseline:
+        v, n, thr = time_oracle(cfg, inp, args.cpu_seconds)
+        out["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s (fwd+bwd)", "cores": thr,
+                               "kind": "oracle",
+                               "sample": f"{n} tokens of the same batch, fp64 numpy oracle: "
+                                         f"brute force over all {cfg.K} keys per head, "
+                                         f"analytic backward; ~{args.cpu_seconds:.0f} s of host time"}
+    return out
+
+
+def _ncu_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, when it is still current."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        j = json.load(open(p))
+        ent = j.get(kernel)
+        if not ent:
+            return None
+        import hashlib
+        h = hashlib.sha256()
+        for f in ent["sources"]:
+            h.update(open(os.path.join(ROOT, f), "rb").read())
+        if h.hexdigest() != ent["source_sha256"]:
+            return None
+        return ent["dram_bytes_per_launch"]
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------- the reference arm
+def run_reference(args, cfg, rank):
+    """The CPU oracle, as it stands, on a bounded sample of the workload per step."""
+    if rank != 0:
+        return None
+    from oracle import pkm_oracle as O
+    inp = make_inputs(cfg, seed=0)
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    per_step = args.ref_tokens
+    times = []
+    for s in range(args.warmup + args.steps):
+        sl = slice((s * per_step) % cfg.N, (s * per_step) % cfg.N + per_step)
+        sub = dict(inp, x=inp["x"][sl], dy=inp["dy"][sl])
+        t0 = time.perf_counter()
+        f = O.forward(sub, cfg)
+        O.backward(sub, cfg, f, sub["dy"])
+        if s >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    ms = 1e3 * float(np.mean(times))
+    v = round(per_step / (ms * 1e-3), 3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s (fwd+bwd)",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": dict(_cfg_json(cfg), parallelism="host cores"),
+        "cpu_baseline": {"value": v, "unit": "tokens/s (fwd+bwd)", "cores": threads,
+                         "kind": "oracle",
+                         "sample": f"{per_step} tokens per step of the same batch; fp64 numpy "
+                                   f"oracle, brute force over all {cfg.K} keys per head"},
+        "e2e": {"value": v, "unit": "tokens/s (fwd+bwd)", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--workload", default=FULL_K1024.name, choices=sorted(CONFIGS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-tokens", type=int, default=8)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    cfg = CONFIGS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if args.impl == "reference":
+        out = run_reference(args, cfg, rank)
+    else:
+        if world > 1:
+            import datetime
+
+            import torch
+            import torch.distributed as tdist
+            torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+            tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+            dist = tdist
+        try:
+            out = run_b200(args, cfg, rank, world, dist)
+        finally:
+            if dist is not None:
+                dist.destroy_process_group()
+    if rank == 0 and out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,188 @@
+/*
+ * pkm.h -- C ABI of the B200 product-key memory (PKM) layer library.
+ *
+ * The layer (sources: "Large Memory Layers with Product Keys", method-details list
+ * and abstract; "Meta AI 可扩展内存层" sections 3.2, 4.3-4.5, 5.1-5.3, 9.2):
+ *
+ *   F1  q = gamma * (x Wq^T - mean) / sqrt(var + eps) + beta     query network
+ *   F2  per head h and half s: scores of q_half against every sub-key of the
+ *       half (C for s = 0, C' for s = 1), then the top-k of each half
+ *   F3  the k x k Cartesian candidates scored s1[a] + s2[b], the best k kept
+ *       (the exact top-k over all C1*C2 product keys), value row i*C2 + j,
+ *       w = softmax(score_scale * (s1 + s2)) over the k winners
+ *   F4  y[t] = sum_h sum_j w[t][h][j] * V[idx[t][h][j]]
+ *   backward: gradients of sum_t dy[t] . y[t] with the selected keys held fixed;
+ *       the value gradient is a scatter-add whose duplicate rows are combined
+ *       before any write (one writer per row, no atomics, deterministic).
+ *
+ * Ordering: per half, (score desc, index asc); candidates, (s1+s2 desc, s1 desc,
+ * s2 desc, flat index asc).  Scores are fp32 on the device.
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer is a DEVICE pointer unless stated otherwise; the caller owns
+ *     all memory.  The library never allocates or frees device memory and never
+ *     synchronises, except pkm_check_status.
+ *   - All work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is
+ *     the legacy default stream) and is asynchronous.
+ *   - Row-major layouts:
+ *       x        [N][d_in]            bf16 (fp32 with PKM_F_FP32)
+ *       Wq       [h*dk][d_in]         bf16 (fp32 with PKM_F_FP32)  Linear weight, out x in
+ *       bn       [4][h*dk]            fp32: running mean, running var, gamma, beta
+ *       subkeys  [h][C1+C2][dk/2]     bf16 (fp32 with PKM_F_FP32)  rows [0,C1) = C, [C1,C1+C2) = C'
+ *       values   [C1*C2][d_v]         bf16 (fp32 with PKM_F_FP32)
+ *       y, dy    [N][d_v]             fp32
+ *   - Gradients of parameters ACCUMULATE (+=) into the caller's buffers; dx is
+ *     overwritten.  A NULL gradient pointer skips that gradient.
+ *   - Host-side validation happens before any launch and returns an error status
+ *     without touching the device.  Device-side problems (a bounded wait that
+ *     expired, an out-of-range index) set a status word that pkm_check_status
+ *     reports; kernels never trap.
+ *   - Limits: 1 <= k <= 32, k <= min(C1, C2), h <= 64, dk/2 <= 1024 (bf16) or 512 (fp32), dk % 32 == 0 (bf16) or dk % 8 == 0
+ *     (fp32), d_in % 8 == 0, d_v % 8 == 0, C1*C2 < 2^31, pointers 16-byte aligned.
+ *     N == 0 is a no-op returning PKM_OK.
+ */
+#ifndef PKM_H_
+#define PKM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PKM_OK = 0,
+  PKM_ERR_INVALID_ARG = 1,     /* null/misaligned pointer, bad size, k > C, ... */
+  PKM_ERR_UNSUPPORTED = 2,     /* legal but outside this build's limits (k > 32, ...) */
+  PKM_ERR_WORKSPACE = 3,       /* workspace pointer NULL or smaller than pkm_workspace_bytes */
+  PKM_ERR_CUDA = 4,            /* a CUDA runtime call failed (launch, attribute, ...) */
+  PKM_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait expired */
+  PKM_ERR_DEVICE_INDEX = 6     /* a device-side index check failed */
+} pkm_status;
+
+/* flags */
+#define PKM_F_FP32 0x1u  /* x, Wq, subkeys, values are fp32 (CUDA-core kernels) */
+#define PKM_F_SIMT 0x2u  /* bf16 storage, but CUDA-core kernels instead of tensor cores */
+
+typedef struct {
+  int64_t N;          /* tokens */
+  int32_t d_in;       /* input width */
+  int32_t h;          /* heads */
+  int32_t dk;         /* query width per head; halves of dk/2 */
+  int32_t C1, C2;     /* |C|, |C'| sub-keys per half */
+  int32_t k;          /* top-k per half and kept product keys per head */
+  int32_t d_v;        /* value width */
+  float bn_eps;       /* BatchNorm epsilon (> 0) */
+  float score_scale;  /* softmax temperature factor (> 0); selection ignores it */
+  uint32_t flags;     /* PKM_F_* */
+} pkm_dims;
+
+/* What the forward writes and the backward reads (caller-owned device buffers).
+ *   q      bf16 storage: [2][N][h*dk] bf16, the query split as q = hi + lo
+ *          (hi = bf16(q), lo = bf16(q - hi)); fp32 storage: [N][h*dk] fp32.
+ *   qhat   optional [N][h*dk] fp32 normalised pre-affine query (x Wq^T - mean) /
+ *          sqrt(var + eps); needed only for the gamma gradient.  May be NULL.
+ *   sub_s  [N][h][2][k] fp32 per-half top-k scores, best first
+ *   sub_i  [N][h][2][k] int32 per-half top-k sub-key indices, best first
+ *   idx    [N][h][k] int32 selected value rows i*C2 + j, best first
+ *   w      [N][h][k] fp32 softmax weights                                     */
+typedef struct {
+  void* q;
+  float* qhat;
+  float* sub_s;
+  int32_t* sub_i;
+  int32_t* idx;
+  float* w;
+} pkm_saved;
+
+#define PKM_SAVED_Q 0
+#define PKM_SAVED_QHAT 1
+#define PKM_SAVED_SUB_S 2
+#define PKM_SAVED_SUB_I 3
+#define PKM_SAVED_IDX 4
+#define PKM_SAVED_W 5
+
+#define PKM_FWD 0
+#define PKM_BWD 1
+
+/* Bytes of one pkm_saved field (PKM_SAVED_*) for these dims; 0 for bad input. */
+size_t pkm_saved_bytes(const pkm_dims* d, int field);
+
+/* Bytes of device workspace pkm_forward (which = PKM_FWD) or pkm_backward
+ * (PKM_BWD) needs.  The workspace is scratch: its contents on entry are ignored
+ * and on return are unspecified.  256-byte alignment is required. */
+size_t pkm_workspace_bytes(const pkm_dims* d, int which);
+
+/* Forward F1..F4 ("Large Memory Layers with Product Keys", method details).
+ *   bn: [4][h*dk] fp32 (mean, var, gamma, beta).  y: [N][d_v] fp32, overwritten.
+ *   saved: every field except qhat must be non-NULL. */
+pkm_status pkm_forward(const pkm_dims* d, const void* x, const void* Wq, const float* bn,
+                       const void* subkeys, const void* values, float* y,
+                       const pkm_saved* saved, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/* Backward of sum_t dy[t].y[t] with the selected keys of `saved` held fixed.
+ *   dx       [N][d_in] fp32, overwritten (NULL: skip)
+ *   dWq      [h*dk][d_in] fp32, += (NULL: skip)
+ *   dbn      [2][h*dk] fp32, += (d gamma, d beta) (NULL: skip; needs saved->qhat)
+ *   dsubkeys [h][C1+C2][dk/2] fp32, += (NULL: skip)
+ *   dvalues  [C1*C2][d_v] fp32, += dense table; only selected rows are touched
+ *            (NULL: skip)
+ *   dw_out   optional [N][h][k] fp32: dL/dw per selected key (NULL: skip)   */
+pkm_status pkm_backward(const pkm_dims* d, const void* x, const void* Wq, const float* bn,
+                        const void* subkeys, const void* values, const pkm_saved* saved,
+                        const float* dy, float* dx, float* dWq, float* dbn, float* dsubkeys,
+                        float* dvalues, float* dw_out, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* ---- the backward's two stages; pkm_backward runs both ----
+ * Value stage (sort of the selections by value row, then one pass per distinct row):
+ *   dw [N][h][k] fp32 out (required), dvalues += (NULL: skip).
+ * Query stage (softmax backward onto the selected sub-keys, query-half and sub-key
+ * gradients, BatchNorm backward, dense query gradients): reads dw from the value
+ * stage.  Both stages take the same workspace (pkm_workspace_bytes(d, PKM_BWD)). */
+pkm_status pkm_value_grad(const pkm_dims* d, const void* values, const pkm_saved* saved,
+                          const float* dy, float* dvalues, float* dw, void* workspace,
+                          size_t workspace_bytes, void* stream);
+pkm_status pkm_query_grad(const pkm_dims* d, const void* x, const void* Wq, const float* bn,
+                          const void* subkeys, const pkm_saved* saved, const float* dw, float* dx,
+                          float* dWq, float* dbn, float* dsubkeys, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/* ---- the forward's steps, each callable alone (same layouts as above) ---- */
+
+/* F1: writes saved->q (and saved->qhat when non-NULL). */
+pkm_status pkm_query(const pkm_dims* d, const void* x, const void* Wq, const float* bn,
+                     const pkm_saved* saved, void* stream);
+
+/* F2 (pkm_subkey_scores): from saved->q, writes saved->sub_s and saved->sub_i. */
+pkm_status pkm_subkey_scores(const pkm_dims* d, const void* subkeys, const pkm_saved* saved,
+                             void* stream);
+
+/* F3 (pkm_candidate_topk): from sub_s/sub_i, writes idx and w. */
+pkm_status pkm_candidate_topk(const pkm_dims* d, const pkm_saved* saved, void* stream);
+
+/* F4 (pkm_gather_bag): y[t] = sum_h sum_j w * V[idx]; y overwritten. */
+pkm_status pkm_gather_bag(const pkm_dims* d, const void* values, const int32_t* idx,
+                          const float* w, float* y, void* stream);
+
+/* Synchronises `stream`, then reads and clears the device status word of the
+ * current device.  Returns PKM_OK, PKM_ERR_DEVICE_TIMEOUT, PKM_ERR_DEVICE_INDEX or
+ * PKM_ERR_CUDA (when the synchronisation itself failed). */
+pkm_status pkm_check_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* pkm_status_string(pkm_status s);
+
+/* Number of kernels this library has launched in this process (diagnostics). */
+unsigned long long pkm_launch_count(void);
+
+/* Build identification string (static). */
+const char* pkm_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKM_H_ */

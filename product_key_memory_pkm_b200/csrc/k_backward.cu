@@ -1,0 +1,557 @@
+// Backward of the product-key memory layer with the selected keys held fixed
+// (the top-k is piecewise constant; "Meta AI 可扩展内存层" 6.1 and 9.2: only the
+// selected slots receive gradient, and the top-k passes gradient only to the
+// selected positions).
+//
+//   B1-B2  sort the N*h*k selections by value row (stable LSD radix), segment table
+//   B3     one warp per distinct row r: read V[r] once, for each selection e of r
+//          dw[e] = dy[t] . V[r] and acc += w[e] * dy[t]; then dV[r] += acc
+//          (duplicates combined before the single write; no atomics)
+//   B4     one warp per (t, h): dS = w (dw - sum w dw), g1/g2 = score_scale * dS
+//          summed onto the selected sub-keys of each half
+//   B5     dq_half = sum_a g[a] C[i_a];  BatchNorm backward dq_pre = dq gamma /
+//          sqrt(var + eps); d gamma, d beta by deterministic two-stage reduction
+//          dC[i] += sum over (t, a) choosing i of g * q_half[t]  (sorted segments)
+//   B7     dx = dq_pre Wq,  dWq += dq_pre^T x
+#include "k_sort.cuh"
+
+namespace pkm {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+
+template <typename T>
+struct VecT;
+template <>
+struct VecT<__nv_bfloat16> {
+  static constexpr int E = 8;
+  __device__ static void load(const __nv_bfloat16* p, float* f) {
+    uint4 u = *reinterpret_cast<const uint4*>(p);
+    bf16x8_to_f32(u, f);
+  }
+};
+template <>
+struct VecT<float> {
+  static constexpr int E = 4;
+  __device__ static void load(const float* p, float* f) {
+    float4 u = *reinterpret_cast<const float4*>(p);
+    f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
+  }
+};
+
+// ------------------------------------------------------------------ B3
+// CH = 16-byte value chunks per lane per column block (column block = 32*CH*E).
+template <typename TV, int CH>
+__global__ void __launch_bounds__(256) value_rows_kernel(
+    const int* __restrict__ seg, const int* __restrict__ U_ptr, const int32_t* __restrict__ rows,
+    const int32_t* __restrict__ ents, const TV* __restrict__ V, const float* __restrict__ w,
+    const float* __restrict__ dy, float* __restrict__ dV, float* __restrict__ dw, int hk, int d_v,
+    int64_t K, int* status) {
+  constexpr int E = VecT<TV>::E;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int U = *U_ptr;
+  const int nvec = d_v / E;
+  for (int64_t u = warp0; u < U; u += nwarps) {
+    const int p0 = seg[u], p1 = seg[u + 1];
+    const int32_t r = rows[p0];
+    if (r < 0 || r >= K) {
+      set_status(status, kDevIndex);
+      continue;
+    }
+    for (int cb = 0; cb < nvec; cb += 32 * CH) {
+      float v[CH][E], acc[CH][E];
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const int vec = cb + lane + 32 * c;
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[c][e] = 0.f;
+        if (vec < nvec)
+          VecT<TV>::load(V + (int64_t)r * d_v + (int64_t)vec * E, v[c]);
+        else
+#pragma unroll
+          for (int e = 0; e < E; ++e) v[c][e] = 0.f;
+      }
+      for (int p = p0; p < p1; ++p) {
+        const int32_t ent = ents[p];
+        const int64_t t = ent / hk;
+        const float wt = w[ent];
+        float dot = 0.f;
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          const int vec = cb + lane + 32 * c;
+          if (vec < nvec) {
+            const float4* g = reinterpret_cast<const float4*>(dy + t * d_v + (int64_t)vec * E);
+#pragma unroll
+            for (int e4 = 0; e4 < E / 4; ++e4) {
+              float4 d4 = g[e4];
+              float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                dot = fmaf(dd[e], v[c][e4 * 4 + e], dot);
+                acc[c][e4 * 4 + e] = fmaf(wt, dd[e], acc[c][e4 * 4 + e]);
+              }
+            }
+          }
+        }
+        dot = warp_sum(dot);
+        if (lane == 0) dw[ent] = (cb == 0) ? dot : dw[ent] + dot;
+      }
+      if (dV) {
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          const int vec = cb + lane + 32 * c;
+          if (vec < nvec) {
+            float4* o = reinterpret_cast<float4*>(dV + (int64_t)r * d_v + (int64_t)vec * E);
+#pragma unroll
+            for (int e4 = 0; e4 < E / 4; ++e4) {
+              float4 x = o[e4];
+              x.x += acc[c][e4 * 4 + 0];
+              x.y += acc[c][e4 * 4 + 1];
+              x.z += acc[c][e4 * 4 + 2];
+              x.w += acc[c][e4 * 4 + 3];
+              o[e4] = x;
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ B4
+__global__ void __launch_bounds__(256) softmax_bwd_kernel(
+    const float* __restrict__ w, const float* __restrict__ dw, const int32_t* __restrict__ idx,
+    const int32_t* __restrict__ sub_i, float* __restrict__ gsub, int64_t NH, int k, int C2,
+    float scale) {
+  const int lane = threadIdx.x & 31;
+  const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (g >= NH) return;
+  const bool live = lane < k;
+  const float wj = live ? w[g * k + lane] : 0.f;
+  const float dwj = live ? dw[g * k + lane] : 0.f;
+  const int32_t ij = live ? idx[g * k + lane] : 0;
+  const float s = warp_sum(wj * dwj);
+  const float dsum = scale * wj * (dwj - s);
+  const int32_t ia = live ? sub_i[g * 2 * k + lane] : -1;
+  const int32_t jb = live ? sub_i[g * 2 * k + k + lane] : -1;
+  float g1 = 0.f, g2 = 0.f;
+  for (int j = 0; j < k; ++j) {
+    const int32_t I = __shfl_sync(kFull, ij / C2, j);
+    const int32_t J = __shfl_sync(kFull, ij % C2, j);
+    const float D = __shfl_sync(kFull, dsum, j);
+    if (ia == I) g1 += D;
+    if (jb == J) g2 += D;
+  }
+  if (live) {
+    gsub[g * 2 * k + lane] = g1;
+    gsub[g * 2 * k + k + lane] = g2;
+  }
+}
+
+// ------------------------------------------------------------------ B5a + B6
+// grid (token blocks, h*2); 8 warps, each warp walks tokens; lane owns 16-byte
+// chunks of the half (MAXC chunks at most).  Writes dq_pre (fp32) and per-block
+// partial sums of dq * qhat and dq for the BatchNorm affine gradients.
+constexpr int kDqTokensPerBlock = 64;
+
+template <typename TS, int MAXC>
+__global__ void __launch_bounds__(256) dq_kernel(
+    const float* __restrict__ gsub, const int32_t* __restrict__ sub_i, const TS* __restrict__ sub,
+    const float* __restrict__ bn, const float* __restrict__ qhat, float* __restrict__ dq_pre,
+    float* __restrict__ part, int64_t N, int h, int dk, int C1, int C2, int k, float eps) {
+  constexpr int E = VecT<TS>::E;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int hs = blockIdx.y, hh = hs >> 1, s = hs & 1;
+  const int half = dk / 2, hq = h * dk;
+  const int nvec = half / E;
+  const TS* Cb = sub + ((int64_t)hh * (C1 + C2) + (s ? C1 : 0)) * half;
+  const int col0 = hh * dk + s * half;
+  float pg[MAXC][E], pb[MAXC][E];
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c)
+#pragma unroll
+    for (int e = 0; e < E; ++e) pg[c][e] = pb[c][e] = 0.f;
+  const int64_t tb = (int64_t)blockIdx.x * kDqTokensPerBlock;
+  for (int tt = wid; tt < kDqTokensPerBlock; tt += 8) {
+    const int64_t t = tb + tt;
+    if (t >= N) break;
+    const int64_t gb = ((t * h + hh) * 2 + s) * k;
+    float acc[MAXC][E];
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c)
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[c][e] = 0.f;
+    for (int a = 0; a < k; ++a) {
+      const float ga = gsub[gb + a];
+      const int32_t row = sub_i[gb + a];
+#pragma unroll
+      for (int c = 0; c < MAXC; ++c) {
+        const int vec = lane + 32 * c;
+        if (vec < nvec) {
+          float f[E];
+          VecT<TS>::load(Cb + (int64_t)row * half + vec * E, f);
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[c][e] = fmaf(ga, f[e], acc[c][e]);
+        }
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+      const int vec = lane + 32 * c;
+      if (vec < nvec) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int col = col0 + vec * E + e;
+          const float gam = bn[2 * hq + col], var = bn[hq + col];
+          dq_pre[t * hq + col] = acc[c][e] * gam / sqrtf(var + eps);
+          if (qhat) pg[c][e] = fmaf(acc[c][e], qhat[t * hq + col], pg[c][e]);
+          pb[c][e] += acc[c][e];
+        }
+      }
+    }
+  }
+  if (!part) return;
+  // reduce partials over the 8 warps in a fixed order
+  __shared__ float red[8][2][32 * 8];
+  for (int c = 0; c < MAXC; ++c) {
+    const int vec = lane + 32 * c;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      red[wid][0][lane * E + e] = pg[c][e];
+      red[wid][1][lane * E + e] = pb[c][e];
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) {
+      float sg = 0.f, sb = 0.f;
+      for (int ww = 0; ww < 8; ++ww) {
+        sg += red[ww][0][i];
+        sb += red[ww][1][i];
+      }
+      const int v2 = i / E + 32 * c;
+      if (v2 < nvec) {
+        const int col = col0 + v2 * E + (i % E);
+        part[((int64_t)blockIdx.x * 2 + 0) * hq + col] = sg;
+        part[((int64_t)blockIdx.x * 2 + 1) * hq + col] = sb;
+      }
+    }
+    __syncthreads();
+    (void)vec;
+  }
+}
+
+__global__ void dbn_reduce_kernel(const float* __restrict__ part, int nblk, int hq,
+                                  float* __restrict__ dbn) {
+  const int col = blockIdx.x * blockDim.x + threadIdx.x;
+  if (col >= 2 * hq) return;
+  const int which = col / hq, c = col % hq;
+  float s = 0.f;
+  for (int b = 0; b < nblk; ++b) s += part[((int64_t)b * 2 + which) * hq + c];
+  dbn[which * hq + c] += s;
+}
+
+// ------------------------------------------------------------------ B5b keys
+__global__ void subkey_keys_kernel(const int32_t* __restrict__ sub_i, int32_t* __restrict__ keys,
+                                   int64_t n, int h, int k, int C1, int C2) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= n) return;
+  const int s = (int)((e / k) % 2);
+  const int hh = (int)((e / (2 * k)) % h);
+  keys[e] = hh * (C1 + C2) + (s ? C1 : 0) + sub_i[e];
+}
+
+// ------------------------------------------------------------------ B5b
+template <bool kSplitQ, int MAXC>
+__global__ void __launch_bounds__(256) subkey_grad_kernel(
+    const int* __restrict__ seg, const int* __restrict__ U_ptr, const int32_t* __restrict__ rows,
+    const int32_t* __restrict__ ents, const float* __restrict__ gsub, const void* __restrict__ q,
+    float* __restrict__ dsub, int64_t N, int h, int dk, int C1, int C2, int k, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int U = *U_ptr;
+  const int half = dk / 2, hq = h * dk;
+  constexpr int E = kSplitQ ? 8 : 4;
+  const int nvec = half / E;
+  const int64_t plane = N * hq;
+  const int rows_total = h * (C1 + C2);
+  for (int64_t u = warp0; u < U; u += nwarps) {
+    const int p0 = seg[u], p1 = seg[u + 1];
+    const int32_t R = rows[p0];
+    if (R < 0 || R >= rows_total) {
+      set_status(status, kDevIndex);
+      continue;
+    }
+    const int hh = R / (C1 + C2);
+    const int s = (R % (C1 + C2)) >= C1 ? 1 : 0;
+    const int64_t colb = (int64_t)hh * dk + s * half;
+    float acc[MAXC][E];
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c)
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[c][e] = 0.f;
+    for (int p = p0; p < p1; ++p) {
+      const int32_t ent = ents[p];
+      const int64_t t = ent / (2 * h * k);
+      const float gv = gsub[ent];
+#pragma unroll
+      for (int c = 0; c < MAXC; ++c) {
+        const int vec = lane + 32 * c;
+        if (vec < nvec) {
+          float f[E];
+          const int64_t off = t * hq + colb + (int64_t)vec * E;
+          if constexpr (kSplitQ) {
+            const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
+            float lo[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4*>(qb + off), f);
+            bf16x8_to_f32(*reinterpret_cast<const uint4*>(qb + plane + off), lo);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] += lo[e];
+          } else {
+            float4 u4 = *reinterpret_cast<const float4*>(static_cast<const float*>(q) + off);
+            f[0] = u4.x; f[1] = u4.y; f[2] = u4.z; f[3] = u4.w;
+          }
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[c][e] = fmaf(gv, f[e], acc[c][e]);
+        }
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+      const int vec = lane + 32 * c;
+      if (vec < nvec) {
+        float* o = dsub + (int64_t)R * half + (int64_t)vec * E;
+#pragma unroll
+        for (int e = 0; e < E; ++e) o[e] += acc[c][e];
+      }
+    }
+  }
+}
+
+inline int bits_for(int64_t maxkey) {
+  int b = 1;
+  while (b < 31 && ((int64_t)1 << b) <= maxkey) ++b;
+  return b;
+}
+
+// ------------------------------------------------------------------ workspace
+struct Layout {
+  size_t keysA, valsA, keysB, valsB, hist, bsum, seg, U, dw, gsub, dq, part, total;
+};
+
+inline size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
+
+Layout layout(const Plan& p) {
+  Layout L{};
+  const int64_t E1 = p.N * p.h * p.k, E2 = 2 * E1;
+  const int64_t En = E2;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t r = o;
+    o += up256(bytes);
+    return r;
+  };
+  L.keysA = take(4 * En);
+  L.valsA = take(4 * En);
+  L.keysB = take(4 * En);
+  L.valsB = take(4 * En);
+  const int64_t hl = sort::radix_hist_len(En);
+  L.hist = take(4 * hl);
+  const int64_t bl = std::max(sort::scan_bsum_len(hl), sort::scan_bsum_len(En));
+  L.bsum = take(4 * bl);
+  L.seg = take(4 * (En + 1));
+  L.U = take(4);
+  L.dw = take(4 * E1);
+  L.gsub = take(4 * E2);
+  L.dq = take(4 * p.N * p.hq);
+  const int64_t nblk = (p.N + kDqTokensPerBlock - 1) / kDqTokensPerBlock;
+  L.part = take(4 * nblk * 2 * p.hq);
+  L.total = o;
+  return L;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+}  // namespace
+
+size_t backward_workspace_bytes(const Plan& p) { return layout(p).total; }
+
+struct BwdCtx {
+  sort::RadixBuffers rb;
+  int* seg;
+  int* U;
+  float* dw;
+  float* gsub;
+  float* dq_pre;
+  float* part;
+};
+
+static BwdCtx bwd_ctx(const Plan& p, void* ws, float* dw_out) {
+  const Layout L = layout(p);
+  BwdCtx c;
+  c.rb = sort::RadixBuffers{at<int32_t>(ws, L.keysA), at<int32_t>(ws, L.valsA),
+                            at<int32_t>(ws, L.keysB), at<int32_t>(ws, L.valsB),
+                            at<int>(ws, L.hist), at<int>(ws, L.bsum)};
+  c.seg = at<int>(ws, L.seg);
+  c.U = at<int>(ws, L.U);
+  c.dw = dw_out ? dw_out : at<float>(ws, L.dw);
+  c.gsub = at<float>(ws, L.gsub);
+  c.dq_pre = at<float>(ws, L.dq);
+  c.part = at<float>(ws, L.part);
+  return c;
+}
+
+cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved& s,
+                              const float* dy, float* dV, float* dw_out, void* ws,
+                              cudaStream_t st) {
+  const int64_t E1 = p.N * p.h * p.k;
+  BwdCtx c = bwd_ctx(p, ws, dw_out);
+  sort::RadixBuffers& rb = c.rb;
+  int* seg = c.seg;
+  int* U = c.U;
+  float* dw = c.dw;
+  cudaError_t e;
+  const int hk = p.h * p.k;
+  const int persist_blocks = p.sm_count * 8;
+
+  // B1-B2: selections sorted by value row
+  const int32_t *rows_sorted, *ents_sorted;
+  e = sort::radix_sort(s.idx, E1, bits_for(p.K - 1), rb, &rows_sorted, &ents_sorted, st);
+  if (e != cudaSuccess) return e;
+  e = sort::segments(rows_sorted, E1, seg, U, rb.bsum, st);
+  if (e != cudaSuccess) return e;
+
+  // B3: value rows
+  {
+    const int E = p.fp32 ? 4 : 8;
+    const int nvec = p.d_v / E;
+    const int chunks = (nvec + 31) / 32;
+#define PKM_B3(TV, CHV)                                                                      \
+  value_rows_kernel<TV, CHV><<<persist_blocks, 256, 0, st>>>(                                \
+      seg, U, rows_sorted, ents_sorted, static_cast<const TV*>(values), s.w, dy, dV, dw, hk, \
+      p.d_v, p.K, p.status)
+    if (p.fp32) {
+      if (chunks <= 1) PKM_B3(float, 1);
+      else if (chunks <= 2) PKM_B3(float, 2);
+      else if (chunks <= 4) PKM_B3(float, 4);
+      else PKM_B3(float, 8);
+    } else {
+      if (chunks <= 1) PKM_B3(__nv_bfloat16, 1);
+      else if (chunks <= 2) PKM_B3(__nv_bfloat16, 2);
+      else if (chunks <= 4) PKM_B3(__nv_bfloat16, 4);
+      else PKM_B3(__nv_bfloat16, 8);
+    }
+#undef PKM_B3
+    PKM_COUNT(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+
+  return cudaSuccess;
+}
+
+cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, const float* bn,
+                              const void* subkeys, const pkm_saved& s, float* dx, float* dWq,
+                              float* dbn, float* dsub, float* dw_out, void* ws, cudaStream_t st) {
+  if (!(dx || dWq || dbn || dsub)) return cudaSuccess;
+  const int64_t E2 = 2 * p.N * p.h * p.k;
+  BwdCtx c = bwd_ctx(p, ws, dw_out);
+  sort::RadixBuffers& rb = c.rb;
+  int* seg = c.seg;
+  int* U = c.U;
+  const float* dw = c.dw;
+  float* gsub = c.gsub;
+  float* dq_pre = c.dq_pre;
+  float* part = c.part;
+  cudaError_t e;
+  const int persist_blocks = p.sm_count * 8;
+
+  // B4: softmax backward onto the selected sub-keys
+  {
+    const int64_t NH = p.N * p.h;
+    softmax_bwd_kernel<<<(unsigned)((NH + 7) / 8), 256, 0, st>>>(s.w, dw, s.idx, s.sub_i, gsub,
+                                                                  NH, p.k, p.C2, p.scale); PKM_COUNT(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+
+  // B5a + B6: dq_pre and BatchNorm affine partials
+  if (dx || dWq || dbn) {
+    const int64_t nblk = (p.N + kDqTokensPerBlock - 1) / kDqTokensPerBlock;
+    dim3 grid((unsigned)nblk, (unsigned)(p.h * 2));
+    float* partp = dbn ? part : nullptr;
+    const float* qh = dbn ? s.qhat : nullptr;
+    if (p.fp32) {
+      const int nv = p.half / 4;
+      if (nv <= 32) dq_kernel<float, 1><<<grid, 256, 0, st>>>(gsub, s.sub_i, (const float*)subkeys, bn, qh, dq_pre, partp, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.eps);
+      else dq_kernel<float, 4><<<grid, 256, 0, st>>>(gsub, s.sub_i, (const float*)subkeys, bn, qh, dq_pre, partp, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.eps); PKM_COUNT(1);
+    } else {
+      const int nv = p.half / 8;
+      if (nv <= 32) dq_kernel<__nv_bfloat16, 1><<<grid, 256, 0, st>>>(gsub, s.sub_i, (const __nv_bfloat16*)subkeys, bn, qh, dq_pre, partp, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.eps);
+      else dq_kernel<__nv_bfloat16, 4><<<grid, 256, 0, st>>>(gsub, s.sub_i, (const __nv_bfloat16*)subkeys, bn, qh, dq_pre, partp, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.eps); PKM_COUNT(1);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (dbn) {
+      dbn_reduce_kernel<<<(2 * p.hq + 255) / 256, 256, 0, st>>>(part, (int)nblk, p.hq, dbn); PKM_COUNT(1);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+  }
+
+  // B5b: sub-key gradients by sorted segments
+  if (dsub) {
+    subkey_keys_kernel<<<(unsigned)((E2 + 255) / 256), 256, 0, st>>>(s.sub_i, rb.keysB, E2, p.h,
+                                                                      p.k, p.C1, p.C2); PKM_COUNT(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int32_t *keys_sorted, *ents2;
+    // the key array lives in keysB: sort from there (the first pass writes A)
+    e = sort::radix_sort(rb.keysB, E2, bits_for((int64_t)p.h * (p.C1 + p.C2) - 1), rb,
+                         &keys_sorted, &ents2, st);
+    if (e != cudaSuccess) return e;
+    e = sort::segments(keys_sorted, E2, seg, U, rb.bsum, st);
+    if (e != cudaSuccess) return e;
+    const int E = p.fp32 ? 4 : 8;
+    const int nv = p.half / E;
+    if (p.fp32) {
+      if (nv <= 32) subkey_grad_kernel<false, 1><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status);
+      else subkey_grad_kernel<false, 4><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status); PKM_COUNT(1);
+    } else {
+      if (nv <= 32) subkey_grad_kernel<true, 1><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status);
+      else subkey_grad_kernel<true, 4><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status); PKM_COUNT(1);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+
+  // B7: dense query gradients
+  if (dx) {
+    e = gemm_simt_f32(p.N, p.d_in, p.hq, dq_pre, false, p.hq, 1, Wq, !p.fp32, 1, p.d_in, dx,
+                      p.d_in, GemmOut::Store, st);
+    if (e != cudaSuccess) return e;
+  }
+  if (dWq) {
+    e = gemm_simt_f32(p.hq, p.d_in, p.N, dq_pre, false, 1, p.hq, x, !p.fp32, 1, p.d_in, dWq,
+                      p.d_in, GemmOut::Accumulate, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace pkm
+
+namespace pkm {
+cudaError_t launch_backward(const Plan& p, const void* x, const void* Wq, const float* bn,
+                            const void* subkeys, const void* values, const pkm_saved& s,
+                            const float* dy, float* dx, float* dWq, float* dbn, float* dsub,
+                            float* dV, float* dw_out, void* ws, cudaStream_t st) {
+  cudaError_t e = launch_value_grad(p, values, s, dy, dV, dw_out, ws, st);
+  if (e != cudaSuccess) return e;
+  return launch_query_grad(p, x, Wq, bn, subkeys, s, dx, dWq, dbn, dsub, dw_out, ws, st);
+}
+}  // namespace pkm

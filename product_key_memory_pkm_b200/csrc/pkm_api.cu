@@ -1,0 +1,322 @@
+// C ABI entry points: host-side validation, plan, launch sequencing.
+#include <atomic>
+#include <mutex>
+
+#include "pkm_internal.cuh"
+
+namespace pkm {
+
+// One device status word per device (first error wins; cleared by pkm_check_status).
+static __device__ int g_status_word;
+
+static std::atomic<unsigned long long> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices];
+int g_sm_count[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+
+// Per-device set-up with that device current: the status word's device address and
+// the SM count.  Returns false if a CUDA call failed.
+bool device_setup(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  bool ok = true;
+  std::call_once(g_dev_once[dev], [&]() {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) {
+      ok = false;
+      return;
+    }
+    g_status_ptr[dev] = static_cast<int*>(p);
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 148;
+    g_sm_count[dev] = sms;
+  });
+  if (!ok || !g_status_ptr[dev]) return false;
+  *dev_out = dev;
+  return true;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+pkm_status validate_dims(const pkm_dims* d) {
+  if (!d) return PKM_ERR_INVALID_ARG;
+  if (d->N < 0 || d->d_in <= 0 || d->h <= 0 || d->dk <= 0 || d->C1 <= 0 || d->C2 <= 0 ||
+      d->k <= 0 || d->d_v <= 0)
+    return PKM_ERR_INVALID_ARG;
+  if (d->k > d->C1 || d->k > d->C2) return PKM_ERR_INVALID_ARG;
+  if (!(d->bn_eps > 0.f) || !(d->score_scale > 0.f) || d->bn_eps != d->bn_eps ||
+      d->score_scale > 3.0e38f)
+    return PKM_ERR_INVALID_ARG;
+  if ((int64_t)d->C1 * d->C2 >= ((int64_t)1 << 31)) return PKM_ERR_INVALID_ARG;
+  if (d->flags & ~(PKM_F_FP32 | PKM_F_SIMT)) return PKM_ERR_INVALID_ARG;
+  const bool fp32 = d->flags & PKM_F_FP32;
+  if (d->dk % 2) return PKM_ERR_INVALID_ARG;
+  if (d->d_in % 8 || d->d_v % 8) return PKM_ERR_INVALID_ARG;
+  if (fp32 ? (d->dk % 8) : (d->dk % 32)) return PKM_ERR_INVALID_ARG;
+  if (d->k > 32 || d->h > 64) return PKM_ERR_UNSUPPORTED;
+  const int half = d->dk / 2;
+  if (fp32 ? (half / 4 > 128) : (half / 8 > 128)) return PKM_ERR_UNSUPPORTED;
+  if (d->N * (int64_t)d->h * d->k * 2 >= ((int64_t)1 << 31)) return PKM_ERR_UNSUPPORTED;
+  if ((int64_t)d->h * d->dk > 65536) return PKM_ERR_UNSUPPORTED;
+  return PKM_OK;
+}
+
+Plan make_plan(const pkm_dims* d, int dev) {
+  Plan p{};
+  p.N = d->N;
+  p.d_in = d->d_in;
+  p.h = d->h;
+  p.dk = d->dk;
+  p.half = d->dk / 2;
+  p.C1 = d->C1;
+  p.C2 = d->C2;
+  p.k = d->k;
+  p.d_v = d->d_v;
+  p.hq = d->h * d->dk;
+  p.K = (int64_t)d->C1 * d->C2;
+  p.eps = d->bn_eps;
+  p.scale = d->score_scale;
+  p.fp32 = d->flags & PKM_F_FP32;
+  p.simt = p.fp32 || (d->flags & PKM_F_SIMT);
+  p.sm_count = g_sm_count[dev];
+  p.status = g_status_ptr[dev];
+  return p;
+}
+
+pkm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA; }
+
+#define PKM_TRY(expr)                  \
+  do {                                 \
+    pkm_status _s = (expr);            \
+    if (_s != PKM_OK) return _s;       \
+  } while (0)
+
+#define PKM_NEED(ptr)                                                   \
+  do {                                                                  \
+    if (!(ptr) || !aligned16(ptr)) return PKM_ERR_INVALID_ARG;          \
+  } while (0)
+
+#define PKM_OPT(ptr)                                                    \
+  do {                                                                  \
+    if ((ptr) && !aligned16(ptr)) return PKM_ERR_INVALID_ARG;           \
+  } while (0)
+
+pkm_status prepare(const pkm_dims* d, Plan* p) {
+  PKM_TRY(validate_dims(d));
+  int dev = 0;
+  if (!device_setup(&dev)) return PKM_ERR_CUDA;
+  *p = make_plan(d, dev);
+  return PKM_OK;
+}
+
+pkm_status check_saved_fwd(const pkm_saved* s) {
+  if (!s) return PKM_ERR_INVALID_ARG;
+  PKM_NEED(s->q);
+  PKM_OPT(s->qhat);
+  PKM_NEED(s->sub_s);
+  PKM_NEED(s->sub_i);
+  PKM_NEED(s->idx);
+  PKM_NEED(s->w);
+  return PKM_OK;
+}
+
+pkm_status check_workspace(size_t need, void* ws, size_t bytes) {
+  if (need == 0) return PKM_OK;
+  if (!ws || bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return PKM_ERR_WORKSPACE;
+  return PKM_OK;
+}
+
+}  // namespace
+}  // namespace pkm
+
+using namespace pkm;
+
+extern "C" {
+
+size_t pkm_saved_bytes(const pkm_dims* d, int field) {
+  if (validate_dims(d) != PKM_OK) return 0;
+  const int64_t N = d->N, hq = (int64_t)d->h * d->dk, sel = N * d->h * d->k;
+  const bool fp32 = d->flags & PKM_F_FP32;
+  switch (field) {
+    case PKM_SAVED_Q: return (size_t)(fp32 ? 4 * N * hq : 2 * 2 * N * hq);
+    case PKM_SAVED_QHAT: return (size_t)(4 * N * hq);
+    case PKM_SAVED_SUB_S:
+    case PKM_SAVED_SUB_I: return (size_t)(4 * 2 * sel);
+    case PKM_SAVED_IDX:
+    case PKM_SAVED_W: return (size_t)(4 * sel);
+    default: return 0;
+  }
+}
+
+size_t pkm_workspace_bytes(const pkm_dims* d, int which) {
+  if (validate_dims(d) != PKM_OK) return 0;
+  if (which == PKM_FWD) return 0;
+  if (which != PKM_BWD || d->N == 0) return 0;
+  Plan p{};
+  p.N = d->N; p.d_in = d->d_in; p.h = d->h; p.dk = d->dk; p.half = d->dk / 2;
+  p.C1 = d->C1; p.C2 = d->C2; p.k = d->k; p.d_v = d->d_v; p.hq = d->h * d->dk;
+  p.K = (int64_t)d->C1 * d->C2; p.fp32 = d->flags & PKM_F_FP32;
+  return backward_workspace_bytes(p);
+}
+
+pkm_status pkm_query(const pkm_dims* d, const void* x, const void* Wq, const float* bn,
+                     const pkm_saved* saved, void* stream) {
+  PKM_TRY(validate_dims(d));
+  if (d->N == 0) return PKM_OK;
+  PKM_NEED(x); PKM_NEED(Wq); PKM_NEED(bn);
+  if (!saved) return PKM_ERR_INVALID_ARG;
+  PKM_NEED(saved->q); PKM_OPT(saved->qhat);
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_query_simt(p, x, Wq, bn, saved->q, saved->qhat, st));
+}
+
+pkm_status pkm_subkey_scores(const pkm_dims* d, const void* subkeys, const pkm_saved* saved,
+                             void* stream) {
+  PKM_TRY(validate_dims(d));
+  if (d->N == 0) return PKM_OK;
+  PKM_NEED(subkeys);
+  if (!saved) return PKM_ERR_INVALID_ARG;
+  PKM_NEED(saved->q); PKM_NEED(saved->sub_s); PKM_NEED(saved->sub_i);
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_scores_simt(p, subkeys, saved->q, saved->sub_s, saved->sub_i, st));
+}
+
+pkm_status pkm_candidate_topk(const pkm_dims* d, const pkm_saved* saved, void* stream) {
+  PKM_TRY(validate_dims(d));
+  if (d->N == 0) return PKM_OK;
+  if (!saved) return PKM_ERR_INVALID_ARG;
+  PKM_NEED(saved->sub_s); PKM_NEED(saved->sub_i); PKM_NEED(saved->idx); PKM_NEED(saved->w);
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_candidates(p, saved->sub_s, saved->sub_i, saved->idx, saved->w, st));
+}
+
+pkm_status pkm_gather_bag(const pkm_dims* d, const void* values, const int32_t* idx,
+                          const float* w, float* y, void* stream) {
+  PKM_TRY(validate_dims(d));
+  if (d->N == 0) return PKM_OK;
+  PKM_NEED(values); PKM_NEED(idx); PKM_NEED(w); PKM_NEED(y);
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_gather(p, values, idx, w, y, st));
+}
+
+pkm_status pkm_forward(const pkm_dims* d, const void* x, const void* Wq, const float* bn,
+                       const void* subkeys, const void* values, float* y,
+                       const pkm_saved* saved, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  PKM_TRY(validate_dims(d));
+  if (d->N == 0) return PKM_OK;
+  PKM_NEED(x); PKM_NEED(Wq); PKM_NEED(bn); PKM_NEED(subkeys); PKM_NEED(values); PKM_NEED(y);
+  PKM_TRY(check_saved_fwd(saved));
+  PKM_TRY(check_workspace(pkm_workspace_bytes(d, PKM_FWD), workspace, workspace_bytes));
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  PKM_TRY(cuda_status(launch_query_simt(p, x, Wq, bn, saved->q, saved->qhat, st)));
+  PKM_TRY(cuda_status(launch_scores_simt(p, subkeys, saved->q, saved->sub_s, saved->sub_i, st)));
+  PKM_TRY(cuda_status(launch_candidates(p, saved->sub_s, saved->sub_i, saved->idx, saved->w, st)));
+  return cuda_status(launch_gather(p, values, saved->idx, saved->w, y, st));
+}
+
+pkm_status pkm_backward(const pkm_dims* d, const void* x, const void* Wq, const float* bn,
+                        const void* subkeys, const void* values, const pkm_saved* saved,
+                        const float* dy, float* dx, float* dWq, float* dbn, float* dsubkeys,
+                        float* dvalues, float* dw_out, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  PKM_TRY(validate_dims(d));
+  if (d->N == 0) return PKM_OK;
+  PKM_NEED(x); PKM_NEED(Wq); PKM_NEED(bn); PKM_NEED(subkeys); PKM_NEED(values); PKM_NEED(dy);
+  PKM_TRY(check_saved_fwd(saved));
+  PKM_OPT(dx); PKM_OPT(dWq); PKM_OPT(dbn); PKM_OPT(dsubkeys); PKM_OPT(dvalues); PKM_OPT(dw_out);
+  if (dbn && !saved->qhat) return PKM_ERR_INVALID_ARG;
+  PKM_TRY(check_workspace(pkm_workspace_bytes(d, PKM_BWD), workspace, workspace_bytes));
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_backward(p, x, Wq, bn, subkeys, values, *saved, dy, dx, dWq, dbn,
+                                     dsubkeys, dvalues, dw_out, workspace, st));
+}
+
+pkm_status pkm_value_grad(const pkm_dims* d, const void* values, const pkm_saved* saved,
+                          const float* dy, float* dvalues, float* dw, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  PKM_TRY(validate_dims(d));
+  if (d->N == 0) return PKM_OK;
+  PKM_NEED(values); PKM_NEED(dy); PKM_NEED(dw); PKM_OPT(dvalues);
+  if (!saved) return PKM_ERR_INVALID_ARG;
+  PKM_NEED(saved->idx); PKM_NEED(saved->w);
+  PKM_TRY(check_workspace(pkm_workspace_bytes(d, PKM_BWD), workspace, workspace_bytes));
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_value_grad(p, values, *saved, dy, dvalues, dw, workspace, st));
+}
+
+pkm_status pkm_query_grad(const pkm_dims* d, const void* x, const void* Wq, const float* bn,
+                          const void* subkeys, const pkm_saved* saved, const float* dw, float* dx,
+                          float* dWq, float* dbn, float* dsubkeys, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  PKM_TRY(validate_dims(d));
+  if (d->N == 0) return PKM_OK;
+  PKM_NEED(x); PKM_NEED(Wq); PKM_NEED(bn); PKM_NEED(subkeys); PKM_NEED(dw);
+  PKM_TRY(check_saved_fwd(saved));
+  PKM_OPT(dx); PKM_OPT(dWq); PKM_OPT(dbn); PKM_OPT(dsubkeys);
+  if (dbn && !saved->qhat) return PKM_ERR_INVALID_ARG;
+  PKM_TRY(check_workspace(pkm_workspace_bytes(d, PKM_BWD), workspace, workspace_bytes));
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_query_grad(p, x, Wq, bn, subkeys, *saved, dx, dWq, dbn, dsubkeys,
+                                       const_cast<float*>(dw), workspace, st));
+}
+
+unsigned long long pkm_launch_count(void) { return g_launches.load(); }
+
+pkm_status pkm_check_status(void* stream) {
+  int dev = 0;
+  if (!device_setup(&dev)) return PKM_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PKM_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, g_status_ptr[dev], sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return PKM_ERR_CUDA;
+  if (v != kDevOk) {
+    int z = 0;
+    if (cudaMemcpy(g_status_ptr[dev], &z, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return PKM_ERR_CUDA;
+  }
+  if (v == kDevTimeout) return PKM_ERR_DEVICE_TIMEOUT;
+  if (v == kDevIndex) return PKM_ERR_DEVICE_INDEX;
+  return PKM_OK;
+}
+
+const char* pkm_status_string(pkm_status s) {
+  switch (s) {
+    case PKM_OK: return "PKM_OK";
+    case PKM_ERR_INVALID_ARG: return "PKM_ERR_INVALID_ARG: invalid argument";
+    case PKM_ERR_UNSUPPORTED: return "PKM_ERR_UNSUPPORTED: outside this build's limits";
+    case PKM_ERR_WORKSPACE: return "PKM_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case PKM_ERR_CUDA: return "PKM_ERR_CUDA: a CUDA runtime call failed";
+    case PKM_ERR_DEVICE_TIMEOUT: return "PKM_ERR_DEVICE_TIMEOUT: a bounded device wait expired";
+    case PKM_ERR_DEVICE_INDEX: return "PKM_ERR_DEVICE_INDEX: a device index check failed";
+  }
+  return "PKM_ERR_UNKNOWN";
+}
+
+const char* pkm_build_info(void) {
+  return "pkm_b200 sm_100a (" __DATE__ ")";
+}
+
+}  // extern "C"

@@ -1,0 +1,91 @@
+// Internal declarations shared by the library's CUDA translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pkm.h"
+
+namespace pkm {
+
+// ---------------------------------------------------------------- device helpers
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Monotone map of a finite fp32 score onto uint32 (larger score -> larger key).
+// -0.0 is first folded onto +0.0 so that equal scores give equal keys.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  v = v + 0.0f;
+  uint32_t b = __float_as_uint(v);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Status codes written by kernels into the device status word (first error wins).
+enum : int { kDevOk = 0, kDevTimeout = 1, kDevIndex = 2 };
+
+__device__ __forceinline__ void set_status(int* st, int code) {
+  if (st) atomicCAS(st, kDevOk, code);
+}
+
+// Unpack 8 bf16 held in a uint4 into floats.
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __bfloat1622float2(p[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+// ---------------------------------------------------------------- launch counter
+// Every kernel launch of the library is counted (host side) for diagnostics.
+void count_launches(int n);
+#define PKM_COUNT(n) ::pkm::count_launches(n)
+
+// ---------------------------------------------------------------- plan
+// Sizes derived once per call from pkm_dims.
+struct Plan {
+  int64_t N;
+  int d_in, h, dk, half, C1, C2, k, d_v, hq;  // hq = h*dk
+  int64_t K;                                 // C1*C2
+  float eps, scale;
+  bool fp32;      // fp32 storage
+  bool simt;      // CUDA-core kernels for bf16 storage
+  int sm_count;
+  int* status;    // device status word
+};
+
+// ---------------------------------------------------------------- forward launches
+cudaError_t launch_query_simt(const Plan& p, const void* x, const void* Wq, const float* bn,
+                              void* q, float* qhat, cudaStream_t st);
+cudaError_t launch_scores_simt(const Plan& p, const void* subkeys, const void* q, float* sub_s,
+                               int32_t* sub_i, cudaStream_t st);
+cudaError_t launch_candidates(const Plan& p, const float* sub_s, const int32_t* sub_i,
+                              int32_t* idx, float* w, cudaStream_t st);
+cudaError_t launch_gather(const Plan& p, const void* values, const int32_t* idx, const float* w,
+                          float* y, cudaStream_t st);
+
+// ---------------------------------------------------------------- backward launches
+struct BwdWs;  // workspace layout, defined in k_backward.cu
+size_t backward_workspace_bytes(const Plan& p);
+cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved& s,
+                              const float* dy, float* dV, float* dw_out, void* ws,
+                              cudaStream_t st);
+cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, const float* bn,
+                              const void* subkeys, const pkm_saved& s, float* dx, float* dWq,
+                              float* dbn, float* dsub, float* dw_out, void* ws, cudaStream_t st);
+cudaError_t launch_backward(const Plan& p, const void* x, const void* Wq, const float* bn,
+                            const void* subkeys, const void* values, const pkm_saved& s,
+                            const float* dy, float* dx, float* dWq, float* dbn, float* dsub,
+                            float* dV, float* dw_out, void* ws, cudaStream_t st);
+
+// ---------------------------------------------------------------- generic CUDA-core GEMM
+// C[m][n] (op)= sum_k A(m,k) * B(n,k), A(m,k) = A[m*sam + k*sak], B(n,k) = B[n*sbn + k*sbk].
+enum class GemmOut { Store, Accumulate };
+cudaError_t gemm_simt_f32(int64_t M, int64_t Nn, int64_t Kk, const void* A, bool a_bf16,
+                          int64_t sam, int64_t sak, const void* B, bool b_bf16, int64_t sbn,
+                          int64_t sbk, float* C, int64_t ldc, GemmOut mode, cudaStream_t st);
+
+}  // namespace pkm

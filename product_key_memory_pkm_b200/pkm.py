@@ -1,0 +1,269 @@
+"""Thin Python binding of the C ABI in ``include/pkm.h`` (ctypes).
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels of
+``libpkm_b200.so``.  PyTorch is used for device memory and streams.  There is no
+CPU fallback: loading fails loudly when the library has not been built.
+
+The functions carry the C names (``pkm_forward``, ``pkm_backward``,
+``pkm_query``, ``pkm_subkey_scores``, ``pkm_candidate_topk``,
+``pkm_gather_bag``, ``pkm_check_status``, ...) and take torch tensors (device
+pointers are read with ``data_ptr()``) or raw integer addresses.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libpkm_b200.so")
+
+PKM_OK = 0
+PKM_ERR_INVALID_ARG = 1
+PKM_ERR_UNSUPPORTED = 2
+PKM_ERR_WORKSPACE = 3
+PKM_ERR_CUDA = 4
+PKM_ERR_DEVICE_TIMEOUT = 5
+PKM_ERR_DEVICE_INDEX = 6
+
+PKM_F_FP32 = 0x1
+PKM_F_SIMT = 0x2
+PKM_FWD, PKM_BWD = 0, 1
+SAVED_FIELDS = ("q", "qhat", "sub_s", "sub_i", "idx", "w")
+
+# every symbol include/pkm.h declares
+EXPORTED = ("pkm_saved_bytes", "pkm_workspace_bytes", "pkm_forward", "pkm_backward", "pkm_query",
+            "pkm_subkey_scores", "pkm_candidate_topk", "pkm_gather_bag", "pkm_check_status",
+            "pkm_status_string", "pkm_build_info", "pkm_value_grad", "pkm_query_grad",
+            "pkm_launch_count")
+
+
+class PKMError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (status {code})")
+
+
+class pkm_dims(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("d_in", ctypes.c_int32), ("h", ctypes.c_int32),
+                ("dk", ctypes.c_int32), ("C1", ctypes.c_int32), ("C2", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("d_v", ctypes.c_int32), ("bn_eps", ctypes.c_float),
+                ("score_scale", ctypes.c_float), ("flags", ctypes.c_uint32)]
+
+
+class pkm_saved(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_void_p) for f in SAVED_FIELDS]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the shared library (once).  Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
+                          "`python -m product_key_memory_pkm_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, S, I, U64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_uint64
+    D = ctypes.POINTER(pkm_dims)
+    SV = ctypes.POINTER(pkm_saved)
+    sig = {
+        "pkm_saved_bytes": (S, [D, I]),
+        "pkm_workspace_bytes": (S, [D, I]),
+        "pkm_forward": (I, [D, P, P, P, P, P, P, SV, P, S, P]),
+        "pkm_backward": (I, [D, P, P, P, P, P, SV, P, P, P, P, P, P, P, P, S, P]),
+        "pkm_query": (I, [D, P, P, P, SV, P]),
+        "pkm_subkey_scores": (I, [D, P, SV, P]),
+        "pkm_candidate_topk": (I, [D, SV, P]),
+        "pkm_gather_bag": (I, [D, P, P, P, P, P]),
+        "pkm_check_status": (I, [P]),
+        "pkm_status_string": (ctypes.c_char_p, [I]),
+        "pkm_build_info": (ctypes.c_char_p, []),
+        "pkm_value_grad": (I, [D, P, SV, P, P, P, P, S, P]),
+        "pkm_query_grad": (I, [D, P, P, P, P, SV, P, P, P, P, P, P, S, P]),
+        "pkm_launch_count": (ctypes.c_ulonglong, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    del U64
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load().pkm_status_string(int(code)).decode()
+
+
+# ----------------------------------------------------------------- marshalling
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(code: int, where: str) -> None:
+    if code != PKM_OK:
+        raise PKMError(code, where)
+
+
+@dataclass
+class Dims:
+    """Python mirror of ``pkm_dims``."""
+    N: int
+    d_in: int
+    h: int
+    dk: int
+    C1: int
+    C2: int
+    k: int
+    d_v: int
+    bn_eps: float = 1e-5
+    score_scale: float = 1.0
+    flags: int = 0
+
+    def c(self) -> pkm_dims:
+        return pkm_dims(self.N, self.d_in, self.h, self.dk, self.C1, self.C2, self.k, self.d_v,
+                        self.bn_eps, self.score_scale, self.flags)
+
+    @classmethod
+    def from_config(cls, cfg, flags: int = 0, N: int | None = None) -> "Dims":
+        f = flags | (PKM_F_FP32 if cfg.dtype == "f32" else 0)
+        return cls(cfg.N if N is None else N, cfg.d_in, cfg.h, cfg.dk, cfg.C1, cfg.C2, cfg.k,
+                   cfg.d_v, cfg.bn_eps, cfg.score_scale, f)
+
+
+def _saved_c(saved: dict) -> pkm_saved:
+    return pkm_saved(*[_ptr(saved.get(f)) for f in SAVED_FIELDS])
+
+
+def pkm_saved_bytes(dims: Dims, field: str) -> int:
+    return int(load().pkm_saved_bytes(ctypes.byref(dims.c()), SAVED_FIELDS.index(field)))
+
+
+def pkm_workspace_bytes(dims: Dims, which: int) -> int:
+    return int(load().pkm_workspace_bytes(ctypes.byref(dims.c()), which))
+
+
+def pkm_forward(dims: Dims, x, Wq, bn, subkeys, values, y, saved: dict, workspace=None,
+                workspace_bytes: int = 0, stream=None) -> None:
+    ws_bytes = workspace_bytes or (workspace.numel() * workspace.element_size()
+                                   if workspace is not None and not isinstance(workspace, int) else 0)
+    s = _saved_c(saved)
+    _check(load().pkm_forward(ctypes.byref(dims.c()), _ptr(x), _ptr(Wq), _ptr(bn), _ptr(subkeys),
+                              _ptr(values), _ptr(y), ctypes.byref(s), _ptr(workspace), ws_bytes,
+                              _stream(stream)), "pkm_forward")
+
+
+def pkm_backward(dims: Dims, x, Wq, bn, subkeys, values, saved: dict, dy, dx=None, dWq=None,
+                 dbn=None, dsubkeys=None, dvalues=None, dw_out=None, workspace=None,
+                 workspace_bytes: int = 0, stream=None) -> None:
+    ws_bytes = workspace_bytes or (workspace.numel() * workspace.element_size()
+                                   if workspace is not None and not isinstance(workspace, int) else 0)
+    s = _saved_c(saved)
+    _check(load().pkm_backward(ctypes.byref(dims.c()), _ptr(x), _ptr(Wq), _ptr(bn), _ptr(subkeys),
+                               _ptr(values), ctypes.byref(s), _ptr(dy), _ptr(dx), _ptr(dWq),
+                               _ptr(dbn), _ptr(dsubkeys), _ptr(dvalues), _ptr(dw_out),
+                               _ptr(workspace), ws_bytes, _stream(stream)), "pkm_backward")
+
+
+def _ws(workspace, workspace_bytes):
+    if workspace_bytes:
+        return workspace_bytes
+    if workspace is None or isinstance(workspace, int):
+        return 0
+    return workspace.numel() * workspace.element_size()
+
+
+def pkm_value_grad(dims: Dims, values, saved: dict, dy, dw, dvalues=None, workspace=None,
+                   workspace_bytes: int = 0, stream=None) -> None:
+    s = _saved_c(saved)
+    _check(load().pkm_value_grad(ctypes.byref(dims.c()), _ptr(values), ctypes.byref(s), _ptr(dy),
+                                 _ptr(dvalues), _ptr(dw), _ptr(workspace),
+                                 _ws(workspace, workspace_bytes), _stream(stream)),
+           "pkm_value_grad")
+
+
+def pkm_query_grad(dims: Dims, x, Wq, bn, subkeys, saved: dict, dw, dx=None, dWq=None, dbn=None,
+                   dsubkeys=None, workspace=None, workspace_bytes: int = 0, stream=None) -> None:
+    s = _saved_c(saved)
+    _check(load().pkm_query_grad(ctypes.byref(dims.c()), _ptr(x), _ptr(Wq), _ptr(bn),
+                                 _ptr(subkeys), ctypes.byref(s), _ptr(dw), _ptr(dx), _ptr(dWq),
+                                 _ptr(dbn), _ptr(dsubkeys), _ptr(workspace),
+                                 _ws(workspace, workspace_bytes), _stream(stream)),
+           "pkm_query_grad")
+
+
+def pkm_launch_count() -> int:
+    return int(load().pkm_launch_count())
+
+
+def pkm_query(dims: Dims, x, Wq, bn, saved: dict, stream=None) -> None:
+    s = _saved_c(saved)
+    _check(load().pkm_query(ctypes.byref(dims.c()), _ptr(x), _ptr(Wq), _ptr(bn), ctypes.byref(s),
+                            _stream(stream)), "pkm_query")
+
+
+def pkm_subkey_scores(dims: Dims, subkeys, saved: dict, stream=None) -> None:
+    s = _saved_c(saved)
+    _check(load().pkm_subkey_scores(ctypes.byref(dims.c()), _ptr(subkeys), ctypes.byref(s),
+                                    _stream(stream)), "pkm_subkey_scores")
+
+
+def pkm_candidate_topk(dims: Dims, saved: dict, stream=None) -> None:
+    s = _saved_c(saved)
+    _check(load().pkm_candidate_topk(ctypes.byref(dims.c()), ctypes.byref(s), _stream(stream)),
+           "pkm_candidate_topk")
+
+
+def pkm_gather_bag(dims: Dims, values, idx, w, y, stream=None) -> None:
+    _check(load().pkm_gather_bag(ctypes.byref(dims.c()), _ptr(values), _ptr(idx), _ptr(w), _ptr(y),
+                                 _stream(stream)), "pkm_gather_bag")
+
+
+def pkm_check_status(stream=None) -> int:
+    """Synchronise the stream and return the device status code (0 = PKM_OK)."""
+    return int(load().pkm_check_status(_stream(stream)))
+
+
+def pkm_build_info() -> str:
+    return load().pkm_build_info().decode()
+
+
+# ----------------------------------------------------------------- allocation helpers
+def alloc_saved(dims: Dims, device="cuda", with_qhat: bool = True) -> dict:
+    """Caller-owned buffers the forward writes and the backward reads (torch)."""
+    import torch
+    N, hq, sel = dims.N, dims.h * dims.dk, dims.N * dims.h * dims.k
+    fp32 = bool(dims.flags & PKM_F_FP32)
+    q = (torch.empty(N, hq, dtype=torch.float32, device=device) if fp32 else
+         torch.empty(2, N, hq, dtype=torch.bfloat16, device=device))
+    return dict(
+        q=q,
+        qhat=torch.empty(N, hq, dtype=torch.float32, device=device) if with_qhat else None,
+        sub_s=torch.empty(N, dims.h, 2, dims.k, dtype=torch.float32, device=device),
+        sub_i=torch.empty(N, dims.h, 2, dims.k, dtype=torch.int32, device=device),
+        idx=torch.empty(N, dims.h, dims.k, dtype=torch.int32, device=device),
+        w=torch.empty(N, dims.h, dims.k, dtype=torch.float32, device=device),
+    )
+
+
+def alloc_workspace(dims: Dims, which: int, device="cuda"):
+    import torch
+    n = pkm_workspace_bytes(dims, which)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)

@@ -1,0 +1,141 @@
+"""The C ABI library loads, exports every symbol ``include/pkm.h`` declares, and its
+host-side validation rejects bad arguments before any device work (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from product_key_memory_pkm_b200 import build as B
+from product_key_memory_pkm_b200 import pkm as P
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return P.load()
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "pkm.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pkm_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared_functions()
+    assert len(declared) >= 10
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) == set(P.EXPORTED)
+
+
+def test_build_targets_sm100a_only():
+    assert B.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_struct_layout_matches_header():
+    assert ctypes.sizeof(P.pkm_dims) == 48
+    assert ctypes.sizeof(P.pkm_saved) == 6 * ctypes.sizeof(ctypes.c_void_p)
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        s = P.status_string(code)
+        assert s.startswith("PKM_")
+    assert "UNKNOWN" in P.status_string(99)
+
+
+def _dims(**kw):
+    base = dict(N=64, d_in=64, h=2, dk=64, C1=32, C2=32, k=8, d_v=64)
+    base.update(kw)
+    return P.Dims(**base)
+
+
+def test_workspace_and_saved_sizes(lib):
+    d = _dims()
+    assert P.pkm_workspace_bytes(d, P.PKM_FWD) == 0
+    assert P.pkm_workspace_bytes(d, P.PKM_BWD) > 0
+    assert P.pkm_saved_bytes(d, "q") == 2 * 2 * 64 * 128
+    assert P.pkm_saved_bytes(d, "idx") == 4 * 64 * 2 * 8
+    assert P.pkm_saved_bytes(d, "sub_i") == 4 * 64 * 2 * 2 * 8
+    d32 = _dims(flags=P.PKM_F_FP32)
+    assert P.pkm_saved_bytes(d32, "q") == 4 * 64 * 128
+    assert P.pkm_saved_bytes(_dims(k=40, C1=32), "q") == 0      # invalid dims -> 0
+    assert P.pkm_workspace_bytes(_dims(N=0), P.PKM_BWD) == 0
+
+
+FAKE = 1 << 20          # a 16-byte-aligned address that is never dereferenced
+
+
+def _fwd(d, **over):
+    args = dict(x=FAKE, Wq=FAKE, bn=FAKE, subkeys=FAKE, values=FAKE, y=FAKE)
+    args.update(over)
+    saved = {f: FAKE for f in P.SAVED_FIELDS}
+    saved.update(over.pop("saved", {}) if "saved" in over else {})
+    return P.load().pkm_forward(ctypes.byref(d.c()), args["x"], args["Wq"], args["bn"],
+                                args["subkeys"], args["values"], args["y"],
+                                ctypes.byref(P._saved_c(saved)), None, 0, None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(k=33, C1=64, C2=64), P.PKM_ERR_UNSUPPORTED),
+    (dict(k=9, C1=8), P.PKM_ERR_INVALID_ARG),
+    (dict(dk=48), P.PKM_ERR_INVALID_ARG),            # bf16 needs dk % 32 == 0
+    (dict(d_in=60), P.PKM_ERR_INVALID_ARG),
+    (dict(d_v=12), P.PKM_ERR_INVALID_ARG),
+    (dict(bn_eps=0.0), P.PKM_ERR_INVALID_ARG),
+    (dict(score_scale=-1.0), P.PKM_ERR_INVALID_ARG),
+    (dict(flags=0x80), P.PKM_ERR_INVALID_ARG),
+    (dict(N=-1), P.PKM_ERR_INVALID_ARG),
+    (dict(C1=65536, C2=65536), P.PKM_ERR_INVALID_ARG),
+])
+def test_forward_rejects_bad_dims(lib, over, code):
+    assert _fwd(_dims(**over)) == code
+
+
+def test_forward_rejects_null_and_misaligned_pointers(lib):
+    d = _dims()
+    assert _fwd(d, x=None) == P.PKM_ERR_INVALID_ARG
+    assert _fwd(d, values=FAKE + 8) == P.PKM_ERR_INVALID_ARG
+    saved = {f: FAKE for f in P.SAVED_FIELDS}
+    saved["idx"] = None
+    rc = P.load().pkm_forward(ctypes.byref(d.c()), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                              ctypes.byref(P._saved_c(saved)), None, 0, None)
+    assert rc == P.PKM_ERR_INVALID_ARG
+
+
+def test_zero_tokens_is_a_noop(lib):
+    assert _fwd(_dims(N=0)) == P.PKM_OK
+    assert _fwd(_dims(N=0), x=None) == P.PKM_OK
+
+
+def test_backward_checks_workspace_and_qhat(lib):
+    d = _dims()
+    saved = {f: FAKE for f in P.SAVED_FIELDS}
+    S = ctypes.byref(P._saved_c(saved))
+    L = P.load()
+    need = P.pkm_workspace_bytes(d, P.PKM_BWD)
+    args = (ctypes.byref(d.c()), FAKE, FAKE, FAKE, FAKE, FAKE, S, FAKE, FAKE, FAKE, FAKE, FAKE,
+            FAKE, None)
+    assert L.pkm_backward(*args, None, 0, None) == P.PKM_ERR_WORKSPACE
+    assert L.pkm_backward(*args, FAKE, need - 1, None) == P.PKM_ERR_WORKSPACE
+    assert L.pkm_backward(*args, FAKE + 16, need, None) == P.PKM_ERR_WORKSPACE  # not 256-aligned
+    saved["qhat"] = None
+    S2 = ctypes.byref(P._saved_c(saved))
+    rc = L.pkm_backward(ctypes.byref(d.c()), FAKE, FAKE, FAKE, FAKE, FAKE, S2, FAKE, None, None,
+                        FAKE, None, None, None, FAKE, need, None)
+    assert rc == P.PKM_ERR_INVALID_ARG      # d gamma needs qhat
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    import importlib
+    mod = importlib.reload(P)
+    try:
+        mod._lib = None
+        with pytest.raises(ImportError):
+            mod.load(str(tmp_path / "missing.so"))
+    finally:
+        importlib.reload(P)

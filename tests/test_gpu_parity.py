@@ -1,0 +1,253 @@
+"""GPU parity of the CUDA path (through the C ABI) against the CPU oracle."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import pkm_oracle as O
+from product_key_memory_pkm_b200 import pkm as P
+from product_key_memory_pkm_b200.inputs import (FULL_K1024, FWD_K512, TINY_FP32, PKMConfig,
+                                                make_inputs)
+from tests import parity as H
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from product_key_memory_pkm_b200 import build as B
+    B.build()
+
+
+def _cfg(**kw):
+    base = dict(name="case", N=300, d_in=128, h=4, dk=64, C1=64, C2=48, k=16, d_v=200,
+                dtype="bf16", score_scale=0.5)
+    base.update(kw)
+    return PKMConfig(**base)
+
+
+CASES = {
+    "tiny_fp32": TINY_FP32,
+    "tiny_bf16": TINY_FP32.with_(name="tiny_bf16", dtype="bf16"),
+    "ragged_multihead_bf16": _cfg(),
+    "ragged_multihead_fp32": _cfg(name="r32", dtype="f32", dk=40),
+    "k_equals_C": _cfg(N=100, h=2, C1=32, C2=32, k=32, d_v=64, dk=64),
+    "k1": _cfg(N=77, k=1, h=2),
+    "one_token": _cfg(N=1),
+    "duplicate_heavy": _cfg(N=512, d_in=64, h=1, dk=64, C1=64, C2=64, k=8, d_v=128,
+                            clustered=8),
+    "unequal_C_wide_dv": _cfg(N=130, h=1, dk=128, C1=96, C2=40, k=24, d_v=2056),
+}
+
+
+def _full_check(cfg, seed=0, flags=0):
+    inp = make_inputs(cfg, seed=seed, random_bn=True)
+    dev = H.to_dev(inp, cfg)
+    dims, saved, y = H.gpu_forward(cfg, dev, flags=flags)
+    of = O.forward(inp, cfg)
+    ranked = H.oracle_gaps(of, cfg)
+    idx = saved["idx"].cpu().numpy()
+    clean = H.check_indices(idx, of, cfg, ranked)
+    yg = y.cpu().numpy()
+    H.assert_rows(yg[clean], of["y"][clean], "y")
+    for t in np.nonzero(~clean)[0]:
+        H.assert_rows(yg[t:t + 1], H.oracle_bag_at(of, cfg, idx, t, inp["values"])[None], "y tie")
+    # softmax weights of clean heads
+    H.assert_rows(saved["w"].cpu().numpy()[clean].reshape(-1, cfg.k),
+                  of["w"][clean].reshape(-1, cfg.k), "w")
+    # backward with dy masked to the clean tokens
+    dy = inp["dy"] * clean[:, None]
+    g = H.gpu_backward(cfg, dims, dev, saved, torch.from_numpy(dy).cuda())
+    ob = O.backward(inp, cfg, of, dy)
+    H.assert_rows(g["dx"].cpu().numpy(), ob["dx"], "dx")
+    H.assert_rows(g["dWq"].cpu().numpy(), ob["dWq"], "dWq")
+    H.assert_rows(g["dbn"].cpu().numpy(), np.stack([ob["dgamma"], ob["dbeta"]]), "dbn")
+    H.assert_rows(g["dsub"].cpu().numpy().reshape(-1, cfg.dk // 2),
+                  ob["dsub"].reshape(-1, cfg.dk // 2), "dsub")
+    dV = g["dV"].cpu().numpy()
+    H.assert_rows(dV[ob["dV_rows"]], ob["dV_vals"], "dV")
+    untouched = np.ones(cfg.K, dtype=bool)
+    untouched[ob["dV_rows"]] = False
+    assert not dV[untouched].any()
+    H.assert_rows(g["dw"].cpu().numpy()[clean].reshape(-1, cfg.k),
+                  ob["dw"][clean].reshape(-1, cfg.k), "dw")
+    return clean
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_end_to_end_parity(name):
+    clean = _full_check(CASES[name])
+    assert clean.mean() > 0.9
+
+
+def test_simt_flag_path_matches_oracle():
+    _full_check(CASES["ragged_multihead_bf16"], flags=P.PKM_F_SIMT)
+
+
+def test_stagewise_scores_given_oracle_query():
+    """F2 alone: fed the oracle's q (as its hi/lo split), the per-half lists match the
+    oracle's per-half top-k computed from the same q."""
+    cfg = _cfg(N=257)
+    inp = make_inputs(cfg, seed=3, random_bn=True)
+    of = O.forward(inp, cfg)
+    q32 = torch.from_numpy(of["q"].astype(np.float32))
+    hi = q32.to(torch.bfloat16)
+    lo = (q32 - hi.float()).to(torch.bfloat16)
+    qrep = (hi.double() + lo.double()).numpy()
+    s1, s2 = O.subkey_scores(qrep, inp["subkeys"], cfg.h, cfg.dk, cfg.C1)
+    dims = P.Dims.from_config(cfg)
+    saved = P.alloc_saved(dims)
+    saved["q"].copy_(torch.stack([hi, lo]).cuda())
+    sub = torch.from_numpy(inp["subkeys"]).to(torch.bfloat16).cuda()
+    P.pkm_subkey_scores(dims, sub, saved)
+    assert P.pkm_check_status() == P.PKM_OK
+    gi = saved["sub_i"].cpu().numpy()
+    gs = saved["sub_s"].cpu().numpy()
+    for t in range(cfg.N):
+        for hh in range(cfg.h):
+            for half, s in ((0, s1[t, hh]), (1, s2[t, hh])):
+                ii, vv = O.half_topk(s, cfg.k + 1)
+                tol = H.GAP_REL * max(abs(vv[cfg.k - 1]), 1e-2)
+                if vv[cfg.k - 1] - vv[cfg.k] > tol:
+                    assert set(gi[t, hh, half].tolist()) == set(ii[:cfg.k].tolist())
+                np.testing.assert_allclose(gs[t, hh, half], s[gi[t, hh, half]], rtol=1e-5,
+                                           atol=1e-5)
+
+
+def test_stagewise_candidates_given_oracle_lists():
+    """F3 alone: fed per-half lists (fp32), the winners and weights match the oracle's
+    product-key combine of the same lists."""
+    cfg = _cfg(N=500, k=32, C1=64, C2=64)
+    rng = np.random.default_rng(5)
+    N, h, k = cfg.N, cfg.h, cfg.k
+    s1 = rng.standard_normal((N, h, cfg.C1)).astype(np.float32)
+    s2 = rng.standard_normal((N, h, cfg.C2)).astype(np.float32)
+    s1[:7] = np.round(s1[:7])      # exact ties in a few tokens
+    s2[:7] = np.round(s2[:7])
+    sub_i = np.zeros((N, h, 2, k), dtype=np.int32)
+    sub_s = np.zeros((N, h, 2, k), dtype=np.float32)
+    for t in range(N):
+        for hh in range(h):
+            for half, s in ((0, s1[t, hh].astype(np.float64)), (1, s2[t, hh].astype(np.float64))):
+                ii, vv = O.half_topk(s, k)
+                sub_i[t, hh, half], sub_s[t, hh, half] = ii, vv
+    dims = P.Dims.from_config(cfg)
+    saved = P.alloc_saved(dims)
+    saved["sub_s"].copy_(torch.from_numpy(sub_s))
+    saved["sub_i"].copy_(torch.from_numpy(sub_i))
+    P.pkm_candidate_topk(dims, saved)
+    assert P.pkm_check_status() == P.PKM_OK
+    gidx = saved["idx"].cpu().numpy()
+    gw = saved["w"].cpu().numpy()
+    for t in range(N):
+        for hh in range(h):
+            a, b = s1[t, hh].astype(np.float64), s2[t, hh].astype(np.float64)
+            ii, jj = O.product_key_topk(a, b, k + 1)
+            S = a[ii] + b[jj]
+            tol = H.GAP_REL * max(abs(S[k - 1]), 1e-2)
+            if S[k - 1] - S[k] > tol:
+                assert set(gidx[t, hh].tolist()) == set((ii[:k] * cfg.C2 + jj[:k]).tolist())
+                w = O.softmax(cfg.score_scale * S[:k])
+                np.testing.assert_allclose(gw[t, hh], w, rtol=2e-3, atol=1e-6)
+            if t < 7:
+                # integer scores: fp32 sums are exact, so the order is the oracle's order
+                assert gidx[t, hh].tolist() == (ii[:k] * cfg.C2 + jj[:k]).tolist()
+
+
+def test_stagewise_gather_given_oracle_selection():
+    cfg = _cfg(N=333, d_v=1032)
+    inp = make_inputs(cfg, seed=6, with_dy=False)
+    of = O.forward(inp, cfg)
+    dims = P.Dims.from_config(cfg)
+    V = torch.from_numpy(inp["values"]).to(torch.bfloat16).cuda()
+    idx = torch.from_numpy(of["idx"].astype(np.int32)).cuda()
+    w32 = of["w"].astype(np.float32)
+    y = torch.empty(cfg.N, cfg.d_v, device="cuda")
+    P.pkm_gather_bag(dims, V, idx, torch.from_numpy(w32).cuda(), y)
+    assert P.pkm_check_status() == P.PKM_OK
+    want = O.bag(w32.astype(np.float64), of["idx"], inp["values"])
+    H.assert_rows(y.cpu().numpy(), want, "y", tol=1e-5)
+
+
+def test_value_gradient_is_deterministic_under_duplicates():
+    cfg = CASES["duplicate_heavy"]
+    inp = make_inputs(cfg, seed=2)
+    dev = H.to_dev(inp, cfg)
+    dims, saved, _ = H.gpu_forward(cfg, dev)
+    idx = saved["idx"].cpu().numpy().ravel()
+    assert np.unique(idx).size < 0.5 * idx.size      # the clustered recipe duplicates rows
+    dy = torch.from_numpy(inp["dy"]).cuda()
+    g1 = H.gpu_backward(cfg, dims, dev, saved, dy)
+    g2 = H.gpu_backward(cfg, dims, dev, saved, dy)
+    for k in ("dV", "dsub", "dWq", "dx", "dbn", "dw"):
+        assert torch.equal(g1[k], g2[k]), k
+
+
+def test_gradients_accumulate_into_caller_buffers():
+    cfg = CASES["tiny_bf16"]
+    inp = make_inputs(cfg, seed=1)
+    dev = H.to_dev(inp, cfg)
+    dims, saved, _ = H.gpu_forward(cfg, dev)
+    dy = torch.from_numpy(inp["dy"]).cuda()
+    g1 = H.gpu_backward(cfg, dims, dev, saved, dy)
+    ws = P.alloc_workspace(dims, P.PKM_BWD)
+    acc = {k: v.clone() for k, v in g1.items()}
+    P.pkm_backward(dims, dev["x"], dev["Wq"], dev["bn"], dev["subkeys"], dev["values"], saved, dy,
+                   dx=acc["dx"], dWq=acc["dWq"], dbn=acc["dbn"], dsubkeys=acc["dsub"],
+                   dvalues=acc["dV"], dw_out=acc["dw"], workspace=ws)
+    torch.cuda.synchronize()
+    for k in ("dWq", "dbn", "dsub", "dV"):
+        torch.testing.assert_close(acc[k], 2 * g1[k], rtol=1e-6, atol=1e-6)
+    torch.testing.assert_close(acc["dx"], g1["dx"], rtol=0, atol=0)      # overwritten
+
+
+def test_zero_tokens_noop_on_device():
+    cfg = _cfg(N=0)
+    dims = P.Dims.from_config(cfg)
+    y = torch.full((1, cfg.d_v), 7.0, device="cuda")
+    saved = P.alloc_saved(P.Dims.from_config(cfg.with_(N=1)))
+    dummy = torch.zeros(1024, device="cuda")
+    P.pkm_forward(dims, dummy, dummy, dummy, dummy, dummy, y, saved)
+    assert P.pkm_check_status() == P.PKM_OK
+    assert torch.all(y == 7.0)
+
+
+def _sampled_full_size(cfg, n_sample, seed=0, backward=True):
+    inp = make_inputs(cfg, seed=seed, random_bn=False)
+    dev = H.to_dev(inp, cfg)
+    dims, saved, y = H.gpu_forward(cfg, dev)
+    rng = np.random.default_rng(123)
+    sample = np.sort(rng.choice(cfg.N, size=n_sample, replace=False))
+    sample[0], sample[-1] = 0, cfg.N - 1
+    sub_inp = dict(inp, x=inp["x"][sample], dy=inp["dy"][sample])
+    of = O.forward(sub_inp, cfg)
+    ranked = H.oracle_gaps(of, cfg)
+    idx = saved["idx"][torch.from_numpy(sample).cuda()].cpu().numpy()
+    clean = H.check_indices(idx, of, cfg, ranked)
+    yg = y[torch.from_numpy(sample).cuda()].cpu().numpy()
+    H.assert_rows(yg[clean], of["y"][clean], "y")
+    if not backward:
+        return
+    dy_s = sub_inp["dy"] * clean[:, None]
+    dy = torch.zeros(cfg.N, cfg.d_v, device="cuda")
+    dy[torch.from_numpy(sample).cuda()] = torch.from_numpy(dy_s).cuda()
+    del dev["dy"]
+    g = H.gpu_backward(cfg, dims, dev, saved, dy)
+    ob = O.backward(sub_inp, cfg, of, dy_s)
+    dx = g["dx"]
+    H.assert_rows(dx[torch.from_numpy(sample).cuda()].cpu().numpy(), ob["dx"], "dx")
+    mask = torch.ones(cfg.N, dtype=torch.bool, device="cuda")
+    mask[torch.from_numpy(sample).cuda()] = False
+    assert not torch.any(dx[mask])
+    H.assert_rows(g["dWq"].cpu().numpy(), ob["dWq"], "dWq")
+    H.assert_rows(g["dsub"].cpu().numpy().reshape(-1, cfg.dk // 2),
+                  ob["dsub"].reshape(-1, cfg.dk // 2), "dsub")
+    H.assert_rows(g["dbn"].cpu().numpy(), np.stack([ob["dgamma"], ob["dbeta"]]), "dbn")
+    rows = torch.from_numpy(ob["dV_rows"]).cuda()
+    H.assert_rows(g["dV"][rows].cpu().numpy(), ob["dV_vals"], "dV")
+    assert int((g["dV"].abs().sum(1) > 0).sum()) <= len(ob["dV_rows"])
+
+
+def test_forward_K512_full_size_sampled():
+    _sampled_full_size(FWD_K512, 48, backward=False)
+
+
+def test_fwd_bwd_K1024_full_size_sampled():
+    _sampled_full_size(FULL_K1024, 24)
