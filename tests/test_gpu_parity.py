@@ -50,8 +50,8 @@ def _full_check(cfg, seed=0, flags=0):
     for t in np.nonzero(~clean)[0]:
         H.assert_rows(yg[t:t + 1], H.oracle_bag_at(of, cfg, idx, t, inp["values"])[None], "y tie")
     # softmax weights of clean heads
-    H.assert_rows(saved["w"].cpu().numpy()[clean].reshape(-1, cfg.k),
-                  of["w"][clean].reshape(-1, cfg.k), "w")
+    wg = H.align_to(idx[clean], of["idx"][clean], saved["w"].cpu().numpy()[clean])
+    H.assert_rows(wg.reshape(-1, cfg.k), of["w"][clean].reshape(-1, cfg.k), "w")
     # backward with dy masked to the clean tokens
     dy = inp["dy"] * clean[:, None]
     g = H.gpu_backward(cfg, dims, dev, saved, torch.from_numpy(dy).cuda())
@@ -66,8 +66,8 @@ def _full_check(cfg, seed=0, flags=0):
     untouched = np.ones(cfg.K, dtype=bool)
     untouched[ob["dV_rows"]] = False
     assert not dV[untouched].any()
-    H.assert_rows(g["dw"].cpu().numpy()[clean].reshape(-1, cfg.k),
-                  ob["dw"][clean].reshape(-1, cfg.k), "dw")
+    dwg = H.align_to(idx[clean], of["idx"][clean], g["dw"].cpu().numpy()[clean])
+    H.assert_rows(dwg.reshape(-1, cfg.k), ob["dw"][clean].reshape(-1, cfg.k), "dw")
     return clean
 
 
