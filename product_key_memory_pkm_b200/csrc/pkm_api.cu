@@ -114,6 +114,18 @@ pkm_status prepare(const pkm_dims* d, Plan* p) {
   return PKM_OK;
 }
 
+cudaError_t run_query(const Plan& p, const void* x, const void* Wq, const float* bn, void* q,
+                      float* qhat, cudaStream_t st) {
+  if (tc_forward_supported(p)) return launch_query_tc(p, x, Wq, bn, q, qhat, st);
+  return launch_query_simt(p, x, Wq, bn, q, qhat, st);
+}
+
+cudaError_t run_scores(const Plan& p, const void* subkeys, const void* q, float* sub_s,
+                       int32_t* sub_i, cudaStream_t st) {
+  if (tc_forward_supported(p)) return launch_scores_tc(p, subkeys, q, sub_s, sub_i, st);
+  return launch_scores_simt(p, subkeys, q, sub_s, sub_i, st);
+}
+
 pkm_status check_saved_fwd(const pkm_saved* s) {
   if (!s) return PKM_ERR_INVALID_ARG;
   PKM_NEED(s->q);
@@ -174,7 +186,7 @@ pkm_status pkm_query(const pkm_dims* d, const void* x, const void* Wq, const flo
   Plan p;
   PKM_TRY(prepare(d, &p));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return cuda_status(launch_query_simt(p, x, Wq, bn, saved->q, saved->qhat, st));
+  return cuda_status(run_query(p, x, Wq, bn, saved->q, saved->qhat, st));
 }
 
 pkm_status pkm_subkey_scores(const pkm_dims* d, const void* subkeys, const pkm_saved* saved,
@@ -187,7 +199,7 @@ pkm_status pkm_subkey_scores(const pkm_dims* d, const void* subkeys, const pkm_s
   Plan p;
   PKM_TRY(prepare(d, &p));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return cuda_status(launch_scores_simt(p, subkeys, saved->q, saved->sub_s, saved->sub_i, st));
+  return cuda_status(run_scores(p, subkeys, saved->q, saved->sub_s, saved->sub_i, st));
 }
 
 pkm_status pkm_candidate_topk(const pkm_dims* d, const pkm_saved* saved, void* stream) {
@@ -224,8 +236,8 @@ pkm_status pkm_forward(const pkm_dims* d, const void* x, const void* Wq, const f
   Plan p;
   PKM_TRY(prepare(d, &p));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  PKM_TRY(cuda_status(launch_query_simt(p, x, Wq, bn, saved->q, saved->qhat, st)));
-  PKM_TRY(cuda_status(launch_scores_simt(p, subkeys, saved->q, saved->sub_s, saved->sub_i, st)));
+  PKM_TRY(cuda_status(run_query(p, x, Wq, bn, saved->q, saved->qhat, st)));
+  PKM_TRY(cuda_status(run_scores(p, subkeys, saved->q, saved->sub_s, saved->sub_i, st)));
   PKM_TRY(cuda_status(launch_candidates(p, saved->sub_s, saved->sub_i, saved->idx, saved->w, st)));
   return cuda_status(launch_gather(p, values, saved->idx, saved->w, y, st));
 }

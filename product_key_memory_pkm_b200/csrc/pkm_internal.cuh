@@ -62,6 +62,12 @@ cudaError_t launch_query_simt(const Plan& p, const void* x, const void* Wq, cons
                               void* q, float* qhat, cudaStream_t st);
 cudaError_t launch_scores_simt(const Plan& p, const void* subkeys, const void* q, float* sub_s,
                                int32_t* sub_i, cudaStream_t st);
+// tcgen05 forward GEMMs (bf16 storage, dk/2 % 64 == 0)
+bool tc_forward_supported(const Plan& p);
+cudaError_t launch_query_tc(const Plan& p, const void* x, const void* Wq, const float* bn,
+                            void* q, float* qhat, cudaStream_t st);
+cudaError_t launch_scores_tc(const Plan& p, const void* subkeys, const void* q, float* sub_s,
+                             int32_t* sub_i, cudaStream_t st);
 cudaError_t launch_candidates(const Plan& p, const float* sub_s, const int32_t* sub_i,
                               int32_t* idx, float* w, cudaStream_t st);
 cudaError_t launch_gather(const Plan& p, const void* values, const int32_t* idx, const float* w,

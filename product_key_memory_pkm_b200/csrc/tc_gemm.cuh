@@ -1,0 +1,221 @@
+// Persistent, warp-specialised tcgen05 GEMM engine for bf16 operands with fp32
+// accumulation in TMEM:  D[128 x 256] = A[128 x K] * B[256 x K]^T per chunk.
+//
+//   warp 0     TMA producer: one lane streams A/B k-blocks (64 wide, 128-byte
+//              swizzle) into a ring of smem stages (full/empty mbarriers)
+//   warp 1     MMA issuer: allocates 512 TMEM columns (two 256-column fp32
+//              accumulators), one lane issues tcgen05.mma K=16 steps, commits each
+//              stage back to the producer and each finished chunk to the epilogue
+//   warps 2-5  epilogue: 128 threads, thread r owns accumulator row r (TMEM lane
+//              r), reads 32-column pieces with tcgen05.ld and hands them to the
+//              problem's epilogue; releases the accumulator with an mbarrier
+//
+// A "unit" is a 128-row block of the output that the problem walks in chunks of
+// 256 columns (the scoring problem keeps a running top-k across the chunks of a
+// row; the query problem has one chunk per unit).  No TMA multicast is used.
+#pragma once
+
+#include "tc_common.cuh"
+
+namespace pkm {
+namespace tc {
+
+constexpr int kBM = 128, kBN = 256, kBK = 64;
+constexpr int kStageA = kBM * kBK * 2;  // 16 KiB
+constexpr int kStageB = kBN * kBK * 2;  // 32 KiB
+constexpr int kStageBytes = kStageA + kStageB;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+
+template <class Prob>
+constexpr size_t smem_bytes() {
+  return 1024 + (size_t)Prob::kStages * kStageBytes + Prob::kEpiSmem;
+}
+
+template <class Prob>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
+                   const __grid_constant__ CUtensorMap tmA1,
+                   const __grid_constant__ CUtensorMap tmB, const typename Prob::Params P) {
+  constexpr int S = Prob::kStages;
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], tfull_bar[2], tempty_bar[2],
+      drain_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ volatile int abort_flag;
+
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* epi_smem = smem + (size_t)S * kStageBytes;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull_bar[b], 1);
+      mbar_init(&tempty_bar[b], 128);
+    }
+    mbar_init(&drain_bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA0);
+    prefetch_tmap(&tmA1);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+  int* status = P.status;
+  const int nunits = Prob::num_units(P);
+  const int nk = Prob::num_kblocks(P);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0;  // stages that received at least one load
+      uint32_t parity_mask = 0;  // bit s: full-barrier parity the last load on s completes
+      bool ok = true;
+      for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+        const int nc = Prob::num_chunks(P, u);
+        for (int c = 0; c < nc && ok; ++c) {
+          for (int kb = 0; kb < nk; ++kb) {
+            if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, status)) {
+              ok = false;
+              break;
+            }
+            unsigned char* sa = smem + (size_t)stage * kStageBytes;
+            mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
+            Prob::load(P, &tmA0, &tmA1, &tmB, u, c, kb, sa, sa + kStageA, &full_bar[stage]);
+            issued_mask |= 1u << stage;
+            parity_mask = (parity_mask & ~(1u << stage)) | (phase << stage);
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+      if (!ok) {
+        // drain: the last load issued on each stage must land before the CTA exits
+        // (earlier loads on a stage completed before the stage was reused)
+        for (int s = 0; s < S; ++s) {
+          if (!((issued_mask >> s) & 1u)) continue;
+          const uint32_t par = (parity_mask >> s) & 1u;
+          const long long t0 = clock64();
+          while (!mbar_try_wait(&full_bar[s], par) && clock64() - t0 < kWaitBudgetCycles) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(kBM, kBN, 0, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+        const int nc = Prob::num_chunks(P, u);
+        for (int c = 0; c < nc && ok; ++c) {
+          if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t dt = tmem_base + (uint32_t)acc * kBN;
+          for (int kb = 0; kb < nk; ++kb) {
+            if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + (size_t)stage * kStageBytes);
+            const uint64_t da = desc_kmajor_sw128(sa);
+            const uint64_t db = desc_kmajor_sw128(sa + kStageA);
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k)
+              mma_bf16(dt, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), idesc,
+                       (kb | k) != 0 ? 1u : 0u);
+            issued = true;
+            umma_commit(&empty_bar[stage]);
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (!ok) break;
+          umma_commit(&tfull_bar[acc]);
+          if (++acc == 2) {
+            acc = 0;
+            acc_phase ^= 1u;
+          }
+        }
+      }
+      if (issued) {
+        // all MMAs of this CTA complete before TMEM is released
+        umma_commit(&drain_bar);
+        const long long t0 = clock64();
+        while (!mbar_try_wait(&drain_bar, 0) && clock64() - t0 < kWaitBudgetCycles) {
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;            // TMEM lanes [32*quarter, 32*quarter + 32)
+    const int row = quarter * 32 + lane;     // accumulator row owned by this thread
+    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+      typename Prob::EpiState es;
+      Prob::epi_begin(P, u, row, epi_smem, es);
+      const int nc = Prob::num_chunks(P, u);
+      for (int c = 0; c < nc; ++c) {
+        // warp-uniform wait: lane 0 waits, the verdict is broadcast, so the warp reaches
+        // the .sync.aligned TMEM loads together or not at all
+        int got = 0;
+        if (lane == 0) got = mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag, status) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        Prob::epi_chunk(P, u, c, row, tmem_base + lane_addr + (uint32_t)acc * kBN, epi_smem, es);
+        tc_fence_before();
+        mbar_arrive(&tempty_bar[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      Prob::epi_end(P, u, row, epi_smem, es);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace tc
+}  // namespace pkm
