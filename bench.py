@@ -192,6 +192,9 @@ def run_b200(args, cfg, rank, world, dist):
                          workspace=ws, stream=st)
         mark(6)
 
+    if args.stage:
+        return run_stage(args, cfg, dims, saved, P, st, step, flush, names, locals())
+
     clocks = ClockSampler(torch.cuda.get_device_properties(dev).uuid and
                           "GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
     clocks.start()
@@ -321,6 +324,43 @@ def run_b200(args, cfg, rank, world, dist):
     return out
 
 
+def run_stage(args, cfg, dims, saved, P, st, step, flush, names, env):
+    """Times one stage alone (after one full step has filled the saved tensors): the
+    per-op view, and the launch that profiling captures target."""
+    import torch
+    step()
+    torch.cuda.synchronize()
+    x, Wq, bn, sub, V, y, dy, dw, ws = (env[k] for k in ("x", "Wq", "bn", "sub", "V", "y", "dy",
+                                                            "dw", "ws"))
+    dV, dx, dWq, dbn, dsub = (env[k] for k in ("dV", "dx", "dWq", "dbn", "dsub"))
+    calls = {
+        "query": lambda: P.pkm_query(dims, x, Wq, bn, saved, stream=st),
+        "subkey_scores": lambda: P.pkm_subkey_scores(dims, sub, saved, stream=st),
+        "candidate_topk": lambda: P.pkm_candidate_topk(dims, saved, stream=st),
+        "gather_bag": lambda: P.pkm_gather_bag(dims, V, saved["idx"], saved["w"], y, stream=st),
+        "value_grad": lambda: P.pkm_value_grad(dims, V, saved, dy, dw, dvalues=dV, workspace=ws,
+                                               stream=st),
+        "query_grad": lambda: P.pkm_query_grad(dims, x, Wq, bn, sub, saved, dw, dx=dx, dWq=dWq,
+                                               dbn=dbn, dsubkeys=dsub, workspace=ws, stream=st),
+    }
+    fn = calls[args.stage]
+    for _ in range(args.warmup):
+        flush.zero_()
+        fn()
+    ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        fn()
+        b.record(st)
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(b))
+    assert P.pkm_check_status(st) == P.PKM_OK
+    return {"stage": args.stage, "workload": cfg.name, "ms_per_call": round(float(np.mean(ms)), 4),
+            "ms_min": round(float(np.min(ms)), 4), "calls": args.steps}
+
+
 def _ncu_traffic(kernel: str):
     """DRAM bytes per launch from a committed ncu summary, when it is still current."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -391,10 +431,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-tokens", type=int, default=8)
+    ap.add_argument("--stage", default=None,
+                    choices=["query", "subkey_scores", "candidate_topk", "gather_bag",
+                             "value_grad", "query_grad"],
+                    help="time one stage alone (per-op benchmark / profiling target)")
+    ap.add_argument("--tokens", type=int, default=None, help="override the token count")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     cfg = CONFIGS[args.workload]
+    if args.tokens:
+        cfg = cfg.with_(N=args.tokens)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     dist = None

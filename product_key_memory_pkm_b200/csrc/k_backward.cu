@@ -46,79 +46,161 @@ struct VecT<float> {
 };
 
 // ------------------------------------------------------------------ B3
-// CH = 16-byte value chunks per lane per column block (column block = 32*CH*E).
+// L2 policies: the upstream gradient rows are re-read once per selection and stay
+// resident (evict_last); value rows and value-gradient rows stream (evict_first).
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ float4 ld_f4_hint(const float* p, uint64_t pol) {
+  float4 v;
+  asm volatile("ld.global.L2::cache_hint.v4.f32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+__device__ __forceinline__ uint4 ld_u4_stream(const void* p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+__device__ __forceinline__ void st_f4_hint(float* p, float4 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1,%2,%3,%4}, %5;" ::"l"(p), "f"(v.x),
+               "f"(v.y), "f"(v.z), "f"(v.w), "l"(pol)
+               : "memory");
+}
+
+template <typename TV>
+__device__ __forceinline__ void load_vals(const TV* p, uint64_t pol, float* f);
+template <>
+__device__ __forceinline__ void load_vals<__nv_bfloat16>(const __nv_bfloat16* p, uint64_t pol,
+                                                          float* f) {
+  bf16x8_to_f32(ld_u4_stream(p, pol), f);
+}
+template <>
+__device__ __forceinline__ void load_vals<float>(const float* p, uint64_t pol, float* f) {
+  uint4 u = ld_u4_stream(p, pol);
+  f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+  f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+}
+
+// One 128-thread CTA per distinct value row r (grid-stride over rows).  Thread j owns
+// 16-byte value chunks j and j + 128 of the row (CH of them).  The row's selections
+// are taken in batches of 64: their entry ids and weights are staged in shared
+// memory, each thread accumulates its chunks of sum_e w_e dy[t_e] in registers and
+// a partial dot dy[t_e] . V[r] per selection; partials are reduced over the 4 warps in
+// a fixed order.  V[r] is read once, dV[r] read and written once.
+constexpr int kB3Threads = 128, kB3Batch = 64;
+
 template <typename TV, int CH>
-__global__ void __launch_bounds__(256) value_rows_kernel(
+__global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
     const int* __restrict__ seg, const int* __restrict__ U_ptr, const int32_t* __restrict__ rows,
     const int32_t* __restrict__ ents, const TV* __restrict__ V, const float* __restrict__ w,
     const float* __restrict__ dy, float* __restrict__ dV, float* __restrict__ dw, int hk, int d_v,
     int64_t K, int* status) {
   constexpr int E = VecT<TV>::E;
-  const int lane = threadIdx.x & 31;
-  const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  __shared__ int s_t[kB3Batch];
+  __shared__ int s_e[kB3Batch];
+  __shared__ float s_w[kB3Batch];
+  __shared__ float s_part[kB3Threads / 32][kB3Batch];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int U = *U_ptr;
   const int nvec = d_v / E;
-  for (int64_t u = warp0; u < U; u += nwarps) {
+  const uint64_t pol_keep = policy_evict_last();
+  const uint64_t pol_stream = policy_evict_first();
+  for (int u = blockIdx.x; u < U; u += gridDim.x) {
     const int p0 = seg[u], p1 = seg[u + 1];
     const int32_t r = rows[p0];
     if (r < 0 || r >= K) {
-      set_status(status, kDevIndex);
-      continue;
+      if (tid == 0) set_status(status, kDevIndex);
+      continue;  // uniform across the CTA
     }
-    for (int cb = 0; cb < nvec; cb += 32 * CH) {
+    const TV* Vr = V + (int64_t)r * d_v;
+    float* dVr = dV ? dV + (int64_t)r * d_v : nullptr;
+    for (int cb = 0; cb < nvec; cb += kB3Threads * CH) {
       float v[CH][E], acc[CH][E];
 #pragma unroll
       for (int c = 0; c < CH; ++c) {
-        const int vec = cb + lane + 32 * c;
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[c][e] = 0.f;
-        if (vec < nvec)
-          VecT<TV>::load(V + (int64_t)r * d_v + (int64_t)vec * E, v[c]);
-        else
-#pragma unroll
-          for (int e = 0; e < E; ++e) v[c][e] = 0.f;
-      }
-      for (int p = p0; p < p1; ++p) {
-        const int32_t ent = ents[p];
-        const int64_t t = ent / hk;
-        const float wt = w[ent];
-        float dot = 0.f;
-#pragma unroll
-        for (int c = 0; c < CH; ++c) {
-          const int vec = cb + lane + 32 * c;
-          if (vec < nvec) {
-            const float4* g = reinterpret_cast<const float4*>(dy + t * d_v + (int64_t)vec * E);
+        const int vec = cb + tid + kB3Threads * c;
+        if (vec < nvec) {
+          load_vals<TV>(Vr + (int64_t)vec * E, pol_stream, v[c]);
+          if (dVr) {
 #pragma unroll
             for (int e4 = 0; e4 < E / 4; ++e4) {
-              float4 d4 = g[e4];
-              float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+              float4 a = ld_f4_hint(dVr + (int64_t)vec * E + 4 * e4, pol_stream);
+              acc[c][4 * e4] = a.x; acc[c][4 * e4 + 1] = a.y;
+              acc[c][4 * e4 + 2] = a.z; acc[c][4 * e4 + 3] = a.w;
+            }
+          } else {
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                dot = fmaf(dd[e], v[c][e4 * 4 + e], dot);
-                acc[c][e4 * 4 + e] = fmaf(wt, dd[e], acc[c][e4 * 4 + e]);
+            for (int e = 0; e < E; ++e) acc[c][e] = 0.f;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < E; ++e) v[c][e] = acc[c][e] = 0.f;
+        }
+      }
+      for (int pb = p0; pb < p1; pb += kB3Batch) {
+        const int nb = min(kB3Batch, p1 - pb);
+        __syncthreads();  // previous batch's staging fully consumed
+        if (tid < nb) {
+          const int32_t ent = ents[pb + tid];
+          s_e[tid] = ent;
+          s_t[tid] = ent / hk;
+          s_w[tid] = w[ent];
+        }
+        __syncthreads();
+        for (int i = 0; i < nb; ++i) {
+          const float* dyt = dy + (int64_t)s_t[i] * d_v;
+          const float wt = s_w[i];
+          float dot = 0.f;
+#pragma unroll
+          for (int c = 0; c < CH; ++c) {
+            const int vec = cb + tid + kB3Threads * c;
+            if (vec < nvec) {
+#pragma unroll
+              for (int e4 = 0; e4 < E / 4; ++e4) {
+                const float4 d4 = ld_f4_hint(dyt + (int64_t)vec * E + 4 * e4, pol_keep);
+                const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  dot = fmaf(dd[e], v[c][4 * e4 + e], dot);
+                  acc[c][4 * e4 + e] = fmaf(wt, dd[e], acc[c][4 * e4 + e]);
+                }
               }
             }
           }
+          dot = warp_sum(dot);
+          if (lane == 0) s_part[wid][i] = dot;
         }
-        dot = warp_sum(dot);
-        if (lane == 0) dw[ent] = (cb == 0) ? dot : dw[ent] + dot;
+        __syncthreads();
+        if (tid < nb) {
+          float sdot = 0.f;
+#pragma unroll
+          for (int ww = 0; ww < kB3Threads / 32; ++ww) sdot += s_part[ww][tid];
+          const int32_t ent = s_e[tid];
+          dw[ent] = (cb == 0) ? sdot : dw[ent] + sdot;
+        }
       }
-      if (dV) {
+      if (dVr) {
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
-          const int vec = cb + lane + 32 * c;
+          const int vec = cb + tid + kB3Threads * c;
           if (vec < nvec) {
-            float4* o = reinterpret_cast<float4*>(dV + (int64_t)r * d_v + (int64_t)vec * E);
 #pragma unroll
-            for (int e4 = 0; e4 < E / 4; ++e4) {
-              float4 x = o[e4];
-              x.x += acc[c][e4 * 4 + 0];
-              x.y += acc[c][e4 * 4 + 1];
-              x.z += acc[c][e4 * 4 + 2];
-              x.w += acc[c][e4 * 4 + 3];
-              o[e4] = x;
-            }
+            for (int e4 = 0; e4 < E / 4; ++e4)
+              st_f4_hint(dVr + (int64_t)vec * E + 4 * e4,
+                         make_float4(acc[c][4 * e4], acc[c][4 * e4 + 1], acc[c][4 * e4 + 2],
+                                     acc[c][4 * e4 + 3]),
+                         pol_stream);
           }
         }
       }
@@ -162,10 +244,10 @@ __global__ void __launch_bounds__(256) softmax_bwd_kernel(
 // partial sums of dq * qhat and dq for the BatchNorm affine gradients.
 constexpr int kDqTokensPerBlock = 64;
 
-template <typename TS, int MAXC>
+template <typename TS, int MAXC, bool kSplit>
 __global__ void __launch_bounds__(256) dq_kernel(
     const float* __restrict__ gsub, const int32_t* __restrict__ sub_i, const TS* __restrict__ sub,
-    const float* __restrict__ bn, const float* __restrict__ qhat, float* __restrict__ dq_pre,
+    const float* __restrict__ bn, const float* __restrict__ qhat, void* __restrict__ dq_out,
     float* __restrict__ part, int64_t N, int h, int dk, int C1, int C2, int k, float eps) {
   constexpr int E = VecT<TS>::E;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -211,7 +293,16 @@ __global__ void __launch_bounds__(256) dq_kernel(
         for (int e = 0; e < E; ++e) {
           const int col = col0 + vec * E + e;
           const float gam = bn[2 * hq + col], var = bn[hq + col];
-          dq_pre[t * hq + col] = acc[c][e] * gam / sqrtf(var + eps);
+          const float val = acc[c][e] * gam / sqrtf(var + eps);
+          if constexpr (kSplit) {
+            // dq_pre as two bf16 planes [2][N][hq]: hi = bf16(v), lo = bf16(v - hi)
+            __nv_bfloat16* pl = static_cast<__nv_bfloat16*>(dq_out);
+            const __nv_bfloat16 hi = __float2bfloat16_rn(val);
+            pl[t * hq + col] = hi;
+            pl[N * hq + t * hq + col] = __float2bfloat16_rn(val - __bfloat162float(hi));
+          } else {
+            static_cast<float*>(dq_out)[t * hq + col] = val;
+          }
           if (qhat) pg[c][e] = fmaf(acc[c][e], qhat[t * hq + col], pg[c][e]);
           pb[c][e] += acc[c][e];
         }
@@ -435,25 +526,22 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
   {
     const int E = p.fp32 ? 4 : 8;
     const int nvec = p.d_v / E;
-    const int chunks = (nvec + 31) / 32;
-#define PKM_B3(TV, CHV)                                                                      \
-  value_rows_kernel<TV, CHV><<<persist_blocks, 256, 0, st>>>(                                \
-      seg, U, rows_sorted, ents_sorted, static_cast<const TV*>(values), s.w, dy, dV, dw, hk, \
-      p.d_v, p.K, p.status)
+    const int blocks = p.sm_count * 6;
+#define PKM_B3(TV, CHV)                                                                  \
+  value_rows_kernel<TV, CHV><<<blocks, kB3Threads, 0, st>>>(                             \
+      seg, U, rows_sorted, ents_sorted, static_cast<const TV*>(values), s.w, dy, dV, dw, \
+      hk, p.d_v, p.K, p.status)
     if (p.fp32) {
-      if (chunks <= 1) PKM_B3(float, 1);
-      else if (chunks <= 2) PKM_B3(float, 2);
-      else if (chunks <= 4) PKM_B3(float, 4);
-      else PKM_B3(float, 8);
+      if (nvec <= kB3Threads) PKM_B3(float, 1);
+      else PKM_B3(float, 2);
     } else {
-      if (chunks <= 1) PKM_B3(__nv_bfloat16, 1);
-      else if (chunks <= 2) PKM_B3(__nv_bfloat16, 2);
-      else if (chunks <= 4) PKM_B3(__nv_bfloat16, 4);
-      else PKM_B3(__nv_bfloat16, 8);
+      if (nvec <= kB3Threads) PKM_B3(__nv_bfloat16, 1);
+      else PKM_B3(__nv_bfloat16, 2);
     }
 #undef PKM_B3
     PKM_COUNT(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    (void)persist_blocks;
   }
 
   return cudaSuccess;
@@ -489,15 +577,23 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
     dim3 grid((unsigned)nblk, (unsigned)(p.h * 2));
     float* partp = dbn ? part : nullptr;
     const float* qh = dbn ? s.qhat : nullptr;
+    const bool split = tc_backward_supported(p);
+#define PKM_DQ(TS, MC, SPL)                                                                 \
+  dq_kernel<TS, MC, SPL><<<grid, 256, 0, st>>>(gsub, s.sub_i, (const TS*)subkeys, bn, qh, \
+                                               dq_pre, partp, p.N, p.h, p.dk, p.C1, p.C2,  \
+                                               p.k, p.eps)
     if (p.fp32) {
-      const int nv = p.half / 4;
-      if (nv <= 32) dq_kernel<float, 1><<<grid, 256, 0, st>>>(gsub, s.sub_i, (const float*)subkeys, bn, qh, dq_pre, partp, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.eps);
-      else dq_kernel<float, 4><<<grid, 256, 0, st>>>(gsub, s.sub_i, (const float*)subkeys, bn, qh, dq_pre, partp, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.eps); PKM_COUNT(1);
+      if (p.half / 4 <= 32) PKM_DQ(float, 1, false);
+      else PKM_DQ(float, 4, false);
+    } else if (split) {
+      if (p.half / 8 <= 32) PKM_DQ(__nv_bfloat16, 1, true);
+      else PKM_DQ(__nv_bfloat16, 4, true);
     } else {
-      const int nv = p.half / 8;
-      if (nv <= 32) dq_kernel<__nv_bfloat16, 1><<<grid, 256, 0, st>>>(gsub, s.sub_i, (const __nv_bfloat16*)subkeys, bn, qh, dq_pre, partp, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.eps);
-      else dq_kernel<__nv_bfloat16, 4><<<grid, 256, 0, st>>>(gsub, s.sub_i, (const __nv_bfloat16*)subkeys, bn, qh, dq_pre, partp, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.eps); PKM_COUNT(1);
+      if (p.half / 8 <= 32) PKM_DQ(__nv_bfloat16, 1, false);
+      else PKM_DQ(__nv_bfloat16, 4, false);
     }
+#undef PKM_DQ
+    PKM_COUNT(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (dbn) {
       dbn_reduce_kernel<<<(2 * p.hq + 255) / 256, 256, 0, st>>>(part, (int)nblk, p.hq, dbn); PKM_COUNT(1);
@@ -530,6 +626,11 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
   }
 
   // B7: dense query gradients
+  if (tc_backward_supported(p)) {
+    if (dx && (e = launch_dx_tc(p, dq_pre, Wq, dx, st)) != cudaSuccess) return e;
+    if (dWq && (e = launch_dwq_tc(p, dq_pre, x, dWq, st)) != cudaSuccess) return e;
+    return cudaSuccess;
+  }
   if (dx) {
     e = gemm_simt_f32(p.N, p.d_in, p.hq, dq_pre, false, p.hq, 1, Wq, !p.fp32, 1, p.d_in, dx,
                       p.d_in, GemmOut::Store, st);

@@ -16,6 +16,7 @@
 #include <mutex>
 
 #include "tc_gemm.cuh"
+#include "tc_launch.cuh"
 
 namespace pkm {
 
@@ -50,6 +51,7 @@ using namespace tc;
 
 // ================================================================== F1 query network
 struct QueryProb {
+  static constexpr int kAMN = 0, kBMN = 0;
   static constexpr int kStages = 4;
   static constexpr int kEpiSmem = 0;
   struct Params {
@@ -131,8 +133,10 @@ struct QueryProb {
 // ================================================================== F2 sub-key scores
 template <int KM>
 struct ScoresProb {
+  static constexpr int kAMN = 0, kBMN = 0;
   static constexpr int kStages = 3;
-  static constexpr int kEpiSmem = KM * kBM * 8;  // heap: KM (score, index) slots per row
+  // heap: KM (score, index) slots per row; staging: one 32-column piece per row
+  static constexpr int kEpiSmem = KM * kBM * 8 + 32 * kBM * 4;
   struct Params {
     int* status;
     float* sub_s;
@@ -165,6 +169,9 @@ struct ScoresProb {
   __device__ static float* hs_(unsigned char* sm) { return reinterpret_cast<float*>(sm); }
   __device__ static int* hi_(unsigned char* sm) {
     return reinterpret_cast<int*>(sm + KM * kBM * 4);
+  }
+  __device__ static float* stage_(unsigned char* sm) {
+    return reinterpret_cast<float*>(sm + KM * kBM * 8);
   }
 
   // worse(a, b): a ranks below b in (score desc, index asc)
@@ -220,18 +227,29 @@ struct ScoresProb {
     const int C = (hs_idx & 1) ? P.C2 : P.C1;
     float* hs = hs_(sm);
     int* hi = hi_(sm);
+    float* stg = stage_(sm);
     for (int piece = 0; piece < kBN / 32; ++piece) {
       const int col0 = c * kBN + piece * 32;
       if (col0 >= C) break;  // warp-uniform
       uint32_t r[32];
       tmem_ld32(taddr + (uint32_t)(piece * 32), r);
       tmem_wait_ld();
+      // candidates of this piece against the threshold at its start
+      uint32_t mask = 0;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float v = __uint_as_float(r[j]);
-        if (v > es.thr && col0 + j < C) {
-          sift_root(hs, hi, row, KM, v, col0 + j);
-          es.thr = hs[row];
+      for (int j = 0; j < 32; ++j) mask |= (__uint_as_float(r[j]) > es.thr ? 1u : 0u) << j;
+      if (C - col0 < 32) mask &= (1u << (C - col0)) - 1u;
+      if (mask) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) stg[j * kBM + row] = __uint_as_float(r[j]);
+        while (mask) {
+          const int j = __ffs(mask) - 1;
+          mask &= mask - 1u;
+          const float v = stg[j * kBM + row];
+          if (v > es.thr) {
+            sift_root(hs, hi, row, KM, v, col0 + j);
+            es.thr = hs[row];
+          }
         }
       }
     }
@@ -257,24 +275,6 @@ struct ScoresProb {
     }
   }
 };
-
-template <class Prob>
-cudaError_t launch_tc(const CUtensorMap& A0, const CUtensorMap& A1, const CUtensorMap& B,
-                      const typename Prob::Params& P, int nunits, int sm_count, cudaStream_t st) {
-  constexpr size_t smem = smem_bytes<Prob>();
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, []() {
-    attr_err = cudaFuncSetAttribute(tc_gemm_kernel<Prob>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  });
-  if (attr_err != cudaSuccess) return attr_err;
-  const int grid = nunits < sm_count ? nunits : sm_count;
-  if (grid <= 0) return cudaSuccess;
-  tc_gemm_kernel<Prob><<<grid, kThreads, smem, st>>>(A0, A1, B, P);
-  PKM_COUNT(1);
-  return cudaGetLastError();
-}
 
 }  // namespace
 

@@ -68,6 +68,12 @@ cudaError_t launch_query_tc(const Plan& p, const void* x, const void* Wq, const 
                             void* q, float* qhat, cudaStream_t st);
 cudaError_t launch_scores_tc(const Plan& p, const void* subkeys, const void* q, float* sub_s,
                              int32_t* sub_i, cudaStream_t st);
+// tcgen05 backward GEMMs (bf16 storage); dq_planes = [2][N][hq] bf16 (hi, lo)
+bool tc_backward_supported(const Plan& p);
+cudaError_t launch_dx_tc(const Plan& p, const void* dq_planes, const void* Wq, float* dx,
+                         cudaStream_t st);
+cudaError_t launch_dwq_tc(const Plan& p, const void* dq_planes, const void* x, float* dWq,
+                          cudaStream_t st);
 cudaError_t launch_candidates(const Plan& p, const float* sub_s, const int32_t* sub_i,
                               int32_t* idx, float* w, cudaStream_t st);
 cudaError_t launch_gather(const Plan& p, const void* values, const int32_t* idx, const float* w,

@@ -12,7 +12,14 @@
 //
 // A "unit" is a 128-row block of the output that the problem walks in chunks of
 // 256 columns (the scoring problem keeps a running top-k across the chunks of a
-// row; the query problem has one chunk per unit).  No TMA multicast is used.
+// row; the other problems have one chunk per unit).  No TMA multicast is used.
+//
+// Operand layouts in a stage (both 128-byte swizzled, as TMA writes them):
+//   K-major  (Prob::kAMN / kBMN == 0): rows of 64 k-elements (128 B), 8-row groups
+//            1024 B apart; one TMA box of 64 x rows.
+//   MN-major (== 1): rows of 64 MN-elements (128 B), one row per k, 8-k groups
+//            1024 B apart (SBO), 64-wide MN blocks 8 KiB apart (LBO); one 64 x 64 TMA
+//            box per MN block.  A K=16 step advances 16 rows = 2 KiB.
 #pragma once
 
 #include "tc_common.cuh"
@@ -122,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(kBM, kBN, 0, 0);
+      constexpr uint32_t idesc = idesc_bf16(kBM, kBN, Prob::kAMN, Prob::kBMN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -145,12 +152,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             const uint32_t sa = smem_u32(smem + (size_t)stage * kStageBytes);
-            const uint64_t da = desc_kmajor_sw128(sa);
-            const uint64_t db = desc_kmajor_sw128(sa + kStageA);
+            const uint32_t sb = sa + kStageA;
 #pragma unroll
-            for (int k = 0; k < kBK / 16; ++k)
-              mma_bf16(dt, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), idesc,
-                       (kb | k) != 0 ? 1u : 0u);
+            for (int k = 0; k < kBK / 16; ++k) {
+              const uint64_t da = Prob::kAMN ? desc_mnmajor_sw128(sa + 2048u * k, 8192u, 1024u)
+                                             : desc_kmajor_sw128(sa) + (uint64_t)(2 * k);
+              const uint64_t db = Prob::kBMN ? desc_mnmajor_sw128(sb + 2048u * k, 8192u, 1024u)
+                                             : desc_kmajor_sw128(sb) + (uint64_t)(2 * k);
+              mma_bf16(dt, da, db, idesc, (kb | k) != 0 ? 1u : 0u);
+            }
             issued = true;
             umma_commit(&empty_bar[stage]);
             if (++stage == S) {
