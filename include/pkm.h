@@ -175,6 +175,12 @@ pkm_status pkm_check_status(void* stream);
 /* Static, human-readable name of a status code. */
 const char* pkm_status_string(pkm_status s);
 
+/* Self-test of the device-side bounded wait: launches one warp that waits on a
+ * barrier nothing arrives on, with a budget of `budget_cycles` SM clocks (1 to 1e8).
+ * The wait gives up and records PKM_ERR_DEVICE_TIMEOUT in the status word, which the
+ * next pkm_check_status returns (and clears).  Faults, traps and hangs nothing. */
+pkm_status pkm_selftest_wait_timeout(uint32_t budget_cycles, void* stream);
+
 /* Number of kernels this library has launched in this process (diagnostics). */
 unsigned long long pkm_launch_count(void);
 

@@ -100,9 +100,13 @@ __device__ __forceinline__ void load_vals<float>(const float* p, uint64_t pol, f
 // a fixed order.  V[r] is read once, dV[r] read and written once.
 constexpr int kB3Threads = 128, kB3Batch = 64;
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 template <typename TV, int CH>
 __global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
-    const int* __restrict__ seg, const int* __restrict__ U_ptr, const int32_t* __restrict__ rows,
+    const int* __restrict__ seg, const int* __restrict__ U_ptr, const int32_t* __restrict__ seg_row,
     const int32_t* __restrict__ ents, const TV* __restrict__ V, const float* __restrict__ w,
     const float* __restrict__ dy, float* __restrict__ dV, float* __restrict__ dw, int hk, int d_v,
     int64_t K, int* status) {
@@ -116,15 +120,25 @@ __global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
   const int nvec = d_v / E;
   const uint64_t pol_keep = policy_evict_last();
   const uint64_t pol_stream = policy_evict_first();
+  const int row_bytes_v = d_v * (int)sizeof(TV), row_bytes_dv = d_v * 4;
   for (int u = blockIdx.x; u < U; u += gridDim.x) {
     const int p0 = seg[u], p1 = seg[u + 1];
-    const int32_t r = rows[p0];
+    const int32_t r = seg_row[u];
     if (r < 0 || r >= K) {
       if (tid == 0) set_status(status, kDevIndex);
       continue;  // uniform across the CTA
     }
     const TV* Vr = V + (int64_t)r * d_v;
     float* dVr = dV ? dV + (int64_t)r * d_v : nullptr;
+    // the next row of this CTA: metadata now, its lines into L2 once known
+    const int un = u + gridDim.x;
+    int np0 = 0, np1 = 0;
+    int32_t nr = -1;
+    if (un < U) {
+      np0 = seg[un];
+      np1 = seg[un + 1];
+      nr = seg_row[un];
+    }
     for (int cb = 0; cb < nvec; cb += kB3Threads * CH) {
       float v[CH][E], acc[CH][E];
 #pragma unroll
@@ -189,6 +203,17 @@ __global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
           const int32_t ent = s_e[tid];
           dw[ent] = (cb == 0) ? sdot : dw[ent] + sdot;
         }
+      }
+      if (cb == 0 && nr >= 0 && nr < K) {
+        const char* nv = reinterpret_cast<const char*>(V + (int64_t)nr * d_v);
+        for (int off = tid * 128; off < row_bytes_v; off += kB3Threads * 128) prefetch_l2(nv + off);
+        if (dV) {
+          const char* nd = reinterpret_cast<const char*>(dV + (int64_t)nr * d_v);
+          for (int off = tid * 128; off < row_bytes_dv; off += kB3Threads * 128)
+            prefetch_l2(nd + off);
+        }
+        if (tid == 0) prefetch_l2(ents + np0);
+        if (tid == 1 && np1 - np0 > 32) prefetch_l2(ents + np0 + 32);
       }
       if (dVr) {
 #pragma unroll
@@ -434,7 +459,7 @@ inline int bits_for(int64_t maxkey) {
 
 // ------------------------------------------------------------------ workspace
 struct Layout {
-  size_t keysA, valsA, keysB, valsB, hist, bsum, seg, U, dw, gsub, dq, part, total;
+  size_t keysA, valsA, keysB, valsB, hist, bsum, seg, segrow, U, dw, gsub, dq, part, total;
 };
 
 inline size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -458,6 +483,7 @@ Layout layout(const Plan& p) {
   const int64_t bl = std::max(sort::scan_bsum_len(hl), sort::scan_bsum_len(En));
   L.bsum = take(4 * bl);
   L.seg = take(4 * (En + 1));
+  L.segrow = take(4 * (En + 1));
   L.U = take(4);
   L.dw = take(4 * E1);
   L.gsub = take(4 * E2);
@@ -480,6 +506,7 @@ size_t backward_workspace_bytes(const Plan& p) { return layout(p).total; }
 struct BwdCtx {
   sort::RadixBuffers rb;
   int* seg;
+  int32_t* seg_row;
   int* U;
   float* dw;
   float* gsub;
@@ -494,6 +521,7 @@ static BwdCtx bwd_ctx(const Plan& p, void* ws, float* dw_out) {
                             at<int32_t>(ws, L.keysB), at<int32_t>(ws, L.valsB),
                             at<int>(ws, L.hist), at<int>(ws, L.bsum)};
   c.seg = at<int>(ws, L.seg);
+  c.seg_row = at<int32_t>(ws, L.segrow);
   c.U = at<int>(ws, L.U);
   c.dw = dw_out ? dw_out : at<float>(ws, L.dw);
   c.gsub = at<float>(ws, L.gsub);
@@ -509,6 +537,7 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
   BwdCtx c = bwd_ctx(p, ws, dw_out);
   sort::RadixBuffers& rb = c.rb;
   int* seg = c.seg;
+  int32_t* seg_row = c.seg_row;
   int* U = c.U;
   float* dw = c.dw;
   cudaError_t e;
@@ -519,7 +548,7 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
   const int32_t *rows_sorted, *ents_sorted;
   e = sort::radix_sort(s.idx, E1, bits_for(p.K - 1), rb, &rows_sorted, &ents_sorted, st);
   if (e != cudaSuccess) return e;
-  e = sort::segments(rows_sorted, E1, seg, U, rb.bsum, st);
+  e = sort::segments(rows_sorted, E1, seg, U, rb.bsum, st, seg_row);
   if (e != cudaSuccess) return e;
 
   // B3: value rows
@@ -529,7 +558,7 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
     const int blocks = p.sm_count * 6;
 #define PKM_B3(TV, CHV)                                                                  \
   value_rows_kernel<TV, CHV><<<blocks, kB3Threads, 0, st>>>(                             \
-      seg, U, rows_sorted, ents_sorted, static_cast<const TV*>(values), s.w, dy, dV, dw, \
+      seg, U, seg_row, ents_sorted, static_cast<const TV*>(values), s.w, dy, dV, dw,     \
       hk, p.d_v, p.K, p.status)
     if (p.fp32) {
       if (nvec <= kB3Threads) PKM_B3(float, 1);

@@ -100,8 +100,13 @@ struct FlagIn {
 struct SegOut {
   int* seg;
   int* U;
+  const int32_t* keys;
+  int32_t* seg_key;
   __device__ void operator()(int64_t i, int excl, int v, int64_t n) const {
-    if (v) seg[excl] = (int)i;
+    if (v) {
+      seg[excl] = (int)i;
+      if (seg_key) seg_key[excl] = keys[i];
+    }
     if (i == n - 1) {
       seg[excl + v] = (int)n;
       *U = excl + v;
@@ -148,8 +153,8 @@ cudaError_t radix_sort(const int32_t* keys_src, int64_t n, int bits_total, const
 }
 
 cudaError_t segments(const int32_t* keys, int64_t n, int* seg, int* U_out, int* bsum,
-                     cudaStream_t st) {
-  return exclusive_scan(FlagIn{keys}, SegOut{seg, U_out}, n, bsum, st);
+                     cudaStream_t st, int32_t* seg_key) {
+  return exclusive_scan(FlagIn{keys}, SegOut{seg, U_out, keys, seg_key}, n, bsum, st);
 }
 
 }  // namespace sort

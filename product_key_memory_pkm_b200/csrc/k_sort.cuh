@@ -115,9 +115,10 @@ cudaError_t radix_sort(const int32_t* keys_src, int64_t n, int bits_total, const
                        const int32_t** keys_out, const int32_t** vals_out, cudaStream_t st);
 
 // Segment table of a sorted key array: seg[u] = first position of the u-th
-// distinct key, seg[U] = n, *U_out = U.
+// distinct key, seg[U] = n, *U_out = U, and (when seg_key is not null)
+// seg_key[u] = that key.
 cudaError_t segments(const int32_t* keys, int64_t n, int* seg, int* U_out, int* bsum,
-                     cudaStream_t st);
+                     cudaStream_t st, int32_t* seg_key = nullptr);
 
 }  // namespace sort
 }  // namespace pkm

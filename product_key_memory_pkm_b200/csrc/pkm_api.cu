@@ -296,6 +296,14 @@ pkm_status pkm_query_grad(const pkm_dims* d, const void* x, const void* Wq, cons
 
 unsigned long long pkm_launch_count(void) { return g_launches.load(); }
 
+pkm_status pkm_selftest_wait_timeout(uint32_t budget_cycles, void* stream) {
+  if (budget_cycles == 0 || budget_cycles > 100000000u) return PKM_ERR_INVALID_ARG;
+  int dev = 0;
+  if (!device_setup(&dev)) return PKM_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_wait_timeout_probe((long long)budget_cycles, g_status_ptr[dev], st));
+}
+
 pkm_status pkm_check_status(void* stream) {
   int dev = 0;
   if (!device_setup(&dev)) return PKM_ERR_CUDA;

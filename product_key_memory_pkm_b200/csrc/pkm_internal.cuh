@@ -93,6 +93,9 @@ cudaError_t launch_backward(const Plan& p, const void* x, const void* Wq, const 
                             const float* dy, float* dx, float* dWq, float* dbn, float* dsub,
                             float* dV, float* dw_out, void* ws, cudaStream_t st);
 
+// ---------------------------------------------------------------- self-test
+cudaError_t launch_wait_timeout_probe(long long budget_cycles, int* status, cudaStream_t st);
+
 // ---------------------------------------------------------------- generic CUDA-core GEMM
 // C[m][n] (op)= sum_k A(m,k) * B(n,k), A(m,k) = A[m*sam + k*sak], B(n,k) = B[n*sbn + k*sbk].
 enum class GemmOut { Store, Accumulate };

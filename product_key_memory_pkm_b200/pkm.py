@@ -35,7 +35,7 @@ SAVED_FIELDS = ("q", "qhat", "sub_s", "sub_i", "idx", "w")
 EXPORTED = ("pkm_saved_bytes", "pkm_workspace_bytes", "pkm_forward", "pkm_backward", "pkm_query",
             "pkm_subkey_scores", "pkm_candidate_topk", "pkm_gather_bag", "pkm_check_status",
             "pkm_status_string", "pkm_build_info", "pkm_value_grad", "pkm_query_grad",
-            "pkm_launch_count")
+            "pkm_launch_count", "pkm_selftest_wait_timeout")
 
 
 class PKMError(RuntimeError):
@@ -85,6 +85,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "pkm_value_grad": (I, [D, P, SV, P, P, P, P, S, P]),
         "pkm_query_grad": (I, [D, P, P, P, P, SV, P, P, P, P, P, P, S, P]),
         "pkm_launch_count": (ctypes.c_ulonglong, []),
+        "pkm_selftest_wait_timeout": (I, [ctypes.c_uint32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -207,6 +208,11 @@ def pkm_query_grad(dims: Dims, x, Wq, bn, subkeys, saved: dict, dw, dx=None, dWq
                                  _ptr(dbn), _ptr(dsubkeys), _ptr(workspace),
                                  _ws(workspace, workspace_bytes), _stream(stream)),
            "pkm_query_grad")
+
+
+def pkm_selftest_wait_timeout(budget_cycles: int = 2_000_000, stream=None) -> None:
+    _check(load().pkm_selftest_wait_timeout(int(budget_cycles), _stream(stream)),
+           "pkm_selftest_wait_timeout")
 
 
 def pkm_launch_count() -> int:

@@ -252,3 +252,13 @@ def test_forward_K512_full_size_sampled():
 
 def test_fwd_bwd_K1024_full_size_sampled():
     _sampled_full_size(FULL_K1024, 24)
+
+
+def test_bounded_wait_expires_with_status_and_context_survives():
+    """A wait on a barrier that nothing completes gives up after its budget, records
+    PKM_ERR_DEVICE_TIMEOUT, and the next call on the same context works."""
+    assert P.pkm_check_status() == P.PKM_OK
+    P.pkm_selftest_wait_timeout(2_000_000)          # ~1 ms at B200 clocks
+    assert P.pkm_check_status() == P.PKM_ERR_DEVICE_TIMEOUT
+    assert P.pkm_check_status() == P.PKM_OK         # read-and-clear
+    _full_check(CASES["tiny_bf16"])                 # the context is still usable
