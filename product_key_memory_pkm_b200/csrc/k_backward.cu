@@ -14,6 +14,7 @@
 //          dC[i] += sum over (t, a) choosing i of g * q_half[t]  (sorted segments)
 //   B7     dx = dq_pre Wq,  dWq += dq_pre^T x
 #include "k_sort.cuh"
+#include "tc_common.cuh"
 
 namespace pkm {
 namespace {
@@ -92,16 +93,38 @@ __device__ __forceinline__ void load_vals<float>(const float* p, uint64_t pol, f
   f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
 }
 
-// One 128-thread CTA per distinct value row r (grid-stride over rows).  Thread j owns
-// 16-byte value chunks j and j + 128 of the row (CH of them).  The row's selections
-// are taken in batches of 64: their entry ids and weights are staged in shared
-// memory, each thread accumulates its chunks of sum_e w_e dy[t_e] in registers and
-// a partial dot dy[t_e] . V[r] per selection; partials are reduced over the 4 warps in
-// a fixed order.  V[r] is read once, dV[r] read and written once.
+// One 128-thread CTA per distinct value row r (grid-stride over rows), with the rows
+// double-buffered in shared memory: while the CTA works on row u, one thread has
+// already issued the 1-D bulk async copies (cp.async.bulk, mbarrier completion, L2
+// evict_first) of V[r'] and dV[r'] for its next row u' into the other buffer, so a
+// row's bytes are in flight during the previous row's arithmetic without costing
+// registers.  Thread j owns 16-byte chunks j, j + 128, ... of the row (CH of them
+// per column block).  A row's selections are taken in batches of 64: entry ids and
+// weights staged in shared memory; each thread accumulates its chunks of
+// sum_e w_e dy[t_e] and a partial dot dy[t_e] . V[r]; partials are reduced over the 4
+// warps in a fixed order.  dV[r] is read once and written once (one writer, no
+// atomics).  Every mbarrier wait is bounded.
 constexpr int kB3Threads = 128, kB3Batch = 64;
 
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(tc::smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(tc::smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+
+template <typename TV>
+__device__ __forceinline__ void smem_vals(const TV* p, float* f);
+template <>
+__device__ __forceinline__ void smem_vals<__nv_bfloat16>(const __nv_bfloat16* p, float* f) {
+  bf16x8_to_f32(*reinterpret_cast<const uint4*>(p), f);
+}
+template <>
+__device__ __forceinline__ void smem_vals<float>(const float* p, float* f) {
+  const float4 u = *reinterpret_cast<const float4*>(p);
+  f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
 }
 
 template <typename TV, int CH>
@@ -111,47 +134,82 @@ __global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
     const float* __restrict__ dy, float* __restrict__ dV, float* __restrict__ dw, int hk, int d_v,
     int64_t K, int* status) {
   constexpr int E = VecT<TV>::E;
+  extern __shared__ __align__(16) unsigned char b3_smem[];
   __shared__ int s_t[kB3Batch];
   __shared__ int s_e[kB3Batch];
   __shared__ float s_w[kB3Batch];
   __shared__ float s_part[kB3Threads / 32][kB3Batch];
+  __shared__ __align__(8) uint64_t bar[2];
+  __shared__ volatile int abort_flag;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int U = *U_ptr;
   const int nvec = d_v / E;
+  const uint32_t vbytes = (uint32_t)d_v * sizeof(TV), dbytes = dV ? (uint32_t)d_v * 4u : 0u;
+  const uint32_t slot_bytes = ((vbytes + 15u) & ~15u) + dbytes;
   const uint64_t pol_keep = policy_evict_last();
   const uint64_t pol_stream = policy_evict_first();
-  const int row_bytes_v = d_v * (int)sizeof(TV), row_bytes_dv = d_v * 4;
-  for (int u = blockIdx.x; u < U; u += gridDim.x) {
+  if (tid == 0) {
+    tc::mbar_init(&bar[0], 1);
+    tc::mbar_init(&bar[1], 1);
+    abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
+
+  // thread 0: start the copies of row u's V and dV lines into buffer b
+  auto issue = [&](int u, int b) {
+    const int32_t r = seg_row[u];
+    unsigned char* buf = b3_smem + (size_t)b * slot_bytes;
+    if (r < 0 || r >= K) {
+      set_status(status, kDevIndex);
+      tc::mbar_arrive(&bar[b]);  // complete the phase without data
+      return;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc::mbar_arrive_expect_tx(&bar[b], vbytes + dbytes);
+    bulk_g2s(buf, V + (int64_t)r * d_v, vbytes, &bar[b], pol_stream);
+    if (dbytes)
+      bulk_g2s(buf + ((vbytes + 15u) & ~15u), dV + (int64_t)r * d_v, dbytes, &bar[b], pol_stream);
+  };
+
+  uint32_t phase_bits = 0u;    // bit b: parity of buffer b's next phase
+  uint32_t pending_bits = 0u;  // bit b: a copy into buffer b not yet waited for (thread 0)
+  if (tid == 0 && (int)blockIdx.x < U) {
+    issue(blockIdx.x, 0);
+    pending_bits |= 1u;
+  }
+  int it = 0;
+  for (int u = blockIdx.x; u < U; u += gridDim.x, ++it) {
+    const int b = it & 1;
+    if (tid == 0 && u + (int)gridDim.x < U) {
+      issue(u + gridDim.x, b ^ 1);
+      pending_bits |= 2u >> b;  // bit (b ^ 1)
+    }
     const int p0 = seg[u], p1 = seg[u + 1];
     const int32_t r = seg_row[u];
-    if (r < 0 || r >= K) {
-      if (tid == 0) set_status(status, kDevIndex);
-      continue;  // uniform across the CTA
-    }
-    const TV* Vr = V + (int64_t)r * d_v;
+    const bool got = tc::mbar_wait(&bar[b], (phase_bits >> b) & 1u, &abort_flag, status);
+    phase_bits ^= 1u << b;
+    pending_bits &= ~(1u << b);
+    __syncthreads();
+    if (abort_flag || !got) break;  // uniform: abort_flag is read after the barrier
+    if (r < 0 || r >= K) continue;  // status already recorded by the issuing thread
+    const TV* sV = reinterpret_cast<const TV*>(b3_smem + (size_t)b * slot_bytes);
+    const float* sD = reinterpret_cast<const float*>(b3_smem + (size_t)b * slot_bytes +
+                                                     ((vbytes + 15u) & ~15u));
     float* dVr = dV ? dV + (int64_t)r * d_v : nullptr;
-    // the next row of this CTA: metadata now, its lines into L2 once known
-    const int un = u + gridDim.x;
-    int np0 = 0, np1 = 0;
-    int32_t nr = -1;
-    if (un < U) {
-      np0 = seg[un];
-      np1 = seg[un + 1];
-      nr = seg_row[un];
-    }
     for (int cb = 0; cb < nvec; cb += kB3Threads * CH) {
       float v[CH][E], acc[CH][E];
 #pragma unroll
       for (int c = 0; c < CH; ++c) {
         const int vec = cb + tid + kB3Threads * c;
         if (vec < nvec) {
-          load_vals<TV>(Vr + (int64_t)vec * E, pol_stream, v[c]);
+          smem_vals<TV>(sV + (int64_t)vec * E, v[c]);
           if (dVr) {
 #pragma unroll
             for (int e4 = 0; e4 < E / 4; ++e4) {
-              float4 a = ld_f4_hint(dVr + (int64_t)vec * E + 4 * e4, pol_stream);
-              acc[c][4 * e4] = a.x; acc[c][4 * e4 + 1] = a.y;
-              acc[c][4 * e4 + 2] = a.z; acc[c][4 * e4 + 3] = a.w;
+              const float4 a4 = *reinterpret_cast<const float4*>(sD + (int64_t)vec * E + 4 * e4);
+              acc[c][4 * e4] = a4.x; acc[c][4 * e4 + 1] = a4.y;
+              acc[c][4 * e4 + 2] = a4.z; acc[c][4 * e4 + 3] = a4.w;
             }
           } else {
 #pragma unroll
@@ -204,17 +262,6 @@ __global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
           dw[ent] = (cb == 0) ? sdot : dw[ent] + sdot;
         }
       }
-      if (cb == 0 && nr >= 0 && nr < K) {
-        const char* nv = reinterpret_cast<const char*>(V + (int64_t)nr * d_v);
-        for (int off = tid * 128; off < row_bytes_v; off += kB3Threads * 128) prefetch_l2(nv + off);
-        if (dV) {
-          const char* nd = reinterpret_cast<const char*>(dV + (int64_t)nr * d_v);
-          for (int off = tid * 128; off < row_bytes_dv; off += kB3Threads * 128)
-            prefetch_l2(nd + off);
-        }
-        if (tid == 0) prefetch_l2(ents + np0);
-        if (tid == 1 && np1 - np0 > 32) prefetch_l2(ents + np0 + 32);
-      }
       if (dVr) {
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
@@ -230,7 +277,23 @@ __global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
         }
       }
     }
+    __syncthreads();  // buffer b may be refilled by the next iteration's issue
   }
+  // copies still in flight (only after an abort) land before the CTA exits
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b) {
+      if (!((pending_bits >> b) & 1u)) continue;
+      const uint32_t par = (phase_bits >> b) & 1u;
+      const long long t0 = clock64();
+      while (!tc::mbar_try_wait(&bar[b], par) && clock64() - t0 < tc::kWaitBudgetCycles) {
+      }
+    }
+  }
+}
+
+inline size_t value_rows_smem(const Plan& p) {
+  const size_t vb = ((size_t)p.d_v * (p.fp32 ? 4 : 2) + 15) & ~size_t(15);
+  return 2 * (vb + (size_t)p.d_v * 4);
 }
 
 // ------------------------------------------------------------------ B4
@@ -556,10 +619,18 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
     const int E = p.fp32 ? 4 : 8;
     const int nvec = p.d_v / E;
     const int blocks = p.sm_count * 6;
-#define PKM_B3(TV, CHV)                                                                  \
-  value_rows_kernel<TV, CHV><<<blocks, kB3Threads, 0, st>>>(                             \
-      seg, U, seg_row, ents_sorted, static_cast<const TV*>(values), s.w, dy, dV, dw,     \
-      hk, p.d_v, p.K, p.status)
+    const size_t smem = value_rows_smem(p);
+#define PKM_B3(TV, CHV)                                                                      \
+  do {                                                                                       \
+    if (smem > 48 * 1024 &&                                                                  \
+        (e = cudaFuncSetAttribute(value_rows_kernel<TV, CHV>,                                \
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != \
+            cudaSuccess)                                                                     \
+      return e;                                                                              \
+    value_rows_kernel<TV, CHV><<<blocks, kB3Threads, smem, st>>>(                            \
+        seg, U, seg_row, ents_sorted, static_cast<const TV*>(values), s.w, dy, dV, dw, hk,   \
+        p.d_v, p.K, p.status);                                                               \
+  } while (0)
     if (p.fp32) {
       if (nvec <= kB3Threads) PKM_B3(float, 1);
       else PKM_B3(float, 2);

@@ -53,7 +53,9 @@ using namespace tc;
 struct QueryProb {
   static constexpr int kAMN = 0, kBMN = 0;
   static constexpr int kStages = 4;
-  static constexpr int kEpiSmem = 0;
+  // per-tile BatchNorm constants (mean, 1/sqrt(var + eps), gamma, beta) for the 256
+  // columns, one private copy per epilogue warp so no barrier spans warps
+  static constexpr int kEpiSmem = 4 * 4 * kBN * 4;
   struct Params {
     int* status;
     const float* bn;
@@ -77,14 +79,39 @@ struct QueryProb {
     tma_load_2d(sb, B, kb * kBK, nt * kBN, bar);
   }
 
-  __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState&) {}
+  __device__ static float* consts(unsigned char* sm, int row) {
+    return reinterpret_cast<float*>(sm) + (row >> 5) * 4 * kBN;
+  }
+
+  __device__ static void epi_begin(const Params& P, int u, int row, unsigned char* sm,
+                                   EpiState&) {
+    const int nt = u % P.n_tiles;
+    float* c = consts(sm, row);
+    __syncwarp();  // this warp's reads of the previous tile's constants are done
+    for (int j = row & 31; j < kBN; j += 32) {
+      const int n = nt * kBN + j;
+      float mean = 0.f, inv = 0.f, gamma = 0.f, beta = 0.f;
+      if (n < P.hq) {
+        mean = P.bn[n];
+        inv = 1.0f / sqrtf(P.bn[P.hq + n] + P.eps);
+        gamma = P.bn[2 * P.hq + n];
+        beta = P.bn[3 * P.hq + n];
+      }
+      c[j] = mean;
+      c[kBN + j] = inv;
+      c[2 * kBN + j] = gamma;
+      c[3 * kBN + j] = beta;
+    }
+    __syncwarp();
+  }
   __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&) {}
 
   __device__ static void epi_chunk(const Params& P, int u, int, int row, uint32_t taddr,
-                                   unsigned char*, EpiState&) {
+                                   unsigned char* sm, EpiState&) {
     const int mt = u / P.n_tiles, nt = u % P.n_tiles;
     const int64_t t = (int64_t)mt * kBM + row;
     const int hq = P.hq;
+    const float* cst = consts(sm, row);
     for (int piece = 0; piece < kBN / 32; ++piece) {
       const int n0 = nt * kBN + piece * 32;
       if (n0 >= hq) break;  // warp-uniform
@@ -99,12 +126,10 @@ struct QueryProb {
         float qq[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int n = n0 + j + e;
-          const float mean = __ldg(P.bn + n), var = __ldg(P.bn + hq + n);
-          const float gamma = __ldg(P.bn + 2 * hq + n), beta = __ldg(P.bn + 3 * hq + n);
-          const float h = (__uint_as_float(r[j + e]) - mean) / sqrtf(var + P.eps);
+          const int jj = piece * 32 + j + e;
+          const float h = (__uint_as_float(r[j + e]) - cst[jj]) * cst[kBN + jj];
           qh[j + e] = h;
-          qq[e] = fmaf(gamma, h, beta);
+          qq[e] = fmaf(cst[2 * kBN + jj], h, cst[3 * kBN + jj]);
         }
         const __nv_bfloat162 hb = __floats2bfloat162_rn(qq[0], qq[1]);
         const float2 hf = __bfloat1622float2(hb);
@@ -131,12 +156,21 @@ struct QueryProb {
 };
 
 // ================================================================== F2 sub-key scores
+// Per-token running top-KM over one half's sub-keys, one epilogue thread per token.
+// The kept keys live in a tournament tree in shared memory: KM leaves hold (score,
+// key) and every node holds the worst key of its subtree, so the root is the current
+// threshold and names the leaf to replace.  A key is packed as (sub-key index << 5 |
+// leaf), so comparing packed keys compares sub-key indices (lower index ranks higher
+// at equal score).  Replacing a leaf rewrites its path to the root; the siblings on
+// that path are known before any comparison, so their loads issue together.
 template <int KM>
 struct ScoresProb {
   static constexpr int kAMN = 0, kBMN = 0;
   static constexpr int kStages = 3;
-  // heap: KM (score, index) slots per row; staging: one 32-column piece per row
-  static constexpr int kEpiSmem = KM * kBM * 8 + 32 * kBM * 4;
+  static constexpr int kLog = KM == 32 ? 5 : (KM == 16 ? 4 : 3);
+  static constexpr int kNodes = 2 * KM;  // nodes 1 .. 2*KM-1; leaves KM .. 2*KM-1
+  // tree: kNodes (score, packed) per row; staging: one 32-column piece per row
+  static constexpr int kEpiSmem = kNodes * kBM * 8 + 32 * kBM * 4;
   struct Params {
     int* status;
     float* sub_s;
@@ -146,6 +180,7 @@ struct ScoresProb {
   };
   struct EpiState {
     float thr;
+    int root_leaf;
   };
 
   __device__ static int num_units(const Params& P) { return P.m_tiles * P.h * 2; }
@@ -166,67 +201,87 @@ struct ScoresProb {
     tma_load_2d(sb, B, kk * kBK, hh * (P.C1 + P.C2) + s * P.C1 + c * kBN, bar);
   }
 
-  __device__ static float* hs_(unsigned char* sm) { return reinterpret_cast<float*>(sm); }
-  __device__ static int* hi_(unsigned char* sm) {
-    return reinterpret_cast<int*>(sm + KM * kBM * 4);
+  __device__ static float* ts_(unsigned char* sm) { return reinterpret_cast<float*>(sm); }
+  __device__ static int* tp_(unsigned char* sm) {
+    return reinterpret_cast<int*>(sm + kNodes * kBM * 4);
   }
   __device__ static float* stage_(unsigned char* sm) {
-    return reinterpret_cast<float*>(sm + KM * kBM * 8);
+    return reinterpret_cast<float*>(sm + kNodes * kBM * 8);
   }
 
-  // worse(a, b): a ranks below b in (score desc, index asc)
-  __device__ static bool worse(float sa, int ia, float sb, int ib) {
-    return sa < sb || (sa == sb && ia > ib);
+  // a ranks below b in (score desc, sub-key index asc)
+  __device__ static bool worse(float sa, int pa, float sb, int pb) {
+    return sa < sb || (sa == sb && pa > pb);
   }
 
-  // Replace the root of the `n`-slot heap with (v, col) and restore the heap.
-  __device__ static void sift_root(float* hs, int* hi, int row, int n, float v, int col) {
-    int pos = 0;
-    while (true) {
-      const int l = 2 * pos + 1;
-      if (l >= n) break;
-      int c = l;
-      float sc = hs[l * kBM + row];
-      int ic = hi[l * kBM + row];
-      const int r = l + 1;
-      if (r < n) {
-        const float sr = hs[r * kBM + row];
-        const int ir = hi[r * kBM + row];
-        if (worse(sr, ir, sc, ic)) {
-          c = r;
-          sc = sr;
-          ic = ir;
-        }
-      }
-      if (worse(sc, ic, v, col)) {
-        hs[pos * kBM + row] = sc;
-        hi[pos * kBM + row] = ic;
-        pos = c;
-      } else {
-        break;
-      }
-    }
-    hs[pos * kBM + row] = v;
-    hi[pos * kBM + row] = col;
+  __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState& es) {
+    es.thr = -INFINITY;
+    es.root_leaf = -1;  // tree not built yet
   }
 
-  __device__ static void epi_begin(const Params&, int, int row, unsigned char* sm, EpiState& es) {
-    float* hs = hs_(sm);
-    int* hi = hi_(sm);
+  // Build the tree from the first KM columns held in registers (columns col0 + j).
+  __device__ static void build(float* ts, int* tp, int row, const uint32_t (&r)[32], int col0,
+                               int C, EpiState& es) {
+    float s[kNodes];
+    int p[kNodes];
 #pragma unroll
     for (int j = 0; j < KM; ++j) {
-      hs[j * kBM + row] = -INFINITY;
-      hi[j * kBM + row] = 0x7fffffff;
+      const bool ok = col0 + j < C;
+      s[KM + j] = ok ? __uint_as_float(r[j]) : -INFINITY;
+      p[KM + j] = ((ok ? col0 + j : 0x3FFFFFF) << 5) | j;
     }
-    es.thr = -INFINITY;
+#pragma unroll
+    for (int n = KM - 1; n >= 1; --n) {
+      const bool rw = worse(s[2 * n + 1], p[2 * n + 1], s[2 * n], p[2 * n]);
+      s[n] = rw ? s[2 * n + 1] : s[2 * n];
+      p[n] = rw ? p[2 * n + 1] : p[2 * n];
+    }
+#pragma unroll
+    for (int n = 1; n < kNodes; ++n) {
+      ts[n * kBM + row] = s[n];
+      tp[n * kBM + row] = p[n];
+    }
+    es.thr = s[1];
+    es.root_leaf = p[1] & 31;
+  }
+
+  // Replace the worst kept key (the root's leaf) with (v, col).
+  __device__ static void replace_root(float* ts, int* tp, int row, float v, int col,
+                                      EpiState& es) {
+    const int leaf = es.root_leaf;
+    int node = KM + leaf;
+    float sib_s[kLog];
+    int sib_p[kLog];
+#pragma unroll
+    for (int l = 0; l < kLog; ++l) {  // siblings along the fixed path, loaded together
+      const int sib = (node >> l) ^ 1;
+      sib_s[l] = ts[sib * kBM + row];
+      sib_p[l] = tp[sib * kBM + row];
+    }
+    float cs = v;
+    int cp = (col << 5) | leaf;
+    ts[node * kBM + row] = cs;
+    tp[node * kBM + row] = cp;
+#pragma unroll
+    for (int l = 0; l < kLog; ++l) {
+      if (worse(sib_s[l], sib_p[l], cs, cp)) {
+        cs = sib_s[l];
+        cp = sib_p[l];
+      }
+      node >>= 1;
+      ts[node * kBM + row] = cs;
+      tp[node * kBM + row] = cp;
+    }
+    es.thr = cs;
+    es.root_leaf = cp & 31;
   }
 
   __device__ static void epi_chunk(const Params& P, int u, int c, int row, uint32_t taddr,
                                    unsigned char* sm, EpiState& es) {
     const int hs_idx = u / P.m_tiles;
     const int C = (hs_idx & 1) ? P.C2 : P.C1;
-    float* hs = hs_(sm);
-    int* hi = hi_(sm);
+    float* ts = ts_(sm);
+    int* tp = tp_(sm);
     float* stg = stage_(sm);
     for (int piece = 0; piece < kBN / 32; ++piece) {
       const int col0 = c * kBN + piece * 32;
@@ -234,10 +289,16 @@ struct ScoresProb {
       uint32_t r[32];
       tmem_ld32(taddr + (uint32_t)(piece * 32), r);
       tmem_wait_ld();
+      int first = 0;
+      if (es.root_leaf < 0) {  // first piece of the unit (uniform across the warp)
+        build(ts, tp, row, r, col0, C, es);
+        first = KM;
+      }
       // candidates of this piece against the threshold at its start
       uint32_t mask = 0;
 #pragma unroll
       for (int j = 0; j < 32; ++j) mask |= (__uint_as_float(r[j]) > es.thr ? 1u : 0u) << j;
+      if (first) mask &= first >= 32 ? 0u : ~((1u << first) - 1u);
       if (C - col0 < 32) mask &= (1u << (C - col0)) - 1u;
       if (mask) {
 #pragma unroll
@@ -246,10 +307,7 @@ struct ScoresProb {
           const int j = __ffs(mask) - 1;
           mask &= mask - 1u;
           const float v = stg[j * kBM + row];
-          if (v > es.thr) {
-            sift_root(hs, hi, row, KM, v, col0 + j);
-            es.thr = hs[row];
-          }
+          if (v > es.thr) replace_root(ts, tp, row, v, col0 + j, es);
         }
       }
     }
@@ -259,19 +317,47 @@ struct ScoresProb {
     const int hs_idx = u / P.m_tiles, mt = u % P.m_tiles;
     const int hh = hs_idx >> 1, s = hs_idx & 1;
     const int64_t t = (int64_t)mt * kBM + row;
-    float* hs = hs_(sm);
-    int* hi = hi_(sm);
-    const bool live = t < P.N;
-    const int64_t o = ((t * P.h + hh) * 2 + s) * P.k;
-    // pop the worst remaining key into the last open position (best-first output)
-    for (int n = KM; n > 0; --n) {
-      const float rs = hs[row];
-      const int ri = hi[row];
-      if (live && n - 1 < P.k) {
-        P.sub_s[o + n - 1] = rs;
-        P.sub_i[o + n - 1] = ri;
+    if (t >= P.N) return;
+    const float* ts = ts_(sm);
+    const int* tp = tp_(sm);
+    float v[KM];
+    int q[KM];
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      v[j] = ts[(KM + j) * kBM + row];
+      q[j] = tp[(KM + j) * kBM + row] >> 5;
+    }
+    // bitonic sort, best first: (score desc, index asc)
+#pragma unroll
+    for (int size = 2; size <= KM; size <<= 1) {
+#pragma unroll
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+        for (int i = 0; i < KM; ++i) {
+          const int j = i ^ stride;
+          if (j > i) {
+            const bool desc = (i & size) == 0;
+            // in a "desc" run the better key goes first
+            const bool jbetter = worse(v[i], q[i], v[j], q[j]);
+            if (jbetter == desc) {
+              const float tv = v[i];
+              v[i] = v[j];
+              v[j] = tv;
+              const int tq = q[i];
+              q[i] = q[j];
+              q[j] = tq;
+            }
+          }
+        }
       }
-      if (n > 1) sift_root(hs, hi, row, n - 1, hs[(n - 1) * kBM + row], hi[(n - 1) * kBM + row]);
+    }
+    const int64_t o = ((t * P.h + hh) * 2 + s) * P.k;
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      if (j < P.k) {
+        P.sub_s[o + j] = v[j];
+        P.sub_i[o + j] = q[j];
+      }
     }
   }
 };
