@@ -49,15 +49,17 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, jobs: int | None = None, verbose: bool = False,
-          extra_flags: list[str] | None = None) -> str:
-    """Compile and link the library; returns its path."""
-    if not force and up_to_date():
+          extra_flags: list[str] | None = None, out: str | None = None) -> str:
+    """Compile and link the library (to ``out``, default the in-tree path); returns it."""
+    lib = out or LIB
+    if out is None and not force and up_to_date():
         return LIB
-    os.makedirs(OBJDIR, exist_ok=True)
+    objdir = OBJDIR if out is None else os.path.join(OBJDIR, os.path.basename(out))
+    os.makedirs(objdir, exist_ok=True)
     flags = NVCC_FLAGS + list(extra_flags or [])
 
     def compile_one(src: str) -> str:
-        obj = os.path.join(OBJDIR, os.path.basename(src) + ".o")
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [nvcc(), *ARCH, *flags, "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
@@ -70,13 +72,13 @@ def build(force: bool = False, jobs: int | None = None, verbose: bool = False,
 
     with ThreadPoolExecutor(max_workers=jobs or min(8, os.cpu_count() or 1)) as ex:
         objs = list(ex.map(compile_one, sources()))
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lcudart"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 def main() -> None:

@@ -127,17 +127,23 @@ __device__ __forceinline__ void smem_vals<float>(const float* p, float* f) {
   f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
 }
 
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
+// ws_sorted[p] = w[ents[p]]: the selection weights in row order, so staging a batch
+// needs two independent loads.
 template <typename TV, int CH>
 __global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
     const int* __restrict__ seg, const int* __restrict__ U_ptr, const int32_t* __restrict__ seg_row,
-    const int32_t* __restrict__ ents, const TV* __restrict__ V, const float* __restrict__ w,
+    const int32_t* __restrict__ ents, const TV* __restrict__ V, const float* __restrict__ ws_sorted,
     const float* __restrict__ dy, float* __restrict__ dV, float* __restrict__ dw, int hk, int d_v,
     int64_t K, int* status) {
   constexpr int E = VecT<TV>::E;
   extern __shared__ __align__(16) unsigned char b3_smem[];
-  __shared__ int s_t[kB3Batch];
-  __shared__ int s_e[kB3Batch];
-  __shared__ float s_w[kB3Batch];
+  __shared__ int s_t[2][kB3Batch];
+  __shared__ int s_e[2][kB3Batch];
+  __shared__ float s_w[2][kB3Batch];
   __shared__ float s_part[kB3Threads / 32][kB3Batch];
   __shared__ __align__(8) uint64_t bar[2];
   __shared__ volatile int abort_flag;
@@ -174,25 +180,63 @@ __global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
 
   uint32_t phase_bits = 0u;    // bit b: parity of buffer b's next phase
   uint32_t pending_bits = 0u;  // bit b: a copy into buffer b not yet waited for (thread 0)
-  if (tid == 0 && (int)blockIdx.x < U) {
-    issue(blockIdx.x, 0);
-    pending_bits |= 1u;
+  if ((int)blockIdx.x < U) {
+    if (tid == 0) {
+      issue(blockIdx.x, 0);
+      pending_bits |= 1u;
+    }
+    const int q0 = seg[blockIdx.x], q1 = seg[blockIdx.x + 1];
+    if (tid < min(kB3Batch, q1 - q0)) {
+      const int32_t ent = ents[q0 + tid];
+      s_e[0][tid] = ent;
+      s_t[0][tid] = ent / hk;
+      s_w[0][tid] = ws_sorted[q0 + tid];
+    }
   }
   int it = 0;
   for (int u = blockIdx.x; u < U; u += gridDim.x, ++it) {
     const int b = it & 1;
-    if (tid == 0 && u + (int)gridDim.x < U) {
-      issue(u + gridDim.x, b ^ 1);
+    const int un = u + (int)gridDim.x;
+    if (tid == 0 && un < U) {
+      issue(un, b ^ 1);
       pending_bits |= 2u >> b;  // bit (b ^ 1)
     }
     const int p0 = seg[u], p1 = seg[u + 1];
     const int32_t r = seg_row[u];
+    // the next row's first batch: loads in flight while this row is processed
+    int nbn = 0;
+    int32_t nent = 0;
+    float nw = 0.f;
+    if (un < U) {
+      const int np0 = seg[un];
+      nbn = min(kB3Batch, seg[un + 1] - np0);
+      if (tid < nbn) {
+        nent = ents[np0 + tid];
+        nw = ws_sorted[np0 + tid];
+      }
+    }
     const bool got = tc::mbar_wait(&bar[b], (phase_bits >> b) & 1u, &abort_flag, status);
     phase_bits ^= 1u << b;
     pending_bits &= ~(1u << b);
     __syncthreads();
     if (abort_flag || !got) break;  // uniform: abort_flag is read after the barrier
-    if (r < 0 || r >= K) continue;  // status already recorded by the issuing thread
+    if (tid < nbn) {  // publish the next row's batch and pull its dy lines into L1
+      const int64_t tn = nent / hk;
+      s_e[b ^ 1][tid] = nent;
+      s_t[b ^ 1][tid] = (int)tn;
+      s_w[b ^ 1][tid] = nw;
+#ifndef PKM_B3_DY_PREFETCH
+#define PKM_B3_DY_PREFETCH 0
+#endif
+      if (PKM_B3_DY_PREFETCH) {
+        const char* row = reinterpret_cast<const char*>(dy + tn * d_v);
+        for (int off = 0; off < d_v * 4; off += 128) prefetch_l1(row + off);
+      }
+    }
+    if (r < 0 || r >= K) {  // status already recorded by the issuing thread
+      __syncthreads();
+      continue;
+    }
     const TV* sV = reinterpret_cast<const TV*>(b3_smem + (size_t)b * slot_bytes);
     const float* sD = reinterpret_cast<const float*>(b3_smem + (size_t)b * slot_bytes +
                                                      ((vbytes + 15u) & ~15u));
@@ -222,17 +266,19 @@ __global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
       }
       for (int pb = p0; pb < p1; pb += kB3Batch) {
         const int nb = min(kB3Batch, p1 - pb);
-        __syncthreads();  // previous batch's staging fully consumed
-        if (tid < nb) {
-          const int32_t ent = ents[pb + tid];
-          s_e[tid] = ent;
-          s_t[tid] = ent / hk;
-          s_w[tid] = w[ent];
+        if (pb != p0 || cb != 0) {  // the first batch was staged ahead of time
+          __syncthreads();          // previous batch's staging fully consumed
+          if (tid < nb) {
+            const int32_t ent = ents[pb + tid];
+            s_e[b][tid] = ent;
+            s_t[b][tid] = ent / hk;
+            s_w[b][tid] = ws_sorted[pb + tid];
+          }
+          __syncthreads();
         }
-        __syncthreads();
         for (int i = 0; i < nb; ++i) {
-          const float* dyt = dy + (int64_t)s_t[i] * d_v;
-          const float wt = s_w[i];
+          const float* dyt = dy + (int64_t)s_t[b][i] * d_v;
+          const float wt = s_w[b][i];
           float dot = 0.f;
 #pragma unroll
           for (int c = 0; c < CH; ++c) {
@@ -258,7 +304,7 @@ __global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
           float sdot = 0.f;
 #pragma unroll
           for (int ww = 0; ww < kB3Threads / 32; ++ww) sdot += s_part[ww][tid];
-          const int32_t ent = s_e[tid];
+          const int32_t ent = s_e[b][tid];
           dw[ent] = (cb == 0) ? sdot : dw[ent] + sdot;
         }
       }
@@ -522,7 +568,8 @@ inline int bits_for(int64_t maxkey) {
 
 // ------------------------------------------------------------------ workspace
 struct Layout {
-  size_t keysA, valsA, keysB, valsB, hist, bsum, seg, segrow, U, dw, gsub, dq, part, total;
+  size_t keysA, valsA, keysB, valsB, hist, bsum, seg, segrow, wsorted, U, dw, gsub, dq, part,
+      total;
 };
 
 inline size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -547,6 +594,7 @@ Layout layout(const Plan& p) {
   L.bsum = take(4 * bl);
   L.seg = take(4 * (En + 1));
   L.segrow = take(4 * (En + 1));
+  L.wsorted = take(4 * E1);
   L.U = take(4);
   L.dw = take(4 * E1);
   L.gsub = take(4 * E2);
@@ -570,6 +618,7 @@ struct BwdCtx {
   sort::RadixBuffers rb;
   int* seg;
   int32_t* seg_row;
+  float* w_sorted;
   int* U;
   float* dw;
   float* gsub;
@@ -585,6 +634,7 @@ static BwdCtx bwd_ctx(const Plan& p, void* ws, float* dw_out) {
                             at<int>(ws, L.hist), at<int>(ws, L.bsum)};
   c.seg = at<int>(ws, L.seg);
   c.seg_row = at<int32_t>(ws, L.segrow);
+  c.w_sorted = at<float>(ws, L.wsorted);
   c.U = at<int>(ws, L.U);
   c.dw = dw_out ? dw_out : at<float>(ws, L.dw);
   c.gsub = at<float>(ws, L.gsub);
@@ -611,7 +661,8 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
   const int32_t *rows_sorted, *ents_sorted;
   e = sort::radix_sort(s.idx, E1, bits_for(p.K - 1), rb, &rows_sorted, &ents_sorted, st);
   if (e != cudaSuccess) return e;
-  e = sort::segments(rows_sorted, E1, seg, U, rb.bsum, st, seg_row);
+  float* w_sorted = c.w_sorted;
+  e = sort::segments(rows_sorted, E1, seg, U, rb.bsum, st, seg_row, ents_sorted, s.w, w_sorted);
   if (e != cudaSuccess) return e;
 
   // B3: value rows
@@ -628,7 +679,8 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
             cudaSuccess)                                                                     \
       return e;                                                                              \
     value_rows_kernel<TV, CHV><<<blocks, kB3Threads, smem, st>>>(                            \
-        seg, U, seg_row, ents_sorted, static_cast<const TV*>(values), s.w, dy, dV, dw, hk,   \
+        seg, U, seg_row, ents_sorted, static_cast<const TV*>(values), w_sorted, dy, dV, dw,  \
+        hk,                                                                                  \
         p.d_v, p.K, p.status);                                                               \
   } while (0)
     if (p.fp32) {

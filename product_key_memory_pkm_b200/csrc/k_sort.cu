@@ -102,7 +102,11 @@ struct SegOut {
   int* U;
   const int32_t* keys;
   int32_t* seg_key;
+  const int32_t* vals;
+  const float* gsrc;
+  float* gdst;
   __device__ void operator()(int64_t i, int excl, int v, int64_t n) const {
+    if (gdst) gdst[i] = gsrc[vals[i]];
     if (v) {
       seg[excl] = (int)i;
       if (seg_key) seg_key[excl] = keys[i];
@@ -153,8 +157,11 @@ cudaError_t radix_sort(const int32_t* keys_src, int64_t n, int bits_total, const
 }
 
 cudaError_t segments(const int32_t* keys, int64_t n, int* seg, int* U_out, int* bsum,
-                     cudaStream_t st, int32_t* seg_key) {
-  return exclusive_scan(FlagIn{keys}, SegOut{seg, U_out, keys, seg_key}, n, bsum, st);
+                     cudaStream_t st, int32_t* seg_key, const int32_t* vals,
+                     const float* gather_src, float* gather_dst) {
+  return exclusive_scan(FlagIn{keys},
+                        SegOut{seg, U_out, keys, seg_key, vals, gather_src, gather_dst}, n, bsum,
+                        st);
 }
 
 }  // namespace sort

@@ -117,8 +117,10 @@ cudaError_t radix_sort(const int32_t* keys_src, int64_t n, int bits_total, const
 // Segment table of a sorted key array: seg[u] = first position of the u-th
 // distinct key, seg[U] = n, *U_out = U, and (when seg_key is not null)
 // seg_key[u] = that key.
+// When gather_src is not null, gather_dst[i] = gather_src[vals[i]] for every position.
 cudaError_t segments(const int32_t* keys, int64_t n, int* seg, int* U_out, int* bsum,
-                     cudaStream_t st, int32_t* seg_key = nullptr);
+                     cudaStream_t st, int32_t* seg_key = nullptr, const int32_t* vals = nullptr,
+                     const float* gather_src = nullptr, float* gather_dst = nullptr);
 
 }  // namespace sort
 }  // namespace pkm

@@ -16,7 +16,8 @@ import os
 from dataclasses import dataclass
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libpkm_b200.so")
+# PKM_B200_LIB overrides the library path (e.g. to compare two builds)
+LIB_PATH = os.environ.get("PKM_B200_LIB") or os.path.join(HERE, "libpkm_b200.so")
 
 PKM_OK = 0
 PKM_ERR_INVALID_ARG = 1
