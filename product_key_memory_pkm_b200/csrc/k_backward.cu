@@ -614,6 +614,8 @@ T* at(void* ws, size_t off) {
 
 size_t backward_workspace_bytes(const Plan& p) { return layout(p).total; }
 
+size_t value_stage_scratch_bytes(const Plan& p) { return layout(p).U + 4; }
+
 struct BwdCtx {
   sort::RadixBuffers rb;
   int* seg;

@@ -340,3 +340,59 @@ const char* pkm_build_info(void) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// Value-gradient stage with a fixed scratch array (no allocation anywhere).
+//
+// The scratch is a file-scope device array: every device that loads this library
+// reserves it for the life of the process.  In host code the array's name is only a
+// host-side stand-in, so its device address is fetched with cudaGetSymbolAddress,
+// once per device, with that device current, and passed to the kernels.
+namespace pkm {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+void* g_noalloc_ptr[kMaxDevices];
+cudaError_t g_noalloc_err[kMaxDevices];
+std::once_flag g_noalloc_once[kMaxDevices];
+
+// Device address of the scratch on the current device (nullptr after a failure).
+void* noalloc_scratch(int dev) {
+  std::call_once(g_noalloc_once[dev], [dev]() {
+    void* ptr = nullptr;
+    g_noalloc_err[dev] = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    g_noalloc_ptr[dev] = g_noalloc_err[dev] == cudaSuccess ? ptr : nullptr;
+  });
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+}  // namespace pkm
+
+extern "C" pkm_status pkm_value_grad_noalloc(const pkm_dims* d, const void* values,
+                                             const pkm_saved* saved, const float* dy,
+                                             float* dvalues, float* dw, void* stream) {
+  PKM_TRY(validate_dims(d));
+  if (d->N == 0) return PKM_OK;
+  PKM_NEED(values); PKM_NEED(dy); PKM_NEED(dw); PKM_OPT(dvalues);
+  if (!saved) return PKM_ERR_INVALID_ARG;
+  PKM_NEED(saved->idx); PKM_NEED(saved->w);
+  {
+    // size check on the host, before any device work
+    Plan q{};
+    q.N = d->N; q.d_in = d->d_in; q.h = d->h; q.dk = d->dk; q.half = d->dk / 2;
+    q.C1 = d->C1; q.C2 = d->C2; q.k = d->k; q.d_v = d->d_v; q.hq = d->h * d->dk;
+    q.K = (int64_t)d->C1 * d->C2; q.fp32 = d->flags & PKM_F_FP32;
+    if (value_stage_scratch_bytes(q) > kNoAllocScratchBytes) return PKM_ERR_WORKSPACE;
+  }
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PKM_ERR_CUDA;
+  void* scratch = noalloc_scratch(dev);
+  if (!scratch) return PKM_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_value_grad(p, values, *saved, dy, dvalues, dw, scratch, st));
+}

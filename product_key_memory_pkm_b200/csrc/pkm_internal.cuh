@@ -82,6 +82,9 @@ cudaError_t launch_gather(const Plan& p, const void* values, const int32_t* idx,
 // ---------------------------------------------------------------- backward launches
 struct BwdWs;  // workspace layout, defined in k_backward.cu
 size_t backward_workspace_bytes(const Plan& p);
+// Leading bytes of the backward workspace that the value stage uses when the caller
+// supplies dw (the value stage touches nothing beyond them).
+size_t value_stage_scratch_bytes(const Plan& p);
 cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved& s,
                               const float* dy, float* dV, float* dw_out, void* ws,
                               cudaStream_t st);

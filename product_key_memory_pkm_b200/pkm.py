@@ -36,7 +36,7 @@ SAVED_FIELDS = ("q", "qhat", "sub_s", "sub_i", "idx", "w")
 EXPORTED = ("pkm_saved_bytes", "pkm_workspace_bytes", "pkm_forward", "pkm_backward", "pkm_query",
             "pkm_subkey_scores", "pkm_candidate_topk", "pkm_gather_bag", "pkm_check_status",
             "pkm_status_string", "pkm_build_info", "pkm_value_grad", "pkm_query_grad",
-            "pkm_launch_count", "pkm_selftest_wait_timeout")
+            "pkm_launch_count", "pkm_selftest_wait_timeout", "pkm_value_grad_noalloc")
 
 
 class PKMError(RuntimeError):
@@ -87,6 +87,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "pkm_query_grad": (I, [D, P, P, P, P, SV, P, P, P, P, P, P, S, P]),
         "pkm_launch_count": (ctypes.c_ulonglong, []),
         "pkm_selftest_wait_timeout": (I, [ctypes.c_uint32, P]),
+        "pkm_value_grad_noalloc": (I, [D, P, SV, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -199,6 +200,16 @@ def pkm_value_grad(dims: Dims, values, saved: dict, dy, dw, dvalues=None, worksp
                                  _ptr(dvalues), _ptr(dw), _ptr(workspace),
                                  _ws(workspace, workspace_bytes), _stream(stream)),
            "pkm_value_grad")
+
+
+def pkm_value_grad_noalloc(dims: Dims, values, saved: dict, dy, dw, dvalues=None,
+                           stream=None) -> None:
+    """pkm_value_grad without a workspace argument: the scratch is a fixed device
+    array inside the library (for callers that cannot allocate device memory)."""
+    s = _saved_c(saved)
+    _check(load().pkm_value_grad_noalloc(ctypes.byref(dims.c()), _ptr(values), ctypes.byref(s),
+                                         _ptr(dy), _ptr(dvalues), _ptr(dw), _stream(stream)),
+           "pkm_value_grad_noalloc")
 
 
 def pkm_query_grad(dims: Dims, x, Wq, bn, subkeys, saved: dict, dw, dx=None, dWq=None, dbn=None,
