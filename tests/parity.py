@@ -104,6 +104,8 @@ def check_indices(idx_gpu: np.ndarray, of: dict, cfg, ranked: np.ndarray):
 
 
 def row_rel_err(got: np.ndarray, want: np.ndarray) -> float:
+    if np.asarray(want).size == 0:
+        return 0.0
     got = np.asarray(got, dtype=np.float64).reshape(want.shape[0], -1)
     want = np.asarray(want, dtype=np.float64).reshape(want.shape[0], -1)
     err = np.abs(got - want).max(axis=1)

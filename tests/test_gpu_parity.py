@@ -215,6 +215,7 @@ def _sampled_full_size(cfg, n_sample, seed=0, backward=True):
     dev = H.to_dev(inp, cfg)
     dims, saved, y = H.gpu_forward(cfg, dev)
     rng = np.random.default_rng(123)
+    n_sample = min(n_sample, cfg.N)
     sample = np.sort(rng.choice(cfg.N, size=n_sample, replace=False))
     sample[0], sample[-1] = 0, cfg.N - 1
     sub_inp = dict(inp, x=inp["x"][sample], dy=inp["dy"][sample])
@@ -262,3 +263,30 @@ def test_bounded_wait_expires_with_status_and_context_survives():
     assert P.pkm_check_status() == P.PKM_ERR_DEVICE_TIMEOUT
     assert P.pkm_check_status() == P.PKM_OK         # read-and-clear
     _full_check(CASES["tiny_bf16"])                 # the context is still usable
+
+
+@pytest.mark.parametrize("n_tok", [1, 8, 64])
+def test_decode_shaped_calls_on_the_full_table(n_tok):
+    """Decode-sized batches (N = 1, 8, 64 tokens) against the full 1024^2 x 1600 bf16
+    table: forward and backward parity for every token."""
+    _sampled_full_size(FULL_K1024.with_(name=f"decode_N{n_tok}", N=n_tok), n_tok)
+
+
+def test_fast_weight_chunk_shape_fp32_values_duplicates():
+    """One 512-token-class chunk of the fast-weight workload (fp32 values, h = 1, k = 8,
+    |K| = 1024^2, d = 1024, queries around 64 centres, so value rows repeat)."""
+    from product_key_memory_pkm_b200.inputs import FASTWEIGHT
+    cfg = FASTWEIGHT.with_(N=192)
+    inp = make_inputs(cfg, seed=0)
+    dev = H.to_dev(inp, cfg)
+    dims, saved, y = H.gpu_forward(cfg, dev)
+    idx = saved["idx"].cpu().numpy()
+    assert np.unique(idx).size < idx.size      # clustered queries share value rows
+    of = O.forward(inp, cfg)
+    ranked = H.oracle_gaps(of, cfg)
+    clean = H.check_indices(idx, of, cfg, ranked)
+    H.assert_rows(y.cpu().numpy()[clean], of["y"][clean], "y")
+    dy = inp["dy"] * clean[:, None]
+    g = H.gpu_backward(cfg, dims, dev, saved, torch.from_numpy(dy).cuda(), want=("dV", "dw"))
+    ob = O.backward(inp, cfg, of, dy)
+    H.assert_rows(g["dV"].cpu().numpy()[ob["dV_rows"]], ob["dV_vals"], "dV")
