@@ -569,7 +569,7 @@ inline int bits_for(int64_t maxkey) {
 // ------------------------------------------------------------------ workspace
 struct Layout {
   size_t keysA, valsA, keysB, valsB, hist, bsum, seg, segrow, wsorted, U, dw, gsub, dq, part,
-      total;
+      G, dqf, dspart, total;
 };
 
 inline size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -601,6 +601,11 @@ Layout layout(const Plan& p) {
   L.dq = take(4 * p.N * p.hq);
   const int64_t nblk = (p.N + kDqTokensPerBlock - 1) / kDqTokensPerBlock;
   L.part = take(4 * nblk * 2 * p.hq);
+  if (!p.fp32) {  // tensor-core sub-key gradients: dense G planes, fp32 dq, split partials
+    L.G = take(2 * (size_t)(2 * p.h) * 2 * subgrad_pad_tokens(p.N) * subgrad_pad_keys(p.C1, p.C2));
+    L.dqf = take(4 * (size_t)p.N * p.hq);
+    L.dspart = take(4 * subgrad_partial_floats(p));
+  }
   L.total = o;
   return L;
 }
@@ -626,6 +631,9 @@ struct BwdCtx {
   float* gsub;
   float* dq_pre;
   float* part;
+  __nv_bfloat16* G;
+  float* dqf;
+  float* dspart;
 };
 
 static BwdCtx bwd_ctx(const Plan& p, void* ws, float* dw_out) {
@@ -642,6 +650,9 @@ static BwdCtx bwd_ctx(const Plan& p, void* ws, float* dw_out) {
   c.gsub = at<float>(ws, L.gsub);
   c.dq_pre = at<float>(ws, L.dq);
   c.part = at<float>(ws, L.part);
+  c.G = at<__nv_bfloat16>(ws, L.G);
+  c.dqf = at<float>(ws, L.dqf);
+  c.dspart = at<float>(ws, L.dspart);
   return c;
 }
 
@@ -725,8 +736,24 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
 
-  // B5a + B6: dq_pre and BatchNorm affine partials
-  if (dx || dWq || dbn) {
+  // B5 + B6 on tensor cores: dense G planes, dq = G C, BatchNorm backward, dC = G^T Q
+  const bool tc_subgrad = tc_backward_supported(p) && p.half % 64 == 0;
+  if (tc_subgrad) {
+    const bool want_dq = dx || dWq || dbn;
+    e = launch_subgrad_tc(p, gsub, s.sub_i, subkeys, s.q, bn, dbn ? s.qhat : nullptr, c.G,
+                          c.dqf, reinterpret_cast<__nv_bfloat16*>(dq_pre), dbn ? part : nullptr,
+                          c.dspart, dsub, want_dq, st);
+    if (e != cudaSuccess) return e;
+    if (dbn) {
+      const int64_t nblk = (p.N + kDqTokensPerBlock - 1) / kDqTokensPerBlock;
+      dbn_reduce_kernel<<<(2 * p.hq + 255) / 256, 256, 0, st>>>(part, (int)nblk, p.hq, dbn);
+      PKM_COUNT(1);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+  }
+
+  // B5a + B6: dq_pre and BatchNorm affine partials (CUDA-core path)
+  if ((dx || dWq || dbn) && !tc_subgrad) {
     const int64_t nblk = (p.N + kDqTokensPerBlock - 1) / kDqTokensPerBlock;
     dim3 grid((unsigned)nblk, (unsigned)(p.h * 2));
     float* partp = dbn ? part : nullptr;
@@ -755,8 +782,8 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
     }
   }
 
-  // B5b: sub-key gradients by sorted segments
-  if (dsub) {
+  // B5b: sub-key gradients by sorted segments (CUDA-core path)
+  if (dsub && !tc_subgrad) {
     subkey_keys_kernel<<<(unsigned)((E2 + 255) / 256), 256, 0, st>>>(s.sub_i, rb.keysB, E2, p.h,
                                                                       p.k, p.C1, p.C2); PKM_COUNT(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -59,7 +59,7 @@ struct DxProb {
   __device__ static int num_chunks(const Params&, int) { return 1; }
   __device__ static int num_kblocks(const Params& P) { return 2 * P.nkh; }
   __device__ static void load(const Params& P, const CUtensorMap* A0, const CUtensorMap* A1,
-                              const CUtensorMap* B, int u, int, int kb, void* sa, void* sb,
+                              const CUtensorMap* B, const CUtensorMap*, int u, int, int kb, void* sa, void* sb,
                               uint64_t* bar) {
     const int mt = u / P.n_tiles, nt = u % P.n_tiles;
     const int plane = kb / P.nkh, kk = kb % P.nkh;
@@ -102,7 +102,7 @@ struct DwqProb {
   __device__ static int num_chunks(const Params&, int) { return 1; }
   __device__ static int num_kblocks(const Params& P) { return 2 * P.nkt; }
   __device__ static void load(const Params& P, const CUtensorMap* A0, const CUtensorMap* A1,
-                              const CUtensorMap* B, int u, int, int kb, void* sa, void* sb,
+                              const CUtensorMap* B, const CUtensorMap*, int u, int, int kb, void* sa, void* sb,
                               uint64_t* bar) {
     const int mt = u / P.n_tiles, nt = u % P.n_tiles;
     const int plane = kb / P.nkt, kk = kb % P.nkt;

@@ -72,7 +72,7 @@ struct QueryProb {
   __device__ static int num_kblocks(const Params& P) { return P.nk; }
 
   __device__ static void load(const Params& P, const CUtensorMap* A0, const CUtensorMap*,
-                              const CUtensorMap* B, int u, int, int kb, void* sa, void* sb,
+                              const CUtensorMap* B, const CUtensorMap*, int u, int, int kb, void* sa, void* sb,
                               uint64_t* bar) {
     const int mt = u / P.n_tiles, nt = u % P.n_tiles;
     tma_load_2d(sa, A0, kb * kBK, mt * kBM, bar);
@@ -192,7 +192,7 @@ struct ScoresProb {
   __device__ static int num_kblocks(const Params& P) { return 2 * P.nkh; }
 
   __device__ static void load(const Params& P, const CUtensorMap* A0, const CUtensorMap* A1,
-                              const CUtensorMap* B, int u, int c, int kb, void* sa, void* sb,
+                              const CUtensorMap* B, const CUtensorMap*, int u, int c, int kb, void* sa, void* sb,
                               uint64_t* bar) {
     const int hs = u / P.m_tiles, mt = u % P.m_tiles;
     const int hh = hs >> 1, s = hs & 1;

@@ -1,0 +1,340 @@
+// Query-half and sub-key gradients (B5) and the BatchNorm backward (B6) on tensor cores.
+//
+// The sub-score gradients of one (head, half) form a sparse matrix G [N x C] with k
+// nonzeros per token row (the selected sub-keys; "Meta AI 可扩展内存层" 9.2: gradient
+// reaches only the selected positions).  It is written densely as bf16 hi/lo planes
+// (zeros elsewhere), and both products become tcgen05 GEMMs:
+//
+//   dq_half = G C_half                 A = G (K-major, K = sub-keys), B = C_half (MN-major)
+//   dC_half = G^T Q_half               A = G^T (MN-major, K = tokens), B = Q_half (MN-major)
+//
+// dq_half uses G_hi + G_lo against the exact bf16 sub-keys; dC_half uses G_hi Q_hi +
+// G_hi Q_lo + G_lo Q_hi (the lo x lo term is below 2^-17 relative).  dC_half is split
+// over the token dimension in kSplits parts written to a partial buffer and added in
+// a fixed order, so results are deterministic.  Padding: G has Np = N rounded up to 64
+// token rows and Cp = max(C1, C2) rounded up to 64 columns, all zero outside the
+// selections, so tiles that run past N or C multiply by exact zeros.
+#include "tc_gemm.cuh"
+#include "tc_launch.cuh"
+
+namespace pkm {
+namespace {
+
+using namespace tc;
+
+constexpr int kMNBox = 64;
+constexpr int kMNBoxBytes = kMNBox * kBK * 2;
+constexpr int kSplits = 2;           // token-dimension split of dC_half
+constexpr int kBnTokens = 64;        // tokens per BatchNorm-backward block (partials layout)
+
+// ------------------------------------------------------------------ dense G planes
+// One warp per (padded token t, head-half hs): zero the row in both planes, then
+// write the k selected entries (distinct within a half, so no accumulation).
+__global__ void __launch_bounds__(256) g_dense_kernel(const float* __restrict__ gsub,
+                                                      const int32_t* __restrict__ sub_i,
+                                                      __nv_bfloat16* __restrict__ G, int64_t N,
+                                                      int64_t Np, int h, int k, int Cp) {
+  const int lane = threadIdx.x & 31;
+  const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int hs2 = 2 * h;
+  if (w >= Np * hs2) return;
+  const int64_t t = w / hs2;
+  const int hs = (int)(w % hs2);
+  __nv_bfloat16* hi = G + ((int64_t)(hs * 2 + 0) * Np + t) * Cp;
+  __nv_bfloat16* lo = G + ((int64_t)(hs * 2 + 1) * Np + t) * Cp;
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  for (int c = lane; c < Cp / 8; c += 32) {
+    reinterpret_cast<uint4*>(hi)[c] = z;
+    reinterpret_cast<uint4*>(lo)[c] = z;
+  }
+  __syncwarp();
+  if (t < N && lane < k) {
+    const int hh = hs >> 1, s = hs & 1;
+    const int64_t o = ((t * h + hh) * 2 + s) * k + lane;
+    const float g = gsub[o];
+    const int32_t i = sub_i[o];
+    const __nv_bfloat16 gh = __float2bfloat16_rn(g);
+    hi[i] = gh;
+    lo[i] = __float2bfloat16_rn(g - __bfloat162float(gh));
+  }
+}
+
+__device__ __forceinline__ void store_piece(float* dst, int n0, int n_lim,
+                                            const uint32_t (&r)[32]) {
+  if (n0 + 32 <= n_lim) {
+    float4* p = reinterpret_cast<float4*>(dst);
+#pragma unroll
+    for (int v = 0; v < 8; ++v)
+      p[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                         __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (n0 + j < n_lim) dst[j] = __uint_as_float(r[j]);
+  }
+}
+
+// ------------------------------------------------------------------ dq_half = G C_half
+struct DqProb {
+  static constexpr int kAMN = 0, kBMN = 1;
+  static constexpr int kStages = 4;
+  static constexpr int kEpiSmem = 0;
+  struct Params {
+    int* status;
+    float* dqf;  // [N][hq]
+    int64_t N, Np;
+    int h, dk, half, C1, C2, Cp, hq, m_tiles, n_tiles, nkc;  // nkc = Cp / 64
+  };
+  struct EpiState {};
+  __device__ static int num_units(const Params& P) { return 2 * P.h * P.m_tiles * P.n_tiles; }
+  __device__ static int num_chunks(const Params&, int) { return 1; }
+  __device__ static int num_kblocks(const Params& P) { return 2 * P.nkc; }
+  __device__ static void decode(const Params& P, int u, int& hs, int& mt, int& nt) {
+    const int per = P.m_tiles * P.n_tiles;
+    hs = u / per;
+    mt = (u % per) / P.n_tiles;
+    nt = u % P.n_tiles;
+  }
+  __device__ static void load(const Params& P, const CUtensorMap* A0, const CUtensorMap*,
+                              const CUtensorMap* B, const CUtensorMap*, int u, int, int kb,
+                              void* sa, void* sb, uint64_t* bar) {
+    int hs, mt, nt;
+    decode(P, u, hs, mt, nt);
+    const int hh = hs >> 1, s = hs & 1;
+    const int plane = kb / P.nkc, kk = kb % P.nkc;
+    tma_load_2d(sa, A0, kk * kBK, (int)((int64_t)(hs * 2 + plane) * P.Np + mt * kBM), bar);
+    unsigned char* b = static_cast<unsigned char*>(sb);
+#pragma unroll
+    for (int j = 0; j < kBN / kMNBox; ++j)
+      tma_load_2d(b + j * kMNBoxBytes, B, nt * kBN + j * kMNBox,
+                  hh * (P.C1 + P.C2) + s * P.C1 + kk * kBK, bar);
+  }
+  __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState&) {}
+  __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&) {}
+  __device__ static void epi_chunk(const Params& P, int u, int, int row, uint32_t taddr,
+                                   unsigned char*, EpiState&) {
+    int hs, mt, nt;
+    decode(P, u, hs, mt, nt);
+    const int hh = hs >> 1, s = hs & 1;
+    const int64_t t = (int64_t)mt * kBM + row;
+    for (int piece = 0; piece < kBN / 32; ++piece) {
+      const int n0 = nt * kBN + piece * 32;
+      if (n0 >= P.half) break;  // warp-uniform
+      uint32_t r[32];
+      tmem_ld32(taddr + (uint32_t)(piece * 32), r);
+      tmem_wait_ld();
+      if (t < P.N) store_piece(P.dqf + t * P.hq + hh * P.dk + s * P.half + n0, n0, P.half, r);
+    }
+  }
+};
+
+// ------------------------------------------------------------------ dC_half = G^T Q_half
+struct DsubProb {
+  static constexpr int kAMN = 1, kBMN = 1;
+  static constexpr int kStages = 4;
+  static constexpr int kEpiSmem = 0;
+  struct Params {
+    int* status;
+    float* part;  // [kSplits][2h][Cp][half]
+    int64_t N, Np;
+    int h, dk, half, C1, C2, Cp, m_tiles, n_tiles, nkt, kper;  // nkt = Np / 64
+  };
+  struct EpiState {};
+  __device__ static int num_units(const Params& P) {
+    return kSplits * 2 * P.h * P.m_tiles * P.n_tiles;
+  }
+  __device__ static int num_chunks(const Params&, int) { return 1; }
+  __device__ static int num_kblocks(const Params& P) { return 3 * P.kper; }
+  __device__ static void decode(const Params& P, int u, int& sp, int& hs, int& mt, int& nt) {
+    const int per = P.m_tiles * P.n_tiles;
+    sp = u / (2 * P.h * per);
+    const int r = u % (2 * P.h * per);
+    hs = r / per;
+    mt = (r % per) / P.n_tiles;
+    nt = r % P.n_tiles;
+  }
+  __device__ static void load(const Params& P, const CUtensorMap* A0, const CUtensorMap*,
+                              const CUtensorMap* B, const CUtensorMap*, int u, int, int kb,
+                              void* sa, void* sb, uint64_t* bar) {
+    int sp, hs, mt, nt;
+    decode(P, u, sp, hs, mt, nt);
+    const int hh = hs >> 1, s = hs & 1;
+    const int pass = kb / P.kper;
+    const int kk = sp * P.kper + kb % P.kper;  // 64-token block
+    const int gplane = pass == 2 ? 1 : 0;    // G_hi Q_hi, G_hi Q_lo, G_lo Q_hi
+    const int qplane = pass == 1 ? 1 : 0;
+    // token blocks past the padded range read beyond both tensors: zero fill
+    const bool live = kk < P.nkt;
+    const int gy = live ? (int)((int64_t)(hs * 2 + gplane) * P.Np + kk * kBK)
+                        : (int)(4 * (int64_t)P.h * P.Np);
+    const int qy = live ? (int)((int64_t)qplane * P.N + kk * kBK) : (int)(2 * P.N);
+    unsigned char* a = static_cast<unsigned char*>(sa);
+    unsigned char* b = static_cast<unsigned char*>(sb);
+#pragma unroll
+    for (int j = 0; j < kBM / kMNBox; ++j)
+      tma_load_2d(a + j * kMNBoxBytes, A0, mt * kBM + j * kMNBox, gy, bar);
+#pragma unroll
+    for (int j = 0; j < kBN / kMNBox; ++j)
+      tma_load_2d(b + j * kMNBoxBytes, B, hh * P.dk + s * P.half + nt * kBN + j * kMNBox, qy,
+                  bar);
+  }
+  __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState&) {}
+  __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&) {}
+  __device__ static void epi_chunk(const Params& P, int u, int, int row, uint32_t taddr,
+                                   unsigned char*, EpiState&) {
+    int sp, hs, mt, nt;
+    decode(P, u, sp, hs, mt, nt);
+    const int C = (hs & 1) ? P.C2 : P.C1;
+    const int c = mt * kBM + row;
+    for (int piece = 0; piece < kBN / 32; ++piece) {
+      const int n0 = nt * kBN + piece * 32;
+      if (n0 >= P.half) break;  // warp-uniform
+      uint32_t r[32];
+      tmem_ld32(taddr + (uint32_t)(piece * 32), r);
+      tmem_wait_ld();
+      if (c < C)
+        store_piece(P.part + (((int64_t)sp * 2 * P.h + hs) * P.Cp + c) * P.half + n0, n0, P.half,
+                    r);
+    }
+  }
+};
+
+// dsub[h][row(s, c)][d] += sum over splits, in split order.
+__global__ void dsub_reduce_kernel(const float* __restrict__ part, float* __restrict__ dsub, int h,
+                                   int C1, int C2, int Cp, int half) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t total = (int64_t)h * (C1 + C2) * half;
+  if (i >= total) return;
+  const int d = (int)(i % half);
+  const int64_t rr = i / half;
+  const int hh = (int)(rr / (C1 + C2));
+  const int within = (int)(rr % (C1 + C2));
+  const int s = within >= C1 ? 1 : 0;
+  const int c = within - s * C1;
+  const int hs = hh * 2 + s;
+  float acc = 0.f;
+#pragma unroll
+  for (int sp = 0; sp < kSplits; ++sp)
+    acc += part[(((int64_t)sp * 2 * h + hs) * Cp + c) * half + d];
+  dsub[i] += acc;
+}
+
+// BatchNorm eval backward: dq_pre = dq gamma / sqrt(var + eps), written as bf16 hi/lo
+// planes for the dense query GEMMs, plus per-64-token partial sums of dq * qhat and
+// dq (the same partial layout the fp32 path produces for dbn_reduce).
+__global__ void __launch_bounds__(256) bn_bwd_kernel(const float* __restrict__ dqf,
+                                                     const float* __restrict__ bn,
+                                                     const float* __restrict__ qhat,
+                                                     __nv_bfloat16* __restrict__ planes,
+                                                     float* __restrict__ part, int64_t N, int hq,
+                                                     float eps) {
+  const int col = blockIdx.y * 256 + threadIdx.x;
+  if (col >= hq) return;
+  const float scale = bn[2 * hq + col] / sqrtf(bn[hq + col] + eps);
+  const int64_t t0 = (int64_t)blockIdx.x * kBnTokens;
+  float pg = 0.f, pb = 0.f;
+  for (int tt = 0; tt < kBnTokens; ++tt) {
+    const int64_t t = t0 + tt;
+    if (t >= N) break;
+    const float dq = dqf[t * hq + col];
+    const float v = dq * scale;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    planes[t * hq + col] = hi;
+    planes[N * hq + t * hq + col] = __float2bfloat16_rn(v - __bfloat162float(hi));
+    if (part) {
+      pg = fmaf(dq, qhat[t * hq + col], pg);
+      pb += dq;
+    }
+  }
+  if (part) {
+    part[((int64_t)blockIdx.x * 2 + 0) * hq + col] = pg;
+    part[((int64_t)blockIdx.x * 2 + 1) * hq + col] = pb;
+  }
+}
+
+}  // namespace
+
+int64_t subgrad_pad_tokens(int64_t N) { return (N + 63) / 64 * 64; }
+int subgrad_pad_keys(int C1, int C2) { return ((C1 > C2 ? C1 : C2) + 63) / 64 * 64; }
+size_t subgrad_partial_floats(const Plan& p) {
+  return (size_t)kSplits * 2 * p.h * subgrad_pad_keys(p.C1, p.C2) * p.half;
+}
+
+cudaError_t launch_subgrad_tc(const Plan& p, const float* gsub, const int32_t* sub_i,
+                              const void* subkeys, const void* q_planes, const float* bn,
+                              const float* qhat, __nv_bfloat16* G, float* dqf,
+                              __nv_bfloat16* dq_planes, float* bn_part, float* dsub_part,
+                              float* dsub, bool want_dq, cudaStream_t st) {
+  const int64_t Np = subgrad_pad_tokens(p.N);
+  const int Cp = subgrad_pad_keys(p.C1, p.C2);
+  const int hs2 = 2 * p.h;
+  cudaError_t e;
+  {
+    const int64_t warps = Np * hs2;
+    g_dense_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(gsub, sub_i, G, p.N, Np, p.h,
+                                                                 p.k, Cp);
+    PKM_COUNT(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (want_dq) {
+    CUtensorMap ta, tb;
+    if (!make_tmap_bf16_2d(&ta, G, Cp, (uint64_t)hs2 * 2 * Np, (uint64_t)Cp * 2, kBK, kBM) ||
+        !make_tmap_bf16_2d(&tb, subkeys, p.half, (uint64_t)p.h * (p.C1 + p.C2),
+                           (uint64_t)p.half * 2, kMNBox, kBK))
+      return cudaErrorInvalidValue;
+    DqProb::Params P{};
+    P.status = p.status;
+    P.dqf = dqf;
+    P.N = p.N;
+    P.Np = Np;
+    P.h = p.h;
+    P.dk = p.dk;
+    P.half = p.half;
+    P.C1 = p.C1;
+    P.C2 = p.C2;
+    P.Cp = Cp;
+    P.hq = p.hq;
+    P.m_tiles = (int)(Np / kBM + (Np % kBM ? 1 : 0));
+    P.n_tiles = (p.half + kBN - 1) / kBN;
+    P.nkc = Cp / kBK;
+    if ((e = launch_tc<DqProb>(ta, ta, tb, P, hs2 * P.m_tiles * P.n_tiles, p.sm_count, st)) !=
+        cudaSuccess)
+      return e;
+    const dim3 grid((unsigned)((p.N + kBnTokens - 1) / kBnTokens), (unsigned)((p.hq + 255) / 256));
+    bn_bwd_kernel<<<grid, 256, 0, st>>>(dqf, bn, qhat, dq_planes, bn_part, p.N, p.hq, p.eps);
+    PKM_COUNT(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (dsub) {
+    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q_planes);
+    CUtensorMap ta, tb;
+    if (!make_tmap_bf16_2d(&ta, G, Cp, (uint64_t)hs2 * 2 * Np, (uint64_t)Cp * 2, kMNBox, kBK) ||
+        !make_tmap_bf16_2d(&tb, qb, p.hq, (uint64_t)2 * p.N, (uint64_t)p.hq * 2, kMNBox, kBK))
+      return cudaErrorInvalidValue;
+    DsubProb::Params P{};
+    P.status = p.status;
+    P.part = dsub_part;
+    P.N = p.N;
+    P.Np = Np;
+    P.h = p.h;
+    P.dk = p.dk;
+    P.half = p.half;
+    P.C1 = p.C1;
+    P.C2 = p.C2;
+    P.Cp = Cp;
+    P.m_tiles = (Cp + kBM - 1) / kBM;
+    P.n_tiles = (p.half + kBN - 1) / kBN;
+    P.nkt = (int)(Np / kBK);
+    P.kper = (P.nkt + kSplits - 1) / kSplits;
+    const int units = kSplits * hs2 * P.m_tiles * P.n_tiles;
+    if ((e = launch_tc<DsubProb>(ta, ta, tb, P, units, p.sm_count, st)) != cudaSuccess) return e;
+    const int64_t total = (int64_t)p.h * (p.C1 + p.C2) * p.half;
+    dsub_reduce_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(dsub_part, dsub, p.h,
+                                                                         p.C1, p.C2, Cp, p.half);
+    PKM_COUNT(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace pkm

@@ -96,6 +96,16 @@ cudaError_t launch_backward(const Plan& p, const void* x, const void* Wq, const 
                             const float* dy, float* dx, float* dWq, float* dbn, float* dsub,
                             float* dV, float* dw_out, void* ws, cudaStream_t st);
 
+// tcgen05 sub-key / query-half gradients and BatchNorm backward (bf16 storage)
+int64_t subgrad_pad_tokens(int64_t N);
+int subgrad_pad_keys(int C1, int C2);
+size_t subgrad_partial_floats(const Plan& p);
+cudaError_t launch_subgrad_tc(const Plan& p, const float* gsub, const int32_t* sub_i,
+                              const void* subkeys, const void* q_planes, const float* bn,
+                              const float* qhat, __nv_bfloat16* G, float* dqf,
+                              __nv_bfloat16* dq_planes, float* bn_part, float* dsub_part,
+                              float* dsub, bool want_dq, cudaStream_t st);
+
 // ---------------------------------------------------------------- self-test
 cudaError_t launch_wait_timeout_probe(long long budget_cycles, int* status, cudaStream_t st);
 

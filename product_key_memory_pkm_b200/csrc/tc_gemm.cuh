@@ -43,7 +43,8 @@ template <class Prob>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
                    const __grid_constant__ CUtensorMap tmA1,
-                   const __grid_constant__ CUtensorMap tmB, const typename Prob::Params P) {
+                   const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmB1, const typename Prob::Params P) {
   constexpr int S = Prob::kStages;
   extern __shared__ unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], tfull_bar[2], tempty_bar[2],
@@ -73,6 +74,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmA0);
     prefetch_tmap(&tmA1);
     prefetch_tmap(&tmB);
+    prefetch_tmap(&tmB1);
   }
   if (warp == 1) {
     tmem_alloc(&tmem_slot, kTmemCols);
@@ -104,7 +106,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             unsigned char* sa = smem + (size_t)stage * kStageBytes;
             mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
-            Prob::load(P, &tmA0, &tmA1, &tmB, u, c, kb, sa, sa + kStageA, &full_bar[stage]);
+            Prob::load(P, &tmA0, &tmA1, &tmB, &tmB1, u, c, kb, sa, sa + kStageA,
+                       &full_bar[stage]);
             issued_mask |= 1u << stage;
             parity_mask = (parity_mask & ~(1u << stage)) | (phase << stage);
             if (++stage == S) {
