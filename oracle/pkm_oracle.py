@@ -228,3 +228,74 @@ def loss(inp, cfg, dy, select="brute"):
     """L = sum_t dy[t] . y[t] (the scalar whose gradient ``backward`` returns)."""
     f = forward(inp, cfg, select=select)
     return float((np.asarray(dy, dtype=np.float64) * f["y"]).sum()), f
+
+
+# ----------------------------------------------------------------------------- fast weights
+class _WrittenRows:
+    """The value table as the fast-weight loop sees it: the initial table, with the
+    rows written so far held in fp64 on top.  Indexing with an array of rows returns
+    those rows as fp64 (what ``bag`` and ``backward`` read), so the loop never copies
+    the whole table."""
+
+    def __init__(self, values):
+        self.base = values
+        self.rows = np.zeros(0, dtype=np.int64)        # sorted
+        self.vals = np.zeros((0, values.shape[1]))
+
+    def __getitem__(self, r):
+        r = np.asarray(r, dtype=np.int64)
+        out = np.asarray(self.base[r], dtype=np.float64)
+        if self.rows.size:
+            pos = np.clip(np.searchsorted(self.rows, r), 0, self.rows.size - 1)
+            hit = self.rows[pos] == r
+            out[hit] = self.vals[pos[hit]]
+        return out
+
+    def sgd(self, r, g, lr):
+        """rows r (unique) <- rows r - lr * g."""
+        new = self[r] - lr * g
+        keep = ~np.isin(self.rows, r)
+        rows = np.concatenate([self.rows[keep], r])
+        vals = np.concatenate([self.vals[keep], new])
+        order = np.argsort(rows, kind="stable")
+        self.rows, self.vals = rows[order], vals[order]
+
+
+def fastweight_chunks(inp, cfg, chunk, lr, targets=None, lookahead=False, select="brute"):
+    """Chunked read-then-write of the fast-weight product-key memory ("Fast-weight
+    Product Key Memory", sections 2.2 and 3, test-time training).
+
+    The token sequence is cut into consecutive chunks of ``chunk`` tokens.  Each chunk
+    first READS: the layer's forward with the current value table.  Then it WRITES:
+    one step of SGD with rate ``lr`` on the value rows it selected, descending the
+    chunk's reconstruction loss L_c = sum_{t in chunk} 1/2 ||y_t - target_t||^2
+    (only the value table is a fast weight here; queries and keys stay fixed).  The
+    next chunk reads the table this chunk wrote.
+
+    Targets: ``targets[t]`` [N][d_v], or with ``lookahead`` the next token's input,
+    target_t = x[t + 1] (needs d_in = d_v); the sequence's last token then has no
+    target and adds nothing to the loss.
+
+    Returns (y [N][d_v] of every read, written rows (sorted), their final values).
+    """
+    N = inp["x"].shape[0]
+    x = np.asarray(inp["x"], dtype=np.float64)
+    if lookahead:
+        assert cfg.d_in == cfg.d_v
+        tg = np.zeros((N, cfg.d_v))
+        tg[:-1] = x[1:]
+        has_target = np.arange(N) < N - 1
+    else:
+        tg = np.asarray(targets, dtype=np.float64)
+        has_target = np.ones(N, dtype=bool)
+    table = _WrittenRows(inp["values"])
+    ys = np.zeros((N, cfg.d_v))
+    for c0 in range(0, N, chunk):
+        c1 = min(N, c0 + chunk)
+        sub = dict(inp, x=inp["x"][c0:c1], values=table)
+        f = forward(sub, cfg, select=select)
+        ys[c0:c1] = f["y"]
+        dy = (f["y"] - tg[c0:c1]) * has_target[c0:c1, None]
+        b = backward(sub, cfg, f, dy)
+        table.sgd(b["dV_rows"], b["dV_vals"], lr)
+    return ys, table.rows, table.vals

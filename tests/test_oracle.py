@@ -309,3 +309,94 @@ def test_backward_central_finite_differences_tiny_config():
         assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, ix, fd, an)
         tested += 1
     assert tested >= 90
+
+
+# --------------------------------------------------------------------------- fast weights
+def _fw_cfg(**kw):
+    base = dict(name="fw", N=48, d_in=6, h=1, dk=8, C1=12, C2=10, k=3, d_v=6, dtype="f32",
+                clustered=4)
+    base.update(kw)
+    return PKMConfig(**base)
+
+
+def test_fastweight_zero_rate_is_plain_forward():
+    cfg = _fw_cfg()
+    inp = make_inputs(cfg, seed=1)
+    tg = np.random.default_rng(0).standard_normal((cfg.N, cfg.d_v))
+    ys, rows, vals = O.fastweight_chunks(inp, cfg, 16, 0.0, targets=tg)
+    np.testing.assert_allclose(ys, O.forward(inp, cfg)["y"], atol=1e-13)
+    np.testing.assert_array_equal(vals, inp["values"][rows])
+
+
+def test_fastweight_one_chunk_is_a_descent_step():
+    """One chunk: the write is -lr times the gradient of the chunk's loss, whose
+    gradient for row r is sum over selections of r of w * (y - target) (closed form,
+    written out here per selection); only selected rows change; and for a small rate
+    the loss at the same selection drops by lr * |grad|^2 to first order."""
+    cfg = _fw_cfg(h=2)
+    inp = make_inputs(cfg, seed=2)
+    tg = np.random.default_rng(1).standard_normal((cfg.N, cfg.d_v))
+    lr = 1e-4
+    _, rows, vals = O.fastweight_chunks(inp, cfg, cfg.N, lr, targets=tg)
+    f = O.forward(inp, cfg)
+    grad = {}
+    for t in range(cfg.N):
+        for hh in range(cfg.h):
+            for j in range(cfg.k):
+                r = int(f["idx"][t, hh, j])
+                grad[r] = grad.get(r, 0.0) + f["w"][t, hh, j] * (f["y"][t] - tg[t])
+    assert sorted(grad) == rows.tolist()
+    for r, v in zip(rows, vals):
+        np.testing.assert_allclose(v, inp["values"][r] - lr * grad[int(r)], atol=1e-13)
+    V1 = np.array(inp["values"], dtype=np.float64)
+    V1[rows] = vals
+    loss0 = 0.5 * ((f["y"] - tg) ** 2).sum()
+    loss1 = 0.5 * ((O.bag(f["w"], f["idx"], V1) - tg) ** 2).sum()
+    g2 = sum((g ** 2).sum() for g in grad.values())
+    np.testing.assert_allclose(loss0 - loss1, lr * g2, rtol=1e-3)
+
+
+def test_fastweight_later_chunks_read_earlier_writes():
+    """Two chunks: the second chunk's reads differ from reading the untouched table
+    exactly on tokens that select a row the first chunk wrote (selection does not
+    depend on the value table)."""
+    cfg = _fw_cfg(C1=16, C2=16, k=2, clustered=0)
+    inp = make_inputs(cfg, seed=3)
+    tg = np.random.default_rng(2).standard_normal((cfg.N, cfg.d_v))
+    ys, rows, _ = O.fastweight_chunks(inp, cfg, 24, 0.5, targets=tg)
+    f0 = O.forward(inp, cfg)
+    first = set(np.unique(f0["idx"][:24]).tolist())
+    np.testing.assert_allclose(ys[:24], f0["y"][:24], atol=1e-14)
+    n_touch = 0
+    for t in range(24, cfg.N):
+        touches = bool(set(f0["idx"][t].ravel().tolist()) & first)
+        n_touch += touches
+        assert np.allclose(ys[t], f0["y"][t], atol=1e-14) == (not touches), t
+    assert 0 < n_touch < cfg.N - 24
+
+
+def test_fastweight_rate_one_on_a_lone_selection_reaches_the_target():
+    """k = 1, one token, w = 1: the gradient of 1/2 ||V[r] - target||^2 is V[r] -
+    target, so a step of rate 1 writes the target into the row exactly."""
+    cfg = _fw_cfg(N=1, k=1)
+    inp = make_inputs(cfg, seed=4)
+    tg = np.random.default_rng(3).standard_normal((1, cfg.d_v))
+    _, rows, vals = O.fastweight_chunks(inp, cfg, 1, 1.0, targets=tg)
+    assert rows.size == 1
+    np.testing.assert_allclose(vals[0], tg[0], atol=1e-14)
+
+
+def test_fastweight_lookahead_targets_are_the_next_input():
+    """Lookahead equals explicit targets x[t + 1] with the last token's target set to
+    its own read (zero residual)."""
+    cfg = _fw_cfg(d_in=6, d_v=6)
+    inp = make_inputs(cfg, seed=5)
+    ys_a, rows_a, vals_a = O.fastweight_chunks(inp, cfg, 16, 0.3, lookahead=True)
+    tg = np.zeros((cfg.N, cfg.d_v))
+    tg[:-1] = np.asarray(inp["x"], dtype=np.float64)[1:]
+    # the last token's target: its read, which no earlier write of its own chunk changes
+    tg[-1] = ys_a[-1]
+    ys_b, rows_b, vals_b = O.fastweight_chunks(inp, cfg, 16, 0.3, targets=tg)
+    np.testing.assert_allclose(ys_a, ys_b, atol=1e-13)
+    assert rows_a.tolist() == rows_b.tolist()
+    np.testing.assert_allclose(vals_a, vals_b, atol=1e-13)
