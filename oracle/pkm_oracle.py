@@ -54,6 +54,16 @@ def query_network(x, Wq, bn, eps):
     return gamma * qhat + beta, qhat
 
 
+def round_bf16(a):
+    """Round to the nearest bfloat16 (ties to even) through fp32, returned as fp64: the
+    fp32 bit pattern u becomes (u + 0x7FFF + ((u >> 16) & 1)) with the low 16 bits
+    cleared (finite inputs).  Used by the single-pass scoring variant, whose scores
+    take q rounded to bf16."""
+    u = np.asarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000).astype(np.uint32)
+    return r.view(np.float32).astype(np.float64)
+
+
 # ----------------------------------------------------------------------------- 2, 3
 def split_halves(q, h, dk):
     """q [N][h*dk] -> (q1, q2), each [N][h][dk/2]."""
@@ -133,8 +143,12 @@ def softmax(S):
 
 
 # ----------------------------------------------------------------------------- 1..6
-def forward(inp, cfg, select="brute"):
+def forward(inp, cfg, select="brute", q_bf16=False):
     """The layer forward for every token of ``inp['x']``.
+
+    ``q_bf16``: the single-pass scoring variant -- the sub-key scores (and through them
+    the selection and the weights) take q rounded to bf16 (``round_bf16``); the dict
+    then also holds that q as ``q_scores``.
 
     Returns a dict with q [N][h*dk], qhat, s1 [N][h][C1], s2 [N][h][C2],
     sub_i/sub_s [N][h][2][k] (per-half top-k, best first), idx [N][h][k]
@@ -143,7 +157,8 @@ def forward(inp, cfg, select="brute"):
     """
     h, dk, C1, C2, k = cfg.h, cfg.dk, cfg.C1, cfg.C2, cfg.k
     q, qhat = query_network(inp["x"], inp["Wq"], inp["bn"], cfg.bn_eps)
-    s1, s2 = subkey_scores(q, inp["subkeys"], h, dk, C1)
+    qs = round_bf16(q) if q_bf16 else q
+    s1, s2 = subkey_scores(qs, inp["subkeys"], h, dk, C1)
     N = q.shape[0]
     pick = brute_force_topk if select == "brute" else product_key_topk
     idx = np.zeros((N, h, k), dtype=np.int64)
@@ -159,8 +174,10 @@ def forward(inp, cfg, select="brute"):
             sub_i[t, hh, 1], sub_s[t, hh, 1] = half_topk(s2[t, hh], k)
     w = softmax(S)
     y = bag(w, idx, inp["values"])
-    return dict(q=q, qhat=qhat, s1=s1, s2=s2, sub_i=sub_i, sub_s=sub_s, idx=idx,
-                S=S, w=w, y=y)
+    out = dict(q=q, qhat=qhat, s1=s1, s2=s2, sub_i=sub_i, sub_s=sub_s, idx=idx, S=S, w=w, y=y)
+    if q_bf16:
+        out["q_scores"] = qs
+    return out
 
 
 def bag(w, idx, values):
@@ -173,6 +190,8 @@ def bag(w, idx, values):
 # ----------------------------------------------------------------------------- backward
 def backward(inp, cfg, fwd, dy):
     """Gradients of L = sum_t dy[t] . y[t] with the selected keys held fixed.
+    After a ``q_bf16`` forward the sub-key gradients take the rounded q the scores
+    used, and the rounding passes the query gradient through unchanged.
 
     Returns dict:
       dw   [N][h][k]   dL/dw            = dy[t] . V[row]
@@ -199,7 +218,7 @@ def backward(inp, cfg, fwd, dy):
     np.add.at(g1, (tt, hh, (idx // C2).reshape(-1)), dsum.reshape(-1))
     np.add.at(g2, (tt, hh, (idx % C2).reshape(-1)), dsum.reshape(-1))
     sub = np.asarray(inp["subkeys"], dtype=np.float64)
-    q1, q2 = split_halves(fwd["q"], h, dk)
+    q1, q2 = split_halves(fwd.get("q_scores", fwd["q"]), h, dk)
     dq1 = np.einsum("thi,hid->thd", g1, sub[:, :C1, :])
     dq2 = np.einsum("thj,hjd->thd", g2, sub[:, C1:, :])
     dsub = np.zeros_like(sub)

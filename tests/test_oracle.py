@@ -400,3 +400,75 @@ def test_fastweight_lookahead_targets_are_the_next_input():
     np.testing.assert_allclose(ys_a, ys_b, atol=1e-13)
     assert rows_a.tolist() == rows_b.tolist()
     np.testing.assert_allclose(vals_a, vals_b, atol=1e-13)
+
+
+# --------------------------------------------------------------------------- bf16 q scoring
+def test_round_bf16_hand_cases_and_library():
+    """Ties go to the even neighbour; everything else to the nearest bf16; agrees with
+    the library's fp32 -> bfloat16 conversion on random values."""
+    e = 2.0 ** -8
+    cases = [(1.0, 1.0), (1 + e, 1.0), (1 + 3 * e, 1 + 4 * e), (1 + e + 2.0 ** -20, 1 + 2 * e),
+             (-(1 + e), -1.0), (3.0, 3.0), (0.0, 0.0), (2.0 ** -130, 2.0 ** -130)]
+    for a, want in cases:
+        assert O.round_bf16(np.array([a]))[0] == want, (a, want)
+    r = np.random.default_rng(0).standard_normal(10000) * 10.0 ** np.random.default_rng(1).integers(-6, 6, 10000)
+    lib = torch.from_numpy(r.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.round_bf16(r), lib)
+
+
+def _bf16_exact_q_case():
+    """Wq = I, BN with var + eps = 1: q = x exactly, and x is bf16."""
+    eps = 2.0 ** -10
+    cfg = _cfg(d_in=16, h=2, dk=8, dtype="bf16", bn_eps=eps)
+    inp = make_inputs(cfg, seed=11)
+    inp["Wq"] = np.eye(16, dtype=np.float32)
+    inp["bn"] = np.stack([np.zeros(16), np.full(16, 1 - eps), np.ones(16), np.zeros(16)])
+    return cfg, inp
+
+
+def test_bf16_q_variant_equals_plain_when_q_is_bf16():
+    cfg, inp = _bf16_exact_q_case()
+    f0, f1 = O.forward(inp, cfg), O.forward(inp, cfg, q_bf16=True)
+    np.testing.assert_array_equal(f1["q_scores"], f0["q"])
+    assert (f0["idx"] == f1["idx"]).all()
+    np.testing.assert_array_equal(f0["y"], f1["y"])
+    b0, b1 = O.backward(inp, cfg, f0, inp["dy"]), O.backward(inp, cfg, f1, inp["dy"])
+    for key in ("dsub", "dx", "dWq", "dgamma", "dbeta", "dV_vals"):
+        np.testing.assert_array_equal(b0[key], b1[key], err_msg=key)
+
+
+def test_bf16_q_scores_within_the_rounding_bound():
+    """|s_b - s| <= sum_d 2^-9 |q_d| |C_d| (half an ulp of bf16 per query coordinate),
+    and the bound is not vacuous (the scores do move)."""
+    cfg = _cfg(h=2, dk=16, C1=20, C2=12)
+    inp = make_inputs(cfg, seed=12, random_bn=True)
+    f0, f1 = O.forward(inp, cfg), O.forward(inp, cfg, q_bf16=True)
+    sub = np.asarray(inp["subkeys"], dtype=np.float64)
+    q1, q2 = O.split_halves(np.abs(f0["q"]), cfg.h, cfg.dk)
+    b1 = 2.0 ** -9 * np.einsum("thd,hid->thi", q1, np.abs(sub[:, :cfg.C1]))
+    b2 = 2.0 ** -9 * np.einsum("thd,hid->thi", q2, np.abs(sub[:, cfg.C1:]))
+    assert np.all(np.abs(f1["s1"] - f0["s1"]) <= b1 * (1 + 1e-12))
+    assert np.all(np.abs(f1["s2"] - f0["s2"]) <= b2 * (1 + 1e-12))
+    assert np.abs(f1["s1"] - f0["s1"]).max() > 0
+
+
+def test_bf16_q_subkey_gradient_by_finite_differences():
+    """The sub-key gradient after a bf16-q forward is the derivative of the loss in the
+    sub-keys with the rounded q (which does not depend on them): central differences."""
+    cfg = _cfg(h=2, dk=8, C1=10, C2=9, k=3)
+    inp = make_inputs(cfg, seed=13, random_bn=True)
+    f = O.forward(inp, cfg, q_bf16=True)
+    g = O.backward(inp, cfg, f, inp["dy"])["dsub"]
+    sub0 = np.asarray(inp["subkeys"], dtype=np.float64)
+    rng = np.random.default_rng(5)
+    for _ in range(12):
+        i = tuple(int(rng.integers(0, n)) for n in sub0.shape)
+        h = 1e-6
+        vals = []
+        for sgn in (1, -1):
+            s = sub0.copy()
+            s[i] += sgn * h
+            fs = O.forward(dict(inp, subkeys=s), cfg, q_bf16=True)
+            assert (fs["idx"] == f["idx"]).all()
+            vals.append((inp["dy"] * fs["y"]).sum())
+        np.testing.assert_allclose((vals[0] - vals[1]) / (2 * h), g[i], rtol=1e-5, atol=1e-8)
