@@ -318,3 +318,43 @@ def fastweight_chunks(inp, cfg, chunk, lr, targets=None, lookahead=False, select
         b = backward(sub, cfg, f, dy)
         table.sgd(b["dV_rows"], b["dV_vals"], lr)
     return ys, table.rows, table.vals
+
+
+# ----------------------------------------------------------------------------- training pieces
+def hit_counts(fwd, cfg):
+    """Hit monitoring of one batch ("Meta AI 可扩展内存层" sections 6.4 and 11.2: how often
+    each slot and each sub-key of each codebook is selected).
+
+    slot [C1*C2]: number of selections (t, h, j) of each value row.
+    sub [h][C1+C2]: per head, how many winners use each sub-key: entry i < C1 counts
+    winners whose first-half sub-key is i, entry C1 + j those whose second-half one is j.
+    """
+    idx = np.asarray(fwd["idx"], dtype=np.int64)
+    slot = np.bincount(idx.ravel(), minlength=cfg.K)
+    sub = np.zeros((cfg.h, cfg.C1 + cfg.C2), dtype=np.int64)
+    for hh in range(cfg.h):
+        sub[hh] += np.bincount(idx[:, hh, :].ravel() // cfg.C2, minlength=cfg.C1 + cfg.C2)
+        sub[hh, cfg.C1:] += np.bincount(idx[:, hh, :].ravel() % cfg.C2, minlength=cfg.C2)
+    return slot, sub
+
+
+def sparse_adam(values, m, v, rows, grads, lr, beta1, beta2, eps, step):
+    """Lazy Adam on the touched value rows only ("Meta AI 可扩展内存层" section 6.3:
+    optimiser state is kept and advanced only for parameters that received a gradient).
+
+    For each touched row r with gradient g (rows unique, e.g. ``backward``'s dV_rows
+    and dV_vals):  m_r <- beta1 m_r + (1 - beta1) g;  v_r <- beta2 v_r + (1 - beta2) g^2;
+    V_r <- V_r - lr * (m_r / (1 - beta1^step)) / (sqrt(v_r / (1 - beta2^step)) + eps),
+    with ``step`` >= 1 the caller's global step count.  Other rows and their state are
+    left as they are.  Returns new (values, m, v) as fp64 copies.
+    """
+    V = np.array(values, dtype=np.float64, copy=True)
+    M = np.array(m, dtype=np.float64, copy=True)
+    S = np.array(v, dtype=np.float64, copy=True)
+    g = np.asarray(grads, dtype=np.float64)
+    M[rows] = beta1 * M[rows] + (1.0 - beta1) * g
+    S[rows] = beta2 * S[rows] + (1.0 - beta2) * g * g
+    mhat = M[rows] / (1.0 - beta1 ** step)
+    vhat = S[rows] / (1.0 - beta2 ** step)
+    V[rows] -= lr * mhat / (np.sqrt(vhat) + eps)
+    return V, M, S

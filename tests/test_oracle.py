@@ -472,3 +472,72 @@ def test_bf16_q_subkey_gradient_by_finite_differences():
             assert (fs["idx"] == f["idx"]).all()
             vals.append((inp["dy"] * fs["y"]).sum())
         np.testing.assert_allclose((vals[0] - vals[1]) / (2 * h), g[i], rtol=1e-5, atol=1e-8)
+
+
+# --------------------------------------------------------------------------- training pieces
+def test_hit_counts_totals_and_argmax_case():
+    """Every token contributes h*k slot hits and 2k sub-key hits per head; with k = 1 the
+    sub-key hits are the per-half argmax counts."""
+    cfg = _cfg(N=40, h=2, k=4)
+    inp = make_inputs(cfg, seed=21)
+    f = O.forward(inp, cfg)
+    slot, sub = O.hit_counts(f, cfg)
+    assert slot.sum() == cfg.N * cfg.h * cfg.k and slot.shape == (cfg.K,)
+    assert (sub.sum(1) == 2 * cfg.N * cfg.k).all()
+    assert (sub[:, :cfg.C1].sum(1) == cfg.N * cfg.k).all()
+    # rows never selected have zero hits; the selected ones at least one
+    assert (slot[np.unique(f["idx"])] > 0).all() and slot.sum() == f["idx"].size
+    cfg1 = _cfg(N=40, h=2, k=1)
+    f1 = O.forward(make_inputs(cfg1, seed=22), cfg1)
+    _, sub1 = O.hit_counts(f1, cfg1)
+    for hh in range(cfg1.h):
+        a1 = np.bincount(np.argmax(f1["s1"][:, hh], axis=1), minlength=cfg1.C1)
+        a2 = np.bincount(np.argmax(f1["s2"][:, hh], axis=1), minlength=cfg1.C2)
+        np.testing.assert_array_equal(sub1[hh], np.concatenate([a1, a2]))
+
+
+def test_sparse_adam_matches_the_library_optimisers():
+    """Lazy Adam against two independent implementations: torch.optim.SparseAdam on
+    changing row sets (it adds eps to sqrt(v) before the bias correction, so eps is made
+    negligible there), and torch.optim.Adam when every row is touched at every step
+    (lazy and dense Adam then coincide; this pins where eps enters)."""
+    rng = np.random.default_rng(23)
+    K, d = 12, 5
+    V0 = rng.standard_normal((K, d))
+    lr, b1, b2 = 0.05, 0.9, 0.99
+    p = torch.nn.Parameter(torch.from_numpy(V0.copy()))
+    opt = torch.optim.SparseAdam([p], lr=lr, betas=(b1, b2), eps=1e-30)
+    V, M, S = V0.copy(), np.zeros((K, d)), np.zeros((K, d))
+    for step, rows in enumerate(([1, 4, 7], [4, 5], [0, 1, 4, 11]), start=1):
+        rows = np.array(rows)
+        g = rng.standard_normal((rows.size, d))
+        V, M, S = O.sparse_adam(V, M, S, rows, g, lr, b1, b2, 1e-30, step)
+        p.grad = torch.sparse_coo_tensor(torch.from_numpy(rows)[None], torch.from_numpy(g), (K, d))
+        opt.step()
+    np.testing.assert_allclose(V, p.detach().numpy(), rtol=1e-12, atol=1e-12)
+
+    eps = 1e-3
+    p = torch.nn.Parameter(torch.from_numpy(V0.copy()))
+    opt = torch.optim.Adam([p], lr=lr, betas=(b1, b2), eps=eps)
+    V, M, S = V0.copy(), np.zeros((K, d)), np.zeros((K, d))
+    for step in range(1, 4):
+        g = rng.standard_normal((K, d)) * 1e-3
+        V, M, S = O.sparse_adam(V, M, S, np.arange(K), g, lr, b1, b2, eps, step)
+        p.grad = torch.from_numpy(g.copy())
+        opt.step()
+    np.testing.assert_allclose(V, p.detach().numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_sparse_adam_first_step_closed_form_and_untouched_rows():
+    """From zero state the first step moves a row by lr * g / (|g| + eps) elementwise;
+    untouched rows and their state stay as they were."""
+    rng = np.random.default_rng(24)
+    V0, M0, S0 = rng.standard_normal((6, 3)), rng.standard_normal((6, 3)), rng.random((6, 3))
+    M0[2] = S0[2] = 0.0
+    g = rng.standard_normal((1, 3))
+    V, M, S = O.sparse_adam(V0, M0, S0, np.array([2]), g, 0.1, 0.9, 0.999, 1e-8, 1)
+    np.testing.assert_allclose(V[2], V0[2] - 0.1 * g[0] / (np.abs(g[0]) + 1e-8), rtol=1e-12)
+    keep = np.arange(6) != 2
+    np.testing.assert_array_equal(V[keep], V0[keep])
+    np.testing.assert_array_equal(M[keep], M0[keep])
+    np.testing.assert_array_equal(S[keep], S0[keep])
