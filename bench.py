@@ -1,7 +1,12 @@
 """Benchmark of the product-key memory layer (forward + sparse backward) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
-                    [--workload NAME] [--no-e2e] [--no-cpu-baseline]
+                    [--workload NAME] [--no-e2e] [--no-cpu-baseline] [--stage S] [--decode]
+
+Default: the full-scale forward + backward workload (16384 tokens, |K| = 1024², h = 4,
+k = 32, d = 1600).  --workload fwpkm_chunk512_K1024x1024_h1_k8_d1024 times the
+fast-weight chunked read-then-write over a 4096-token sequence; --decode times
+decode-shaped forward calls (N = 1, 8, 64); --stage times one stage alone.
 
 One step = one pass of the whole layer over one batch of synthetic tokens: query
 network, sub-key scoring with per-half top-k, candidate top-k with softmax, value
@@ -30,9 +35,12 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from product_key_memory_pkm_b200.inputs import CONFIGS, FULL_K1024, make_inputs  # noqa: E402
+from product_key_memory_pkm_b200.inputs import (CONFIGS, FASTWEIGHT, FULL_K1024,  # noqa: E402
+                                              make_inputs, make_targets)
 
 METRIC = "PKM layer tokens/s (fwd, fwd+bwd) at |K|=1024²,h=4,k=32; gather HBM GB/s vs peak"
+FW_METRIC = "FwPKM chunked read-then-write tokens/s over the sequence (8 chunks of 512)"
+FW_CHUNK, FW_LR = 512, 1.0
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -49,7 +57,7 @@ def _peaks():
 def _cfg_json(cfg):
     return {"workload": cfg.name, "N_tokens": cfg.N, "d_in": cfg.d_in, "h": cfg.h, "dk": cfg.dk,
             "C1": cfg.C1, "C2": cfg.C2, "K": cfg.K, "k": cfg.k, "d_v": cfg.d_v,
-            "value_dtype": cfg.dtype, "l2": "flushed before every timed step (256 MiB write)"}
+            "input_dtype": cfg.dtype, "value_dtype": cfg.vdtype, "l2": "flushed before every timed step (256 MiB write)"}
 
 
 # ---------------------------------------------------------------- clocks
@@ -161,7 +169,7 @@ def run_b200(args, cfg, rank, world, dist):
     dy = torch.from_numpy(inp["dy"]).to(dev)
     gen_s = time.perf_counter() - t_gen
 
-    dims = P.Dims.from_config(cfg)
+    dims = P.Dims.from_config(cfg, flags=P.PKM_F_BF16_Q if args.bf16_q else 0)
     saved = P.alloc_saved(dims, with_qhat=True)
     y = torch.empty(cfg.N, cfg.d_v, device=dev)
     dx = torch.empty(cfg.N, cfg.d_in, device=dev)
@@ -302,7 +310,9 @@ def run_b200(args, cfg, rank, world, dist):
         "ms_per_step": round(step_ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded; tables random-init, no trained weights)",
-        "config": dict(_cfg_json(cfg), parallelism=f"replicas{world}" if world > 1 else "single"),
+        "config": dict(_cfg_json(cfg), parallelism=f"replicas{world}" if world > 1 else "single",
+                       scoring="single-pass, q rounded to bf16" if args.bf16_q else
+                       "q as bf16 hi + lo (two passes)"),
         "fwd": {"value": round(cfg.N * world / (fwd_ms * 1e-3), 1), "unit": "tokens/s (fwd)",
                 "ms": round(fwd_ms, 4)},
         "stage_ms": {n: round(float(v), 4) for n, v in zip(names, st_mean)},
@@ -325,6 +335,342 @@ def run_b200(args, cfg, rank, world, dist):
                                          f"brute force over all {cfg.K} keys per head, "
                                          f"analytic backward; ~{args.cpu_seconds:.0f} s of host time"}
     return out
+
+
+# ---------------------------------------------------------------- fast-weight workload
+def time_oracle_fastweight(cfg, inp, targets, seconds: float, n: int = 32):
+    """The oracle's chunk loop on successive n-token slices (one chunk each) until
+    ``seconds`` of host time have passed.  Returns (tokens/s, tokens, threads)."""
+    from oracle import pkm_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    done, t0 = 0, time.perf_counter()
+    while True:
+        sl = slice(done % cfg.N, done % cfg.N + n)
+        sub = dict(inp, x=inp["x"][sl])
+        O.fastweight_chunks(sub, cfg, n, FW_LR, targets=targets[sl])
+        done += n
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            return done / el, done, threads
+
+
+def run_fastweight(args, cfg, rank, world, dist):
+    """One step = the whole chunk loop over the sequence: every chunk reads (query,
+    scoring, candidates, bag + residual) and then writes (sparse SGD on its rows).
+    Headline: the loop captured once into a CUDA graph and replayed; the eager loop
+    and a per-stage breakdown (each stage timed alone over the 8 chunks) beside it."""
+    import torch
+
+    from product_key_memory_pkm_b200 import build as B
+    from product_key_memory_pkm_b200 import pkm as P
+
+    if not os.path.exists(B.LIB):
+        B.build()
+    P.load()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    t_gen = time.perf_counter()
+    inp = make_inputs(cfg, seed=0, with_dy=False)
+    tg_np = make_targets(cfg, seed=0)
+    if world > 1:   # each rank its own sequence; the same initial tables
+        inp["x"] = make_inputs(cfg, seed=1000 + rank, with_dy=False)["x"]
+        tg_np = make_targets(cfg, seed=1000 + rank)
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev)
+    sto = (lambda a: f32(a).to(torch.bfloat16)) if cfg.dtype == "bf16" else f32
+    x, Wq, bn, sub, V, tg = (sto(inp["x"]), sto(inp["Wq"]), f32(inp["bn"]), sto(inp["subkeys"]),
+                             f32(inp["values"]), f32(tg_np))
+    gen_s = time.perf_counter() - t_gen
+    dims = P.Dims.from_config(cfg)
+    y = torch.empty(cfg.N, cfg.d_v, device=dev)
+    ws = P.alloc_fastweight_workspace(dims, FW_CHUNK, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    side = torch.cuda.Stream(device=dev)
+
+    def loop(stream):
+        P.pkm_fastweight_chunks(dims, FW_CHUNK, FW_LR, x, Wq, bn, sub, V, y, targets=tg,
+                                workspace=ws, stream=stream)
+
+    clocks = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    clocks.start()
+    with torch.cuda.stream(side):
+        for _ in range(args.warmup):
+            flush.zero_()
+            loop(side)
+        side.synchronize()
+        if P.pkm_check_status(side) != P.PKM_OK:
+            raise RuntimeError("device status after warm-up is not OK")
+        l0 = P.pkm_launch_count()
+        loop(side)
+        side.synchronize()
+        launches_per_step = P.pkm_launch_count() - l0
+
+        def timed(fn):
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            if dist is not None:
+                dist.barrier()
+            torch.cuda.synchronize()
+            for a, b in evs:
+                flush.zero_()
+                a.record(side)
+                fn()
+                b.record(side)
+            torch.cuda.synchronize()
+            if dist is not None:
+                dist.barrier()
+            return float(np.mean([a.elapsed_time(b) for a, b in evs]))
+
+        eager_ms = timed(lambda: loop(side))
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            loop(side)
+        for _ in range(args.warmup):
+            graph.replay()
+        graph_ms = timed(graph.replay)
+        if P.pkm_check_status(side) != P.PKM_OK:
+            raise RuntimeError("device status after the timed steps is not OK")
+
+        # per-stage view through the stage entry points, as the loop runs them: the
+        # selection of the whole sequence at once (it does not read the table), then
+        # per chunk the bag and the write (pkm_value_sgd sorts its own chunk)
+        names = ["query", "subkey_scores", "candidate_topk", "gather_bag", "value_sgd"]
+        sdims = P.Dims.from_config(cfg)
+        cdims = P.Dims.from_config(cfg, N=FW_CHUNK)
+        saved = P.alloc_saved(sdims, with_qhat=False)
+        bws = P.alloc_workspace(cdims, P.PKM_BWD, device=dev)
+        dyc = torch.empty(FW_CHUNK, cfg.d_v, device=dev)
+        nch = cfg.N // FW_CHUNK
+        hk = cfg.h * cfg.k
+        stage_ms = np.zeros(len(names))
+        U_tot = 0
+
+        def ev_time(fn):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            flush.zero_()
+            a.record(side)
+            fn()
+            b.record(side)
+            b.synchronize()
+            return a.elapsed_time(b)
+        for rep in range(args.steps):
+            stage_ms[0] += ev_time(lambda: P.pkm_query(sdims, x, Wq, bn, saved, stream=side))
+            stage_ms[1] += ev_time(lambda: P.pkm_subkey_scores(sdims, sub, saved, stream=side))
+            stage_ms[2] += ev_time(lambda: P.pkm_candidate_topk(sdims, saved, stream=side))
+            for c in range(nch):
+                r0, r1 = c * FW_CHUNK, (c + 1) * FW_CHUNK
+                sc = {"idx": saved["idx"][r0:r1], "w": saved["w"][r0:r1]}
+                stage_ms[3] += ev_time(lambda: P.pkm_gather_bag(cdims, V, sc["idx"], sc["w"],
+                                                                y[r0:r1], stream=side))
+                if rep == 0:
+                    torch.sub(y[r0:r1], tg[r0:r1], out=dyc)
+                    U_tot += int(torch.unique(sc["idx"]).numel())
+                stage_ms[4] += ev_time(lambda: P.pkm_value_sgd(cdims, FW_LR, V, sc, dyc,
+                                                               workspace=bws, stream=side))
+        stage_ms /= args.steps
+    clk = clocks.stop()
+    vals = torch.tensor([graph_ms, eager_ms], device=dev, dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    graph_ms, eager_ms = (float(v) for v in vals.tolist())
+    if rank != 0:
+        return None
+
+    pk = _peaks()
+    sel = FW_CHUNK * cfg.h * cfg.k
+    per_launch = {"query": 1, "subkey_scores": 1, "candidate_topk": 1, "gather_bag": nch,
+                  "value_sgd": nch}
+    # algorithmic bytes over the sequence (the bag and the write are HBM-bound)
+    alg = {
+        "gather_bag": nch * (sel * cfg.d_v * 4 + FW_CHUNK * cfg.d_v * 4 + sel * 8),
+        "value_sgd": U_tot * cfg.d_v * 8 + nch * (FW_CHUNK * cfg.d_v * 4 + sel * 8),
+    }
+    tc = cfg.dtype == "bf16"       # tensor-core query and scoring (q as hi + lo: 2 passes)
+    flops = {"query": 2.0 * cfg.N * cfg.d_in * cfg.h * cfg.dk,
+             "subkey_scores": (2 if tc else 1) * 2.0 * cfg.N * cfg.h * (cfg.C1 + cfg.C2) *
+             cfg.dk / 2}
+    # fp32 CUDA-core peak: 148 SMs x 128 FMA lanes x 2 flops x max SM clock
+    fp32_peak = 148 * 128 * 2 * (clk.get("sm_max_mhz") or 1965) * 1e6 / 1e12
+    dom_i = int(np.argmax(stage_ms))
+    dom = names[dom_i]
+    launch_ms = stage_ms[dom_i] / per_launch[dom]
+    if dom in alg:
+        ach = alg[dom] / (stage_ms[dom_i] * 1e-3) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm"],
+                "unit": "GB/s", "frac": round(ach / pk["hbm"], 4), "traffic": None,
+                "algorithmic_bytes": int(alg[dom] / per_launch[dom]), "peak_source": pk["src"]}
+    elif dom in flops:
+        ach = flops[dom] / (stage_ms[dom_i] * 1e-3) / 1e12
+        peak = pk["bf16"] if tc else round(fp32_peak, 1)
+        roof = {"kernel": dom, "bound": "tensor" if tc else "alu", "achieved": round(ach, 2),
+                "peak": peak, "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+                "algorithmic_flops": flops[dom],
+                "peak_source": pk["src"] if tc else "fp32 FMA lanes x max SM clock"}
+    else:
+        roof = {"kernel": dom, "bound": "latency", "achieved": None, "peak": None, "unit": None,
+                "frac": None, "traffic": None}
+    roof["ms_per_launch"] = round(float(launch_ms), 4)
+
+    # e2e: the sequence's inputs from pinned host memory, every read back to the host
+    xh, tgh = x.cpu().pin_memory(), tg.cpu().pin_memory()
+    yh = torch.empty(cfg.N, cfg.d_v).pin_memory()
+    with torch.cuda.stream(side):
+        def e2e():
+            x.copy_(xh, non_blocking=True)
+            tg.copy_(tgh, non_blocking=True)
+            graph.replay()
+            yh.copy_(y, non_blocking=True)
+        e2e()
+        e2e_ms = timed(e2e)
+    del graph
+
+    out = {
+        "metric": FW_METRIC,
+        "value": round(cfg.N * world / (graph_ms * 1e-3), 1),
+        "unit": "tokens/s (read + write, whole sequence)",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(graph_ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if cfg.dtype == "f32" else "bf16 inputs, f32 value table",
+        "data": "synthetic (seeded; 64 input clusters, N(0,1) targets)",
+        "config": dict(_cfg_json(cfg), chunk=FW_CHUNK, lr=FW_LR,
+                       parallelism=f"replicas{world}" if world > 1 else "single"),
+        "eager": {"ms": round(eager_ms, 4), "value": round(cfg.N * world / (eager_ms * 1e-3), 1)},
+        "stage_ms_per_sequence": {n: round(float(v), 4) for n, v in zip(names, stage_ms)},
+        "distinct_rows_per_chunk": round(U_tot / nch, 1),
+        "roofline": roof,
+        "clocks": clk,
+        "gpu_launches": int(launches_per_step * args.steps),
+        "input_gen_s": round(gen_s, 1),
+        "e2e": {"value": round(cfg.N * world / (e2e_ms * 1e-3), 1),
+                "unit": "tokens/s (host x and targets in, y out)",
+                "h2d_bytes_per_step": int(xh.numel() * xh.element_size() +
+                                          tgh.numel() * tgh.element_size()),
+                "d2h_bytes_per_step": int(cfg.N * cfg.d_v * 4), "ms": round(e2e_ms, 4)},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        v, n, thr = time_oracle_fastweight(cfg, inp, tg_np, args.cpu_seconds)
+        out["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s (read + write)",
+                               "cores": thr, "kind": "oracle",
+                               "sample": f"{n} tokens, 32-token chunks of the same sequence; fp64 "
+                                         f"numpy oracle, brute force over all {cfg.K} keys"}
+    return out
+
+
+# ---------------------------------------------------------------- decode latency
+DECODE_METRIC = "PKM decode forward latency (us/call) at |K|=1024², h=4, k=32, d=1600"
+
+
+def run_decode(args, cfg, rank, world, dist):
+    """Decode-shaped forward calls (N = 1, 8, 64 tokens) against the full table: the
+    four forward steps captured once per size into a CUDA graph and replayed, timed per
+    call with the L2 warm (back-to-back replays) and flushed (a 256 MiB write before
+    each call, outside its events); the eager call sequence beside it."""
+    import torch
+
+    from product_key_memory_pkm_b200 import build as B
+    from product_key_memory_pkm_b200 import pkm as P
+
+    if not os.path.exists(B.LIB):
+        B.build()
+    P.load()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    sizes = (1, 8, 64)
+    inp = make_inputs(cfg.with_(N=max(sizes)), seed=0, with_dy=False)
+    bf = torch.bfloat16
+    x_all = torch.from_numpy(inp["x"]).to(bf).to(dev)
+    Wq = torch.from_numpy(inp["Wq"]).to(bf).to(dev)
+    bn = torch.from_numpy(inp["bn"]).to(dev)
+    sub = torch.from_numpy(inp["subkeys"]).to(bf).to(dev)
+    V = torch.from_numpy(inp["values"]).to(bf).to(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    side = torch.cuda.Stream(device=dev)
+    reps = max(50, args.steps * 20)
+    clocks = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    clocks.start()
+    res, launches = {}, 0
+    with torch.cuda.stream(side):
+        for n in sizes:
+            dims = P.Dims.from_config(cfg, N=n)
+            saved = P.alloc_saved(dims, with_qhat=False)
+            x = x_all[:n].contiguous()
+            y = torch.empty(n, cfg.d_v, device=dev)
+
+            def call():
+                P.pkm_forward(dims, x, Wq, bn, sub, V, y, saved, stream=side)
+            for _ in range(args.warmup):
+                call()
+            side.synchronize()
+            l0 = P.pkm_launch_count()
+            call()
+            side.synchronize()
+            per_call = P.pkm_launch_count() - l0
+
+            def burst(fn):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(side)
+                for _ in range(reps):
+                    fn()
+                b.record(side)
+                b.synchronize()
+                return 1e3 * a.elapsed_time(b) / reps
+
+            def cold(fn):
+                out = []
+                for _ in range(args.steps * 5):
+                    a, b = (torch.cuda.Event(enable_timing=True),
+                            torch.cuda.Event(enable_timing=True))
+                    flush.zero_()
+                    a.record(side)
+                    fn()
+                    b.record(side)
+                    b.synchronize()
+                    out.append(1e3 * a.elapsed_time(b))
+                return float(np.median(out))
+            eager_warm = burst(call)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                call()
+            g.replay()
+            graph_warm = burst(g.replay)
+            graph_cold = cold(g.replay)
+            eager_cold = cold(call)
+            launches += per_call * (reps + args.steps * 5) * 2
+            assert P.pkm_check_status(side) == P.PKM_OK
+            # bytes a call must move: Wq and the sub-keys once, then n*h*k value rows
+            alg = (cfg.h * cfg.dk * cfg.d_in * 2 + cfg.h * (cfg.C1 + cfg.C2) * cfg.dk // 2 * 2 +
+                   n * cfg.h * cfg.k * cfg.d_v * 2 + n * (cfg.d_in * 2 + cfg.d_v * 4))
+            res[n] = {"graph_us_l2_warm": round(graph_warm, 2),
+                      "graph_us_l2_flushed": round(graph_cold, 2),
+                      "eager_us_l2_warm": round(eager_warm, 2),
+                      "eager_us_l2_flushed": round(eager_cold, 2),
+                      "kernels_per_call": int(per_call), "algorithmic_bytes": int(alg)}
+            del g
+    clk = clocks.stop()
+    if rank != 0:
+        return None
+    pk = _peaks()
+    top = res[max(sizes)]
+    ach = top["algorithmic_bytes"] / (top["graph_us_l2_flushed"] * 1e-6) / 1e9
+    return {
+        "metric": DECODE_METRIC, "value": res[1]["graph_us_l2_flushed"],
+        "unit": "us per forward call at N=1 (CUDA graph, L2 flushed)",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(res[1]["graph_us_l2_flushed"] / 1e3, 5),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; tables random-init)",
+        "config": dict(_cfg_json(cfg), N_tokens=list(sizes), parallelism="single"),
+        "per_size": {str(n): v for n, v in res.items()},
+        "roofline": {"kernel": "forward call at N=64 (graph, flushed)", "bound": "hbm",
+                     "achieved": round(ach, 1), "peak": pk["hbm"], "unit": "GB/s",
+                     "frac": round(ach / pk["hbm"], 4), "traffic": None,
+                     "algorithmic_bytes": top["algorithmic_bytes"], "peak_source": pk["src"]},
+        "clocks": clk, "gpu_launches": int(launches),
+    }
 
 
 def run_stage(args, cfg, dims, saved, P, st, step, flush, names, env):
@@ -441,6 +787,10 @@ def main():
                              "value_grad", "query_grad"],
                     help="time one stage alone (per-op benchmark / profiling target)")
     ap.add_argument("--tokens", type=int, default=None, help="override the token count")
+    ap.add_argument("--bf16-q", action="store_true",
+                    help="single-pass scoring (PKM_F_BF16_Q: q rounded to bf16 for the scores)")
+    ap.add_argument("--decode", action="store_true",
+                    help="decode-shaped forward latency (N = 1, 8, 64) on the workload's table")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -462,7 +812,9 @@ def main():
             tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
             dist = tdist
         try:
-            out = run_b200(args, cfg, rank, world, dist)
+            run = (run_decode if args.decode else
+                   run_fastweight if cfg.name == FASTWEIGHT.name else run_b200)
+            out = run(args, cfg, rank, world, dist)
         finally:
             if dist is not None:
                 dist.destroy_process_group()

@@ -29,7 +29,7 @@
  *       Wq       [h*dk][d_in]         bf16 (fp32 with PKM_F_FP32)  Linear weight, out x in
  *       bn       [4][h*dk]            fp32: running mean, running var, gamma, beta
  *       subkeys  [h][C1+C2][dk/2]     bf16 (fp32 with PKM_F_FP32)  rows [0,C1) = C, [C1,C1+C2) = C'
- *       values   [C1*C2][d_v]         bf16 (fp32 with PKM_F_FP32)
+ *       values   [C1*C2][d_v]         bf16 (fp32 with PKM_F_FP32 or PKM_F_VALUES_FP32)
  *       y, dy    [N][d_v]             fp32
  *   - Gradients of parameters ACCUMULATE (+=) into the caller's buffers; dx is
  *     overwritten.  A NULL gradient pointer skips that gradient.
@@ -64,6 +64,13 @@ typedef enum {
 /* flags */
 #define PKM_F_FP32 0x1u  /* x, Wq, subkeys, values are fp32 (CUDA-core kernels) */
 #define PKM_F_SIMT 0x2u  /* bf16 storage, but CUDA-core kernels instead of tensor cores */
+#define PKM_F_VALUES_FP32 0x4u  /* values (the table) fp32; x, Wq, subkeys stay bf16 */
+/* Single-pass scoring: the sub-key scores (so the selection and the weights) take q
+ * rounded to bf16 instead of q = hi + lo (half the scoring MMA work; scores move by up
+ * to half a bf16 ulp of q per coordinate, ~2e-4 relative).  The sub-key gradient
+ * uses the same rounded q; the query gradient passes the rounding unchanged.  bf16
+ * storage only (PKM_ERR_INVALID_ARG with PKM_F_FP32). */
+#define PKM_F_BF16_Q 0x8u
 
 typedef struct {
   int64_t N;          /* tokens */
@@ -166,6 +173,91 @@ pkm_status pkm_candidate_topk(const pkm_dims* d, const pkm_saved* saved, void* s
 /* F4 (pkm_gather_bag): y[t] = sum_h sum_j w * V[idx]; y overwritten. */
 pkm_status pkm_gather_bag(const pkm_dims* d, const void* values, const int32_t* idx,
                           const float* w, float* y, void* stream);
+
+/* ---- training-time pieces ("Meta AI 可扩展内存层" sections 6.1, 6.3, 6.4, 11.2) ---- */
+
+/* Value-gradient stage with a compact (sparse-rows) result instead of the dense table:
+ * num_rows (device int, written) = U, the number of distinct selected rows;
+ * rows_out[u] (ascending) = the u-th distinct row and dvalues_rows[u][:] = its gradient
+ * sum over selections (overwritten) for u < U.  Capacity: min(N*h*k, C1*C2) rows.
+ * dw [N][h][k] as in pkm_value_grad (NULL: not returned).  Moves d_v*(2 or 4) bytes of
+ * V and d_v*4 of result per distinct row, against d_v*(2 or 4) + 8 for the dense form.
+ * Workspace: pkm_workspace_bytes(d, PKM_BWD). */
+pkm_status pkm_value_grad_rows(const pkm_dims* d, const void* values, const pkm_saved* saved,
+                               const float* dy, float* dw, int32_t* rows_out,
+                               float* dvalues_rows, int* num_rows, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* Lazy Adam on the selected rows only: with g_r = sum over the selections of row r of
+ * w * dy[t] (the value gradient of sum_t dy[t] . y[t]),
+ *   m_r <- beta1 m_r + (1 - beta1) g_r,   v_r <- beta2 v_r + (1 - beta2) g_r^2,
+ *   V_r <- V_r - lr * (m_r / (1 - beta1^step)) / (sqrt(v_r / (1 - beta2^step)) + eps);
+ * rows not selected, and their m and v, are left unchanged.  values, m, v: [C1*C2][d_v]
+ * fp32, updated in place (fp32 tables required: PKM_F_FP32 or PKM_F_VALUES_FP32).
+ * step >= 1 is the caller's global step count.  0 <= beta < 1, eps > 0.
+ * Workspace: pkm_workspace_bytes(d, PKM_BWD). */
+pkm_status pkm_value_adam(const pkm_dims* d, float lr, float beta1, float beta2, float eps,
+                          int64_t step, float* values, float* m, float* v,
+                          const pkm_saved* saved, const float* dy, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/* Hit monitoring: slot_hits[r] += number of selections of value row r ([C1*C2] int32);
+ * subkey_hits[h][i] += number of winners of head h whose first-half sub-key is i, and
+ * [h][C1 + j] those whose second-half sub-key is j ([h][C1+C2] int32).  Either may be
+ * NULL.  Reads idx [N][h][k] (saved->idx of a forward). */
+pkm_status pkm_hit_counts(const pkm_dims* d, const int32_t* idx, int32_t* slot_hits,
+                          int32_t* subkey_hits, void* stream);
+
+/* ---- fast-weight memory: chunked read-then-write ----
+ * "Fast-weight Product Key Memory", sections 2.2 and 3 (test-time training): the
+ * value table is a fast weight.  The N tokens of one sequence are cut into
+ * consecutive chunks of `chunk` tokens (the last may be shorter).  Each chunk first
+ * READS (F1..F4 with the current table, y of its tokens written), then WRITES: one
+ * SGD step of rate `lr` on the value rows the chunk selected, descending
+ *     L_c = sum_{t in chunk} 1/2 ||y[t] - target[t]||^2,
+ * i.e. V[r] -= lr * sum_{selections (t, h, j) of r} w[t][h][j] * (y[t] - target[t]),
+ * duplicates combined before the single write of each row (deterministic).  The
+ * next chunk reads what this one wrote; queries, keys and BatchNorm stay fixed.
+ *   d        d->N is the sequence length; the value table must be fp32 (PKM_F_FP32,
+ *            or PKM_F_VALUES_FP32 beside bf16 x, Wq, subkeys), otherwise
+ *            PKM_ERR_UNSUPPORTED.
+ *   chunk    >= 1 tokens per chunk.   lr: finite.
+ *   mode     0: target[t] = targets[t], targets [N][d_v] fp32 (required);
+ *            PKM_FW_LOOKAHEAD: target[t] = x[t + 1], the next token's input, in
+ *            x's storage type (needs d_in == d_v; `targets` is ignored and may be
+ *            NULL); the last token of
+ *            the sequence has no target and adds nothing to the loss.
+ *   values   [C1*C2][d_v] fp32, updated IN PLACE.
+ *   y        [N][d_v] fp32 out: every chunk's read.
+ *   workspace  pkm_fastweight_workspace_bytes(d, chunk, mode) bytes, 256-byte aligned.
+ * Everything is enqueued on `stream` with no host synchronisation, so the whole loop
+ * can be captured into one CUDA graph. */
+/* The write step alone: one sparse SGD step on the value rows `saved` selected,
+ *     V[r] -= lr * sum_{selections (t, h, j) of r} w[t][h][j] * dy[t],
+ * i.e. rate lr on the value gradient of sum_t dy[t] . y[t], applied only to touched
+ * rows, duplicates combined before the single write of each row (deterministic).
+ *   values  [C1*C2][d_v] fp32, updated IN PLACE (PKM_F_FP32 or PKM_F_VALUES_FP32
+ *           required, otherwise PKM_ERR_UNSUPPORTED).   saved: idx and w are read.   dy: [N][d_v] fp32.
+ *   workspace  pkm_workspace_bytes(d, PKM_BWD) bytes. */
+pkm_status pkm_value_sgd(const pkm_dims* d, float lr, float* values, const pkm_saved* saved,
+                         const float* dy, void* workspace, size_t workspace_bytes, void* stream);
+
+#define PKM_FW_LOOKAHEAD 0x1u
+/* Strategy overrides (results are the same; for tests and tuning).  By default every
+ * chunk's writes are sorted before the loop -- in shared memory, one CTA per chunk, when a
+ * chunk has at most 16384 selections, else by one global radix sort while
+ * (number of chunks) * C1*C2 < 2^31 -- and otherwise each chunk selects and sorts on its
+ * own.  PKM_FW_SORT_GLOBAL asks for the global sort (per-chunk steps when it does not
+ * fit); PKM_FW_PER_CHUNK for the per-chunk steps. */
+#define PKM_FW_SORT_GLOBAL 0x2u
+#define PKM_FW_PER_CHUNK 0x4u
+/* Workspace bytes of pkm_fastweight_chunks for these dims, chunk size and mode bits. */
+size_t pkm_fastweight_workspace_bytes(const pkm_dims* d, int64_t chunk, uint32_t mode);
+pkm_status pkm_fastweight_chunks(const pkm_dims* d, int64_t chunk, float lr, uint32_t mode,
+                                 const void* x, const void* Wq, const float* bn,
+                                 const void* subkeys, float* values, const float* targets,
+                                 float* y, void* workspace, size_t workspace_bytes,
+                                 void* stream);
 
 /* Synchronises `stream`, then reads and clears the device status word of the
  * current device.  Returns PKM_OK, PKM_ERR_DEVICE_TIMEOUT, PKM_ERR_DEVICE_INDEX or

@@ -13,6 +13,8 @@
 //          sqrt(var + eps); d gamma, d beta by deterministic two-stage reduction
 //          dC[i] += sum over (t, a) choosing i of g * q_half[t]  (sorted segments)
 //   B7     dx = dq_pre Wq,  dWq += dq_pre^T x
+#include <cmath>
+
 #include "k_sort.cuh"
 #include "tc_common.cuh"
 
@@ -138,7 +140,8 @@ __global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
     const int* __restrict__ seg, const int* __restrict__ U_ptr, const int32_t* __restrict__ seg_row,
     const int32_t* __restrict__ ents, const TV* __restrict__ V, const float* __restrict__ ws_sorted,
     const float* __restrict__ dy, float* __restrict__ dV, float* __restrict__ dw, int hk, int d_v,
-    int64_t K, int* status) {
+    int64_t K, int* status, float* __restrict__ dVc, int32_t* __restrict__ rows_out,
+    int* __restrict__ U_out) {
   constexpr int E = VecT<TV>::E;
   extern __shared__ __align__(16) unsigned char b3_smem[];
   __shared__ int s_t[2][kB3Batch];
@@ -178,6 +181,7 @@ __global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
       bulk_g2s(buf + ((vbytes + 15u) & ~15u), dV + (int64_t)r * d_v, dbytes, &bar[b], pol_stream);
   };
 
+  if (U_out && blockIdx.x == 0 && tid == 0) *U_out = U;
   uint32_t phase_bits = 0u;    // bit b: parity of buffer b's next phase
   uint32_t pending_bits = 0u;  // bit b: a copy into buffer b not yet waited for (thread 0)
   if ((int)blockIdx.x < U) {
@@ -240,7 +244,9 @@ __global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
     const TV* sV = reinterpret_cast<const TV*>(b3_smem + (size_t)b * slot_bytes);
     const float* sD = reinterpret_cast<const float*>(b3_smem + (size_t)b * slot_bytes +
                                                      ((vbytes + 15u) & ~15u));
-    float* dVr = dV ? dV + (int64_t)r * d_v : nullptr;
+    // dense table (+=) or compact rows (u-th distinct row, overwritten)
+    float* dVr = dV ? dV + (int64_t)r * d_v : (dVc ? dVc + (int64_t)u * d_v : nullptr);
+    if (rows_out && tid == 0) rows_out[u] = r;
     for (int cb = 0; cb < nvec; cb += kB3Threads * CH) {
       float v[CH][E], acc[CH][E];
 #pragma unroll
@@ -248,7 +254,7 @@ __global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
         const int vec = cb + tid + kB3Threads * c;
         if (vec < nvec) {
           smem_vals<TV>(sV + (int64_t)vec * E, v[c]);
-          if (dVr) {
+          if (dV) {  // accumulate onto the dense table's row (staged with V)
 #pragma unroll
             for (int e4 = 0; e4 < E / 4; ++e4) {
               const float4 a4 = *reinterpret_cast<const float4*>(sD + (int64_t)vec * E + 4 * e4);
@@ -337,8 +343,99 @@ __global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
   }
 }
 
+// Fast-weight write ("Fast-weight Product Key Memory", section 2.2: the chunk's
+// reconstruction loss is descended by sparse gradient steps on the selected value
+// rows): for each distinct row r, V[r] <- V[r] - lr * sum_{selections e of r}
+// w_e * dy[t_e].  One 256-thread CTA per row (grid-stride), thread j owning float4
+// columns j, j + 256, ...; the row's selections are taken in row order (stable
+// sort), four at a time so four dy lines are in flight.  One writer per row: no
+// atomics, deterministic.  fp32 tables only.
+//
+// kAdam: the same pass applies lazy Adam instead ("Meta AI 可扩展内存层" section 6.3:
+// optimiser state only for rows that received a gradient): with g the row's gradient,
+// m <- b1 m + (1 - b1) g, v <- b2 v + (1 - b2) g^2, V <- V - lr (m / bc1) / (sqrt(v / bc2)
+// + eps), bc = 1 - beta^step; m and v are fp32 tables shaped like V.
+constexpr int kSgdThreads = 256;
+
+struct AdamArgs {
+  float* m;
+  float* v;
+  float b1, b2, eps, inv_bc1, inv_bc2;
+};
+
+//
+// The segments may carry composite keys (chunk * K + row, sorted once for a whole
+// sequence): then `bounds` gives this chunk's segment range [bounds[0], bounds[1]) and
+// the row is key - key_base.  Without bounds the range is [0, U) and key_base is 0.
+template <bool kAdam>
+__global__ void __launch_bounds__(kSgdThreads) rows_step_kernel(
+    const int* __restrict__ seg, const int* __restrict__ U_ptr,
+    const int32_t* __restrict__ seg_row, const int32_t* __restrict__ ents,
+    const float* __restrict__ ws_sorted, const float* __restrict__ dy, float* __restrict__ V,
+    float lr, int hk, int d_v, int64_t K, int* status, const int* __restrict__ bounds,
+    int64_t key_base, AdamArgs ad) {
+  const int u0 = bounds ? bounds[0] : 0;
+  const int u1 = bounds ? bounds[1] : *U_ptr;
+  const int nvec = d_v / 4;
+  for (int u = u0 + blockIdx.x; u < u1; u += gridDim.x) {
+    const int64_t r = (int64_t)seg_row[u] - key_base;
+    if (r < 0 || r >= K) {
+      if (threadIdx.x == 0) set_status(status, kDevIndex);
+      continue;
+    }
+    const int p0 = seg[u], p1 = seg[u + 1];
+    float4* Vr = reinterpret_cast<float4*>(V + (int64_t)r * d_v);
+    for (int c = threadIdx.x; c < nvec; c += kSgdThreads) {
+      const float4 v = Vr[c];
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      int q = p0;
+      for (; q + 4 <= p1; q += 4) {
+        float4 d[4];
+        float wt[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          wt[i] = ws_sorted[q + i];
+          d[i] = reinterpret_cast<const float4*>(dy + (int64_t)(ents[q + i] / hk) * d_v)[c];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc.x = fmaf(wt[i], d[i].x, acc.x); acc.y = fmaf(wt[i], d[i].y, acc.y);
+          acc.z = fmaf(wt[i], d[i].z, acc.z); acc.w = fmaf(wt[i], d[i].w, acc.w);
+        }
+      }
+      for (; q < p1; ++q) {
+        const float wt = ws_sorted[q];
+        const float4 d = reinterpret_cast<const float4*>(dy + (int64_t)(ents[q] / hk) * d_v)[c];
+        acc.x = fmaf(wt, d.x, acc.x); acc.y = fmaf(wt, d.y, acc.y);
+        acc.z = fmaf(wt, d.z, acc.z); acc.w = fmaf(wt, d.w, acc.w);
+      }
+      if constexpr (kAdam) {
+        float4* Mr = reinterpret_cast<float4*>(ad.m + r * d_v);
+        float4* Sr = reinterpret_cast<float4*>(ad.v + r * d_v);
+        float4 m = Mr[c], s = Sr[c];
+        const float g[4] = {acc.x, acc.y, acc.z, acc.w};
+        float* mm = &m.x;
+        float* ss = &s.x;
+        float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          mm[i] = fmaf(ad.b1, mm[i], (1.f - ad.b1) * g[i]);
+          ss[i] = fmaf(ad.b2, ss[i], (1.f - ad.b2) * g[i] * g[i]);
+          vv[i] -= lr * (mm[i] * ad.inv_bc1) / (sqrtf(ss[i] * ad.inv_bc2) + ad.eps);
+        }
+        Mr[c] = m;
+        Sr[c] = s;
+        Vr[c] = make_float4(vv[0], vv[1], vv[2], vv[3]);
+      } else {
+        Vr[c] = make_float4(fmaf(-lr, acc.x, v.x), fmaf(-lr, acc.y, v.y),
+                            fmaf(-lr, acc.z, v.z), fmaf(-lr, acc.w, v.w));
+      }
+    }
+  }
+}
+
 inline size_t value_rows_smem(const Plan& p) {
-  const size_t vb = ((size_t)p.d_v * (p.fp32 ? 4 : 2) + 15) & ~size_t(15);
+  const size_t vb = ((size_t)p.d_v * (p.vfp32 ? 4 : 2) + 15) & ~size_t(15);
   return 2 * (vb + (size_t)p.d_v * 4);
 }
 
@@ -497,7 +594,8 @@ template <bool kSplitQ, int MAXC>
 __global__ void __launch_bounds__(256) subkey_grad_kernel(
     const int* __restrict__ seg, const int* __restrict__ U_ptr, const int32_t* __restrict__ rows,
     const int32_t* __restrict__ ents, const float* __restrict__ gsub, const void* __restrict__ q,
-    float* __restrict__ dsub, int64_t N, int h, int dk, int C1, int C2, int k, int* status) {
+    float* __restrict__ dsub, int64_t N, int h, int dk, int C1, int C2, int k, int* status,
+    float lo_scale) {
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -538,7 +636,7 @@ __global__ void __launch_bounds__(256) subkey_grad_kernel(
             bf16x8_to_f32(*reinterpret_cast<const uint4*>(qb + off), f);
             bf16x8_to_f32(*reinterpret_cast<const uint4*>(qb + plane + off), lo);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] += lo[e];
+            for (int e = 0; e < 8; ++e) f[e] += lo_scale * lo[e];
           } else {
             float4 u4 = *reinterpret_cast<const float4*>(static_cast<const float*>(q) + off);
             f[0] = u4.x; f[1] = u4.y; f[2] = u4.z; f[3] = u4.w;
@@ -658,7 +756,7 @@ static BwdCtx bwd_ctx(const Plan& p, void* ws, float* dw_out) {
 
 cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved& s,
                               const float* dy, float* dV, float* dw_out, void* ws,
-                              cudaStream_t st) {
+                              cudaStream_t st, float* dVc, int32_t* rows_out, int* U_out) {
   const int64_t E1 = p.N * p.h * p.k;
   BwdCtx c = bwd_ctx(p, ws, dw_out);
   sort::RadixBuffers& rb = c.rb;
@@ -680,7 +778,7 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
 
   // B3: value rows
   {
-    const int E = p.fp32 ? 4 : 8;
+    const int E = p.vfp32 ? 4 : 8;
     const int nvec = p.d_v / E;
     const int blocks = p.sm_count * 6;
     const size_t smem = value_rows_smem(p);
@@ -693,10 +791,9 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
       return e;                                                                              \
     value_rows_kernel<TV, CHV><<<blocks, kB3Threads, smem, st>>>(                            \
         seg, U, seg_row, ents_sorted, static_cast<const TV*>(values), w_sorted, dy, dV, dw,  \
-        hk,                                                                                  \
-        p.d_v, p.K, p.status);                                                               \
+        hk, p.d_v, p.K, p.status, dVc, rows_out, U_out);                                     \
   } while (0)
-    if (p.fp32) {
+    if (p.vfp32) {
       if (nvec <= kB3Threads) PKM_B3(float, 1);
       else PKM_B3(float, 2);
     } else {
@@ -710,6 +807,308 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
   }
 
   return cudaSuccess;
+}
+
+cudaError_t launch_value_sgd(const Plan& p, float* values, const pkm_saved& s, const float* dy,
+                             float lr, void* ws, cudaStream_t st) {
+  const int64_t E1 = p.N * p.h * p.k;
+  BwdCtx c = bwd_ctx(p, ws, nullptr);
+  cudaError_t e;
+  const int32_t *rows_sorted, *ents_sorted;
+  e = sort::radix_sort(s.idx, E1, bits_for(p.K - 1), c.rb, &rows_sorted, &ents_sorted, st);
+  if (e != cudaSuccess) return e;
+  e = sort::segments(rows_sorted, E1, c.seg, c.U, c.rb.bsum, st, c.seg_row, ents_sorted, s.w,
+                     c.w_sorted);
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = std::min<int64_t>(E1, (int64_t)p.sm_count * 8);
+  rows_step_kernel<false><<<(unsigned)blocks, kSgdThreads, 0, st>>>(
+      c.seg, c.U, c.seg_row, ents_sorted, c.w_sorted, dy, values, lr, p.h * p.k, p.d_v, p.K,
+      p.status, nullptr, 0, AdamArgs{});
+  PKM_COUNT(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_value_adam(const Plan& p, float* values, float* m, float* v,
+                              const pkm_saved& s, const float* dy, float lr, float beta1,
+                              float beta2, float eps, int64_t step, void* ws, cudaStream_t st) {
+  const int64_t E1 = p.N * p.h * p.k;
+  BwdCtx c = bwd_ctx(p, ws, nullptr);
+  cudaError_t e;
+  const int32_t *rows_sorted, *ents_sorted;
+  e = sort::radix_sort(s.idx, E1, bits_for(p.K - 1), c.rb, &rows_sorted, &ents_sorted, st);
+  if (e != cudaSuccess) return e;
+  e = sort::segments(rows_sorted, E1, c.seg, c.U, c.rb.bsum, st, c.seg_row, ents_sorted, s.w,
+                     c.w_sorted);
+  if (e != cudaSuccess) return e;
+  AdamArgs ad{m, v, beta1, beta2, eps,
+              (float)(1.0 / (1.0 - std::pow((double)beta1, (double)step))),
+              (float)(1.0 / (1.0 - std::pow((double)beta2, (double)step)))};
+  const int64_t blocks = std::min<int64_t>(E1, (int64_t)p.sm_count * 8);
+  rows_step_kernel<true><<<(unsigned)blocks, kSgdThreads, 0, st>>>(
+      c.seg, c.U, c.seg_row, ents_sorted, c.w_sorted, dy, values, lr, p.h * p.k, p.d_v, p.K,
+      p.status, nullptr, 0, ad);
+  PKM_COUNT(1);
+  return cudaGetLastError();
+}
+
+// Hit monitoring ("Meta AI 可扩展内存层" sections 6.4 and 11.2): one thread per
+// selection adds 1 to its slot and to the two sub-keys of its head.  Integer atomics:
+// the counts do not depend on the order.
+namespace {
+__global__ void hit_counts_kernel(const int32_t* __restrict__ idx, int64_t E, int h, int k,
+                                  int C1, int C2, int64_t K, int32_t* __restrict__ slot,
+                                  int32_t* __restrict__ sub, int* status) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < E;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t r = idx[e];
+    if (r < 0 || r >= K) {
+      set_status(status, kDevIndex);
+      continue;
+    }
+    if (slot) atomicAdd(slot + r, 1);
+    if (sub) {
+      const int hh = (int)((e / k) % h);
+      int32_t* row = sub + (int64_t)hh * (C1 + C2);
+      atomicAdd(row + r / C2, 1);
+      atomicAdd(row + C1 + r % C2, 1);
+    }
+  }
+}
+}  // namespace
+
+cudaError_t launch_hit_counts(const Plan& p, const int32_t* idx, int32_t* slot, int32_t* sub,
+                              cudaStream_t st) {
+  const int64_t E = p.N * p.h * p.k;
+  const int64_t blocks = std::min<int64_t>((E + 255) / 256, (int64_t)p.sm_count * 16);
+  hit_counts_kernel<<<(unsigned)blocks, 256, 0, st>>>(idx, E, p.h, p.k, p.C1, p.C2, p.K, slot,
+                                                      sub, p.status);
+  PKM_COUNT(1);
+  return cudaGetLastError();
+}
+
+// ---- a whole sequence's writes sorted at once (the selection does not read the table)
+namespace {
+
+__global__ void fw_keys_kernel(const int32_t* __restrict__ idx, int64_t E, int hk, int64_t chunk,
+                               int64_t K, int32_t* __restrict__ keys, int* status) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= E) return;
+  const int64_t c = (e / hk) / chunk;
+  int64_t r = idx[e];
+  if (r < 0 || r >= K) {
+    set_status(status, kDevIndex);
+    r = 0;
+  }
+  keys[e] = (int32_t)(c * K + r);
+}
+
+// bounds[c] = first segment whose key is >= c * K (lower bound), c in [0, nch]
+__global__ void fw_bounds_kernel(const int32_t* __restrict__ seg_key, const int* __restrict__ U_ptr,
+                                 int nch, int64_t K, int* __restrict__ bounds) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c > nch) return;
+  const int U = *U_ptr;
+  const int64_t want = (int64_t)c * K;
+  int lo = 0, hi = U;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if ((int64_t)seg_key[mid] < want) lo = mid + 1;
+    else hi = mid;
+  }
+  bounds[c] = lo;
+}
+
+// One CTA per chunk sorts the chunk's selections by value row in shared memory (the
+// selections of a chunk are contiguous) and writes the chunk's segment table at a fixed
+// stride: seg[u] (position of the u-th distinct row's first selection), seg_row[u],
+// seg[U_c] = n_c, U_c; ents[i] (global selection id) and w_sorted[i] in row order.
+// Keys are (row << 32 | local selection id), so a bitonic network over unique keys
+// gives the stable order (rows ascending, selections of a row in id order).
+constexpr int kFwSortThreads = 1024, kFwSortMax = 16384;
+
+__global__ void __launch_bounds__(kFwSortThreads) fw_chunk_sort_kernel(
+    const int32_t* __restrict__ idx, const float* __restrict__ w, int64_t N, int64_t chunk,
+    int hk, int64_t K, int stride, int npow2, int* __restrict__ seg,
+    int32_t* __restrict__ seg_row, int32_t* __restrict__ ents, float* __restrict__ w_sorted,
+    int* __restrict__ U_out, int* status) {
+  extern __shared__ __align__(16) unsigned long long fw_keys[];
+  __shared__ int warp_tot[kFwSortThreads / 32];
+  const int c = blockIdx.x, tid = threadIdx.x;
+  const int64_t t0 = (int64_t)c * chunk;
+  const int64_t nt = (N - t0 < chunk) ? N - t0 : chunk;
+  const int n = (int)(nt * hk);
+  const int64_t e0 = t0 * hk;
+  const int64_t base = (int64_t)c * stride;
+  for (int i = tid; i < npow2; i += kFwSortThreads) {
+    unsigned long long key = ~0ull;
+    if (i < n) {
+      int64_t r = idx[e0 + i];
+      if (r < 0 || r >= K) {
+        set_status(status, kDevIndex);
+        r = 0;
+      }
+      key = ((unsigned long long)r << 32) | (unsigned)i;
+    }
+    fw_keys[i] = key;
+  }
+  __syncthreads();
+  for (int size = 2; size <= npow2; size <<= 1) {
+    for (int half = size >> 1; half > 0; half >>= 1) {
+      for (int j = tid; j < (npow2 >> 1); j += kFwSortThreads) {
+        const int lo = 2 * j - (j & (half - 1));
+        const int hi = lo + half;
+        const bool up = (lo & size) == 0;
+        const unsigned long long a = fw_keys[lo], b = fw_keys[hi];
+        if ((a > b) == up) {
+          fw_keys[lo] = b;
+          fw_keys[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // segment starts: block-wide exclusive scan of the start flags over thread-owned runs
+  const int per = (n + kFwSortThreads - 1) / kFwSortThreads;
+  const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
+  int cnt = 0;
+  for (int i = i0; i < i1; ++i)
+    cnt += (i == 0 || (fw_keys[i] >> 32) != (fw_keys[i - 1] >> 32)) ? 1 : 0;
+  const int lane = tid & 31, wid = tid >> 5;
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_tot[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    int v = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
+    }
+    warp_tot[lane] = v;  // inclusive over warps
+  }
+  __syncthreads();
+  int u = incl - cnt + (wid ? warp_tot[wid - 1] : 0);
+  for (int i = i0; i < i1; ++i) {
+    const unsigned long long key = fw_keys[i];
+    const int32_t row = (int32_t)(key >> 32);
+    if (i == 0 || row != (int32_t)(fw_keys[i - 1] >> 32)) {
+      seg[base + u] = i;
+      seg_row[base + u] = row;
+      ++u;
+    }
+    const int64_t e = e0 + (int64_t)(unsigned)(key & 0xffffffffu);
+    ents[base + i] = (int32_t)e;
+    w_sorted[base + i] = w[e];
+  }
+  if (tid == kFwSortThreads - 1) {
+    const int U = warp_tot[kFwSortThreads / 32 - 1];
+    seg[base + U] = n;
+    U_out[c] = U;
+  }
+}
+
+}  // namespace
+
+bool fw_presort_fits(const Plan& p, int64_t chunk) {
+  const int64_t nch = (p.N + chunk - 1) / chunk;
+  return nch * p.K < ((int64_t)1 << 31);
+}
+
+cudaError_t launch_fw_presort(const Plan& p, int64_t chunk, const int32_t* idx, const float* w,
+                              int32_t* keys, int* bounds, void* ws, cudaStream_t st) {
+  const int64_t E1 = p.N * p.h * p.k;
+  const int64_t nch = (p.N + chunk - 1) / chunk;
+  BwdCtx c = bwd_ctx(p, ws, nullptr);
+  fw_keys_kernel<<<(unsigned)((E1 + 255) / 256), 256, 0, st>>>(idx, E1, p.h * p.k, chunk, p.K,
+                                                               keys, p.status);
+  PKM_COUNT(1);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int32_t *keys_sorted, *ents_sorted;
+  e = sort::radix_sort(keys, E1, bits_for(nch * p.K - 1), c.rb, &keys_sorted, &ents_sorted, st);
+  if (e != cudaSuccess) return e;
+  e = sort::segments(keys_sorted, E1, c.seg, c.U, c.rb.bsum, st, c.seg_row, ents_sorted, w,
+                     c.w_sorted);
+  if (e != cudaSuccess) return e;
+  fw_bounds_kernel<<<(unsigned)((nch + 1 + 255) / 256), 256, 0, st>>>(c.seg_row, c.U, (int)nch,
+                                                                      p.K, bounds);
+  PKM_COUNT(1);
+  return cudaGetLastError();
+}
+
+bool fw_chunk_sort_fits(const Plan& p, int64_t chunk) {
+  return std::min<int64_t>(chunk, p.N) * p.h * p.k <= kFwSortMax;
+}
+
+size_t fw_chunk_sort_bytes(const Plan& p, int64_t chunk) {
+  const int64_t nch = (p.N + chunk - 1) / chunk;
+  const int64_t stride = std::min<int64_t>(chunk, p.N) * p.h * p.k + 1;
+  // seg, seg_row, ents, w_sorted at `stride` per chunk, then U per chunk
+  return (size_t)(4 * 4 * nch * stride + 4 * nch);
+}
+
+cudaError_t launch_fw_chunk_sort(const Plan& p, int64_t chunk, const int32_t* idx, const float* w,
+                                 void* buf, cudaStream_t st) {
+  const int64_t nch = (p.N + chunk - 1) / chunk;
+  const int n_max = (int)(std::min<int64_t>(chunk, p.N) * p.h * p.k);
+  const int stride = n_max + 1;
+  int npow2 = 1;
+  while (npow2 < n_max) npow2 <<= 1;
+  int* seg = static_cast<int*>(buf);
+  int32_t* seg_row = seg + nch * stride;
+  int32_t* ents = seg_row + nch * stride;
+  float* w_sorted = reinterpret_cast<float*>(ents + nch * stride);
+  int* U = reinterpret_cast<int*>(w_sorted + nch * stride);
+  const size_t smem = (size_t)npow2 * 8;
+  cudaError_t e;
+  if (smem > 48 * 1024 &&
+      (e = cudaFuncSetAttribute(fw_chunk_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem)) != cudaSuccess)
+    return e;
+  fw_chunk_sort_kernel<<<(unsigned)nch, kFwSortThreads, smem, st>>>(
+      idx, w, p.N, chunk, p.h * p.k, p.K, stride, npow2, seg, seg_row, ents, w_sorted, U,
+      p.status);
+  PKM_COUNT(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fw_chunk_write(const Plan& p, int64_t chunk, int64_t ci, const void* buf,
+                                  const float* dy, float* values, float lr, cudaStream_t st) {
+  const int64_t nch = (p.N + chunk - 1) / chunk;
+  const int n_max = (int)(std::min<int64_t>(chunk, p.N) * p.h * p.k);
+  const int64_t stride = n_max + 1;
+  const int* seg = static_cast<const int*>(buf);
+  const int32_t* seg_row = seg + nch * stride;
+  const int32_t* ents = seg_row + nch * stride;
+  const float* w_sorted = reinterpret_cast<const float*>(ents + nch * stride);
+  const int* U = reinterpret_cast<const int*>(w_sorted + nch * stride);
+  const int64_t n_c = std::min<int64_t>(chunk, p.N - ci * chunk) * p.h * p.k;
+  const int64_t blocks = std::min<int64_t>(n_c, (int64_t)p.sm_count * 8);
+  const int64_t o = ci * stride;
+  rows_step_kernel<false><<<(unsigned)blocks, kSgdThreads, 0, st>>>(
+      seg + o, U + ci, seg_row + o, ents + o, w_sorted + o, dy, values, lr, p.h * p.k, p.d_v,
+      p.K, p.status, nullptr, 0, AdamArgs{});
+  PKM_COUNT(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fw_write(const Plan& p, int64_t chunk, int64_t ci, const int* bounds,
+                            const float* dy, float* values, float lr, void* ws, cudaStream_t st) {
+  BwdCtx c = bwd_ctx(p, ws, nullptr);
+  const int32_t* ents_sorted =
+      sort::radix_sorted_vals(c.rb, bits_for(((p.N + chunk - 1) / chunk) * p.K - 1));
+  const int64_t n_c = std::min<int64_t>(chunk, p.N - ci * chunk);
+  const int64_t blocks = std::min<int64_t>(n_c * p.h * p.k, (int64_t)p.sm_count * 8);
+  rows_step_kernel<false><<<(unsigned)blocks, kSgdThreads, 0, st>>>(
+      c.seg, c.U, c.seg_row, ents_sorted, c.w_sorted, dy, values, lr, p.h * p.k, p.d_v, p.K,
+      p.status, bounds + ci, ci * p.K, AdamArgs{});
+  PKM_COUNT(1);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, const float* bn,
@@ -797,11 +1196,11 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
     const int E = p.fp32 ? 4 : 8;
     const int nv = p.half / E;
     if (p.fp32) {
-      if (nv <= 32) subkey_grad_kernel<false, 1><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status);
-      else subkey_grad_kernel<false, 4><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status); PKM_COUNT(1);
+      if (nv <= 32) subkey_grad_kernel<false, 1><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status, p.bf16q ? 0.f : 1.f);
+      else subkey_grad_kernel<false, 4><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status, p.bf16q ? 0.f : 1.f); PKM_COUNT(1);
     } else {
-      if (nv <= 32) subkey_grad_kernel<true, 1><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status);
-      else subkey_grad_kernel<true, 4><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status); PKM_COUNT(1);
+      if (nv <= 32) subkey_grad_kernel<true, 1><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status, p.bf16q ? 0.f : 1.f);
+      else subkey_grad_kernel<true, 4><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status, p.bf16q ? 0.f : 1.f); PKM_COUNT(1);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

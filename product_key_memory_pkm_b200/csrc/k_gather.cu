@@ -30,12 +30,33 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   return r;
 }
 
-template <typename TV, int UNROLL>
+// Fast-weight read (kResid): the same bag, and beside y the reconstruction residual
+// dy[t] = y[t] - tgt[t] (tgt rows tgt_ld elements apart, fp32 or bf16) for
+// t < n_target, 0 after it.
+struct Resid {
+  const void* tgt;
+  int64_t tgt_ld, n_target;
+  float* dy;
+  bool tgt_bf16;
+};
+
+__device__ __forceinline__ float4 load_target4(const Resid& r, int64_t t, int64_t col) {
+  if (r.tgt_bf16) {
+    const uint2 u = *reinterpret_cast<const uint2*>(
+        static_cast<const __nv_bfloat16*>(r.tgt) + t * r.tgt_ld + col);
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                       __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+  }
+  return *reinterpret_cast<const float4*>(static_cast<const float*>(r.tgt) + t * r.tgt_ld + col);
+}
+
+template <typename TV, int UNROLL, bool kResid = false>
 __global__ void __launch_bounds__(256) gather_bag_kernel(const TV* __restrict__ V,
                                                          const int32_t* __restrict__ idx,
                                                          const float* __restrict__ w,
                                                          float* __restrict__ y, int64_t N, int hk,
-                                                         int d_v, int64_t K, int* status) {
+                                                         int d_v, int64_t K, int* status,
+                                                         Resid res = Resid{}) {
   constexpr int E = Vec<TV>::kElems;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   int32_t* s_idx = reinterpret_cast<int32_t*>(smem_raw);
@@ -92,6 +113,18 @@ __global__ void __launch_bounds__(256) gather_bag_kernel(const TV* __restrict__ 
     float4* yo = reinterpret_cast<float4*>(y + t * d_v + (int64_t)c * E);
 #pragma unroll
     for (int e = 0; e < E; e += 4) yo[e / 4] = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+    if constexpr (kResid) {
+      float4* d = reinterpret_cast<float4*>(res.dy + t * d_v + (int64_t)c * E);
+      const bool has = t < res.n_target;
+#pragma unroll
+      for (int e = 0; e < E; e += 4) {
+        const float4 tv = has ? load_target4(res, t, (int64_t)c * E + e)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        d[e / 4] = has ? make_float4(acc[e] - tv.x, acc[e + 1] - tv.y, acc[e + 2] - tv.z,
+                                     acc[e + 3] - tv.w)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
   }
 }
 
@@ -101,7 +134,7 @@ cudaError_t launch_gather(const Plan& p, const void* values, const int32_t* idx,
                           float* y, cudaStream_t st) {
   const int hk = p.h * p.k;
   const size_t smem = (size_t)hk * 8;
-  if (p.fp32) {
+  if (p.vfp32) {
     const int nvec = p.d_v / 4;
     const int threads = min(256, ((nvec + 31) / 32) * 32);
     gather_bag_kernel<float, 8><<<(unsigned)p.N, threads, smem, st>>>(
@@ -112,6 +145,20 @@ cudaError_t launch_gather(const Plan& p, const void* values, const int32_t* idx,
     gather_bag_kernel<__nv_bfloat16, 8><<<(unsigned)p.N, threads, smem, st>>>(
         static_cast<const __nv_bfloat16*>(values), idx, w, y, p.N, hk, p.d_v, p.K, p.status); PKM_COUNT(1);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_resid(const Plan& p, const float* values, const int32_t* idx,
+                                const float* w, float* y, const void* tgt, bool tgt_bf16,
+                                int64_t tgt_ld, int64_t n_target, float* dy, cudaStream_t st) {
+  const int hk = p.h * p.k;
+  const size_t smem = (size_t)hk * 8;
+  const int nvec = p.d_v / 4;
+  const int threads = min(256, ((nvec + 31) / 32) * 32);
+  gather_bag_kernel<float, 8, true><<<(unsigned)p.N, threads, smem, st>>>(
+      values, idx, w, y, p.N, hk, p.d_v, p.K, p.status,
+      Resid{tgt, tgt_ld, n_target, dy, tgt_bf16});
+  PKM_COUNT(1);
   return cudaGetLastError();
 }
 

@@ -15,11 +15,13 @@ namespace {
 
 constexpr int TT = 64, TC = 64, BK = 16, TPB = 256;
 
+// lo_scale = 0 drops the lo plane: q rounded to bf16 (single-pass scoring)
 template <bool kSplitQ>
-__device__ __forceinline__ float load_q(const void* q, int64_t plane, int64_t off) {
+__device__ __forceinline__ float load_q(const void* q, int64_t plane, int64_t off,
+                                        float lo_scale) {
   if constexpr (kSplitQ) {
     const __nv_bfloat16* b = static_cast<const __nv_bfloat16*>(q);
-    return __bfloat162float(b[off]) + __bfloat162float(b[plane + off]);
+    return __bfloat162float(b[off]) + lo_scale * __bfloat162float(b[plane + off]);
   } else {
     return static_cast<const float*>(q)[off];
   }
@@ -30,7 +32,8 @@ __global__ void __launch_bounds__(TPB) scores_topk_simt(const void* __restrict__
                                                         const TS* __restrict__ sub,
                                                         float* __restrict__ sub_s,
                                                         int32_t* __restrict__ sub_i, int64_t N,
-                                                        int h, int dk, int C1, int C2, int k) {
+                                                        int h, int dk, int C1, int C2, int k,
+                                                        float lo_scale) {
   __shared__ __align__(16) float Qs[BK][TT + 4];
   __shared__ __align__(16) float Cs[BK][TC + 4];
   __shared__ float Ssc[TT][TC + 1];
@@ -65,7 +68,7 @@ __global__ void __launch_bounds__(TPB) scores_topk_simt(const void* __restrict__
         int r = e / BK, dd = e % BK;
         int64_t t = t0 + r;
         float v = 0.f;
-        if (t < N && d0 + dd < half) v = load_q<kSplitQ>(q, plane, t * hq + qoff + d0 + dd);
+        if (t < N && d0 + dd < half) v = load_q<kSplitQ>(q, plane, t * hq + qoff + d0 + dd, lo_scale);
         Qs[dd][r] = v;
         int c = c0 + r;
         float u = 0.f;
@@ -129,7 +132,8 @@ cudaError_t dispatch_km(const Plan& p, const void* subkeys, const void* q, float
   const TS* sub = static_cast<const TS*>(subkeys);
 #define PKM_LAUNCH(KMV)                                                                     \
   scores_topk_simt<kSplitQ, TS, KMV><<<grid, TPB, 0, st>>>(q, sub, sub_s, sub_i, p.N, p.h, \
-                                                           p.dk, p.C1, p.C2, p.k)
+                                                           p.dk, p.C1, p.C2, p.k,       \
+                                                           p.bf16q ? 0.f : 1.f)
   if (p.k <= 8)
     PKM_LAUNCH(8);
   else if (p.k <= 16)

@@ -114,6 +114,13 @@ inline int64_t radix_hist_len(int64_t n) { return (int64_t)(1 << kRadixMaxBits) 
 cudaError_t radix_sort(const int32_t* keys_src, int64_t n, int bits_total, const RadixBuffers& b,
                        const int32_t** keys_out, const int32_t** vals_out, cudaStream_t st);
 
+// Where radix_sort(bits_total) leaves the sorted payloads (*vals_out of that call).
+inline const int32_t* radix_sorted_vals(const RadixBuffers& b, int bits_total) {
+  if (bits_total < 1) bits_total = 1;
+  const int passes = (bits_total + kRadixMaxBits - 1) / kRadixMaxBits;
+  return (passes & 1) ? b.valsA : b.valsB;
+}
+
 // Segment table of a sorted key array: seg[u] = first position of the u-th
 // distinct key, seg[U] = n, *U_out = U, and (when seg_key is not null)
 // seg_key[u] = that key.

@@ -177,6 +177,7 @@ struct ScoresProb {
     int32_t* sub_i;
     int64_t N;
     int h, dk, half, C1, C2, k, m_tiles, nkh;  // nkh = half / 64
+    int planes;  // 2: q_hi and q_lo K-blocks; 1: q_hi only (q rounded to bf16)
   };
   struct EpiState {
     float thr;
@@ -189,7 +190,7 @@ struct ScoresProb {
     const int C = (hs & 1) ? P.C2 : P.C1;
     return (C + kBN - 1) / kBN;
   }
-  __device__ static int num_kblocks(const Params& P) { return 2 * P.nkh; }
+  __device__ static int num_kblocks(const Params& P) { return P.planes * P.nkh; }
 
   __device__ static void load(const Params& P, const CUtensorMap* A0, const CUtensorMap* A1,
                               const CUtensorMap* B, const CUtensorMap*, int u, int c, int kb, void* sa, void* sb,
@@ -402,7 +403,8 @@ cudaError_t launch_scores_tc(const Plan& p, const void* subkeys, const void* q, 
 #define PKM_SC(KMV)                                                                   \
   do {                                                                                \
     typename ScoresProb<KMV>::Params P{p.status, sub_s, sub_i, p.N, p.h, p.dk, p.half, \
-                                       p.C1, p.C2, p.k, m_tiles, p.half / kBK};       \
+                                       p.C1, p.C2, p.k, m_tiles, p.half / kBK,        \
+                                       p.bf16q ? 1 : 2};                             \
     return launch_tc<ScoresProb<KMV>>(thi, tlo, tb, P, nunits, p.sm_count, st);      \
   } while (0)
   if (p.k <= 8) PKM_SC(8);

@@ -138,13 +138,14 @@ struct DsubProb {
     float* part;  // [kSplits][2h][Cp][half]
     int64_t N, Np;
     int h, dk, half, C1, C2, Cp, m_tiles, n_tiles, nkt, kper;  // nkt = Np / 64
+    int npass;  // 3: G_hi Q_hi, G_hi Q_lo, G_lo Q_hi; 2: without G_hi Q_lo (q rounded)
   };
   struct EpiState {};
   __device__ static int num_units(const Params& P) {
     return kSplits * 2 * P.h * P.m_tiles * P.n_tiles;
   }
   __device__ static int num_chunks(const Params&, int) { return 1; }
-  __device__ static int num_kblocks(const Params& P) { return 3 * P.kper; }
+  __device__ static int num_kblocks(const Params& P) { return P.npass * P.kper; }
   __device__ static void decode(const Params& P, int u, int& sp, int& hs, int& mt, int& nt) {
     const int per = P.m_tiles * P.n_tiles;
     sp = u / (2 * P.h * per);
@@ -159,7 +160,7 @@ struct DsubProb {
     int sp, hs, mt, nt;
     decode(P, u, sp, hs, mt, nt);
     const int hh = hs >> 1, s = hs & 1;
-    const int pass = kb / P.kper;
+    const int pass = (P.npass == 2 && kb >= P.kper) ? 2 : kb / P.kper;
     const int kk = sp * P.kper + kb % P.kper;  // 64-token block
     const int gplane = pass == 2 ? 1 : 0;    // G_hi Q_hi, G_hi Q_lo, G_lo Q_hi
     const int qplane = pass == 1 ? 1 : 0;
@@ -326,6 +327,7 @@ cudaError_t launch_subgrad_tc(const Plan& p, const float* gsub, const int32_t* s
     P.n_tiles = (p.half + kBN - 1) / kBN;
     P.nkt = (int)(Np / kBK);
     P.kper = (P.nkt + kSplits - 1) / kSplits;
+    P.npass = p.bf16q ? 2 : 3;
     const int units = kSplits * hs2 * P.m_tiles * P.n_tiles;
     if ((e = launch_tc<DsubProb>(ta, ta, tb, P, units, p.sm_count, st)) != cudaSuccess) return e;
     const int64_t total = (int64_t)p.h * (p.C1 + p.C2) * p.half;

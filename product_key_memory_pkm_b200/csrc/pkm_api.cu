@@ -1,4 +1,5 @@
 // C ABI entry points: host-side validation, plan, launch sequencing.
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -53,7 +54,9 @@ pkm_status validate_dims(const pkm_dims* d) {
       d->score_scale > 3.0e38f)
     return PKM_ERR_INVALID_ARG;
   if ((int64_t)d->C1 * d->C2 >= ((int64_t)1 << 31)) return PKM_ERR_INVALID_ARG;
-  if (d->flags & ~(PKM_F_FP32 | PKM_F_SIMT)) return PKM_ERR_INVALID_ARG;
+  if (d->flags & ~(PKM_F_FP32 | PKM_F_SIMT | PKM_F_VALUES_FP32 | PKM_F_BF16_Q))
+    return PKM_ERR_INVALID_ARG;
+  if ((d->flags & PKM_F_BF16_Q) && (d->flags & PKM_F_FP32)) return PKM_ERR_INVALID_ARG;
   const bool fp32 = d->flags & PKM_F_FP32;
   if (d->dk % 2) return PKM_ERR_INVALID_ARG;
   if (d->d_in % 8 || d->d_v % 8) return PKM_ERR_INVALID_ARG;
@@ -82,7 +85,9 @@ Plan make_plan(const pkm_dims* d, int dev) {
   p.eps = d->bn_eps;
   p.scale = d->score_scale;
   p.fp32 = d->flags & PKM_F_FP32;
+  p.vfp32 = p.fp32 || (d->flags & PKM_F_VALUES_FP32);
   p.simt = p.fp32 || (d->flags & PKM_F_SIMT);
+  p.bf16q = d->flags & PKM_F_BF16_Q;
   p.sm_count = g_sm_count[dev];
   p.status = g_status_ptr[dev];
   return p;
@@ -173,6 +178,7 @@ size_t pkm_workspace_bytes(const pkm_dims* d, int which) {
   p.N = d->N; p.d_in = d->d_in; p.h = d->h; p.dk = d->dk; p.half = d->dk / 2;
   p.C1 = d->C1; p.C2 = d->C2; p.k = d->k; p.d_v = d->d_v; p.hq = d->h * d->dk;
   p.K = (int64_t)d->C1 * d->C2; p.fp32 = d->flags & PKM_F_FP32;
+  p.vfp32 = p.fp32 || (d->flags & PKM_F_VALUES_FP32);
   return backward_workspace_bytes(p);
 }
 
@@ -292,6 +298,250 @@ pkm_status pkm_query_grad(const pkm_dims* d, const void* x, const void* Wq, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return cuda_status(launch_query_grad(p, x, Wq, bn, subkeys, *saved, dx, dWq, dbn, dsubkeys,
                                        const_cast<float*>(dw), workspace, st));
+}
+
+// ---------------------------------------------------------------- fast weights
+}  // extern "C"
+
+namespace pkm {
+namespace {
+
+// The selection (query, scores, candidates) does not read the value table, so when the
+// (chunk, row) keys of a whole sequence fit in 31 bits the loop selects and sorts every
+// chunk's writes in one pass up front and each chunk then only reads (bag + residual)
+// and writes (SGD on its rows).  Otherwise each chunk runs the whole sequence of steps.
+// How the chunk loop sorts its writes.  The selection (query, scores, candidates) does
+// not read the value table, so the whole sequence is selected in one pass up front and
+// each chunk's writes are sorted before the loop; each chunk then only reads (bag +
+// residual) and writes (SGD on its rows).
+//   kChunkSort  a chunk has at most 16384 selections: one CTA per chunk sorts them in
+//               shared memory (one launch for all chunks);
+//   kPresort    otherwise, while chunks * K fits in 31 bits: one global radix sort of
+//               every selection by (chunk, row);
+//   kPerChunk   otherwise each chunk runs the whole sequence of steps itself.
+enum FwMode { kChunkSort, kPresort, kPerChunk };
+
+Plan fw_shape(const pkm_dims* d) {
+  Plan p{};
+  p.N = d->N; p.h = d->h; p.k = d->k; p.K = (int64_t)d->C1 * d->C2;
+  return p;
+}
+
+bool fw_presort_fits(const pkm_dims* d, int64_t chunk) {
+  const int64_t nch = (d->N + chunk - 1) / chunk;
+  return nch * ((int64_t)d->C1 * d->C2) < ((int64_t)1 << 31);
+}
+
+// The fastest strategy that fits, unless the caller's mode bits ask for another one
+// (PKM_FW_SORT_GLOBAL falls back to the per-chunk steps when its keys do not fit).
+FwMode fw_mode(const pkm_dims* d, int64_t chunk, uint32_t mode) {
+  if (mode & PKM_FW_PER_CHUNK) return kPerChunk;
+  const bool presort = fw_presort_fits(d, chunk);
+  if (mode & PKM_FW_SORT_GLOBAL) return presort ? kPresort : kPerChunk;
+  if (fw_chunk_sort_fits(fw_shape(d), chunk)) return kChunkSort;
+  return presort ? kPresort : kPerChunk;
+}
+
+// Workspace of the chunk loop (each part 256-byte aligned): the saved forward state and
+// the residual of the whole sequence (one chunk's for kPerChunk), then the sort state:
+// the per-chunk segment tables (kChunkSort), or the sort keys, per-chunk segment bounds
+// and the value stage's sort buffers.
+struct FwLayout {
+  FwMode mode;
+  size_t q, sub_s, sub_i, idx, w, dy, keys, bounds, csort, bwd, total;
+};
+
+FwLayout fw_layout(const pkm_dims* d, int64_t chunk, uint32_t mode) {
+  FwLayout L{};
+  L.mode = fw_mode(d, chunk, mode);
+  pkm_dims dc = *d;
+  if (L.mode == kPerChunk) dc.N = std::min<int64_t>(chunk, d->N);
+  const int64_t nch = (d->N + chunk - 1) / chunk;
+  const auto up = [](size_t v) { return (v + 255) & ~size_t(255); };
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t r = o;
+    o += up(bytes);
+    return r;
+  };
+  L.q = take(pkm_saved_bytes(&dc, PKM_SAVED_Q));
+  L.sub_s = take(pkm_saved_bytes(&dc, PKM_SAVED_SUB_S));
+  L.sub_i = take(pkm_saved_bytes(&dc, PKM_SAVED_SUB_I));
+  L.idx = take(pkm_saved_bytes(&dc, PKM_SAVED_IDX));
+  L.w = take(pkm_saved_bytes(&dc, PKM_SAVED_W));
+  L.dy = take((size_t)dc.N * d->d_v * 4);
+  L.keys = take(L.mode == kPresort ? (size_t)4 * dc.N * d->h * d->k : 0);
+  L.bounds = take(L.mode == kPresort ? (size_t)4 * (nch + 1) : 0);
+  L.csort = take(L.mode == kChunkSort ? fw_chunk_sort_bytes(fw_shape(d), chunk) : 0);
+  L.bwd = take(L.mode == kChunkSort ? 0 : pkm_workspace_bytes(&dc, PKM_BWD));
+  L.total = o;
+  return L;
+}
+
+pkm_status validate_fw(const pkm_dims* d, int64_t chunk, float lr, uint32_t mode) {
+  PKM_TRY(validate_dims(d));
+  if (chunk < 1 || !(lr == lr) || lr > 3.0e38f || lr < -3.0e38f) return PKM_ERR_INVALID_ARG;
+  if (mode & ~(PKM_FW_LOOKAHEAD | PKM_FW_SORT_GLOBAL | PKM_FW_PER_CHUNK))
+    return PKM_ERR_INVALID_ARG;
+  if ((mode & PKM_FW_LOOKAHEAD) && d->d_in != d->d_v) return PKM_ERR_INVALID_ARG;
+  if (!(d->flags & (PKM_F_FP32 | PKM_F_VALUES_FP32))) return PKM_ERR_UNSUPPORTED;
+  return PKM_OK;
+}
+
+}  // namespace
+}  // namespace pkm
+
+extern "C" {
+
+pkm_status pkm_value_sgd(const pkm_dims* d, float lr, float* values, const pkm_saved* saved,
+                         const float* dy, void* workspace, size_t workspace_bytes, void* stream) {
+  PKM_TRY(validate_fw(d, 1, lr, 0));
+  if (d->N == 0) return PKM_OK;
+  PKM_NEED(values); PKM_NEED(dy);
+  if (!saved) return PKM_ERR_INVALID_ARG;
+  PKM_NEED(saved->idx); PKM_NEED(saved->w);
+  PKM_TRY(check_workspace(pkm_workspace_bytes(d, PKM_BWD), workspace, workspace_bytes));
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_value_sgd(p, values, *saved, dy, lr, workspace, st));
+}
+
+size_t pkm_fastweight_workspace_bytes(const pkm_dims* d, int64_t chunk, uint32_t mode) {
+  if (validate_dims(d) != PKM_OK || chunk < 1 || d->N == 0) return 0;
+  return fw_layout(d, chunk, mode).total;
+}
+
+pkm_status pkm_fastweight_chunks(const pkm_dims* d, int64_t chunk, float lr, uint32_t mode,
+                                 const void* x, const void* Wq, const float* bn,
+                                 const void* subkeys, float* values, const float* targets,
+                                 float* y, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  PKM_TRY(validate_fw(d, chunk, lr, mode));
+  if (d->N == 0) return PKM_OK;
+  const bool lookahead = mode & PKM_FW_LOOKAHEAD;
+  PKM_NEED(x); PKM_NEED(Wq); PKM_NEED(bn); PKM_NEED(subkeys); PKM_NEED(values); PKM_NEED(y);
+  if (!lookahead) PKM_NEED(targets);
+  const FwLayout L = fw_layout(d, chunk, mode);
+  PKM_TRY(check_workspace(L.total, workspace, workspace_bytes));
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  pkm_saved s{};
+  s.q = ws + L.q;
+  s.qhat = nullptr;
+  s.sub_s = reinterpret_cast<float*>(ws + L.sub_s);
+  s.sub_i = reinterpret_cast<int32_t*>(ws + L.sub_i);
+  s.idx = reinterpret_cast<int32_t*>(ws + L.idx);
+  s.w = reinterpret_cast<float*>(ws + L.w);
+  float* dy = reinterpret_cast<float*>(ws + L.dy);
+  const size_t xsz = p.fp32 ? 4 : 2;
+  const char* xb = static_cast<const char*>(x);
+  const int hk = d->h * d->k;
+  const bool tgt_bf16 = lookahead && !p.fp32;
+  // the chunk's residual target: the next input (lookahead) or the caller's targets
+  auto target = [&](int64_t c0, int64_t n, const void** tgt, int64_t* ld, int64_t* nt) {
+    *tgt = lookahead ? static_cast<const void*>(xb + (c0 + 1) * d->d_in * xsz)
+                     : static_cast<const void*>(targets + c0 * d->d_v);
+    *ld = lookahead ? d->d_in : d->d_v;
+    *nt = lookahead ? std::min<int64_t>(n, d->N - 1 - c0) : n;
+  };
+  if (L.mode != kPerChunk) {
+    PKM_TRY(cuda_status(run_query(p, x, Wq, bn, s.q, nullptr, st)));
+    PKM_TRY(cuda_status(run_scores(p, subkeys, s.q, s.sub_s, s.sub_i, st)));
+    PKM_TRY(cuda_status(launch_candidates(p, s.sub_s, s.sub_i, s.idx, s.w, st)));
+    int* bounds = reinterpret_cast<int*>(ws + L.bounds);
+    if (L.mode == kChunkSort)
+      PKM_TRY(cuda_status(launch_fw_chunk_sort(p, chunk, s.idx, s.w, ws + L.csort, st)));
+    else
+      PKM_TRY(cuda_status(launch_fw_presort(p, chunk, s.idx, s.w,
+                                            reinterpret_cast<int32_t*>(ws + L.keys), bounds,
+                                            ws + L.bwd, st)));
+    for (int64_t c0 = 0, ci = 0; c0 < d->N; c0 += chunk, ++ci) {
+      Plan pc = p;
+      pc.N = std::min<int64_t>(chunk, d->N - c0);
+      const void* tgt;
+      int64_t ld, nt;
+      target(c0, pc.N, &tgt, &ld, &nt);
+      PKM_TRY(cuda_status(launch_gather_resid(pc, values, s.idx + c0 * hk, s.w + c0 * hk,
+                                              y + c0 * d->d_v, tgt, tgt_bf16, ld, nt,
+                                              dy + c0 * d->d_v, st)));
+      if (L.mode == kChunkSort)
+        PKM_TRY(cuda_status(launch_fw_chunk_write(p, chunk, ci, ws + L.csort, dy, values, lr, st)));
+      else
+        PKM_TRY(cuda_status(launch_fw_write(p, chunk, ci, bounds, dy, values, lr, ws + L.bwd,
+                                            st)));
+    }
+    return PKM_OK;
+  }
+  for (int64_t c0 = 0; c0 < d->N; c0 += chunk) {
+    Plan pc = p;
+    pc.N = std::min<int64_t>(chunk, d->N - c0);
+    const void* xc = xb + c0 * d->d_in * xsz;
+    // read
+    PKM_TRY(cuda_status(run_query(pc, xc, Wq, bn, s.q, nullptr, st)));
+    PKM_TRY(cuda_status(run_scores(pc, subkeys, s.q, s.sub_s, s.sub_i, st)));
+    PKM_TRY(cuda_status(launch_candidates(pc, s.sub_s, s.sub_i, s.idx, s.w, st)));
+    const void* tgt;
+    int64_t ld, nt;
+    target(c0, pc.N, &tgt, &ld, &nt);
+    PKM_TRY(cuda_status(launch_gather_resid(pc, values, s.idx, s.w, y + c0 * d->d_v, tgt,
+                                            tgt_bf16, ld, nt, dy, st)));
+    // write
+    PKM_TRY(cuda_status(launch_value_sgd(pc, values, s, dy, lr, ws + L.bwd, st)));
+  }
+  return PKM_OK;
+}
+
+pkm_status pkm_value_grad_rows(const pkm_dims* d, const void* values, const pkm_saved* saved,
+                               const float* dy, float* dw, int32_t* rows_out,
+                               float* dvalues_rows, int* num_rows, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  PKM_TRY(validate_dims(d));
+  if (d->N == 0) return PKM_OK;
+  PKM_NEED(values); PKM_NEED(dy); PKM_OPT(dw);
+  PKM_NEED(rows_out); PKM_NEED(dvalues_rows);
+  if (!num_rows) return PKM_ERR_INVALID_ARG;
+  if (!saved) return PKM_ERR_INVALID_ARG;
+  PKM_NEED(saved->idx); PKM_NEED(saved->w);
+  PKM_TRY(check_workspace(pkm_workspace_bytes(d, PKM_BWD), workspace, workspace_bytes));
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_value_grad(p, values, *saved, dy, nullptr, dw, workspace, st,
+                                       dvalues_rows, rows_out, num_rows));
+}
+
+pkm_status pkm_value_adam(const pkm_dims* d, float lr, float beta1, float beta2, float eps,
+                          int64_t step, float* values, float* m, float* v,
+                          const pkm_saved* saved, const float* dy, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  PKM_TRY(validate_fw(d, 1, lr, 0));
+  if (!(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f) || !(eps > 0.f) ||
+      eps > 3.0e38f || step < 1)
+    return PKM_ERR_INVALID_ARG;
+  if (d->N == 0) return PKM_OK;
+  PKM_NEED(values); PKM_NEED(m); PKM_NEED(v); PKM_NEED(dy);
+  if (!saved) return PKM_ERR_INVALID_ARG;
+  PKM_NEED(saved->idx); PKM_NEED(saved->w);
+  PKM_TRY(check_workspace(pkm_workspace_bytes(d, PKM_BWD), workspace, workspace_bytes));
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_value_adam(p, values, m, v, *saved, dy, lr, beta1, beta2, eps, step,
+                                       workspace, st));
+}
+
+pkm_status pkm_hit_counts(const pkm_dims* d, const int32_t* idx, int32_t* slot_hits,
+                          int32_t* subkey_hits, void* stream) {
+  PKM_TRY(validate_dims(d));
+  if (d->N == 0 || (!slot_hits && !subkey_hits)) return PKM_OK;
+  PKM_NEED(idx); PKM_OPT(slot_hits); PKM_OPT(subkey_hits);
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_hit_counts(p, idx, slot_hits, subkey_hits, st));
 }
 
 unsigned long long pkm_launch_count(void) { return g_launches.load(); }

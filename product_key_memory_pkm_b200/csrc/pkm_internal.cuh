@@ -52,6 +52,8 @@ struct Plan {
   int64_t K;                                 // C1*C2
   float eps, scale;
   bool fp32;      // fp32 storage
+  bool vfp32;     // fp32 value table (fp32, or bf16 x/Wq/subkeys beside fp32 values)
+  bool bf16q;     // scores (and the sub-key gradient) take q rounded to bf16 (hi plane)
   bool simt;      // CUDA-core kernels for bf16 storage
   int sm_count;
   int* status;    // device status word
@@ -85,9 +87,42 @@ size_t backward_workspace_bytes(const Plan& p);
 // Leading bytes of the backward workspace that the value stage uses when the caller
 // supplies dw (the value stage touches nothing beyond them).
 size_t value_stage_scratch_bytes(const Plan& p);
+// Fast-weight pieces (fp32 tables): the bag plus the residual y - target, and the
+// SGD step on the distinct selected rows.
+cudaError_t launch_gather_resid(const Plan& p, const float* values, const int32_t* idx,
+                                const float* w, float* y, const void* tgt, bool tgt_bf16,
+                                int64_t tgt_ld, int64_t n_target, float* dy, cudaStream_t st);
+cudaError_t launch_value_sgd(const Plan& p, float* values, const pkm_saved& s, const float* dy,
+                             float lr, void* ws, cudaStream_t st);
+// Lazy Adam on the distinct selected rows (m, v: fp32 tables like the values).
+cudaError_t launch_value_adam(const Plan& p, float* values, float* m, float* v,
+                              const pkm_saved& s, const float* dy, float lr, float beta1,
+                              float beta2, float eps, int64_t step, void* ws, cudaStream_t st);
+// Selection counts: slot[r] += selections of row r, sub[h][C1+C2] += winners per sub-key.
+cudaError_t launch_hit_counts(const Plan& p, const int32_t* idx, int32_t* slot, int32_t* sub,
+                              cudaStream_t st);
+// A whole sequence's chunked writes, sorted once by (chunk, row) when chunk count * K
+// fits in 31 bits (fw_presort_fits); then each chunk's write reads its segment range.
+bool fw_presort_fits(const Plan& p, int64_t chunk);
+cudaError_t launch_fw_presort(const Plan& p, int64_t chunk, const int32_t* idx, const float* w,
+                              int32_t* keys, int* bounds, void* ws, cudaStream_t st);
+// Per-chunk sorts in shared memory (one CTA per chunk) when a chunk has at most 16384
+// selections: one launch for every chunk's segment table; the write of chunk ci then
+// reads its own table from `buf` (fw_chunk_sort_bytes bytes).
+bool fw_chunk_sort_fits(const Plan& p, int64_t chunk);
+size_t fw_chunk_sort_bytes(const Plan& p, int64_t chunk);
+cudaError_t launch_fw_chunk_sort(const Plan& p, int64_t chunk, const int32_t* idx, const float* w,
+                                 void* buf, cudaStream_t st);
+cudaError_t launch_fw_chunk_write(const Plan& p, int64_t chunk, int64_t ci, const void* buf,
+                                  const float* dy, float* values, float lr, cudaStream_t st);
+cudaError_t launch_fw_write(const Plan& p, int64_t chunk, int64_t ci, const int* bounds,
+                            const float* dy, float* values, float lr, void* ws, cudaStream_t st);
+// dV (dense table, +=) or, when dVc is given, the compact form: dVc[u] = the gradient of
+// the u-th distinct selected row (ascending), rows_out[u] = that row, *U_out = U.
 cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved& s,
                               const float* dy, float* dV, float* dw_out, void* ws,
-                              cudaStream_t st);
+                              cudaStream_t st, float* dVc = nullptr, int32_t* rows_out = nullptr,
+                              int* U_out = nullptr);
 cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, const float* bn,
                               const void* subkeys, const pkm_saved& s, float* dx, float* dWq,
                               float* dbn, float* dsub, float* dw_out, void* ws, cudaStream_t st);

@@ -45,6 +45,7 @@ class PKMConfig:
     k: int          # top-k per half and in the final selection
     d_v: int        # value width
     dtype: str = "bf16"     # storage of x, Wq, subkeys, values: "bf16" or "f32"
+    value_dtype: str = ""   # "f32": an fp32 value table beside bf16 x, Wq, subkeys
     bn_eps: float = 1e-5
     score_scale: float = 1.0
     clustered: int = 0      # >0: x drawn around this many centres (duplicate-heavy)
@@ -52,6 +53,11 @@ class PKMConfig:
     @property
     def K(self) -> int:
         return self.C1 * self.C2
+
+    @property
+    def vdtype(self) -> str:
+        """Storage of the value table."""
+        return self.value_dtype or self.dtype
 
     def with_(self, **kw) -> "PKMConfig":
         return dataclasses.replace(self, **kw)
@@ -65,7 +71,8 @@ FWD_K512 = PKMConfig("pkm_fwd_K512x512_h4_k32_d1024", N=4096, d_in=1024, h=4, dk
 FULL_K1024 = PKMConfig("pkm_fwdbwd_K1024x1024_h4_k32_d1600", N=16384, d_in=1600, h=4,
                        dk=512, C1=1024, C2=1024, k=32, d_v=1600)
 FASTWEIGHT = PKMConfig("fwpkm_chunk512_K1024x1024_h1_k8_d1024", N=4096, d_in=1024, h=1,
-                       dk=512, C1=1024, C2=1024, k=8, d_v=1024, dtype="f32", clustered=64)
+                       dk=512, C1=1024, C2=1024, k=8, d_v=1024, value_dtype="f32",
+                       clustered=64)
 
 CONFIGS = {c.name: c for c in (TINY_FP32, FWD_K512, FULL_K1024, FASTWEIGHT)}
 
@@ -153,7 +160,9 @@ def make_inputs(cfg: PKMConfig, seed: int = 0, with_dy: bool = True,
     else:
         bn = np.stack([np.zeros(hq), np.ones(hq), np.ones(hq), np.zeros(hq)]).astype(np.float32)
     if cfg.dtype == "bf16":
-        x, Wq, sub, V = (_round_bf16(a) for a in (x, Wq, sub, V))
+        x, Wq, sub = (_round_bf16(a) for a in (x, Wq, sub))
+    if cfg.vdtype == "bf16":
+        V = _round_bf16(V)
     out = dict(x=x, Wq=Wq, bn=bn, subkeys=sub, values=V)
     if with_dy:
         out["dy"] = _draw(seed, "dy", cfg.N, cfg.d_v, "normal", 1.0, _rows_per_block(cfg.d_v))

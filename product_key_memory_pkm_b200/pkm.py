@@ -29,14 +29,21 @@ PKM_ERR_DEVICE_INDEX = 6
 
 PKM_F_FP32 = 0x1
 PKM_F_SIMT = 0x2
+PKM_F_VALUES_FP32 = 0x4
+PKM_F_BF16_Q = 0x8
 PKM_FWD, PKM_BWD = 0, 1
+PKM_FW_LOOKAHEAD = 0x1
+PKM_FW_SORT_GLOBAL = 0x2
+PKM_FW_PER_CHUNK = 0x4
 SAVED_FIELDS = ("q", "qhat", "sub_s", "sub_i", "idx", "w")
 
 # every symbol include/pkm.h declares
 EXPORTED = ("pkm_saved_bytes", "pkm_workspace_bytes", "pkm_forward", "pkm_backward", "pkm_query",
             "pkm_subkey_scores", "pkm_candidate_topk", "pkm_gather_bag", "pkm_check_status",
             "pkm_status_string", "pkm_build_info", "pkm_value_grad", "pkm_query_grad",
-            "pkm_launch_count", "pkm_selftest_wait_timeout", "pkm_value_grad_noalloc")
+            "pkm_launch_count", "pkm_selftest_wait_timeout", "pkm_value_grad_noalloc",
+            "pkm_fastweight_workspace_bytes", "pkm_fastweight_chunks", "pkm_value_sgd",
+            "pkm_value_grad_rows", "pkm_value_adam", "pkm_hit_counts")
 
 
 class PKMError(RuntimeError):
@@ -88,6 +95,14 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "pkm_launch_count": (ctypes.c_ulonglong, []),
         "pkm_selftest_wait_timeout": (I, [ctypes.c_uint32, P]),
         "pkm_value_grad_noalloc": (I, [D, P, SV, P, P, P, P]),
+        "pkm_value_sgd": (I, [D, ctypes.c_float, P, SV, P, P, S, P]),
+        "pkm_value_grad_rows": (I, [D, P, SV, P, P, P, P, P, P, S, P]),
+        "pkm_value_adam": (I, [D, ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                               ctypes.c_int64, P, P, P, SV, P, P, S, P]),
+        "pkm_hit_counts": (I, [D, P, P, P, P]),
+        "pkm_fastweight_workspace_bytes": (S, [D, ctypes.c_int64, ctypes.c_uint32]),
+        "pkm_fastweight_chunks": (I, [D, ctypes.c_int64, ctypes.c_float, ctypes.c_uint32, P, P, P,
+                                      P, P, P, P, P, S, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -147,6 +162,8 @@ class Dims:
     @classmethod
     def from_config(cls, cfg, flags: int = 0, N: int | None = None) -> "Dims":
         f = flags | (PKM_F_FP32 if cfg.dtype == "f32" else 0)
+        if cfg.dtype != "f32" and cfg.vdtype == "f32":
+            f |= PKM_F_VALUES_FP32
         return cls(cfg.N if N is None else N, cfg.d_in, cfg.h, cfg.dk, cfg.C1, cfg.C2, cfg.k,
                    cfg.d_v, cfg.bn_eps, cfg.score_scale, f)
 
@@ -210,6 +227,69 @@ def pkm_value_grad_noalloc(dims: Dims, values, saved: dict, dy, dw, dvalues=None
     _check(load().pkm_value_grad_noalloc(ctypes.byref(dims.c()), _ptr(values), ctypes.byref(s),
                                          _ptr(dy), _ptr(dvalues), _ptr(dw), _stream(stream)),
            "pkm_value_grad_noalloc")
+
+
+def pkm_value_sgd(dims: Dims, lr: float, values, saved: dict, dy, workspace=None,
+                  workspace_bytes: int = 0, stream=None) -> None:
+    """values[r] -= lr * (sum of w * dy over the selections of r), in place (fp32)."""
+    s = _saved_c(saved)
+    _check(load().pkm_value_sgd(ctypes.byref(dims.c()), float(lr), _ptr(values), ctypes.byref(s),
+                                _ptr(dy), _ptr(workspace), _ws(workspace, workspace_bytes),
+                                _stream(stream)), "pkm_value_sgd")
+
+
+def pkm_value_grad_rows(dims: Dims, values, saved: dict, dy, rows_out, dvalues_rows, num_rows,
+                        dw=None, workspace=None, workspace_bytes: int = 0, stream=None) -> None:
+    """Compact value gradient: num_rows[0] = U, rows_out[:U] (ascending), dvalues_rows[:U]."""
+    s = _saved_c(saved)
+    _check(load().pkm_value_grad_rows(ctypes.byref(dims.c()), _ptr(values), ctypes.byref(s),
+                                      _ptr(dy), _ptr(dw), _ptr(rows_out), _ptr(dvalues_rows),
+                                      _ptr(num_rows), _ptr(workspace),
+                                      _ws(workspace, workspace_bytes), _stream(stream)),
+           "pkm_value_grad_rows")
+
+
+def pkm_value_adam(dims: Dims, lr: float, beta1: float, beta2: float, eps: float, step: int,
+                   values, m, v, saved: dict, dy, workspace=None, workspace_bytes: int = 0,
+                   stream=None) -> None:
+    """Lazy Adam on the selected value rows (values, m, v fp32, in place)."""
+    s = _saved_c(saved)
+    _check(load().pkm_value_adam(ctypes.byref(dims.c()), float(lr), float(beta1), float(beta2),
+                                 float(eps), int(step), _ptr(values), _ptr(m), _ptr(v),
+                                 ctypes.byref(s), _ptr(dy), _ptr(workspace),
+                                 _ws(workspace, workspace_bytes), _stream(stream)),
+           "pkm_value_adam")
+
+
+def pkm_hit_counts(dims: Dims, idx, slot_hits=None, subkey_hits=None, stream=None) -> None:
+    """slot_hits [C1*C2] int32 and subkey_hits [h][C1+C2] int32 accumulate (+=)."""
+    _check(load().pkm_hit_counts(ctypes.byref(dims.c()), _ptr(idx), _ptr(slot_hits),
+                                 _ptr(subkey_hits), _stream(stream)), "pkm_hit_counts")
+
+
+def pkm_fastweight_workspace_bytes(dims: Dims, chunk: int, mode: int = 0) -> int:
+    return int(load().pkm_fastweight_workspace_bytes(ctypes.byref(dims.c()), int(chunk),
+                                                     int(mode)))
+
+
+def alloc_fastweight_workspace(dims: Dims, chunk: int, mode: int = 0, device="cuda"):
+    import torch
+    return torch.empty(max(pkm_fastweight_workspace_bytes(dims, chunk, mode), 256),
+                       dtype=torch.uint8, device=device)
+
+
+def pkm_fastweight_chunks(dims: Dims, chunk: int, lr: float, x, Wq, bn, subkeys, values, y,
+                          targets=None, lookahead: bool = False, strategy: int = 0,
+                          workspace=None, workspace_bytes: int = 0, stream=None) -> None:
+    """Chunked read-then-write of the fast-weight memory: ``values`` (fp32) is updated
+    in place, ``y`` receives every chunk's read.  ``strategy``: 0, PKM_FW_SORT_GLOBAL or
+    PKM_FW_PER_CHUNK (same results)."""
+    mode = (PKM_FW_LOOKAHEAD if lookahead else 0) | int(strategy)
+    _check(load().pkm_fastweight_chunks(ctypes.byref(dims.c()), int(chunk), float(lr), mode,
+                                        _ptr(x), _ptr(Wq), _ptr(bn), _ptr(subkeys),
+                                        _ptr(values), _ptr(targets), _ptr(y), _ptr(workspace),
+                                        _ws(workspace, workspace_bytes), _stream(stream)),
+           "pkm_fastweight_chunks")
 
 
 def pkm_query_grad(dims: Dims, x, Wq, bn, subkeys, saved: dict, dw, dx=None, dWq=None, dbn=None,

@@ -34,8 +34,10 @@ def to_dev(inp: dict, cfg, device="cuda") -> dict:
     out = {}
     for k, v in inp.items():
         t = torch.from_numpy(np.ascontiguousarray(v, dtype=np.float32))
-        if k in ("x", "Wq", "subkeys", "values"):
+        if k in ("x", "Wq", "subkeys"):
             t = t.to(st)
+        elif k == "values" and cfg.vdtype == "bf16":
+            t = t.to(torch.bfloat16)
         out[k] = t.to(device)
     return out
 
@@ -68,13 +70,16 @@ def gpu_backward(cfg, dims, dev: dict, saved: dict, dy: torch.Tensor, want=("dx"
     return g
 
 
-def oracle_gaps(of: dict, cfg):
-    """Per (t, h): the oracle's ranked scores of the best k+1 keys (unscaled sums)."""
+def oracle_gaps(of: dict, cfg, select: str = "brute"):
+    """Per (t, h): the oracle's ranked scores of the best k+1 keys (unscaled sums).
+    ``select="product"`` takes them by the product-key search (exact, and far cheaper
+    over a million keys)."""
     N = of["s1"].shape[0]
     ranked = np.zeros((N, cfg.h, cfg.k + 1))
+    pick = O.brute_force_topk if select == "brute" else O.product_key_topk
     for t in range(N):
         for hh in range(cfg.h):
-            ii, jj = O.brute_force_topk(of["s1"][t, hh], of["s2"][t, hh], cfg.k + 1)
+            ii, jj = pick(of["s1"][t, hh], of["s2"][t, hh], cfg.k + 1)
             ranked[t, hh] = of["s1"][t, hh, ii] + of["s2"][t, hh, jj]
     return ranked
 

@@ -89,6 +89,7 @@ def _fwd(d, **over):
     (dict(bn_eps=0.0), P.PKM_ERR_INVALID_ARG),
     (dict(score_scale=-1.0), P.PKM_ERR_INVALID_ARG),
     (dict(flags=0x80), P.PKM_ERR_INVALID_ARG),
+    (dict(flags=P.PKM_F_BF16_Q | P.PKM_F_FP32), P.PKM_ERR_INVALID_ARG),   # no q planes
     (dict(N=-1), P.PKM_ERR_INVALID_ARG),
     (dict(C1=65536, C2=65536), P.PKM_ERR_INVALID_ARG),
 ])
@@ -130,6 +131,55 @@ def test_backward_checks_workspace_and_qhat(lib):
     assert rc == P.PKM_ERR_INVALID_ARG      # d gamma needs qhat
 
 
+def test_fastweight_validation(lib):
+    """Host-side checks of the chunked fast-weight entry point."""
+    L = P.load()
+    d = _dims(flags=P.PKM_F_FP32)
+    need = P.pkm_fastweight_workspace_bytes(d, 16)
+    assert need > 0
+    ws = lambda dd, ch, m=0: P.pkm_fastweight_workspace_bytes(dd, ch, m)
+    # the whole sequence is selected and sorted up front: space grows with N ...
+    assert ws(_dims(N=640, flags=P.PKM_F_FP32), 16) > need
+    # ... except for the per-chunk steps: one chunk's worth whatever N is
+    per = P.PKM_FW_PER_CHUNK
+    assert ws(_dims(N=3000, flags=P.PKM_F_FP32), 16, per) == ws(d, 16, per)
+    # the global sort falls back to the per-chunk steps when (chunks x K) overflows 31 bits
+    big = dict(C1=1024, C2=1024, flags=P.PKM_F_FP32)
+    glob = P.PKM_FW_SORT_GLOBAL
+    assert ws(_dims(N=3000, **big), 1, glob) == ws(_dims(N=3000, **big), 1, per)
+    assert ws(_dims(N=2000, **big), 1, glob) > ws(_dims(N=2000, **big), 1, per)
+    assert ws(d, 0) == 0
+
+    def call(dd=d, chunk=16, lr=0.5, mode=0, targets=FAKE, ws=FAKE, wsb=need, values=FAKE):
+        return L.pkm_fastweight_chunks(ctypes.byref(dd.c()), chunk, lr, mode, FAKE, FAKE, FAKE,
+                                       FAKE, values, targets, FAKE, ws, wsb, None)
+
+    assert call(dd=_dims()) == P.PKM_ERR_UNSUPPORTED              # bf16 tables
+    # bf16 inputs beside an fp32 table pass validation (then the workspace check)
+    assert call(dd=_dims(flags=P.PKM_F_VALUES_FP32), ws=None) == P.PKM_ERR_WORKSPACE
+    assert call(chunk=0) == P.PKM_ERR_INVALID_ARG
+    assert call(lr=float("nan")) == P.PKM_ERR_INVALID_ARG
+    assert call(mode=0x8) == P.PKM_ERR_INVALID_ARG
+    assert call(targets=None) == P.PKM_ERR_INVALID_ARG             # explicit targets needed
+    assert call(dd=_dims(d_v=72, flags=P.PKM_F_FP32), mode=P.PKM_FW_LOOKAHEAD,
+                targets=None) == P.PKM_ERR_INVALID_ARG             # lookahead needs d_in == d_v
+    assert call(values=FAKE + 4) == P.PKM_ERR_INVALID_ARG
+    assert call(ws=None) == P.PKM_ERR_WORKSPACE
+    assert call(wsb=need - 1) == P.PKM_ERR_WORKSPACE
+    assert call(dd=_dims(N=0, flags=P.PKM_F_FP32), ws=None, wsb=0) == P.PKM_OK
+    # the write step alone
+    S = ctypes.byref(P._saved_c({f: FAKE for f in P.SAVED_FIELDS}))
+    nb = P.pkm_workspace_bytes(d, P.PKM_BWD)
+    assert L.pkm_value_sgd(ctypes.byref(_dims().c()), 0.5, FAKE, S, FAKE, FAKE, nb,
+                           None) == P.PKM_ERR_UNSUPPORTED
+    assert L.pkm_value_sgd(ctypes.byref(d.c()), float("inf"), FAKE, S, FAKE, FAKE, nb,
+                           None) == P.PKM_ERR_INVALID_ARG
+    assert L.pkm_value_sgd(ctypes.byref(d.c()), 0.5, FAKE, S, None, FAKE, nb,
+                           None) == P.PKM_ERR_INVALID_ARG
+    assert L.pkm_value_sgd(ctypes.byref(d.c()), 0.5, FAKE, S, FAKE, FAKE, nb - 1,
+                           None) == P.PKM_ERR_WORKSPACE
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     import importlib
     mod = importlib.reload(P)
@@ -139,3 +189,37 @@ def test_binding_fails_loudly_without_library(tmp_path):
             mod.load(str(tmp_path / "missing.so"))
     finally:
         importlib.reload(P)
+
+
+def test_training_pieces_validation(lib):
+    L = P.load()
+    d = _dims()
+    d32 = _dims(flags=P.PKM_F_VALUES_FP32)
+    S = ctypes.byref(P._saved_c({f: FAKE for f in P.SAVED_FIELDS}))
+    nb = P.pkm_workspace_bytes(d, P.PKM_BWD)
+    # compact value gradient
+    rows = lambda **kw: L.pkm_value_grad_rows(
+        ctypes.byref(kw.get("d", d).c()), FAKE, S, FAKE, kw.get("dw", None), kw.get("ro", FAKE),
+        kw.get("dvr", FAKE), kw.get("nr", FAKE), FAKE, kw.get("nb", nb), None)
+    assert rows(ro=None) == P.PKM_ERR_INVALID_ARG
+    assert rows(nr=None) == P.PKM_ERR_INVALID_ARG
+    assert rows(dvr=FAKE + 4) == P.PKM_ERR_INVALID_ARG
+    assert rows(nb=nb - 1) == P.PKM_ERR_WORKSPACE
+    assert rows(d=_dims(N=0), ro=None) == P.PKM_OK
+    # lazy Adam
+    adam = lambda **kw: L.pkm_value_adam(
+        ctypes.byref(kw.get("d", d32).c()), 0.01, kw.get("b1", 0.9), kw.get("b2", 0.99),
+        kw.get("eps", 1e-8), kw.get("step", 1), FAKE, FAKE, kw.get("v", FAKE), S, FAKE, FAKE,
+        nb, None)
+    assert adam(d=d) == P.PKM_ERR_UNSUPPORTED          # bf16 table
+    assert adam(b1=1.0) == P.PKM_ERR_INVALID_ARG
+    assert adam(b2=-0.1) == P.PKM_ERR_INVALID_ARG
+    assert adam(eps=0.0) == P.PKM_ERR_INVALID_ARG
+    assert adam(step=0) == P.PKM_ERR_INVALID_ARG
+    assert adam(v=None) == P.PKM_ERR_INVALID_ARG
+    # hit counts
+    hits = lambda **kw: L.pkm_hit_counts(ctypes.byref(kw.get("d", d).c()), kw.get("idx", FAKE),
+                                         kw.get("slot", FAKE), kw.get("sub", FAKE), None)
+    assert hits(idx=None) == P.PKM_ERR_INVALID_ARG
+    assert hits(slot=FAKE + 2) == P.PKM_ERR_INVALID_ARG
+    assert hits(idx=None, slot=None, sub=None) == P.PKM_OK    # nothing asked

@@ -35,14 +35,16 @@ CASES = {
     "one_token": _cfg(N=1),
     "duplicate_heavy": _cfg(N=512, d_in=64, h=1, C1=64, C2=64, k=8, d_v=128, clustered=8),
     "unequal_C_wide_dv": _cfg(N=130, h=1, dk=128, C1=96, C2=40, k=24, d_v=2056),
+    "fp32_values_bf16_rest": _cfg(N=211, value_dtype="f32", d_v=136),
 }
 
 
-def _full_check(cfg, seed=0, flags=0):
-    inp = make_inputs(cfg, seed=seed, random_bn=True)
+def _full_check(cfg, seed=0, flags=0, inp=None, q_bf16=False):
+    if inp is None:
+        inp = make_inputs(cfg, seed=seed, random_bn=True)
     dev = H.to_dev(inp, cfg)
     dims, saved, y = H.gpu_forward(cfg, dev, flags=flags)
-    of = O.forward(inp, cfg)
+    of = O.forward(inp, cfg, q_bf16=q_bf16)
     ranked = H.oracle_gaps(of, cfg)
     idx = saved["idx"].cpu().numpy()
     clean = H.check_indices(idx, of, cfg, ranked)
@@ -80,6 +82,36 @@ def test_end_to_end_parity(name):
 
 def test_simt_flag_path_matches_oracle():
     _full_check(CASES["ragged_multihead_bf16"], flags=P.PKM_F_SIMT)
+
+
+def _exact_query_inputs(cfg, seed):
+    """x and Wq with few significant bits and an identity BatchNorm (var + eps = 1):
+    every product and partial sum of q = x Wq^T is exact in fp32, so the device and the
+    oracle hold the same q and round it to bf16 the same way."""
+    inp = make_inputs(cfg, seed=seed)
+    rng = np.random.default_rng(seed + 100)
+    inp["x"] = (rng.integers(-8, 9, (cfg.N, cfg.d_in)) / 8).astype(np.float32)
+    inp["Wq"] = (rng.integers(-64, 65, (cfg.h * cfg.dk, cfg.d_in)) / 64).astype(np.float32)
+    eps = 2.0 ** -10
+    hq = cfg.h * cfg.dk
+    inp["bn"] = np.stack([np.zeros(hq), np.full(hq, 1 - eps), np.ones(hq),
+                          np.zeros(hq)]).astype(np.float32)
+    return inp, cfg.with_(bn_eps=eps)
+
+
+@pytest.mark.parametrize("simt", [False, True])
+def test_single_pass_bf16_q_scoring(simt):
+    """PKM_F_BF16_Q: scores from q rounded to bf16 (one tensor-core pass, or the CUDA-core
+    kernel dropping the lo plane), the sub-key gradient from the same rounded q, the
+    query gradient straight through -- against the oracle's bf16-q variant."""
+    cfg = _cfg(N=300)
+    inp, cfg = _exact_query_inputs(cfg, 5)
+    # the variant is visible: its scores move well beyond the index tolerance
+    f0, f1 = O.forward(inp, cfg), O.forward(inp, cfg, q_bf16=True)
+    assert np.abs(f1["s1"] - f0["s1"]).max() > 1e-3 * np.abs(f0["s1"]).max()
+    flags = P.PKM_F_BF16_Q | (P.PKM_F_SIMT if simt else 0)
+    clean = _full_check(cfg, flags=flags, inp=inp, q_bf16=True)
+    assert clean.mean() > 0.5
 
 
 def test_stagewise_scores_given_oracle_query():
