@@ -54,6 +54,32 @@ def query_network(x, Wq, bn, eps):
     return gamma * qhat + beta, qhat
 
 
+def query_network_train(x, Wq, bn, eps):
+    """Training-mode BatchNorm on the query: the statistics are the batch's own, over the
+    N tokens of the call (per column of x Wq^T: mean mu and the biased variance var);
+    q-hat = (x Wq^T - mu) / sqrt(var + eps), q = gamma * q-hat + beta.  Returns
+    (q, q-hat, mu, var).  The BatchNorm on the query is the first page's remark on
+    query normalisation ("Large Memory Layers with Product Keys", key results); training
+    mode is the plain reading of that layer when the batch trains it."""
+    x = np.asarray(x, dtype=np.float64)
+    Wq = np.asarray(Wq, dtype=np.float64)
+    gamma, beta = (np.asarray(r, dtype=np.float64) for r in bn[2:4])
+    pre = x @ Wq.T
+    mu = pre.mean(axis=0)
+    var = ((pre - mu) ** 2).mean(axis=0)
+    qhat = (pre - mu) / np.sqrt(var + eps)
+    return gamma * qhat + beta, qhat, mu, var
+
+
+def running_stats_update(bn, mu, var, n, momentum):
+    """Running statistics after a training batch of n tokens: mean <- (1 - m) mean + m mu,
+    var <- (1 - m) var + m * var_batch * n / (n - 1) (the unbiased batch variance)."""
+    out = np.array(bn, dtype=np.float64, copy=True)
+    out[0] = (1.0 - momentum) * out[0] + momentum * mu
+    out[1] = (1.0 - momentum) * out[1] + momentum * var * n / (n - 1)
+    return out
+
+
 def round_bf16(a):
     """Round to the nearest bfloat16 (ties to even) through fp32, returned as fp64: the
     fp32 bit pattern u becomes (u + 0x7FFF + ((u >> 16) & 1)) with the low 16 bits
@@ -143,8 +169,11 @@ def softmax(S):
 
 
 # ----------------------------------------------------------------------------- 1..6
-def forward(inp, cfg, select="brute", q_bf16=False):
+def forward(inp, cfg, select="brute", q_bf16=False, bn_train=False):
     """The layer forward for every token of ``inp['x']``.
+
+    ``bn_train``: BatchNorm with the batch's statistics (``query_network_train``); the
+    dict then also holds them as ``bn_batch`` = (mu, var).
 
     ``q_bf16``: the single-pass scoring variant -- the sub-key scores (and through them
     the selection and the weights) take q rounded to bf16 (``round_bf16``); the dict
@@ -156,7 +185,10 @@ def forward(inp, cfg, select="brute", q_bf16=False):
     w [N][h][k] (softmax weights) and y [N][d_v].
     """
     h, dk, C1, C2, k = cfg.h, cfg.dk, cfg.C1, cfg.C2, cfg.k
-    q, qhat = query_network(inp["x"], inp["Wq"], inp["bn"], cfg.bn_eps)
+    if bn_train:
+        q, qhat, mu, var = query_network_train(inp["x"], inp["Wq"], inp["bn"], cfg.bn_eps)
+    else:
+        q, qhat = query_network(inp["x"], inp["Wq"], inp["bn"], cfg.bn_eps)
     qs = round_bf16(q) if q_bf16 else q
     s1, s2 = subkey_scores(qs, inp["subkeys"], h, dk, C1)
     N = q.shape[0]
@@ -177,6 +209,8 @@ def forward(inp, cfg, select="brute", q_bf16=False):
     out = dict(q=q, qhat=qhat, s1=s1, s2=s2, sub_i=sub_i, sub_s=sub_s, idx=idx, S=S, w=w, y=y)
     if q_bf16:
         out["q_scores"] = qs
+    if bn_train:
+        out["bn_batch"] = (mu, var)
     return out
 
 
@@ -226,9 +260,16 @@ def backward(inp, cfg, fwd, dy):
     dsub[:, C1:, :] = np.einsum("thj,thd->hjd", g2, q2)
     dq = np.concatenate([dq1, dq2], axis=2).reshape(N, h * dk)
     mean, var, gamma, beta = (np.asarray(r, dtype=np.float64) for r in inp["bn"])
-    dq_pre = dq * gamma / np.sqrt(var + cfg.bn_eps)
     dgamma = (dq * fwd["qhat"]).sum(axis=0)
     dbeta = dq.sum(axis=0)
+    if "bn_batch" in fwd:
+        # batch statistics depend on every token: d pre = gamma / sqrt(var + eps) *
+        # (dq - mean_t dq - q-hat * mean_t (dq q-hat))
+        var_b = fwd["bn_batch"][1]
+        n = dq.shape[0]
+        dq_pre = gamma / np.sqrt(var_b + cfg.bn_eps) * (dq - dbeta / n - fwd["qhat"] * dgamma / n)
+    else:
+        dq_pre = dq * gamma / np.sqrt(var + cfg.bn_eps)
     x = np.asarray(inp["x"], dtype=np.float64)
     Wq = np.asarray(inp["Wq"], dtype=np.float64)
     dWq = dq_pre.T @ x

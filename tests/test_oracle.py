@@ -211,13 +211,18 @@ def test_subkey_scores_of_one_hot_queries_are_subkey_columns():
 
 
 # --------------------------------------------------------------------------- backward
-def _torch_loss_fixed_selection(inp, cfg, idx, dy):
-    """An independent forward in torch fp64 that touches only the selected keys."""
+def _torch_loss_fixed_selection(inp, cfg, idx, dy, bn_train=False):
+    """An independent forward in torch fp64 that touches only the selected keys (with
+    ``bn_train`` the library's training-mode batch_norm normalises the query)."""
     t = lambda a: torch.tensor(np.asarray(a, dtype=np.float64), requires_grad=True)
     x, Wq, sub, V = t(inp["x"]), t(inp["Wq"]), t(inp["subkeys"]), t(inp["values"])
     mean, var = (torch.tensor(np.asarray(r, dtype=np.float64)) for r in inp["bn"][:2])
     gamma, beta = t(inp["bn"][2]), t(inp["bn"][3])
-    q = (x @ Wq.T - mean) / torch.sqrt(var + cfg.bn_eps) * gamma + beta
+    if bn_train:
+        q = torch.nn.functional.batch_norm(x @ Wq.T, None, None, gamma, beta, training=True,
+                                           eps=cfg.bn_eps)
+    else:
+        q = (x @ Wq.T - mean) / torch.sqrt(var + cfg.bn_eps) * gamma + beta
     N = q.shape[0]
     qh = q.reshape(N, cfg.h, cfg.dk)
     half = cfg.dk // 2
@@ -237,18 +242,65 @@ def _torch_loss_fixed_selection(inp, cfg, idx, dy):
                 dV=V.grad.numpy(), dgamma=gamma.grad.numpy(), dbeta=beta.grad.numpy())
 
 
-@pytest.mark.parametrize("scale", [1.0, 0.37])
-def test_backward_matches_autograd_of_independent_forward(scale):
+@pytest.mark.parametrize("scale,bn_train", [(1.0, False), (0.37, False), (0.6, True)])
+def test_backward_matches_autograd_of_independent_forward(scale, bn_train):
     cfg = _cfg(score_scale=scale, N=10, h=2)
     inp = make_inputs(cfg, seed=8, random_bn=True)
-    f = O.forward(inp, cfg)
+    f = O.forward(inp, cfg, bn_train=bn_train)
     b = O.backward(inp, cfg, f, inp["dy"])
-    ref = _torch_loss_fixed_selection(inp, cfg, f["idx"], inp["dy"])
+    ref = _torch_loss_fixed_selection(inp, cfg, f["idx"], inp["dy"], bn_train=bn_train)
     for key in ("dx", "dWq", "dsub", "dgamma", "dbeta"):
         np.testing.assert_allclose(b[key], ref[key], rtol=1e-10, atol=1e-12, err_msg=key)
     dV = np.zeros_like(ref["dV"])
     dV[b["dV_rows"]] = b["dV_vals"]
     np.testing.assert_allclose(dV, ref["dV"], rtol=1e-10, atol=1e-12)
+
+
+def test_training_batch_norm_matches_the_library():
+    """Training-mode BatchNorm: q and the running-statistics update equal the library's
+    batch_norm(training=True) (biased variance to normalise, unbiased for the running
+    variance); each column of q-hat has mean 0 and mean square var / (var + eps)."""
+    cfg = _cfg(N=24)
+    inp = make_inputs(cfg, seed=30, with_dy=False, random_bn=True)
+    q, qhat, mu, var = O.query_network_train(inp["x"], inp["Wq"], inp["bn"], cfg.bn_eps)
+    t = lambda a: torch.from_numpy(np.array(a, dtype=np.float64))
+    rm, rv = t(inp["bn"][0]), t(inp["bn"][1])
+    ref = torch.nn.functional.batch_norm(t(inp["x"]) @ t(inp["Wq"]).T, rm, rv, t(inp["bn"][2]),
+                                         t(inp["bn"][3]), training=True, momentum=0.1,
+                                         eps=cfg.bn_eps)
+    np.testing.assert_allclose(q, ref.numpy(), rtol=1e-12, atol=1e-12)
+    upd = O.running_stats_update(inp["bn"], mu, var, cfg.N, 0.1)
+    np.testing.assert_allclose(upd[0], rm.numpy(), rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(upd[1], rv.numpy(), rtol=1e-12, atol=1e-14)
+    np.testing.assert_array_equal(upd[2:], np.asarray(inp["bn"][2:], dtype=np.float64))
+    np.testing.assert_allclose(qhat.mean(0), 0.0, atol=1e-12)
+    np.testing.assert_allclose((qhat ** 2).mean(0), var / (var + cfg.bn_eps), rtol=1e-12)
+
+
+def test_training_batch_norm_dx_by_finite_differences():
+    """Training mode couples every token through the batch statistics: central
+    differences of the loss in x (any token) match the analytic dx."""
+    cfg = _cfg(N=8, h=2)
+    inp = make_inputs(cfg, seed=31, random_bn=True)
+    inp = {k: np.asarray(v, dtype=np.float64) for k, v in inp.items()}
+    f0 = O.forward(inp, cfg, bn_train=True)
+    b = O.backward(inp, cfg, f0, inp["dy"])
+    rng = np.random.default_rng(32)
+    tested = 0
+    for _ in range(30):
+        ix = tuple(int(rng.integers(0, s)) for s in inp["x"].shape)
+        vals, ok = [], True
+        for sgn in (1, -1):
+            p = {k: v.copy() for k, v in inp.items()}
+            p["x"][ix] += sgn * 1e-6
+            f = O.forward(p, cfg, bn_train=True)
+            ok &= np.array_equal(f["idx"], f0["idx"])
+            vals.append((inp["dy"] * f["y"]).sum())
+        if ok:
+            np.testing.assert_allclose((vals[0] - vals[1]) / 2e-6, b["dx"][ix], rtol=1e-5,
+                                       atol=1e-8)
+            tested += 1
+    assert tested >= 20
 
 
 def test_value_gradient_row_sum_closed_form():
