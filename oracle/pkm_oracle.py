@@ -169,8 +169,13 @@ def softmax(S):
 
 
 # ----------------------------------------------------------------------------- 1..6
-def forward(inp, cfg, select="brute", q_bf16=False, bn_train=False):
+def forward(inp, cfg, select="brute", q_bf16=False, bn_train=False, all_k2=False):
     """The layer forward for every token of ``inp['x']``.
+
+    ``all_k2``: the variant of the code snippet in "Meta AI 可扩展内存层" section 10 --
+    no second top-k: every one of the k x k candidates top-k(s1) x top-k(s2) is kept
+    (a-major: candidate a*k + b pairs the a-th key of the first half with the b-th of the
+    second) and the softmax runs over all k^2 of them; idx, S, w are then [N][h][k*k].
 
     ``bn_train``: BatchNorm with the batch's statistics (``query_network_train``); the
     dict then also holds them as ``bn_batch`` = (mu, var).
@@ -193,17 +198,22 @@ def forward(inp, cfg, select="brute", q_bf16=False, bn_train=False):
     s1, s2 = subkey_scores(qs, inp["subkeys"], h, dk, C1)
     N = q.shape[0]
     pick = brute_force_topk if select == "brute" else product_key_topk
-    idx = np.zeros((N, h, k), dtype=np.int64)
-    S = np.zeros((N, h, k))
+    ksel = k * k if all_k2 else k
+    idx = np.zeros((N, h, ksel), dtype=np.int64)
+    S = np.zeros((N, h, ksel))
     sub_i = np.zeros((N, h, 2, k), dtype=np.int64)
     sub_s = np.zeros((N, h, 2, k))
     for t in range(N):
         for hh in range(h):
-            ii, jj = pick(s1[t, hh], s2[t, hh], k)
-            idx[t, hh] = ii * C2 + jj
-            S[t, hh] = cfg.score_scale * (s1[t, hh, ii] + s2[t, hh, jj])
             sub_i[t, hh, 0], sub_s[t, hh, 0] = half_topk(s1[t, hh], k)
             sub_i[t, hh, 1], sub_s[t, hh, 1] = half_topk(s2[t, hh], k)
+            if all_k2:
+                ii = np.repeat(sub_i[t, hh, 0], k)
+                jj = np.tile(sub_i[t, hh, 1], k)
+            else:
+                ii, jj = pick(s1[t, hh], s2[t, hh], k)
+            idx[t, hh] = ii * C2 + jj
+            S[t, hh] = cfg.score_scale * (s1[t, hh, ii] + s2[t, hh, jj])
     w = softmax(S)
     y = bag(w, idx, inp["values"])
     out = dict(q=q, qhat=qhat, s1=s1, s2=s2, sub_i=sub_i, sub_s=sub_s, idx=idx, S=S, w=w, y=y)
@@ -235,10 +245,10 @@ def backward(inp, cfg, fwd, dy):
       dsub [h][C1+C2][dk/2]
       dV_rows (sorted unique rows), dV_vals [len][d_v]  (all other rows are zero)
     """
-    h, dk, C1, C2, k = cfg.h, cfg.dk, cfg.C1, cfg.C2, cfg.k
+    h, dk, C1, C2 = cfg.h, cfg.dk, cfg.C1, cfg.C2
     dy = np.asarray(dy, dtype=np.float64)
     idx, w = fwd["idx"], fwd["w"]
-    N = idx.shape[0]
+    N, k = idx.shape[0], idx.shape[2]      # selections per head (k, or k*k for all_k2)
     V = inp["values"]
     rows = np.asarray(V[idx.reshape(-1)], dtype=np.float64).reshape(N, h, k, -1)
     dw = np.einsum("td,thjd->thj", dy, rows)

@@ -593,3 +593,55 @@ def test_sparse_adam_first_step_closed_form_and_untouched_rows():
     np.testing.assert_array_equal(V[keep], V0[keep])
     np.testing.assert_array_equal(M[keep], M0[keep])
     np.testing.assert_array_equal(S[keep], S0[keep])
+
+
+# --------------------------------------------------------------------------- all k^2 variant
+def test_all_k2_with_full_halves_is_softmax_attention_over_every_key():
+    """k = C1 = C2: the k x k candidates are every product key, so the variant is a dense
+    softmax over all C1*C2 keys: y = softmax(scale * (s1[i] + s2[j])) @ V, written here
+    with plain matrix operations."""
+    cfg = _cfg(C1=6, C2=6, k=6, h=2, N=7, score_scale=0.8)
+    inp = make_inputs(cfg, seed=40)
+    f = O.forward(inp, cfg, all_k2=True)
+    assert f["idx"].shape == (cfg.N, cfg.h, 36)
+    V = np.asarray(inp["values"], dtype=np.float64)
+    want = np.zeros((cfg.N, cfg.d_v))
+    for hh in range(cfg.h):
+        S = cfg.score_scale * (f["s1"][:, hh, :, None] + f["s2"][:, hh, None, :]).reshape(cfg.N, -1)
+        P = np.exp(S - S.max(1, keepdims=True))
+        want += (P / P.sum(1, keepdims=True)) @ V
+    np.testing.assert_allclose(f["y"], want, rtol=1e-12, atol=1e-13)
+
+
+def test_all_k2_candidates_and_gradient():
+    """The variant keeps exactly top-k(s1) x top-k(s2) (a-major), its weights sum to one,
+    and its backward matches central differences in the sub-keys and x (the candidate
+    set held fixed)."""
+    cfg = _cfg(C1=9, C2=7, k=3, h=2, N=5)
+    inp = make_inputs(cfg, seed=41, random_bn=True)
+    inp = {k_: np.asarray(v, dtype=np.float64) for k_, v in inp.items()}
+    f = O.forward(inp, cfg, all_k2=True)
+    for t in range(cfg.N):
+        for hh in range(cfg.h):
+            a, b = O.half_topk(f["s1"][t, hh], 3)[0], O.half_topk(f["s2"][t, hh], 3)[0]
+            want = [int(i) * cfg.C2 + int(j) for i in a for j in b]
+            assert f["idx"][t, hh].tolist() == want
+    np.testing.assert_allclose(f["w"].sum(-1), 1.0, atol=1e-12)
+    b = O.backward(inp, cfg, f, inp["dy"])
+    rng = np.random.default_rng(42)
+    tested = 0
+    for name, key in (("subkeys", "dsub"), ("x", "dx")):
+        for _ in range(12):
+            ix = tuple(int(rng.integers(0, s)) for s in inp[name].shape)
+            vals, ok = [], True
+            for sgn in (1, -1):
+                p = {k_: v.copy() for k_, v in inp.items()}
+                p[name][ix] += sgn * 1e-6
+                fs = O.forward(p, cfg, all_k2=True)
+                ok &= np.array_equal(fs["idx"], f["idx"])
+                vals.append((inp["dy"] * fs["y"]).sum())
+            if ok:
+                np.testing.assert_allclose((vals[0] - vals[1]) / 2e-6, b[key][ix], rtol=1e-5,
+                                           atol=1e-8)
+                tested += 1
+    assert tested >= 16
