@@ -106,6 +106,22 @@ def subkey_scores(q, subkeys, h, dk, C1):
     return s1, s2
 
 
+IDW_EPS = 1e-12
+
+
+def subkey_scores_idw(q, subkeys, h, dk, C1):
+    """Inverse-distance scores ("Fast-weight Product Key Memory", section 2.2, practical
+    techniques: the negative log of the Euclidean distance replaces the dot product):
+    s1[t][h][i] = -1/2 log(||q1[t][h] - C[h][i]||^2 + IDW_EPS), likewise s2 with C'.
+    IDW_EPS only keeps a zero distance finite.  The softmax of scale * (s1 + s2) then
+    weighs a key by (d1 d2)^(-scale): inverse distance weighting.  fp64."""
+    sub = np.asarray(subkeys, dtype=np.float64)
+    q1, q2 = split_halves(q, h, dk)
+    d1 = ((q1[:, :, None, :] - sub[None, :, :C1, :]) ** 2).sum(-1)
+    d2 = ((q2[:, :, None, :] - sub[None, :, C1:, :]) ** 2).sum(-1)
+    return -0.5 * np.log(d1 + IDW_EPS), -0.5 * np.log(d2 + IDW_EPS)
+
+
 # ----------------------------------------------------------------------------- 4
 def half_topk(s, k):
     """Top-k of one half's scores s [C] by (score desc, index asc) -> (index, score)."""
@@ -169,8 +185,11 @@ def softmax(S):
 
 
 # ----------------------------------------------------------------------------- 1..6
-def forward(inp, cfg, select="brute", q_bf16=False, bn_train=False, all_k2=False):
+def forward(inp, cfg, select="brute", q_bf16=False, bn_train=False, all_k2=False, idw=False):
     """The layer forward for every token of ``inp['x']``.
+
+    ``idw``: inverse-distance sub-key scores (``subkey_scores_idw``) instead of dot
+    products; selection and softmax are unchanged.
 
     ``all_k2``: the variant of the code snippet in "Meta AI 可扩展内存层" section 10 --
     no second top-k: every one of the k x k candidates top-k(s1) x top-k(s2) is kept
@@ -195,7 +214,8 @@ def forward(inp, cfg, select="brute", q_bf16=False, bn_train=False, all_k2=False
     else:
         q, qhat = query_network(inp["x"], inp["Wq"], inp["bn"], cfg.bn_eps)
     qs = round_bf16(q) if q_bf16 else q
-    s1, s2 = subkey_scores(qs, inp["subkeys"], h, dk, C1)
+    score = subkey_scores_idw if idw else subkey_scores
+    s1, s2 = score(qs, inp["subkeys"], h, dk, C1)
     N = q.shape[0]
     pick = brute_force_topk if select == "brute" else product_key_topk
     ksel = k * k if all_k2 else k
@@ -221,6 +241,8 @@ def forward(inp, cfg, select="brute", q_bf16=False, bn_train=False, all_k2=False
         out["q_scores"] = qs
     if bn_train:
         out["bn_batch"] = (mu, var)
+    if idw:
+        out["idw"] = True
     return out
 
 
@@ -263,11 +285,25 @@ def backward(inp, cfg, fwd, dy):
     np.add.at(g2, (tt, hh, (idx % C2).reshape(-1)), dsum.reshape(-1))
     sub = np.asarray(inp["subkeys"], dtype=np.float64)
     q1, q2 = split_halves(fwd.get("q_scores", fwd["q"]), h, dk)
-    dq1 = np.einsum("thi,hid->thd", g1, sub[:, :C1, :])
-    dq2 = np.einsum("thj,hjd->thd", g2, sub[:, C1:, :])
-    dsub = np.zeros_like(sub)
-    dsub[:, :C1, :] = np.einsum("thi,thd->hid", g1, q1)
-    dsub[:, C1:, :] = np.einsum("thj,thd->hjd", g2, q2)
+    if fwd.get("idw"):
+        # s = -1/2 log(||q - c||^2 + eps): ds/dq = (c - q) / (||q - c||^2 + eps) = -ds/dc;
+        # with u = g / (||q - c||^2 + eps) = g * exp(2 s):
+        #   dq = sum_i u_i c_i - q sum_i u_i,  dc_i = sum_t u_ti q_t - c_i sum_t u_ti
+        u1 = g1 * np.exp(2.0 * fwd["s1"])
+        u2 = g2 * np.exp(2.0 * fwd["s2"])
+        dq1 = np.einsum("thi,hid->thd", u1, sub[:, :C1, :]) - q1 * u1.sum(-1)[..., None]
+        dq2 = np.einsum("thj,hjd->thd", u2, sub[:, C1:, :]) - q2 * u2.sum(-1)[..., None]
+        dsub = np.zeros_like(sub)
+        dsub[:, :C1, :] = (np.einsum("thi,thd->hid", u1, q1) -
+                           sub[:, :C1, :] * u1.sum(0)[..., None])
+        dsub[:, C1:, :] = (np.einsum("thj,thd->hjd", u2, q2) -
+                           sub[:, C1:, :] * u2.sum(0)[..., None])
+    else:
+        dq1 = np.einsum("thi,hid->thd", g1, sub[:, :C1, :])
+        dq2 = np.einsum("thj,hjd->thd", g2, sub[:, C1:, :])
+        dsub = np.zeros_like(sub)
+        dsub[:, :C1, :] = np.einsum("thi,thd->hid", g1, q1)
+        dsub[:, C1:, :] = np.einsum("thj,thd->hjd", g2, q2)
     dq = np.concatenate([dq1, dq2], axis=2).reshape(N, h * dk)
     mean, var, gamma, beta = (np.asarray(r, dtype=np.float64) for r in inp["bn"])
     dgamma = (dq * fwd["qhat"]).sum(axis=0)

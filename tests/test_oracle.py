@@ -645,3 +645,67 @@ def test_all_k2_candidates_and_gradient():
                                            atol=1e-8)
                 tested += 1
     assert tested >= 16
+
+
+# --------------------------------------------------------------------------- IDW scores
+def test_idw_scores_closed_form():
+    """With q at the origin and sub-keys at known distances, s = -log(distance); the
+    softmax weights are proportional to (d1 d2)^(-scale)."""
+    cfg = _cfg(N=1, h=1, dk=4, C1=3, C2=2, k=2, score_scale=1.5)
+    sub = np.zeros((1, 5, 2))
+    sub[0, 0] = [1.0, 0.0]     # C: distances 1, 2, 4 from the origin
+    sub[0, 1] = [0.0, 2.0]
+    sub[0, 2] = [4.0, 0.0]
+    sub[0, 3] = [3.0, 4.0]     # C': distances 5, 0.5
+    sub[0, 4] = [0.0, -0.5]
+    q = np.zeros((1, 4))
+    s1, s2 = O.subkey_scores_idw(q, sub, 1, 4, 3)
+    np.testing.assert_allclose(s1[0, 0], -np.log([1.0, 2.0, 4.0]), atol=1e-11)
+    np.testing.assert_allclose(s2[0, 0], -np.log([5.0, 0.5]), atol=1e-11)
+    # the layer with these sub-keys: x = 0 and BN beta = 0 give q = 0
+    inp = dict(x=np.zeros((1, 16)), Wq=np.zeros((4, 16)),
+               bn=np.stack([np.zeros(4), np.ones(4), np.ones(4), np.zeros(4)]), subkeys=sub,
+               values=np.eye(6))
+    cfg = cfg.with_(d_in=16, d_v=6)
+    f = O.forward(inp, cfg, idw=True)
+    # the two closest products: (d1, d2) = (1, 0.5) and (2, 0.5), rows 0*2+1 and 1*2+1
+    assert f["idx"][0, 0].tolist() == [1, 3]
+    wr = (1.0 * 0.5) ** -1.5, (2.0 * 0.5) ** -1.5
+    np.testing.assert_allclose(f["w"][0, 0], np.array(wr) / sum(wr), rtol=1e-10)
+
+
+def test_idw_gradient_by_finite_differences():
+    """The inverse-distance backward against central differences in x, the sub-keys and
+    the values (selection held fixed)."""
+    cfg = _cfg(N=6, h=2, dk=8, C1=9, C2=7, k=3)
+    inp = make_inputs(cfg, seed=50, random_bn=True)
+    inp = {k_: np.asarray(v, dtype=np.float64) for k_, v in inp.items()}
+    f = O.forward(inp, cfg, idw=True)
+    b = O.backward(inp, cfg, f, inp["dy"])
+    rng = np.random.default_rng(51)
+    tested = 0
+    for name, key in (("subkeys", "dsub"), ("x", "dx"), ("Wq", "dWq")):
+        for _ in range(10):
+            ix = tuple(int(rng.integers(0, s)) for s in inp[name].shape)
+            vals, ok = [], True
+            for sgn in (1, -1):
+                p = {k_: v.copy() for k_, v in inp.items()}
+                p[name][ix] += sgn * 1e-6
+                fs = O.forward(p, cfg, idw=True)
+                ok &= np.array_equal(fs["idx"], f["idx"])
+                vals.append((inp["dy"] * fs["y"]).sum())
+            if ok:
+                np.testing.assert_allclose((vals[0] - vals[1]) / 2e-6, b[key][ix], rtol=1e-5,
+                                           atol=1e-8)
+                tested += 1
+    assert tested >= 24
+
+
+def test_idw_product_key_search_is_exact():
+    """The scores are still a sum over the two halves, so the product-key search reaches
+    the brute-force winners."""
+    cfg = _cfg(N=12, h=2, dk=8, C1=16, C2=12, k=5)
+    inp = make_inputs(cfg, seed=52)
+    fb = O.forward(inp, cfg, idw=True)
+    fp = O.forward(inp, cfg, idw=True, select="product")
+    np.testing.assert_array_equal(fb["idx"], fp["idx"])
