@@ -116,8 +116,14 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- CPU oracle timing
-def time_oracle(cfg, inp, seconds: float, batch: int = 8):
-    """Oracle forward (brute force over all keys) + backward on successive token batches
+def _oracle_kw(variant: str) -> dict:
+    return {"bf16_q": dict(q_bf16=True), "bn_train": dict(bn_train=True),
+            "all_k2": dict(all_k2=True)}.get(variant, {})
+
+
+def time_oracle(cfg, inp, seconds: float, batch: int = 8, variant: str = "none",
+                backward: bool = True):
+    """Oracle forward (brute force over all keys) [+ backward] on successive token batches
     until ``seconds`` of host time have passed.  Returns (tokens/s, tokens, threads)."""
     from oracle import pkm_oracle as O
     try:
@@ -128,9 +134,10 @@ def time_oracle(cfg, inp, seconds: float, batch: int = 8):
     done, t0 = 0, time.perf_counter()
     while True:
         sl = slice(done % cfg.N, done % cfg.N + batch)
-        sub = dict(inp, x=inp["x"][sl], dy=inp["dy"][sl])
-        f = O.forward(sub, cfg)
-        O.backward(sub, cfg, f, sub["dy"])
+        sub = dict(inp, x=inp["x"][sl])
+        f = O.forward(sub, cfg, **_oracle_kw(variant))
+        if backward:
+            O.backward(sub, cfg, f, inp["dy"][sl])
         done += sub["x"].shape[0]
         el = time.perf_counter() - t0
         if el >= seconds:
@@ -169,7 +176,10 @@ def run_b200(args, cfg, rank, world, dist):
     dy = torch.from_numpy(inp["dy"]).to(dev)
     gen_s = time.perf_counter() - t_gen
 
-    dims = P.Dims.from_config(cfg, flags=P.PKM_F_BF16_Q if args.bf16_q else 0)
+    vflags = {"none": 0, "bf16_q": P.PKM_F_BF16_Q, "bn_train": P.PKM_F_BN_TRAIN,
+              "all_k2": P.PKM_F_ALL_K2}[args.variant]
+    dims = P.Dims.from_config(cfg, flags=vflags)
+    ksel = cfg.k * cfg.k if args.variant == "all_k2" else cfg.k
     saved = P.alloc_saved(dims, with_qhat=True)
     y = torch.empty(cfg.N, cfg.d_v, device=dev)
     dx = torch.empty(cfg.N, cfg.d_in, device=dev)
@@ -178,7 +188,7 @@ def run_b200(args, cfg, rank, world, dist):
     dsub = torch.zeros(cfg.h, cfg.C1 + cfg.C2, cfg.dk // 2, device=dev)
     dV = (torch.zeros(cfg.K, cfg.d_v, device=dev)
           if args.stage in (None, "value_grad", "query_grad") else None)
-    dw = torch.empty(cfg.N, cfg.h, cfg.k, device=dev)
+    dw = torch.empty(cfg.N, cfg.h, ksel, device=dev)
     ws = P.alloc_workspace(dims, P.PKM_BWD, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
@@ -283,7 +293,7 @@ def run_b200(args, cfg, rank, world, dist):
 
     pk = _peaks()
     st_mean = stage_ms.mean(0)
-    hk = cfg.h * cfg.k
+    hk = cfg.h * ksel
     sel = cfg.N * hk
     bytes_gather = sel * cfg.d_v * 2 + cfg.N * cfg.d_v * 4 + sel * 8
     bytes_value = U * cfg.d_v * (2 + 8) + cfg.N * cfg.d_v * 4 + sel * 12
@@ -311,8 +321,7 @@ def run_b200(args, cfg, rank, world, dist):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded; tables random-init, no trained weights)",
         "config": dict(_cfg_json(cfg), parallelism=f"replicas{world}" if world > 1 else "single",
-                       scoring="single-pass, q rounded to bf16" if args.bf16_q else
-                       "q as bf16 hi + lo (two passes)"),
+                       variant=args.variant),
         "fwd": {"value": round(cfg.N * world / (fwd_ms * 1e-3), 1), "unit": "tokens/s (fwd)",
                 "ms": round(fwd_ms, 4)},
         "stage_ms": {n: round(float(v), 4) for n, v in zip(names, st_mean)},
@@ -328,7 +337,7 @@ def run_b200(args, cfg, rank, world, dist):
                       "h2d_bytes_per_step": int(e2e["h2d"]), "d2h_bytes_per_step": int(e2e["d2h"]),
                       "ms": round(e2e_ms, 4)}
     if world == 1 and not args.no_cpu_baseline:
-        v, n, thr = time_oracle(cfg, inp, args.cpu_seconds)
+        v, n, thr = time_oracle(cfg, inp, args.cpu_seconds, variant=args.variant)
         out["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s (fwd+bwd)", "cores": thr,
                                "kind": "oracle",
                                "sample": f"{n} tokens of the same batch, fp64 numpy oracle: "
@@ -654,6 +663,14 @@ def run_decode(args, cfg, rank, world, dist):
     if rank != 0:
         return None
     pk = _peaks()
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        tps, n_tok, thr = time_oracle(cfg.with_(N=max(sizes)), inp, min(args.cpu_seconds, 8.0),
+                                      batch=1, backward=False)
+        cpu = {"value": round(1e6 / tps, 1), "unit": "us per forward call at N=1", "cores": thr,
+               "kind": "oracle",
+               "sample": f"{n_tok} single-token forward calls; fp64 numpy oracle, brute force "
+                         f"over all {cfg.K} keys per head"}
     top = res[max(sizes)]
     ach = top["algorithmic_bytes"] / (top["graph_us_l2_flushed"] * 1e-6) / 1e9
     return {
@@ -670,6 +687,7 @@ def run_decode(args, cfg, rank, world, dist):
                      "frac": round(ach / pk["hbm"], 4), "traffic": None,
                      "algorithmic_bytes": top["algorithmic_bytes"], "peak_source": pk["src"]},
         "clocks": clk, "gpu_launches": int(launches),
+        **({"cpu_baseline": cpu} if cpu else {}),
     }
 
 
@@ -691,10 +709,41 @@ def run_stage(args, cfg, dims, saved, P, st, step, flush, names, env):
                                                dbn=dbn, dsubkeys=dsub, workspace=ws, stream=st),
     }
     order = list(calls)
-    for prev in order[: order.index(args.stage)]:   # fill the saved tensors the stage reads
-        calls[prev]()
-    torch.cuda.synchronize()
-    fn = calls[args.stage]
+    extra = {}
+    if args.stage in ("value_grad_rows", "value_adam", "hit_counts"):
+        # training-time stages after the forward: compact value gradient, lazy Adam on the
+        # selected rows (fp32 table and state), hit histograms
+        for prev in order[:4]:
+            calls[prev]()
+        torch.cuda.synchronize()
+        U = int(torch.unique(saved["idx"]).numel())
+        sel = cfg.N * cfg.h * cfg.k
+        if args.stage == "value_grad_rows":
+            cap = min(sel, cfg.K)
+            rows = torch.empty(cap, dtype=torch.int32, device=x.device)
+            dvr = torch.empty(cap, cfg.d_v, device=x.device)
+            nr = torch.empty(1, dtype=torch.int32, device=x.device)
+            fn = lambda: P.pkm_value_grad_rows(dims, V, saved, dy, rows, dvr, nr, dw=dw,
+                                               workspace=ws, stream=st)
+            alg = U * cfg.d_v * (2 + 4) + cfg.N * cfg.d_v * 4 + sel * 12
+        elif args.stage == "value_adam":
+            d32 = P.Dims.from_config(cfg.with_(value_dtype="f32"))
+            V32, m, v = V.float(), torch.zeros(cfg.K, cfg.d_v, device=x.device), None
+            v = torch.zeros_like(m)
+            fn = lambda: P.pkm_value_adam(d32, 1e-3, 0.9, 0.999, 1e-8, 1, V32, m, v, saved, dy,
+                                          workspace=ws, stream=st)
+            alg = U * cfg.d_v * 4 * 6 + cfg.N * cfg.d_v * 4 + sel * 12
+        else:
+            slot = torch.zeros(cfg.K, dtype=torch.int32, device=x.device)
+            subh = torch.zeros(cfg.h, cfg.C1 + cfg.C2, dtype=torch.int32, device=x.device)
+            fn = lambda: P.pkm_hit_counts(dims, saved["idx"], slot, subh, stream=st)
+            alg = sel * 4
+        extra = {"distinct_rows": U, "algorithmic_bytes": int(alg)}
+    else:
+        for prev in order[: order.index(args.stage)]:   # fill the saved tensors the stage reads
+            calls[prev]()
+        torch.cuda.synchronize()
+        fn = calls[args.stage]
     for _ in range(args.warmup):
         flush.zero_()
         fn()
@@ -708,8 +757,13 @@ def run_stage(args, cfg, dims, saved, P, st, step, flush, names, env):
         torch.cuda.synchronize()
         ms.append(a.elapsed_time(b))
     assert P.pkm_check_status(st) == P.PKM_OK
-    return {"stage": args.stage, "workload": cfg.name, "ms_per_call": round(float(np.mean(ms)), 4),
-            "ms_min": round(float(np.min(ms)), 4), "calls": args.steps}
+    out = {"stage": args.stage, "workload": cfg.name, "variant": args.variant,
+           "ms_per_call": round(float(np.mean(ms)), 4), "ms_min": round(float(np.min(ms)), 4),
+           "calls": args.steps}
+    if extra:
+        out.update(extra)
+        out["GB_per_s"] = round(extra["algorithmic_bytes"] / (np.mean(ms) * 1e-3) / 1e9, 1)
+    return out
 
 
 def _ncu_traffic(kernel: str):
@@ -784,11 +838,13 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=8)
     ap.add_argument("--stage", default=None,
                     choices=["query", "subkey_scores", "candidate_topk", "gather_bag",
-                             "value_grad", "query_grad"],
+                             "value_grad", "query_grad", "value_grad_rows", "value_adam",
+                             "hit_counts"],
                     help="time one stage alone (per-op benchmark / profiling target)")
     ap.add_argument("--tokens", type=int, default=None, help="override the token count")
-    ap.add_argument("--bf16-q", action="store_true",
-                    help="single-pass scoring (PKM_F_BF16_Q: q rounded to bf16 for the scores)")
+    ap.add_argument("--variant", default="none", choices=["none", "bf16_q", "bn_train", "all_k2"],
+                    help="layer variant for the whole step: single-pass bf16-q scoring, "
+                         "training-mode BatchNorm, or the all-k^2 softmax")
     ap.add_argument("--decode", action="store_true",
                     help="decode-shaped forward latency (N = 1, 8, 64) on the workload's table")
     args = ap.parse_args()

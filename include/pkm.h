@@ -71,6 +71,23 @@ typedef enum {
  * uses the same rounded q; the query gradient passes the rounding unchanged.  bf16
  * storage only (PKM_ERR_INVALID_ARG with PKM_F_FP32). */
 #define PKM_F_BF16_Q 0x8u
+/* Training-mode BatchNorm on the query: the forward normalises with the batch's own
+ * statistics (per column of x Wq^T over the call's N tokens: mean and biased variance),
+ * records them in saved->bn_batch and needs saved->qhat; the backward differentiates
+ * through them (every token's gradient depends on all tokens).  bn's running mean and
+ * variance are not read; pkm_bn_running_update folds a batch into them. */
+#define PKM_F_BN_TRAIN 0x10u
+/* The all-k^2 variant (the code snippet of "Meta AI 可扩展内存层" section 10): no second
+ * top-k -- every one of the k*k candidates top-k(s1) x top-k(s2) is kept, a-major
+ * (selection a*k + b pairs the a-th sub-key of the first half with the b-th of the second),
+ * and the softmax runs over all of them.  idx, w and dw then hold k*k selections per head:
+ * [N][h][k*k] (pkm_saved_bytes accounts for it). */
+#define PKM_F_ALL_K2 0x20u
+/* Inverse-distance sub-key scores ("Fast-weight Product Key Memory", section 2.2):
+ * s = -1/2 log(||q_half - c||^2 + 1e-12) instead of q_half . c; selection and softmax as
+ * usual, so the weights fall off as (d1 d2)^(-score_scale).  Scoring and the sub-key /
+ * query-half gradients run on the CUDA-core kernels. */
+#define PKM_F_IDW 0x40u
 
 typedef struct {
   int64_t N;          /* tokens */
@@ -93,7 +110,10 @@ typedef struct {
  *   sub_s  [N][h][2][k] fp32 per-half top-k scores, best first
  *   sub_i  [N][h][2][k] int32 per-half top-k sub-key indices, best first
  *   idx    [N][h][k] int32 selected value rows i*C2 + j, best first
- *   w      [N][h][k] fp32 softmax weights                                     */
+ *   w      [N][h][k] fp32 softmax weights
+ *   bn_batch  [2][h*dk] fp32 batch mean and biased batch variance of x Wq^T: written by
+ *          the forward and read by the backward with PKM_F_BN_TRAIN (with it, qhat is
+ *          required too); otherwise unused and may be NULL.                     */
 typedef struct {
   void* q;
   float* qhat;
@@ -101,6 +121,7 @@ typedef struct {
   int32_t* sub_i;
   int32_t* idx;
   float* w;
+  float* bn_batch;
 } pkm_saved;
 
 #define PKM_SAVED_Q 0
@@ -109,6 +130,7 @@ typedef struct {
 #define PKM_SAVED_SUB_I 3
 #define PKM_SAVED_IDX 4
 #define PKM_SAVED_W 5
+#define PKM_SAVED_BN_BATCH 6
 
 #define PKM_FWD 0
 #define PKM_BWD 1
@@ -175,6 +197,13 @@ pkm_status pkm_gather_bag(const pkm_dims* d, const void* values, const int32_t* 
                           const float* w, float* y, void* stream);
 
 /* ---- training-time pieces ("Meta AI 可扩展内存层" sections 6.1, 6.3, 6.4, 11.2) ---- */
+
+/* Running statistics after a training-mode batch (PKM_F_BN_TRAIN forward):
+ *   bn[0] <- (1 - momentum) bn[0] + momentum * mean_batch,
+ *   bn[1] <- (1 - momentum) bn[1] + momentum * var_batch * N / (N - 1)   (N >= 2),
+ * bn [4][h*dk] updated in place (rows 2-3 untouched), bn_batch = saved->bn_batch. */
+pkm_status pkm_bn_running_update(const pkm_dims* d, float* bn, const float* bn_batch,
+                                 float momentum, void* stream);
 
 /* Value-gradient stage with a compact (sparse-rows) result instead of the dense table:
  * num_rows (device int, written) = U, the number of distinct selected rows;

@@ -374,6 +374,8 @@ __global__ void __launch_bounds__(kSgdThreads) rows_step_kernel(
     const float* __restrict__ ws_sorted, const float* __restrict__ dy, float* __restrict__ V,
     float lr, int hk, int d_v, int64_t K, int* status, const int* __restrict__ bounds,
     int64_t key_base, AdamArgs ad) {
+  grid_dependency_wait();  // the residual (and the table's last reader) precede this write
+  allow_dependent_launch();
   const int u0 = bounds ? bounds[0] : 0;
   const int u1 = bounds ? bounds[1] : *U_ptr;
   const int nvec = d_v / 4;
@@ -439,6 +441,42 @@ inline size_t value_rows_smem(const Plan& p) {
   return 2 * (vb + (size_t)p.d_v * 4);
 }
 
+// ------------------------------------------------------------------ B4 (inverse distance)
+__global__ void idw_scale_kernel(float* __restrict__ gsub, const float* __restrict__ sub_s,
+                                 int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    gsub[i] *= expf(2.f * sub_s[i]);
+}
+
+// ------------------------------------------------------------------ B4 (all-k^2 variant)
+// Every candidate (a, b) of the k x k grid is selected: dS_ab = scale w_ab (dw_ab -
+// sum w dw); the first half's a-th sub-key collects the row sum over b, the second
+// half's b-th the column sum over a.  One warp per (token, head).
+__global__ void __launch_bounds__(256) softmax_bwd_all_kernel(
+    const float* __restrict__ w, const float* __restrict__ dw, float* __restrict__ gsub,
+    int64_t NH, int k, float scale) {
+  const int lane = threadIdx.x & 31;
+  const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (g >= NH) return;
+  const int kk = k * k;
+  const float* wg = w + g * kk;
+  const float* dg = dw + g * kk;
+  float s = 0.f;
+  for (int c = lane; c < kk; c += 32) s = fmaf(wg[c], dg[c], s);
+  s = warp_sum(s);
+  if (lane < k) {
+    float g1 = 0.f, g2 = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int ca = lane * k + j, cb = j * k + lane;
+      g1 += scale * wg[ca] * (dg[ca] - s);
+      g2 += scale * wg[cb] * (dg[cb] - s);
+    }
+    gsub[g * 2 * k + lane] = g1;
+    gsub[g * 2 * k + k + lane] = g2;
+  }
+}
+
 // ------------------------------------------------------------------ B4
 __global__ void __launch_bounds__(256) softmax_bwd_kernel(
     const float* __restrict__ w, const float* __restrict__ dw, const int32_t* __restrict__ idx,
@@ -479,7 +517,10 @@ template <typename TS, int MAXC, bool kSplit>
 __global__ void __launch_bounds__(256) dq_kernel(
     const float* __restrict__ gsub, const int32_t* __restrict__ sub_i, const TS* __restrict__ sub,
     const float* __restrict__ bn, const float* __restrict__ qhat, void* __restrict__ dq_out,
-    float* __restrict__ part, int64_t N, int h, int dk, int C1, int C2, int k, float eps) {
+    float* __restrict__ part, int64_t N, int h, int dk, int C1, int C2, int k, float eps,
+    const void* __restrict__ q_idw) {
+  // q_idw (inverse-distance scores; gsub then holds u = g / ||q - c||^2): subtract
+  // q * sum_a u_a, q read from the saved query (bf16 hi + lo planes, or fp32)
   constexpr int E = VecT<TS>::E;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int hs = blockIdx.y, hh = hs >> 1, s = hs & 1;
@@ -502,8 +543,10 @@ __global__ void __launch_bounds__(256) dq_kernel(
     for (int c = 0; c < MAXC; ++c)
 #pragma unroll
       for (int e = 0; e < E; ++e) acc[c][e] = 0.f;
+    float usum = 0.f;
     for (int a = 0; a < k; ++a) {
       const float ga = gsub[gb + a];
+      usum += ga;
       const int32_t row = sub_i[gb + a];
 #pragma unroll
       for (int c = 0; c < MAXC; ++c) {
@@ -523,6 +566,16 @@ __global__ void __launch_bounds__(256) dq_kernel(
 #pragma unroll
         for (int e = 0; e < E; ++e) {
           const int col = col0 + vec * E + e;
+          if (q_idw) {
+            float qv;
+            if constexpr (E == 8) {
+              const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q_idw);
+              qv = __bfloat162float(qb[t * hq + col]) + __bfloat162float(qb[N * hq + t * hq + col]);
+            } else {
+              qv = static_cast<const float*>(q_idw)[t * hq + col];
+            }
+            acc[c][e] = fmaf(-usum, qv, acc[c][e]);
+          }
           const float gam = bn[2 * hq + col], var = bn[hq + col];
           const float val = acc[c][e] * gam / sqrtf(var + eps);
           if constexpr (kSplit) {
@@ -595,7 +648,8 @@ __global__ void __launch_bounds__(256) subkey_grad_kernel(
     const int* __restrict__ seg, const int* __restrict__ U_ptr, const int32_t* __restrict__ rows,
     const int32_t* __restrict__ ents, const float* __restrict__ gsub, const void* __restrict__ q,
     float* __restrict__ dsub, int64_t N, int h, int dk, int C1, int C2, int k, int* status,
-    float lo_scale) {
+    float lo_scale, const void* __restrict__ sub_idw) {
+  // sub_idw (inverse-distance scores; gsub holds u): subtract c_R * sum u over the segment
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -620,10 +674,12 @@ __global__ void __launch_bounds__(256) subkey_grad_kernel(
     for (int c = 0; c < MAXC; ++c)
 #pragma unroll
       for (int e = 0; e < E; ++e) acc[c][e] = 0.f;
+    float usum = 0.f;
     for (int p = p0; p < p1; ++p) {
       const int32_t ent = ents[p];
       const int64_t t = ent / (2 * h * k);
       const float gv = gsub[ent];
+      usum += gv;
 #pragma unroll
       for (int c = 0; c < MAXC; ++c) {
         const int vec = lane + 32 * c;
@@ -651,6 +707,16 @@ __global__ void __launch_bounds__(256) subkey_grad_kernel(
       const int vec = lane + 32 * c;
       if (vec < nvec) {
         float* o = dsub + (int64_t)R * half + (int64_t)vec * E;
+        if (sub_idw) {
+          const int64_t so = (int64_t)R * half + (int64_t)vec * E;
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const float cv = kSplitQ
+                                 ? __bfloat162float(static_cast<const __nv_bfloat16*>(sub_idw)[so + e])
+                                 : static_cast<const float*>(sub_idw)[so + e];
+            acc[c][e] = fmaf(-usum, cv, acc[c][e]);
+          }
+        }
 #pragma unroll
         for (int e = 0; e < E; ++e) o[e] += acc[c][e];
       }
@@ -667,15 +733,16 @@ inline int bits_for(int64_t maxkey) {
 // ------------------------------------------------------------------ workspace
 struct Layout {
   size_t keysA, valsA, keysB, valsB, hist, bsum, seg, segrow, wsorted, U, dw, gsub, dq, part,
-      G, dqf, dspart, total;
+      G, dqf, dspart, bneff, bntot, total;
 };
 
 inline size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
 
 Layout layout(const Plan& p) {
   Layout L{};
-  const int64_t E1 = p.N * p.h * p.k, E2 = 2 * E1;
-  const int64_t En = E2;
+  // E1 selections (value pass), E2 per-half list entries (sub-key pass)
+  const int64_t E1 = p.N * p.h * p.ksel, E2 = 2 * p.N * p.h * p.k;
+  const int64_t En = std::max(E1, E2);
   size_t o = 0;
   auto take = [&](size_t bytes) {
     size_t r = o;
@@ -704,6 +771,8 @@ Layout layout(const Plan& p) {
     L.dqf = take(4 * (size_t)p.N * p.hq);
     L.dspart = take(4 * subgrad_partial_floats(p));
   }
+  L.bneff = take(4 * 4 * (size_t)p.hq);  // training-mode BatchNorm: (mean, var, gamma, beta)
+  L.bntot = take(4 * 2 * (size_t)p.hq);  // and the column sums (d gamma, d beta)
   L.total = o;
   return L;
 }
@@ -732,6 +801,8 @@ struct BwdCtx {
   __nv_bfloat16* G;
   float* dqf;
   float* dspart;
+  float* bneff;
+  float* bntot;
 };
 
 static BwdCtx bwd_ctx(const Plan& p, void* ws, float* dw_out) {
@@ -751,13 +822,15 @@ static BwdCtx bwd_ctx(const Plan& p, void* ws, float* dw_out) {
   c.G = at<__nv_bfloat16>(ws, L.G);
   c.dqf = at<float>(ws, L.dqf);
   c.dspart = at<float>(ws, L.dspart);
+  c.bneff = at<float>(ws, L.bneff);
+  c.bntot = at<float>(ws, L.bntot);
   return c;
 }
 
 cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved& s,
                               const float* dy, float* dV, float* dw_out, void* ws,
                               cudaStream_t st, float* dVc, int32_t* rows_out, int* U_out) {
-  const int64_t E1 = p.N * p.h * p.k;
+  const int64_t E1 = p.N * p.h * p.ksel;
   BwdCtx c = bwd_ctx(p, ws, dw_out);
   sort::RadixBuffers& rb = c.rb;
   int* seg = c.seg;
@@ -765,7 +838,7 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
   int* U = c.U;
   float* dw = c.dw;
   cudaError_t e;
-  const int hk = p.h * p.k;
+  const int hk = p.h * p.ksel;
   const int persist_blocks = p.sm_count * 8;
 
   // B1-B2: selections sorted by value row
@@ -811,7 +884,7 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
 
 cudaError_t launch_value_sgd(const Plan& p, float* values, const pkm_saved& s, const float* dy,
                              float lr, void* ws, cudaStream_t st) {
-  const int64_t E1 = p.N * p.h * p.k;
+  const int64_t E1 = p.N * p.h * p.ksel;
   BwdCtx c = bwd_ctx(p, ws, nullptr);
   cudaError_t e;
   const int32_t *rows_sorted, *ents_sorted;
@@ -822,7 +895,7 @@ cudaError_t launch_value_sgd(const Plan& p, float* values, const pkm_saved& s, c
   if (e != cudaSuccess) return e;
   const int64_t blocks = std::min<int64_t>(E1, (int64_t)p.sm_count * 8);
   rows_step_kernel<false><<<(unsigned)blocks, kSgdThreads, 0, st>>>(
-      c.seg, c.U, c.seg_row, ents_sorted, c.w_sorted, dy, values, lr, p.h * p.k, p.d_v, p.K,
+      c.seg, c.U, c.seg_row, ents_sorted, c.w_sorted, dy, values, lr, p.h * p.ksel, p.d_v, p.K,
       p.status, nullptr, 0, AdamArgs{});
   PKM_COUNT(1);
   return cudaGetLastError();
@@ -831,7 +904,7 @@ cudaError_t launch_value_sgd(const Plan& p, float* values, const pkm_saved& s, c
 cudaError_t launch_value_adam(const Plan& p, float* values, float* m, float* v,
                               const pkm_saved& s, const float* dy, float lr, float beta1,
                               float beta2, float eps, int64_t step, void* ws, cudaStream_t st) {
-  const int64_t E1 = p.N * p.h * p.k;
+  const int64_t E1 = p.N * p.h * p.ksel;
   BwdCtx c = bwd_ctx(p, ws, nullptr);
   cudaError_t e;
   const int32_t *rows_sorted, *ents_sorted;
@@ -845,7 +918,7 @@ cudaError_t launch_value_adam(const Plan& p, float* values, float* m, float* v,
               (float)(1.0 / (1.0 - std::pow((double)beta2, (double)step)))};
   const int64_t blocks = std::min<int64_t>(E1, (int64_t)p.sm_count * 8);
   rows_step_kernel<true><<<(unsigned)blocks, kSgdThreads, 0, st>>>(
-      c.seg, c.U, c.seg_row, ents_sorted, c.w_sorted, dy, values, lr, p.h * p.k, p.d_v, p.K,
+      c.seg, c.U, c.seg_row, ents_sorted, c.w_sorted, dy, values, lr, p.h * p.ksel, p.d_v, p.K,
       p.status, nullptr, 0, ad);
   PKM_COUNT(1);
   return cudaGetLastError();
@@ -878,9 +951,9 @@ __global__ void hit_counts_kernel(const int32_t* __restrict__ idx, int64_t E, in
 
 cudaError_t launch_hit_counts(const Plan& p, const int32_t* idx, int32_t* slot, int32_t* sub,
                               cudaStream_t st) {
-  const int64_t E = p.N * p.h * p.k;
+  const int64_t E = p.N * p.h * p.ksel;
   const int64_t blocks = std::min<int64_t>((E + 255) / 256, (int64_t)p.sm_count * 16);
-  hit_counts_kernel<<<(unsigned)blocks, 256, 0, st>>>(idx, E, p.h, p.k, p.C1, p.C2, p.K, slot,
+  hit_counts_kernel<<<(unsigned)blocks, 256, 0, st>>>(idx, E, p.h, p.ksel, p.C1, p.C2, p.K, slot,
                                                       sub, p.status);
   PKM_COUNT(1);
   return cudaGetLastError();
@@ -952,6 +1025,9 @@ __global__ void __launch_bounds__(kFwSortThreads) fw_chunk_sort_kernel(
     fw_keys[i] = key;
   }
   __syncthreads();
+  // A stage with distance `half` <= 32 pairs elements inside the 64-element blocks that
+  // one warp's 32 consecutive pair indices cover, so between two such stages a warp
+  // barrier suffices; a block barrier is needed around stages of larger distance.
   for (int size = 2; size <= npow2; size <<= 1) {
     for (int half = size >> 1; half > 0; half >>= 1) {
       for (int j = tid; j < (npow2 >> 1); j += kFwSortThreads) {
@@ -964,9 +1040,14 @@ __global__ void __launch_bounds__(kFwSortThreads) fw_chunk_sort_kernel(
           fw_keys[hi] = a;
         }
       }
-      __syncthreads();
+      const int next_half = half == 1 ? size : half >> 1;
+      if (half > 32 || next_half > 32)
+        __syncthreads();
+      else
+        __syncwarp();
     }
   }
+  __syncthreads();
   // segment starts: block-wide exclusive scan of the start flags over thread-owned runs
   const int per = (n + kFwSortThreads - 1) / kFwSortThreads;
   const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
@@ -1090,11 +1171,11 @@ cudaError_t launch_fw_chunk_write(const Plan& p, int64_t chunk, int64_t ci, cons
   const int64_t n_c = std::min<int64_t>(chunk, p.N - ci * chunk) * p.h * p.k;
   const int64_t blocks = std::min<int64_t>(n_c, (int64_t)p.sm_count * 8);
   const int64_t o = ci * stride;
-  rows_step_kernel<false><<<(unsigned)blocks, kSgdThreads, 0, st>>>(
-      seg + o, U + ci, seg_row + o, ents + o, w_sorted + o, dy, values, lr, p.h * p.k, p.d_v,
-      p.K, p.status, nullptr, 0, AdamArgs{});
   PKM_COUNT(1);
-  return cudaGetLastError();
+  return launch_dependent(rows_step_kernel<false>, dim3((unsigned)blocks), dim3(kSgdThreads), 0,
+                          st, seg + o, U + ci, seg_row + o, ents + o, w_sorted + o, dy, values, lr,
+                          p.h * p.k, p.d_v, p.K, p.status, (const int*)nullptr, (int64_t)0,
+                          AdamArgs{});
 }
 
 cudaError_t launch_fw_write(const Plan& p, int64_t chunk, int64_t ci, const int* bounds,
@@ -1104,11 +1185,10 @@ cudaError_t launch_fw_write(const Plan& p, int64_t chunk, int64_t ci, const int*
       sort::radix_sorted_vals(c.rb, bits_for(((p.N + chunk - 1) / chunk) * p.K - 1));
   const int64_t n_c = std::min<int64_t>(chunk, p.N - ci * chunk);
   const int64_t blocks = std::min<int64_t>(n_c * p.h * p.k, (int64_t)p.sm_count * 8);
-  rows_step_kernel<false><<<(unsigned)blocks, kSgdThreads, 0, st>>>(
-      c.seg, c.U, c.seg_row, ents_sorted, c.w_sorted, dy, values, lr, p.h * p.k, p.d_v, p.K,
-      p.status, bounds + ci, ci * p.K, AdamArgs{});
   PKM_COUNT(1);
-  return cudaGetLastError();
+  return launch_dependent(rows_step_kernel<false>, dim3((unsigned)blocks), dim3(kSgdThreads), 0,
+                          st, c.seg, c.U, c.seg_row, ents_sorted, c.w_sorted, dy, values, lr,
+                          p.h * p.k, p.d_v, p.K, p.status, bounds + ci, ci * p.K, AdamArgs{});
 }
 
 cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, const float* bn,
@@ -1126,26 +1206,54 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
   float* part = c.part;
   cudaError_t e;
   const int persist_blocks = p.sm_count * 8;
+  // Training-mode BatchNorm: the eval-mode kernels below run with the batch statistics,
+  // the d gamma / d beta column sums are always formed, and dq_pre is corrected for the
+  // statistics' dependence on every token before the dense query gradients.
+  const bool train = p.bn_train && (dx || dWq || dbn);
+  if (train) {
+    if ((e = cudaMemcpyAsync(c.bneff, s.bn_batch, 2 * sizeof(float) * p.hq,
+                             cudaMemcpyDeviceToDevice, st)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(c.bneff + 2 * p.hq, bn + 2 * p.hq, 2 * sizeof(float) * p.hq,
+                             cudaMemcpyDeviceToDevice, st)) != cudaSuccess)
+      return e;
+    bn = c.bneff;
+  }
+  float* dbn_acc = train ? c.bntot : dbn;  // where the partial column sums are reduced
 
   // B4: softmax backward onto the selected sub-keys
   {
     const int64_t NH = p.N * p.h;
-    softmax_bwd_kernel<<<(unsigned)((NH + 7) / 8), 256, 0, st>>>(s.w, dw, s.idx, s.sub_i, gsub,
-                                                                  NH, p.k, p.C2, p.scale); PKM_COUNT(1);
+    if (p.ksel != p.k)
+      softmax_bwd_all_kernel<<<(unsigned)((NH + 7) / 8), 256, 0, st>>>(s.w, dw, gsub, NH, p.k,
+                                                                       p.scale);
+    else
+      softmax_bwd_kernel<<<(unsigned)((NH + 7) / 8), 256, 0, st>>>(s.w, dw, s.idx, s.sub_i, gsub,
+                                                                    NH, p.k, p.C2, p.scale);
+    PKM_COUNT(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (p.idw) {  // inverse-distance scores: u = g / (||q - c||^2 + eps) = g exp(2 s)
+    const int64_t n = 2 * p.N * p.h * p.k;
+    idw_scale_kernel<<<(unsigned)std::min<int64_t>((n + 255) / 256, (int64_t)p.sm_count * 16),
+                       256, 0, st>>>(gsub, s.sub_s, n);
+    PKM_COUNT(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
 
   // B5 + B6 on tensor cores: dense G planes, dq = G C, BatchNorm backward, dC = G^T Q
-  const bool tc_subgrad = tc_backward_supported(p) && p.half % 64 == 0;
+  // (the inverse-distance variant's corrections run on the CUDA-core path)
+  const bool tc_subgrad = tc_backward_supported(p) && p.half % 64 == 0 && !p.idw;
   if (tc_subgrad) {
     const bool want_dq = dx || dWq || dbn;
-    e = launch_subgrad_tc(p, gsub, s.sub_i, subkeys, s.q, bn, dbn ? s.qhat : nullptr, c.G,
-                          c.dqf, reinterpret_cast<__nv_bfloat16*>(dq_pre), dbn ? part : nullptr,
-                          c.dspart, dsub, want_dq, st);
+    e = launch_subgrad_tc(p, gsub, s.sub_i, subkeys, s.q, bn, dbn_acc ? s.qhat : nullptr,
+                          c.G, c.dqf, reinterpret_cast<__nv_bfloat16*>(dq_pre),
+                          dbn_acc ? part : nullptr, c.dspart, dsub, want_dq, st);
     if (e != cudaSuccess) return e;
-    if (dbn) {
+    if (dbn_acc) {
       const int64_t nblk = (p.N + kDqTokensPerBlock - 1) / kDqTokensPerBlock;
-      dbn_reduce_kernel<<<(2 * p.hq + 255) / 256, 256, 0, st>>>(part, (int)nblk, p.hq, dbn);
+      if (train && (e = cudaMemsetAsync(c.bntot, 0, 2 * sizeof(float) * p.hq, st)) != cudaSuccess)
+        return e;
+      dbn_reduce_kernel<<<(2 * p.hq + 255) / 256, 256, 0, st>>>(part, (int)nblk, p.hq, dbn_acc);
       PKM_COUNT(1);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -1155,13 +1263,13 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
   if ((dx || dWq || dbn) && !tc_subgrad) {
     const int64_t nblk = (p.N + kDqTokensPerBlock - 1) / kDqTokensPerBlock;
     dim3 grid((unsigned)nblk, (unsigned)(p.h * 2));
-    float* partp = dbn ? part : nullptr;
-    const float* qh = dbn ? s.qhat : nullptr;
+    float* partp = dbn_acc ? part : nullptr;
+    const float* qh = dbn_acc ? s.qhat : nullptr;
     const bool split = tc_backward_supported(p);
 #define PKM_DQ(TS, MC, SPL)                                                                 \
   dq_kernel<TS, MC, SPL><<<grid, 256, 0, st>>>(gsub, s.sub_i, (const TS*)subkeys, bn, qh, \
                                                dq_pre, partp, p.N, p.h, p.dk, p.C1, p.C2,  \
-                                               p.k, p.eps)
+                                               p.k, p.eps, p.idw ? s.q : nullptr)
     if (p.fp32) {
       if (p.half / 4 <= 32) PKM_DQ(float, 1, false);
       else PKM_DQ(float, 4, false);
@@ -1175,8 +1283,22 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
 #undef PKM_DQ
     PKM_COUNT(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (dbn) {
-      dbn_reduce_kernel<<<(2 * p.hq + 255) / 256, 256, 0, st>>>(part, (int)nblk, p.hq, dbn); PKM_COUNT(1);
+    if (dbn_acc) {
+      if (train && (e = cudaMemsetAsync(c.bntot, 0, 2 * sizeof(float) * p.hq, st)) != cudaSuccess)
+        return e;
+      dbn_reduce_kernel<<<(2 * p.hq + 255) / 256, 256, 0, st>>>(part, (int)nblk, p.hq, dbn_acc); PKM_COUNT(1);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+  }
+  if (train) {
+    // dq_pre is bf16 hi/lo planes wherever the dense query gradients run on tensor cores
+    e = launch_bn_train_correct(p, dq_pre, tc_backward_supported(p), s.qhat, c.bneff, c.bntot,
+                                st);
+    if (e != cudaSuccess) return e;
+    if (dbn) {  // the caller's (d gamma, d beta) += the column sums
+      const int64_t nblk = (p.N + kDqTokensPerBlock - 1) / kDqTokensPerBlock;
+      dbn_reduce_kernel<<<(2 * p.hq + 255) / 256, 256, 0, st>>>(part, (int)nblk, p.hq, dbn);
+      PKM_COUNT(1);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
   }
@@ -1196,11 +1318,11 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
     const int E = p.fp32 ? 4 : 8;
     const int nv = p.half / E;
     if (p.fp32) {
-      if (nv <= 32) subkey_grad_kernel<false, 1><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status, p.bf16q ? 0.f : 1.f);
-      else subkey_grad_kernel<false, 4><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status, p.bf16q ? 0.f : 1.f); PKM_COUNT(1);
+      if (nv <= 32) subkey_grad_kernel<false, 1><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status, p.bf16q ? 0.f : 1.f, p.idw ? subkeys : nullptr);
+      else subkey_grad_kernel<false, 4><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status, p.bf16q ? 0.f : 1.f, p.idw ? subkeys : nullptr); PKM_COUNT(1);
     } else {
-      if (nv <= 32) subkey_grad_kernel<true, 1><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status, p.bf16q ? 0.f : 1.f);
-      else subkey_grad_kernel<true, 4><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status, p.bf16q ? 0.f : 1.f); PKM_COUNT(1);
+      if (nv <= 32) subkey_grad_kernel<true, 1><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status, p.bf16q ? 0.f : 1.f, p.idw ? subkeys : nullptr);
+      else subkey_grad_kernel<true, 4><<<persist_blocks, 256, 0, st>>>(seg, U, keys_sorted, ents2, gsub, s.q, dsub, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.status, p.bf16q ? 0.f : 1.f, p.idw ? subkeys : nullptr); PKM_COUNT(1);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

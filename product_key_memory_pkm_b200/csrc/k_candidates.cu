@@ -20,6 +20,8 @@ constexpr unsigned kFull = 0xffffffffu;
 __global__ void __launch_bounds__(256) candidate_topk_kernel(
     const float* __restrict__ sub_s, const int32_t* __restrict__ sub_i, int32_t* __restrict__ idx,
     float* __restrict__ w_out, int64_t NH, int k, int C2, float scale) {
+  grid_dependency_wait();  // the per-half lists come from the previous kernel
+  allow_dependent_launch();
   const int lane = threadIdx.x & 31;
   const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (g >= NH) return;  // warp-uniform
@@ -82,6 +84,39 @@ __global__ void __launch_bounds__(256) candidate_topk_kernel(
   }
 }
 
+// The all-k^2 variant (the code snippet of "Meta AI 可扩展内存层" section 10): every one
+// of the k*k candidates is kept, a-major (candidate a*k + b pairs the a-th key of the
+// first half with the b-th of the second), and the softmax runs over all of them.  One
+// warp per (token, head); lanes stride over the candidates.
+__global__ void __launch_bounds__(256) candidate_all_kernel(
+    const float* __restrict__ sub_s, const int32_t* __restrict__ sub_i, int32_t* __restrict__ idx,
+    float* __restrict__ w_out, int64_t NH, int k, int C2, float scale) {
+  grid_dependency_wait();  // the per-half lists come from the previous kernel
+  allow_dependent_launch();
+  const int lane = threadIdx.x & 31;
+  const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (g >= NH) return;  // warp-uniform
+  const int kk = k * k;
+  const float* s1 = sub_s + g * 2 * k;
+  const float* s2 = s1 + k;
+  const int32_t* i1 = sub_i + g * 2 * k;
+  const int32_t* i2 = i1 + k;
+  float mx = -INFINITY;
+  for (int c = lane; c < kk; c += 32) mx = fmaxf(mx, scale * (s1[c / k] + s2[c % k]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+  float sum = 0.f;
+  for (int c = lane; c < kk; c += 32) sum += expf(scale * (s1[c / k] + s2[c % k]) - mx);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
+  const float inv = 1.f / sum;
+  for (int c = lane; c < kk; c += 32) {
+    const int a = c / k, b = c % k;
+    idx[g * kk + c] = i1[a] * C2 + i2[b];
+    w_out[g * kk + c] = expf(scale * (s1[a] + s2[b]) - mx) * inv;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_candidates(const Plan& p, const float* sub_s, const int32_t* sub_i,
@@ -89,9 +124,16 @@ cudaError_t launch_candidates(const Plan& p, const float* sub_s, const int32_t* 
   const int64_t NH = p.N * p.h;
   const int warps = 8;
   const int64_t blocks = (NH + warps - 1) / warps;
-  candidate_topk_kernel<<<(unsigned)blocks, warps * 32, 0, st>>>(sub_s, sub_i, idx, w, NH, p.k,
-                                                                 p.C2, p.scale); PKM_COUNT(1);
-  return cudaGetLastError();
+  if (p.ksel != p.k) {
+    cudaError_t e = launch_dependent(candidate_all_kernel, dim3((unsigned)blocks), dim3(warps * 32),
+                                     0, st, sub_s, sub_i, idx, w, NH, p.k, p.C2, p.scale);
+    PKM_COUNT(1);
+    return e;
+  }
+  cudaError_t e = launch_dependent(candidate_topk_kernel, dim3((unsigned)blocks), dim3(warps * 32),
+                                   0, st, sub_s, sub_i, idx, w, NH, p.k, p.C2, p.scale);
+  PKM_COUNT(1);
+  return e;
 }
 
 }  // namespace pkm

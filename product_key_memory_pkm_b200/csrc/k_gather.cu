@@ -6,6 +6,8 @@
 // column slice of the value width and walks the token's h*k rows, keeping UNROLL
 // independent 16-byte loads in flight.  Indices and weights are staged in shared
 // memory once per token.  fp32 accumulation in registers, one coalesced store.
+#include <cooperative_groups.h>
+
 #include "pkm_internal.cuh"
 
 namespace pkm {
@@ -57,6 +59,8 @@ __global__ void __launch_bounds__(256) gather_bag_kernel(const TV* __restrict__ 
                                                          float* __restrict__ y, int64_t N, int hk,
                                                          int d_v, int64_t K, int* status,
                                                          Resid res = Resid{}) {
+  grid_dependency_wait();  // idx and w (and V's last write) come from earlier kernels
+  allow_dependent_launch();
   constexpr int E = Vec<TV>::kElems;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   int32_t* s_idx = reinterpret_cast<int32_t*>(smem_raw);
@@ -128,38 +132,153 @@ __global__ void __launch_bounds__(256) gather_bag_kernel(const TV* __restrict__ 
   }
 }
 
+// Few tokens (decode): one token's h*k rows are split over the S CTAs of a thread-block
+// cluster, CTA r taking rows r, r + S, ...; each keeps its partial sums in shared memory
+// and, after a cluster barrier, CTA 0 adds the S partials in rank order (reading the
+// others' shared memory directly) and stores y.  S times the loads in flight per token
+// of the one-CTA-per-token kernel; deterministic.
+template <typename TV, int S>
+__global__ void __cluster_dims__(S, 1, 1) __launch_bounds__(256)
+    gather_bag_split_kernel(const TV* __restrict__ V, const int32_t* __restrict__ idx,
+                            const float* __restrict__ w, float* __restrict__ y, int hk, int d_v,
+                            int64_t K, int* status) {
+  grid_dependency_wait();
+  allow_dependent_launch();
+  namespace cg = cooperative_groups;
+  constexpr int E = Vec<TV>::kElems;
+  extern __shared__ __align__(16) float part[];  // [d_v] partial sums of this CTA
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int64_t t = blockIdx.x / S;
+  const int nvec = d_v / E;
+  for (int c = threadIdx.x; c < nvec; c += blockDim.x) {
+    float acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    int r = rank;
+    constexpr int kAhead = 8;  // rows in flight per thread
+    for (; r + (kAhead - 1) * S < hk; r += kAhead * S) {
+      uint4 u[kAhead];
+      float wt[kAhead];
+#pragma unroll
+      for (int q = 0; q < kAhead; ++q) {
+        int32_t row = idx[t * hk + r + q * S];
+        if (row < 0 || row >= K) {
+          set_status(status, kDevIndex);
+          row = 0;
+        }
+        wt[q] = w[t * hk + r + q * S];
+        u[q] = ld_stream(reinterpret_cast<const uint4*>(V + (int64_t)row * d_v) + c);
+      }
+#pragma unroll
+      for (int q = 0; q < kAhead; ++q) {
+        float f[E];
+        if constexpr (E == 8) {
+          bf16x8_to_f32(u[q], f);
+        } else {
+          f[0] = __uint_as_float(u[q].x); f[1] = __uint_as_float(u[q].y);
+          f[2] = __uint_as_float(u[q].z); f[3] = __uint_as_float(u[q].w);
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = fmaf(wt[q], f[e], acc[e]);
+      }
+    }
+    for (; r < hk; r += S) {
+      int32_t row = idx[t * hk + r];
+      if (row < 0 || row >= K) {
+        set_status(status, kDevIndex);
+        row = 0;
+      }
+      const float wt = w[t * hk + r];
+      const uint4 u = ld_stream(reinterpret_cast<const uint4*>(V + (int64_t)row * d_v) + c);
+      float f[E];
+      if constexpr (E == 8) {
+        bf16x8_to_f32(u, f);
+      } else {
+        f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+        f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = fmaf(wt, f[e], acc[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) part[c * E + e] = acc[e];
+  }
+  cluster.sync();
+  if (rank == 0) {
+    for (int i = threadIdx.x; i < d_v / 4; i += blockDim.x) {
+      float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < S; ++q) {
+        const float4 v = reinterpret_cast<const float4*>(cluster.map_shared_rank(part, q))[i];
+        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+      }
+      reinterpret_cast<float4*>(y + t * d_v)[i] = s;
+    }
+  }
+  cluster.sync();  // the partials stay readable until CTA 0 has summed them
+}
+
+template <typename TV>
+cudaError_t launch_gather_split(const Plan& p, const TV* V, const int32_t* idx, const float* w,
+                                float* y, cudaStream_t st) {
+  constexpr int S = 8;
+  const int hk = p.h * p.ksel;
+  const int nvec = p.d_v / Vec<TV>::kElems;
+  const int threads = min(256, ((nvec + 31) / 32) * 32);
+  const size_t smem = (size_t)p.d_v * 4;
+  cudaError_t e;
+  if (smem > 48 * 1024 &&
+      (e = cudaFuncSetAttribute(gather_bag_split_kernel<TV, S>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+          cudaSuccess)
+    return e;
+  e = launch_dependent(gather_bag_split_kernel<TV, S>, dim3((unsigned)(p.N * S)), dim3(threads),
+                       smem, st, V, idx, w, y, hk, p.d_v, p.K, p.status);
+  PKM_COUNT(1);
+  return e;
+}
+
 }  // namespace
 
 cudaError_t launch_gather(const Plan& p, const void* values, const int32_t* idx, const float* w,
                           float* y, cudaStream_t st) {
-  const int hk = p.h * p.k;
+  const int hk = p.h * p.ksel;
   const size_t smem = (size_t)hk * 8;
+  // few tokens: split each token's rows over a cluster of CTAs (d_v*4 bytes of partials)
+  if (p.N < (int64_t)p.sm_count && hk >= 16 && (size_t)p.d_v * 4 <= 200 * 1024) {
+    if (p.vfp32)
+      return launch_gather_split(p, static_cast<const float*>(values), idx, w, y, st);
+    return launch_gather_split(p, static_cast<const __nv_bfloat16*>(values), idx, w, y, st);
+  }
   if (p.vfp32) {
     const int nvec = p.d_v / 4;
     const int threads = min(256, ((nvec + 31) / 32) * 32);
-    gather_bag_kernel<float, 8><<<(unsigned)p.N, threads, smem, st>>>(
-        static_cast<const float*>(values), idx, w, y, p.N, hk, p.d_v, p.K, p.status); PKM_COUNT(1);
+    PKM_COUNT(1);
+    return launch_dependent(gather_bag_kernel<float, 8, false>, dim3((unsigned)p.N), dim3(threads),
+                            smem, st, static_cast<const float*>(values), idx, w, y, p.N, hk,
+                            p.d_v, p.K, p.status, Resid{});
   } else {
     const int nvec = p.d_v / 8;
     const int threads = min(256, ((nvec + 31) / 32) * 32);
-    gather_bag_kernel<__nv_bfloat16, 8><<<(unsigned)p.N, threads, smem, st>>>(
-        static_cast<const __nv_bfloat16*>(values), idx, w, y, p.N, hk, p.d_v, p.K, p.status); PKM_COUNT(1);
+    PKM_COUNT(1);
+    return launch_dependent(gather_bag_kernel<__nv_bfloat16, 8, false>, dim3((unsigned)p.N),
+                            dim3(threads), smem, st, static_cast<const __nv_bfloat16*>(values), idx,
+                            w, y, p.N, hk, p.d_v, p.K, p.status, Resid{});
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_gather_resid(const Plan& p, const float* values, const int32_t* idx,
                                 const float* w, float* y, const void* tgt, bool tgt_bf16,
                                 int64_t tgt_ld, int64_t n_target, float* dy, cudaStream_t st) {
-  const int hk = p.h * p.k;
+  const int hk = p.h * p.ksel;
   const size_t smem = (size_t)hk * 8;
   const int nvec = p.d_v / 4;
   const int threads = min(256, ((nvec + 31) / 32) * 32);
-  gather_bag_kernel<float, 8, true><<<(unsigned)p.N, threads, smem, st>>>(
-      values, idx, w, y, p.N, hk, p.d_v, p.K, p.status,
-      Resid{tgt, tgt_ld, n_target, dy, tgt_bf16});
   PKM_COUNT(1);
-  return cudaGetLastError();
+  return launch_dependent(gather_bag_kernel<float, 8, true>, dim3((unsigned)p.N), dim3(threads),
+                          smem, st, values, idx, w, y, p.N, hk, p.d_v, p.K, p.status,
+                          Resid{tgt, tgt_ld, n_target, dy, tgt_bf16});
 }
 
 }  // namespace pkm

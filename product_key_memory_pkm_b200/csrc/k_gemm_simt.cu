@@ -115,9 +115,12 @@ struct EpiQuery {
   void* q;
   float* qhat;
   __device__ void operator()(int64_t m, int64_t n, float v) const {
-    float mean = bn[n], var = bn[hq + n], gamma = bn[2 * hq + n], beta = bn[3 * hq + n];
-    float qh = (v - mean) / sqrtf(var + eps);
-    float qq = fmaf(gamma, qh, beta);
+    float qh = v, qq = v;  // no bn: identity (training-mode BatchNorm follows)
+    if (bn) {
+      const float mean = bn[n], var = bn[hq + n], gamma = bn[2 * hq + n], beta = bn[3 * hq + n];
+      qh = (v - mean) / sqrtf(var + eps);
+      qq = fmaf(gamma, qh, beta);
+    }
     int64_t o = m * hq + n;
     if (split) {
       __nv_bfloat16 hi = __float2bfloat16_rn(qq);

@@ -27,7 +27,11 @@ __device__ __forceinline__ float load_q(const void* q, int64_t plane, int64_t of
   }
 }
 
-template <bool kSplitQ, typename TS, int KM>
+// kIdw: inverse-distance scores -1/2 log(||q - c||^2 + eps) ("Fast-weight Product Key
+// Memory", section 2.2), ||q - c||^2 = ||q||^2 + ||c||^2 - 2 q.c from the same tiles.
+constexpr float kIdwEps = 1e-12f;
+
+template <bool kSplitQ, typename TS, int KM, bool kIdw>
 __global__ void __launch_bounds__(TPB) scores_topk_simt(const void* __restrict__ q,
                                                         const TS* __restrict__ sub,
                                                         float* __restrict__ sub_s,
@@ -55,7 +59,7 @@ __global__ void __launch_bounds__(TPB) scores_topk_simt(const void* __restrict__
   }
 
   for (int c0 = 0; c0 < C; c0 += TC) {
-    float acc[4][4];
+    float acc[4][4], qn[4] = {0.f, 0.f, 0.f, 0.f}, cn[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -85,13 +89,24 @@ __global__ void __launch_bounds__(TPB) scores_topk_simt(const void* __restrict__
         for (int i = 0; i < 4; ++i)
 #pragma unroll
           for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        if constexpr (kIdw) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            qn[i] = fmaf(av[i], av[i], qn[i]);
+            cn[i] = fmaf(bv[i], bv[i], cn[i]);
+          }
+        }
       }
       __syncthreads();
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) Ssc[ty * 4 + i][tx * 4 + j] = acc[i][j];
+      for (int j = 0; j < 4; ++j) {
+        float v = acc[i][j];
+        if constexpr (kIdw) v = -0.5f * logf(fmaxf(qn[i] + cn[j] - 2.f * v, 0.f) + kIdwEps);
+        Ssc[ty * 4 + i][tx * 4 + j] = v;
+      }
     __syncthreads();
     if (tid < TT) {
       const int r = tid;
@@ -125,15 +140,14 @@ __global__ void __launch_bounds__(TPB) scores_topk_simt(const void* __restrict__
   }
 }
 
-template <bool kSplitQ, typename TS>
+template <bool kSplitQ, typename TS, bool kIdw>
 cudaError_t dispatch_km(const Plan& p, const void* subkeys, const void* q, float* sub_s,
                         int32_t* sub_i, cudaStream_t st) {
   dim3 grid((unsigned)((p.N + TT - 1) / TT), (unsigned)(p.h * 2));
   const TS* sub = static_cast<const TS*>(subkeys);
-#define PKM_LAUNCH(KMV)                                                                     \
-  scores_topk_simt<kSplitQ, TS, KMV><<<grid, TPB, 0, st>>>(q, sub, sub_s, sub_i, p.N, p.h, \
-                                                           p.dk, p.C1, p.C2, p.k,       \
-                                                           p.bf16q ? 0.f : 1.f)
+#define PKM_LAUNCH(KMV)                                                                      \
+  scores_topk_simt<kSplitQ, TS, KMV, kIdw><<<grid, TPB, 0, st>>>(                          \
+      q, sub, sub_s, sub_i, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.bf16q ? 0.f : 1.f)
   if (p.k <= 8)
     PKM_LAUNCH(8);
   else if (p.k <= 16)
@@ -149,8 +163,12 @@ cudaError_t dispatch_km(const Plan& p, const void* subkeys, const void* q, float
 
 cudaError_t launch_scores_simt(const Plan& p, const void* subkeys, const void* q, float* sub_s,
                                int32_t* sub_i, cudaStream_t st) {
-  if (p.fp32) return dispatch_km<false, float>(p, subkeys, q, sub_s, sub_i, st);
-  return dispatch_km<true, __nv_bfloat16>(p, subkeys, q, sub_s, sub_i, st);
+  if (p.idw) {
+    if (p.fp32) return dispatch_km<false, float, true>(p, subkeys, q, sub_s, sub_i, st);
+    return dispatch_km<true, __nv_bfloat16, true>(p, subkeys, q, sub_s, sub_i, st);
+  }
+  if (p.fp32) return dispatch_km<false, float, false>(p, subkeys, q, sub_s, sub_i, st);
+  return dispatch_km<true, __nv_bfloat16, false>(p, subkeys, q, sub_s, sub_i, st);
 }
 
 }  // namespace pkm

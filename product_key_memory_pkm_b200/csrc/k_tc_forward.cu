@@ -91,7 +91,10 @@ struct QueryProb {
     for (int j = row & 31; j < kBN; j += 32) {
       const int n = nt * kBN + j;
       float mean = 0.f, inv = 0.f, gamma = 0.f, beta = 0.f;
-      if (n < P.hq) {
+      if (n < P.hq && !P.bn) {  // identity: q = x Wq^T (training-mode BatchNorm follows)
+        inv = 1.f;
+        gamma = 1.f;
+      } else if (n < P.hq) {
         mean = P.bn[n];
         inv = 1.0f / sqrtf(P.bn[P.hq + n] + P.eps);
         gamma = P.bn[2 * P.hq + n];

@@ -54,7 +54,8 @@ pkm_status validate_dims(const pkm_dims* d) {
       d->score_scale > 3.0e38f)
     return PKM_ERR_INVALID_ARG;
   if ((int64_t)d->C1 * d->C2 >= ((int64_t)1 << 31)) return PKM_ERR_INVALID_ARG;
-  if (d->flags & ~(PKM_F_FP32 | PKM_F_SIMT | PKM_F_VALUES_FP32 | PKM_F_BF16_Q))
+  if (d->flags & ~(PKM_F_FP32 | PKM_F_SIMT | PKM_F_VALUES_FP32 | PKM_F_BF16_Q | PKM_F_BN_TRAIN |
+                   PKM_F_ALL_K2 | PKM_F_IDW))
     return PKM_ERR_INVALID_ARG;
   if ((d->flags & PKM_F_BF16_Q) && (d->flags & PKM_F_FP32)) return PKM_ERR_INVALID_ARG;
   const bool fp32 = d->flags & PKM_F_FP32;
@@ -64,7 +65,8 @@ pkm_status validate_dims(const pkm_dims* d) {
   if (d->k > 32 || d->h > 64) return PKM_ERR_UNSUPPORTED;
   const int half = d->dk / 2;
   if (fp32 ? (half / 4 > 128) : (half / 8 > 128)) return PKM_ERR_UNSUPPORTED;
-  if (d->N * (int64_t)d->h * d->k * 2 >= ((int64_t)1 << 31)) return PKM_ERR_UNSUPPORTED;
+  const int64_t ksel = (d->flags & PKM_F_ALL_K2) ? (int64_t)d->k * d->k : d->k;
+  if (d->N * (int64_t)d->h * ksel * 2 >= ((int64_t)1 << 31)) return PKM_ERR_UNSUPPORTED;
   if ((int64_t)d->h * d->dk > 65536) return PKM_ERR_UNSUPPORTED;
   return PKM_OK;
 }
@@ -88,6 +90,9 @@ Plan make_plan(const pkm_dims* d, int dev) {
   p.vfp32 = p.fp32 || (d->flags & PKM_F_VALUES_FP32);
   p.simt = p.fp32 || (d->flags & PKM_F_SIMT);
   p.bf16q = d->flags & PKM_F_BF16_Q;
+  p.bn_train = d->flags & PKM_F_BN_TRAIN;
+  p.ksel = (d->flags & PKM_F_ALL_K2) ? d->k * d->k : d->k;
+  p.idw = d->flags & PKM_F_IDW;
   p.sm_count = g_sm_count[dev];
   p.status = g_status_ptr[dev];
   return p;
@@ -119,16 +124,35 @@ pkm_status prepare(const pkm_dims* d, Plan* p) {
   return PKM_OK;
 }
 
-cudaError_t run_query(const Plan& p, const void* x, const void* Wq, const float* bn, void* q,
-                      float* qhat, cudaStream_t st) {
+cudaError_t run_query_gemm(const Plan& p, const void* x, const void* Wq, const float* bn, void* q,
+                           float* qhat, cudaStream_t st) {
+  if (small_n_supported(p)) return launch_query_small(p, x, Wq, bn, q, qhat, st);
   if (tc_forward_supported(p)) return launch_query_tc(p, x, Wq, bn, q, qhat, st);
   return launch_query_simt(p, x, Wq, bn, q, qhat, st);
 }
 
+// F1.  Training-mode BatchNorm: the GEMM without BatchNorm leaves x Wq^T in q-hat, whose
+// column statistics then normalise it (bn_batch receives them).
+cudaError_t run_query(const Plan& p, const void* x, const void* Wq, const float* bn, void* q,
+                      float* qhat, cudaStream_t st, float* bn_batch = nullptr) {
+  if (!p.bn_train) return run_query_gemm(p, x, Wq, bn, q, qhat, st);
+  cudaError_t e = run_query_gemm(p, x, Wq, nullptr, q, qhat, st);
+  if (e != cudaSuccess) return e;
+  return launch_bn_train_forward(p, bn, qhat, q, bn_batch, st);
+}
+
 cudaError_t run_scores(const Plan& p, const void* subkeys, const void* q, float* sub_s,
                        int32_t* sub_i, cudaStream_t st) {
-  if (tc_forward_supported(p)) return launch_scores_tc(p, subkeys, q, sub_s, sub_i, st);
+  if (small_n_supported(p)) return launch_scores_small(p, subkeys, q, sub_s, sub_i, st);
+  if (tc_forward_supported(p) && !p.idw) return launch_scores_tc(p, subkeys, q, sub_s, sub_i, st);
   return launch_scores_simt(p, subkeys, q, sub_s, sub_i, st);
+}
+
+pkm_status check_bn_train(const pkm_dims* d, const pkm_saved* s) {
+  if (!(d->flags & PKM_F_BN_TRAIN)) return PKM_OK;
+  if (!s || !s->qhat || !s->bn_batch) return PKM_ERR_INVALID_ARG;
+  PKM_NEED(s->qhat); PKM_NEED(s->bn_batch);
+  return PKM_OK;
 }
 
 pkm_status check_saved_fwd(const pkm_saved* s) {
@@ -157,15 +181,17 @@ extern "C" {
 
 size_t pkm_saved_bytes(const pkm_dims* d, int field) {
   if (validate_dims(d) != PKM_OK) return 0;
-  const int64_t N = d->N, hq = (int64_t)d->h * d->dk, sel = N * d->h * d->k;
+  const int64_t ksel = (d->flags & PKM_F_ALL_K2) ? (int64_t)d->k * d->k : d->k;
+  const int64_t N = d->N, hq = (int64_t)d->h * d->dk, sel = N * d->h * ksel;
   const bool fp32 = d->flags & PKM_F_FP32;
   switch (field) {
     case PKM_SAVED_Q: return (size_t)(fp32 ? 4 * N * hq : 2 * 2 * N * hq);
     case PKM_SAVED_QHAT: return (size_t)(4 * N * hq);
     case PKM_SAVED_SUB_S:
-    case PKM_SAVED_SUB_I: return (size_t)(4 * 2 * sel);
+    case PKM_SAVED_SUB_I: return (size_t)(4 * 2 * N * d->h * d->k);
     case PKM_SAVED_IDX:
     case PKM_SAVED_W: return (size_t)(4 * sel);
+    case PKM_SAVED_BN_BATCH: return (size_t)(4 * 2 * hq);
     default: return 0;
   }
 }
@@ -179,6 +205,7 @@ size_t pkm_workspace_bytes(const pkm_dims* d, int which) {
   p.C1 = d->C1; p.C2 = d->C2; p.k = d->k; p.d_v = d->d_v; p.hq = d->h * d->dk;
   p.K = (int64_t)d->C1 * d->C2; p.fp32 = d->flags & PKM_F_FP32;
   p.vfp32 = p.fp32 || (d->flags & PKM_F_VALUES_FP32);
+  p.ksel = (d->flags & PKM_F_ALL_K2) ? d->k * d->k : d->k;
   return backward_workspace_bytes(p);
 }
 
@@ -189,10 +216,11 @@ pkm_status pkm_query(const pkm_dims* d, const void* x, const void* Wq, const flo
   PKM_NEED(x); PKM_NEED(Wq); PKM_NEED(bn);
   if (!saved) return PKM_ERR_INVALID_ARG;
   PKM_NEED(saved->q); PKM_OPT(saved->qhat);
+  PKM_TRY(check_bn_train(d, saved));
   Plan p;
   PKM_TRY(prepare(d, &p));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return cuda_status(run_query(p, x, Wq, bn, saved->q, saved->qhat, st));
+  return cuda_status(run_query(p, x, Wq, bn, saved->q, saved->qhat, st, saved->bn_batch));
 }
 
 pkm_status pkm_subkey_scores(const pkm_dims* d, const void* subkeys, const pkm_saved* saved,
@@ -238,11 +266,12 @@ pkm_status pkm_forward(const pkm_dims* d, const void* x, const void* Wq, const f
   if (d->N == 0) return PKM_OK;
   PKM_NEED(x); PKM_NEED(Wq); PKM_NEED(bn); PKM_NEED(subkeys); PKM_NEED(values); PKM_NEED(y);
   PKM_TRY(check_saved_fwd(saved));
+  PKM_TRY(check_bn_train(d, saved));
   PKM_TRY(check_workspace(pkm_workspace_bytes(d, PKM_FWD), workspace, workspace_bytes));
   Plan p;
   PKM_TRY(prepare(d, &p));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  PKM_TRY(cuda_status(run_query(p, x, Wq, bn, saved->q, saved->qhat, st)));
+  PKM_TRY(cuda_status(run_query(p, x, Wq, bn, saved->q, saved->qhat, st, saved->bn_batch)));
   PKM_TRY(cuda_status(run_scores(p, subkeys, saved->q, saved->sub_s, saved->sub_i, st)));
   PKM_TRY(cuda_status(launch_candidates(p, saved->sub_s, saved->sub_i, saved->idx, saved->w, st)));
   return cuda_status(launch_gather(p, values, saved->idx, saved->w, y, st));
@@ -259,6 +288,7 @@ pkm_status pkm_backward(const pkm_dims* d, const void* x, const void* Wq, const 
   PKM_TRY(check_saved_fwd(saved));
   PKM_OPT(dx); PKM_OPT(dWq); PKM_OPT(dbn); PKM_OPT(dsubkeys); PKM_OPT(dvalues); PKM_OPT(dw_out);
   if (dbn && !saved->qhat) return PKM_ERR_INVALID_ARG;
+  PKM_TRY(check_bn_train(d, saved));
   PKM_TRY(check_workspace(pkm_workspace_bytes(d, PKM_BWD), workspace, workspace_bytes));
   Plan p;
   PKM_TRY(prepare(d, &p));
@@ -292,6 +322,7 @@ pkm_status pkm_query_grad(const pkm_dims* d, const void* x, const void* Wq, cons
   PKM_TRY(check_saved_fwd(saved));
   PKM_OPT(dx); PKM_OPT(dWq); PKM_OPT(dbn); PKM_OPT(dsubkeys);
   if (dbn && !saved->qhat) return PKM_ERR_INVALID_ARG;
+  PKM_TRY(check_bn_train(d, saved));
   PKM_TRY(check_workspace(pkm_workspace_bytes(d, PKM_BWD), workspace, workspace_bytes));
   Plan p;
   PKM_TRY(prepare(d, &p));
@@ -323,7 +354,7 @@ enum FwMode { kChunkSort, kPresort, kPerChunk };
 
 Plan fw_shape(const pkm_dims* d) {
   Plan p{};
-  p.N = d->N; p.h = d->h; p.k = d->k; p.K = (int64_t)d->C1 * d->C2;
+  p.N = d->N; p.h = d->h; p.k = d->k; p.ksel = d->k; p.K = (int64_t)d->C1 * d->C2;
   return p;
 }
 
@@ -418,6 +449,8 @@ pkm_status pkm_fastweight_chunks(const pkm_dims* d, int64_t chunk, float lr, uin
                                  float* y, void* workspace, size_t workspace_bytes,
                                  void* stream) {
   PKM_TRY(validate_fw(d, chunk, lr, mode));
+  // the loop's BatchNorm is eval; its writes are sorted per k selections
+  if (d->flags & (PKM_F_BN_TRAIN | PKM_F_ALL_K2)) return PKM_ERR_INVALID_ARG;
   if (d->N == 0) return PKM_OK;
   const bool lookahead = mode & PKM_FW_LOOKAHEAD;
   PKM_NEED(x); PKM_NEED(Wq); PKM_NEED(bn); PKM_NEED(subkeys); PKM_NEED(values); PKM_NEED(y);
@@ -544,6 +577,17 @@ pkm_status pkm_hit_counts(const pkm_dims* d, const int32_t* idx, int32_t* slot_h
   return cuda_status(launch_hit_counts(p, idx, slot_hits, subkey_hits, st));
 }
 
+pkm_status pkm_bn_running_update(const pkm_dims* d, float* bn, const float* bn_batch,
+                                 float momentum, void* stream) {
+  PKM_TRY(validate_dims(d));
+  if (d->N < 2 || !(momentum >= 0.f && momentum <= 1.f)) return PKM_ERR_INVALID_ARG;
+  PKM_NEED(bn); PKM_NEED(bn_batch);
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(launch_bn_running(p, bn, bn_batch, momentum, st));
+}
+
 unsigned long long pkm_launch_count(void) { return g_launches.load(); }
 
 pkm_status pkm_selftest_wait_timeout(uint32_t budget_cycles, void* stream) {
@@ -635,6 +679,7 @@ extern "C" pkm_status pkm_value_grad_noalloc(const pkm_dims* d, const void* valu
     q.N = d->N; q.d_in = d->d_in; q.h = d->h; q.dk = d->dk; q.half = d->dk / 2;
     q.C1 = d->C1; q.C2 = d->C2; q.k = d->k; q.d_v = d->d_v; q.hq = d->h * d->dk;
     q.K = (int64_t)d->C1 * d->C2; q.fp32 = d->flags & PKM_F_FP32;
+    q.ksel = (d->flags & PKM_F_ALL_K2) ? d->k * d->k : d->k;
     if (value_stage_scratch_bytes(q) > kNoAllocScratchBytes) return PKM_ERR_WORKSPACE;
   }
   Plan p;

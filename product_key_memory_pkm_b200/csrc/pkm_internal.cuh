@@ -39,6 +39,35 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
   }
 }
 
+// ---------------------------------------------------------------- dependent launches
+// A kernel launched with launch_dependent may start while the previous kernel on the
+// stream is finishing; before it reads anything that kernel wrote it waits in
+// grid_dependency_wait (returns at once when launched the ordinary way).  A producer may
+// call allow_dependent_launch once its dependents may begin their prologue; the wait
+// still covers all of its memory operations.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ---------------------------------------------------------------- launch counter
 // Every kernel launch of the library is counted (host side) for diagnostics.
 void count_launches(int n);
@@ -54,6 +83,9 @@ struct Plan {
   bool fp32;      // fp32 storage
   bool vfp32;     // fp32 value table (fp32, or bf16 x/Wq/subkeys beside fp32 values)
   bool bf16q;     // scores (and the sub-key gradient) take q rounded to bf16 (hi plane)
+  bool bn_train;  // training-mode BatchNorm (batch statistics)
+  int ksel;       // selections per head: k, or k*k for the all-k^2 variant
+  bool idw;       // inverse-distance sub-key scores
   bool simt;      // CUDA-core kernels for bf16 storage
   int sm_count;
   int* status;    // device status word
@@ -78,6 +110,22 @@ cudaError_t launch_dwq_tc(const Plan& p, const void* dq_planes, const void* x, f
                           cudaStream_t st);
 cudaError_t launch_candidates(const Plan& p, const float* sub_s, const int32_t* sub_i,
                               int32_t* idx, float* w, cudaStream_t st);
+// Training-mode BatchNorm: statistics of pre (left in the q-hat buffer by an identity-BN
+// query GEMM), then q-hat and q; the backward's correction of dq_pre for the batch
+// statistics (tot = column sums (d gamma, d beta)); the running-statistics update.
+cudaError_t launch_bn_train_forward(const Plan& p, const float* bn, float* qhat_pre, void* q,
+                                    float* bn_batch, cudaStream_t st);
+cudaError_t launch_bn_train_correct(const Plan& p, void* dq_pre, bool planes, const float* qhat,
+                                    const float* bn_eff, const float* tot, cudaStream_t st);
+cudaError_t launch_bn_running(const Plan& p, float* bn, const float* bn_batch, float momentum,
+                              cudaStream_t st);
+// Few tokens (decode): CUDA-core F1 and F2 spread over many CTAs (bf16 storage).
+constexpr int64_t kSmallTokens = 16;
+bool small_n_supported(const Plan& p);
+cudaError_t launch_query_small(const Plan& p, const void* x, const void* Wq, const float* bn,
+                               void* q, float* qhat, cudaStream_t st);
+cudaError_t launch_scores_small(const Plan& p, const void* subkeys, const void* q, float* sub_s,
+                                int32_t* sub_i, cudaStream_t st);
 cudaError_t launch_gather(const Plan& p, const void* values, const int32_t* idx, const float* w,
                           float* y, cudaStream_t st);
 

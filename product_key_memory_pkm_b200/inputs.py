@@ -74,7 +74,11 @@ FASTWEIGHT = PKMConfig("fwpkm_chunk512_K1024x1024_h1_k8_d1024", N=4096, d_in=102
                        dk=512, C1=1024, C2=1024, k=8, d_v=1024, value_dtype="f32",
                        clustered=64)
 
-CONFIGS = {c.name: c for c in (TINY_FP32, FWD_K512, FULL_K1024, FASTWEIGHT)}
+# the full workload with unequal sub-key sets (|C| = 2048, |C'| = 512: the same 1M slots)
+FULL_K2048x512 = PKMConfig("pkm_fwdbwd_K2048x512_h4_k32_d1600", N=16384, d_in=1600, h=4,
+                           dk=512, C1=2048, C2=512, k=32, d_v=1600)
+
+CONFIGS = {c.name: c for c in (TINY_FP32, FWD_K512, FULL_K1024, FASTWEIGHT, FULL_K2048x512)}
 
 
 def _round_bf16(a: np.ndarray) -> np.ndarray:

@@ -31,11 +31,14 @@ PKM_F_FP32 = 0x1
 PKM_F_SIMT = 0x2
 PKM_F_VALUES_FP32 = 0x4
 PKM_F_BF16_Q = 0x8
+PKM_F_BN_TRAIN = 0x10
+PKM_F_ALL_K2 = 0x20
+PKM_F_IDW = 0x40
 PKM_FWD, PKM_BWD = 0, 1
 PKM_FW_LOOKAHEAD = 0x1
 PKM_FW_SORT_GLOBAL = 0x2
 PKM_FW_PER_CHUNK = 0x4
-SAVED_FIELDS = ("q", "qhat", "sub_s", "sub_i", "idx", "w")
+SAVED_FIELDS = ("q", "qhat", "sub_s", "sub_i", "idx", "w", "bn_batch")
 
 # every symbol include/pkm.h declares
 EXPORTED = ("pkm_saved_bytes", "pkm_workspace_bytes", "pkm_forward", "pkm_backward", "pkm_query",
@@ -43,7 +46,7 @@ EXPORTED = ("pkm_saved_bytes", "pkm_workspace_bytes", "pkm_forward", "pkm_backwa
             "pkm_status_string", "pkm_build_info", "pkm_value_grad", "pkm_query_grad",
             "pkm_launch_count", "pkm_selftest_wait_timeout", "pkm_value_grad_noalloc",
             "pkm_fastweight_workspace_bytes", "pkm_fastweight_chunks", "pkm_value_sgd",
-            "pkm_value_grad_rows", "pkm_value_adam", "pkm_hit_counts")
+            "pkm_value_grad_rows", "pkm_value_adam", "pkm_hit_counts", "pkm_bn_running_update")
 
 
 class PKMError(RuntimeError):
@@ -100,6 +103,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "pkm_value_adam": (I, [D, ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_float,
                                ctypes.c_int64, P, P, P, SV, P, P, S, P]),
         "pkm_hit_counts": (I, [D, P, P, P, P]),
+        "pkm_bn_running_update": (I, [D, P, P, ctypes.c_float, P]),
         "pkm_fastweight_workspace_bytes": (S, [D, ctypes.c_int64, ctypes.c_uint32]),
         "pkm_fastweight_chunks": (I, [D, ctypes.c_int64, ctypes.c_float, ctypes.c_uint32, P, P, P,
                                       P, P, P, P, P, S, P]),
@@ -267,6 +271,13 @@ def pkm_hit_counts(dims: Dims, idx, slot_hits=None, subkey_hits=None, stream=Non
                                  _ptr(subkey_hits), _stream(stream)), "pkm_hit_counts")
 
 
+def pkm_bn_running_update(dims: Dims, bn, bn_batch, momentum: float = 0.1, stream=None) -> None:
+    """Fold a training-mode batch's statistics into bn's running mean and variance."""
+    _check(load().pkm_bn_running_update(ctypes.byref(dims.c()), _ptr(bn), _ptr(bn_batch),
+                                        float(momentum), _stream(stream)),
+           "pkm_bn_running_update")
+
+
 def pkm_fastweight_workspace_bytes(dims: Dims, chunk: int, mode: int = 0) -> int:
     return int(load().pkm_fastweight_workspace_bytes(ctypes.byref(dims.c()), int(chunk),
                                                      int(mode)))
@@ -347,7 +358,8 @@ def pkm_build_info() -> str:
 def alloc_saved(dims: Dims, device="cuda", with_qhat: bool = True) -> dict:
     """Caller-owned buffers the forward writes and the backward reads (torch)."""
     import torch
-    N, hq, sel = dims.N, dims.h * dims.dk, dims.N * dims.h * dims.k
+    N, hq = dims.N, dims.h * dims.dk
+    ksel = dims.k * dims.k if dims.flags & PKM_F_ALL_K2 else dims.k
     fp32 = bool(dims.flags & PKM_F_FP32)
     q = (torch.empty(N, hq, dtype=torch.float32, device=device) if fp32 else
          torch.empty(2, N, hq, dtype=torch.bfloat16, device=device))
@@ -356,8 +368,9 @@ def alloc_saved(dims: Dims, device="cuda", with_qhat: bool = True) -> dict:
         qhat=torch.empty(N, hq, dtype=torch.float32, device=device) if with_qhat else None,
         sub_s=torch.empty(N, dims.h, 2, dims.k, dtype=torch.float32, device=device),
         sub_i=torch.empty(N, dims.h, 2, dims.k, dtype=torch.int32, device=device),
-        idx=torch.empty(N, dims.h, dims.k, dtype=torch.int32, device=device),
-        w=torch.empty(N, dims.h, dims.k, dtype=torch.float32, device=device),
+        idx=torch.empty(N, dims.h, ksel, dtype=torch.int32, device=device),
+        w=torch.empty(N, dims.h, ksel, dtype=torch.float32, device=device),
+        bn_batch=torch.empty(2, hq, dtype=torch.float32, device=device),
     )
 
 

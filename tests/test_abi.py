@@ -38,7 +38,7 @@ def test_build_targets_sm100a_only():
 
 def test_struct_layout_matches_header():
     assert ctypes.sizeof(P.pkm_dims) == 48
-    assert ctypes.sizeof(P.pkm_saved) == 6 * ctypes.sizeof(ctypes.c_void_p)
+    assert ctypes.sizeof(P.pkm_saved) == 7 * ctypes.sizeof(ctypes.c_void_p)
 
 
 def test_status_strings(lib):
@@ -191,6 +191,24 @@ def test_binding_fails_loudly_without_library(tmp_path):
         importlib.reload(P)
 
 
+def test_training_batch_norm_validation(lib):
+    L = P.load()
+    d = _dims(flags=P.PKM_F_BN_TRAIN)
+    saved = {f: FAKE for f in P.SAVED_FIELDS}
+    for missing in ("qhat", "bn_batch"):
+        s = dict(saved, **{missing: None})
+        rc = L.pkm_forward(ctypes.byref(d.c()), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                           ctypes.byref(P._saved_c(s)), None, 0, None)
+        assert rc == P.PKM_ERR_INVALID_ARG, missing
+    upd = lambda dd, m: L.pkm_bn_running_update(ctypes.byref(dd.c()), FAKE, FAKE, m, None)
+    assert upd(_dims(N=1), 0.1) == P.PKM_ERR_INVALID_ARG        # unbiased variance needs N >= 2
+    assert upd(d, 1.5) == P.PKM_ERR_INVALID_ARG
+    fw = _dims(flags=P.PKM_F_BN_TRAIN | P.PKM_F_FP32)
+    rc = L.pkm_fastweight_chunks(ctypes.byref(fw.c()), 16, 0.5, 0, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                 FAKE, FAKE, FAKE, 1 << 30, None)
+    assert rc == P.PKM_ERR_INVALID_ARG                          # the loop's BatchNorm is eval
+
+
 def test_training_pieces_validation(lib):
     L = P.load()
     d = _dims()
@@ -223,3 +241,15 @@ def test_training_pieces_validation(lib):
     assert hits(idx=None) == P.PKM_ERR_INVALID_ARG
     assert hits(slot=FAKE + 2) == P.PKM_ERR_INVALID_ARG
     assert hits(idx=None, slot=None, sub=None) == P.PKM_OK    # nothing asked
+
+
+def test_all_k2_sizes(lib):
+    """The all-k^2 variant keeps k*k selections per head: idx and w grow, the per-half
+    lists do not."""
+    d, d2 = _dims(), _dims(flags=P.PKM_F_ALL_K2)
+    assert P.pkm_saved_bytes(d2, "idx") == d.k * P.pkm_saved_bytes(d, "idx")
+    assert P.pkm_saved_bytes(d2, "w") == d.k * P.pkm_saved_bytes(d, "w")
+    assert P.pkm_saved_bytes(d2, "sub_i") == P.pkm_saved_bytes(d, "sub_i")
+    assert P.pkm_workspace_bytes(d2, P.PKM_BWD) > P.pkm_workspace_bytes(d, P.PKM_BWD)
+    big = _dims(N=1 << 18, k=32, h=4, flags=P.PKM_F_ALL_K2)       # 2^18*4*1024*2 = 2^31
+    assert _fwd(big) == P.PKM_ERR_UNSUPPORTED

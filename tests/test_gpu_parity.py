@@ -36,15 +36,21 @@ CASES = {
     "duplicate_heavy": _cfg(N=512, d_in=64, h=1, C1=64, C2=64, k=8, d_v=128, clustered=8),
     "unequal_C_wide_dv": _cfg(N=130, h=1, dk=128, C1=96, C2=40, k=24, d_v=2056),
     "fp32_values_bf16_rest": _cfg(N=211, value_dtype="f32", d_v=136),
+    # few tokens (N <= 16): CUDA-core query and cluster-split scoring and bag
+    "few_tokens_unequal_C_k8": _cfg(N=13, h=2, dk=64, C1=96, C2=40, k=8),
+    "few_tokens_k32_small_C": _cfg(N=16, h=3, k=32, C1=40, C2=33, d_v=72),
+    "split_bag_37_tokens": _cfg(N=37, h=2, dk=64, C1=96, C2=40, k=8),
 }
 
 
-def _full_check(cfg, seed=0, flags=0, inp=None, q_bf16=False):
+def _full_check(cfg, seed=0, flags=0, inp=None, q_bf16=False, bn_train=False, idw=False):
     if inp is None:
         inp = make_inputs(cfg, seed=seed, random_bn=True)
     dev = H.to_dev(inp, cfg)
     dims, saved, y = H.gpu_forward(cfg, dev, flags=flags)
-    of = O.forward(inp, cfg, q_bf16=q_bf16)
+    of = O.forward(inp, cfg, q_bf16=q_bf16, bn_train=bn_train, idw=idw)
+    if bn_train:   # the batch statistics the forward recorded
+        H.assert_rows(saved["bn_batch"].cpu().numpy(), np.stack(of["bn_batch"]), "bn_batch")
     ranked = H.oracle_gaps(of, cfg)
     idx = saved["idx"].cpu().numpy()
     clean = H.check_indices(idx, of, cfg, ranked)
@@ -99,12 +105,13 @@ def _exact_query_inputs(cfg, seed):
     return inp, cfg.with_(bn_eps=eps)
 
 
-@pytest.mark.parametrize("simt", [False, True])
-def test_single_pass_bf16_q_scoring(simt):
-    """PKM_F_BF16_Q: scores from q rounded to bf16 (one tensor-core pass, or the CUDA-core
-    kernel dropping the lo plane), the sub-key gradient from the same rounded q, the
-    query gradient straight through -- against the oracle's bf16-q variant."""
-    cfg = _cfg(N=300)
+@pytest.mark.parametrize("simt,n", [(False, 300), (True, 300), (False, 12)])
+def test_single_pass_bf16_q_scoring(simt, n):
+    """PKM_F_BF16_Q: scores from q rounded to bf16 (one tensor-core pass, the CUDA-core
+    kernel, or the few-token kernel dropping the lo plane), the sub-key gradient from the
+    same rounded q, the query gradient straight through -- against the oracle's bf16-q
+    variant."""
+    cfg = _cfg(N=n)
     inp, cfg = _exact_query_inputs(cfg, 5)
     # the variant is visible: its scores move well beyond the index tolerance
     f0, f1 = O.forward(inp, cfg), O.forward(inp, cfg, q_bf16=True)
@@ -112,6 +119,34 @@ def test_single_pass_bf16_q_scoring(simt):
     flags = P.PKM_F_BF16_Q | (P.PKM_F_SIMT if simt else 0)
     clean = _full_check(cfg, flags=flags, inp=inp, q_bf16=True)
     assert clean.mean() > 0.5
+
+
+@pytest.mark.parametrize("case", ["tensor_core", "simt", "fp32", "few_tokens"])
+def test_training_mode_batch_norm(case):
+    """PKM_F_BN_TRAIN: the query normalised with the batch's statistics, the backward
+    through them (every token's dx depends on all tokens), and the running-statistics
+    update -- against the oracle's training-mode BatchNorm."""
+    cfg, flags = {
+        "tensor_core": (_cfg(N=300), 0),
+        "simt": (_cfg(N=300), P.PKM_F_SIMT),
+        "fp32": (_cfg(N=200, dtype="f32", dk=40), 0),
+        "few_tokens": (_cfg(N=12), 0),
+    }[case]
+    inp = make_inputs(cfg, seed=12, random_bn=True)
+    clean = _full_check(cfg, flags=flags | P.PKM_F_BN_TRAIN, inp=inp, bn_train=True)
+    assert clean.mean() > 0.5
+    # running statistics: fold the batch into bn
+    dims = P.Dims.from_config(cfg, flags=flags | P.PKM_F_BN_TRAIN)
+    dev = H.to_dev(inp, cfg)
+    saved = P.alloc_saved(dims)
+    y = torch.empty(cfg.N, cfg.d_v, device="cuda")
+    P.pkm_forward(dims, dev["x"], dev["Wq"], dev["bn"], dev["subkeys"], dev["values"], y, saved)
+    bn = dev["bn"].clone()
+    P.pkm_bn_running_update(dims, bn, saved["bn_batch"], 0.1)
+    assert P.pkm_check_status() == P.PKM_OK
+    of = O.forward(inp, cfg, bn_train=True)
+    want = O.running_stats_update(inp["bn"], *of["bn_batch"], cfg.N, 0.1)
+    H.assert_rows(bn.cpu().numpy(), want, "running statistics")
 
 
 def test_stagewise_scores_given_oracle_query():
@@ -322,3 +357,70 @@ def test_fast_weight_chunk_shape_fp32_values_duplicates():
     g = H.gpu_backward(cfg, dims, dev, saved, torch.from_numpy(dy).cuda(), want=("dV", "dw"))
     ob = O.backward(inp, cfg, of, dy)
     H.assert_rows(g["dV"].cpu().numpy()[ob["dV_rows"]], ob["dV_vals"], "dV")
+
+
+@pytest.mark.parametrize("n", [200, 12])
+def test_all_k2_variant(n):
+    """PKM_F_ALL_K2: every candidate of top-k(s1) x top-k(s2) is kept and the softmax runs
+    over all k^2 of them.  A head's candidate set is unique where both halves separate
+    their k-th from their (k+1)-th sub-key by more than the tolerance; other tokens are
+    left out of the output comparison and their upstream gradient is masked."""
+    cfg = _cfg(N=n, h=2, k=8, C1=64, C2=48)
+    inp = make_inputs(cfg, seed=13, random_bn=True)
+    dev = H.to_dev(inp, cfg)
+    dims, saved, y = H.gpu_forward(cfg, dev, flags=P.PKM_F_ALL_K2)
+    of = O.forward(inp, cfg, all_k2=True)
+    k, kk = cfg.k, cfg.k * cfg.k
+    idx = saved["idx"].cpu().numpy()
+    assert idx.shape == (cfg.N, cfg.h, kk)
+    clean = np.ones(cfg.N, dtype=bool)
+    for t in range(cfg.N):
+        for hh in range(cfg.h):
+            for s in (of["s1"][t, hh], of["s2"][t, hh]):
+                r = np.sort(s)[::-1]
+                if r[k - 1] - r[k] <= H.GAP_REL * max(abs(r[k - 1]), 1e-2):
+                    clean[t] = False
+            if clean[t]:
+                assert set(idx[t, hh].tolist()) == set(of["idx"][t, hh].tolist()), (t, hh)
+    assert clean.mean() > 0.5
+    H.assert_rows(y.cpu().numpy()[clean], of["y"][clean], "y")
+    wg = H.align_to(idx[clean], of["idx"][clean], saved["w"].cpu().numpy()[clean])
+    H.assert_rows(wg.reshape(-1, kk), of["w"][clean].reshape(-1, kk), "w")
+    dy = inp["dy"] * clean[:, None]
+    z = lambda *s: torch.zeros(*s, dtype=torch.float32, device="cuda")
+    g = dict(dx=z(cfg.N, cfg.d_in), dWq=z(cfg.h * cfg.dk, cfg.d_in), dbn=z(2, cfg.h * cfg.dk),
+             dsub=z(cfg.h, cfg.C1 + cfg.C2, cfg.dk // 2), dV=z(cfg.K, cfg.d_v),
+             dw=z(cfg.N, cfg.h, kk))
+    ws = P.alloc_workspace(dims, P.PKM_BWD)
+    P.pkm_backward(dims, dev["x"], dev["Wq"], dev["bn"], dev["subkeys"], dev["values"], saved,
+                   torch.from_numpy(dy).cuda(), dx=g["dx"], dWq=g["dWq"], dbn=g["dbn"],
+                   dsubkeys=g["dsub"], dvalues=g["dV"], dw_out=g["dw"], workspace=ws)
+    assert P.pkm_check_status() == P.PKM_OK
+    ob = O.backward(inp, cfg, of, dy)
+    H.assert_rows(g["dx"].cpu().numpy(), ob["dx"], "dx")
+    H.assert_rows(g["dWq"].cpu().numpy(), ob["dWq"], "dWq")
+    H.assert_rows(g["dbn"].cpu().numpy(), np.stack([ob["dgamma"], ob["dbeta"]]), "dbn")
+    H.assert_rows(g["dsub"].cpu().numpy().reshape(-1, cfg.dk // 2),
+                  ob["dsub"].reshape(-1, cfg.dk // 2), "dsub")
+    H.assert_rows(g["dV"].cpu().numpy()[ob["dV_rows"]], ob["dV_vals"], "dV")
+    dwg = H.align_to(idx[clean], of["idx"][clean], g["dw"].cpu().numpy()[clean])
+    H.assert_rows(dwg.reshape(-1, kk), ob["dw"][clean].reshape(-1, kk), "dw")
+
+
+@pytest.mark.parametrize("case", ["bf16", "fp32", "few_tokens"])
+def test_inverse_distance_scores(case):
+    """PKM_F_IDW: sub-key scores -1/2 log(||q_half - c||^2 + eps), on the CUDA-core and the
+    few-token kernels, and their backward (u = g / d^2 corrections) -- against the oracle's
+    inverse-distance scorer.  Sub-keys ~ N(0, 1), at the queries' scale, so that distances
+    differ across keys."""
+    cfg = {"bf16": _cfg(N=200, h=2, dk=64, C1=64, C2=48, k=16, d_v=64),
+           "fp32": _cfg(N=200, h=2, dk=64, C1=64, C2=48, k=16, d_v=64, dtype="f32"),
+           "few_tokens": _cfg(N=14, h=2, dk=64, C1=64, C2=48, k=16, d_v=64)}[case]
+    inp = make_inputs(cfg, seed=14, random_bn=True)
+    rng = np.random.default_rng(99)
+    sub = rng.standard_normal(inp["subkeys"].shape).astype(np.float32)
+    if cfg.dtype == "bf16":
+        sub = torch.from_numpy(sub).bfloat16().float().numpy()
+    inp["subkeys"] = sub
+    clean = _full_check(cfg, flags=P.PKM_F_IDW, inp=inp, idw=True)
+    assert clean.mean() > 0.5
