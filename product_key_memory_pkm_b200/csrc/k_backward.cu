@@ -528,7 +528,7 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
   {
     const int E = p.vfp32 ? 4 : 8;
     const int nvec = p.d_v / E;
-    const int blocks = p.sm_count * 6;
+    const int blocks = p.sm_count * PKM_B3_MIN_BLOCKS;
     const size_t smem = value_rows_smem(p);
 #define PKM_B3(TV, CHV)                                                                      \
   do {                                                                                       \

@@ -128,7 +128,12 @@ __device__ __forceinline__ void prefetch_l1(const void* p) {
 // ws_sorted[p] = w[ents[p]]: the selection weights in row order, so staging a batch
 // needs two independent loads.
 template <typename TV, int CH>
-__global__ void __launch_bounds__(kB3Threads, 6) value_rows_kernel(
+// resident CTAs per SM the pass is compiled and launched for (a tuning value)
+#ifndef PKM_B3_MIN_BLOCKS
+#define PKM_B3_MIN_BLOCKS 6
+#endif
+
+__global__ void __launch_bounds__(kB3Threads, PKM_B3_MIN_BLOCKS) value_rows_kernel(
     const int* __restrict__ seg, const int* __restrict__ U_ptr, const int32_t* __restrict__ seg_row,
     const int32_t* __restrict__ ents, const TV* __restrict__ V, const float* __restrict__ ws_sorted,
     const float* __restrict__ dy, float* __restrict__ dV, float* __restrict__ dw, int hk, int d_v,
