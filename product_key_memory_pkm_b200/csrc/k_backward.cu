@@ -560,6 +560,11 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
 cudaError_t launch_value_sgd(const Plan& p, float* values, const pkm_saved& s, const float* dy,
                              float lr, void* ws, cudaStream_t st) {
   const int64_t E1 = p.N * p.h * p.ksel;
+  if (fw_chunk_sort_fits(p, p.N)) {  // few selections: one CTA sorts them in shared memory
+    cudaError_t e = launch_fw_chunk_sort(p, p.N, s.idx, s.w, ws, st);
+    if (e != cudaSuccess) return e;
+    return launch_fw_chunk_write(p, p.N, 0, ws, dy, values, lr, st);
+  }
   BwdCtx c = bwd_ctx(p, ws, nullptr);
   cudaError_t e;
   const int32_t *rows_sorted, *ents_sorted;
@@ -777,10 +782,10 @@ bool fw_presort_fits(const Plan& p, int64_t chunk) {
 
 cudaError_t launch_fw_presort(const Plan& p, int64_t chunk, const int32_t* idx, const float* w,
                               int32_t* keys, int* bounds, void* ws, cudaStream_t st) {
-  const int64_t E1 = p.N * p.h * p.k;
+  const int64_t E1 = p.N * p.h * p.ksel;
   const int64_t nch = (p.N + chunk - 1) / chunk;
   BwdCtx c = bwd_ctx(p, ws, nullptr);
-  fw_keys_kernel<<<(unsigned)((E1 + 255) / 256), 256, 0, st>>>(idx, E1, p.h * p.k, chunk, p.K,
+  fw_keys_kernel<<<(unsigned)((E1 + 255) / 256), 256, 0, st>>>(idx, E1, p.h * p.ksel, chunk, p.K,
                                                                keys, p.status);
   PKM_COUNT(1);
   cudaError_t e = cudaGetLastError();
@@ -798,12 +803,12 @@ cudaError_t launch_fw_presort(const Plan& p, int64_t chunk, const int32_t* idx, 
 }
 
 bool fw_chunk_sort_fits(const Plan& p, int64_t chunk) {
-  return std::min<int64_t>(chunk, p.N) * p.h * p.k <= kFwSortMax;
+  return std::min<int64_t>(chunk, p.N) * p.h * p.ksel <= kFwSortMax;
 }
 
 size_t fw_chunk_sort_bytes(const Plan& p, int64_t chunk) {
   const int64_t nch = (p.N + chunk - 1) / chunk;
-  const int64_t stride = std::min<int64_t>(chunk, p.N) * p.h * p.k + 1;
+  const int64_t stride = std::min<int64_t>(chunk, p.N) * p.h * p.ksel + 1;
   // seg, seg_row, ents, w_sorted at `stride` per chunk, then U per chunk
   return (size_t)(4 * 4 * nch * stride + 4 * nch);
 }
@@ -811,7 +816,7 @@ size_t fw_chunk_sort_bytes(const Plan& p, int64_t chunk) {
 cudaError_t launch_fw_chunk_sort(const Plan& p, int64_t chunk, const int32_t* idx, const float* w,
                                  void* buf, cudaStream_t st) {
   const int64_t nch = (p.N + chunk - 1) / chunk;
-  const int n_max = (int)(std::min<int64_t>(chunk, p.N) * p.h * p.k);
+  const int n_max = (int)(std::min<int64_t>(chunk, p.N) * p.h * p.ksel);
   const int stride = n_max + 1;
   int npow2 = 1;
   while (npow2 < n_max) npow2 <<= 1;
@@ -827,7 +832,7 @@ cudaError_t launch_fw_chunk_sort(const Plan& p, int64_t chunk, const int32_t* id
                                 (int)smem)) != cudaSuccess)
     return e;
   fw_chunk_sort_kernel<<<(unsigned)nch, kFwSortThreads, smem, st>>>(
-      idx, w, p.N, chunk, p.h * p.k, p.K, stride, npow2, seg, seg_row, ents, w_sorted, U,
+      idx, w, p.N, chunk, p.h * p.ksel, p.K, stride, npow2, seg, seg_row, ents, w_sorted, U,
       p.status);
   PKM_COUNT(1);
   return cudaGetLastError();
@@ -836,20 +841,20 @@ cudaError_t launch_fw_chunk_sort(const Plan& p, int64_t chunk, const int32_t* id
 cudaError_t launch_fw_chunk_write(const Plan& p, int64_t chunk, int64_t ci, const void* buf,
                                   const float* dy, float* values, float lr, cudaStream_t st) {
   const int64_t nch = (p.N + chunk - 1) / chunk;
-  const int n_max = (int)(std::min<int64_t>(chunk, p.N) * p.h * p.k);
+  const int n_max = (int)(std::min<int64_t>(chunk, p.N) * p.h * p.ksel);
   const int64_t stride = n_max + 1;
   const int* seg = static_cast<const int*>(buf);
   const int32_t* seg_row = seg + nch * stride;
   const int32_t* ents = seg_row + nch * stride;
   const float* w_sorted = reinterpret_cast<const float*>(ents + nch * stride);
   const int* U = reinterpret_cast<const int*>(w_sorted + nch * stride);
-  const int64_t n_c = std::min<int64_t>(chunk, p.N - ci * chunk) * p.h * p.k;
+  const int64_t n_c = std::min<int64_t>(chunk, p.N - ci * chunk) * p.h * p.ksel;
   const int64_t blocks = std::min<int64_t>(n_c, (int64_t)p.sm_count * 8);
   const int64_t o = ci * stride;
   PKM_COUNT(1);
   return launch_dependent(rows_step_kernel<false>, dim3((unsigned)blocks), dim3(kSgdThreads), 0,
                           st, seg + o, U + ci, seg_row + o, ents + o, w_sorted + o, dy, values, lr,
-                          p.h * p.k, p.d_v, p.K, p.status, (const int*)nullptr, (int64_t)0,
+                          p.h * p.ksel, p.d_v, p.K, p.status, (const int*)nullptr, (int64_t)0,
                           AdamArgs{});
 }
 
@@ -859,11 +864,11 @@ cudaError_t launch_fw_write(const Plan& p, int64_t chunk, int64_t ci, const int*
   const int32_t* ents_sorted =
       sort::radix_sorted_vals(c.rb, bits_for(((p.N + chunk - 1) / chunk) * p.K - 1));
   const int64_t n_c = std::min<int64_t>(chunk, p.N - ci * chunk);
-  const int64_t blocks = std::min<int64_t>(n_c * p.h * p.k, (int64_t)p.sm_count * 8);
+  const int64_t blocks = std::min<int64_t>(n_c * p.h * p.ksel, (int64_t)p.sm_count * 8);
   PKM_COUNT(1);
   return launch_dependent(rows_step_kernel<false>, dim3((unsigned)blocks), dim3(kSgdThreads), 0,
                           st, c.seg, c.U, c.seg_row, ents_sorted, c.w_sorted, dy, values, lr,
-                          p.h * p.k, p.d_v, p.K, p.status, bounds + ci, ci * p.K, AdamArgs{});
+                          p.h * p.ksel, p.d_v, p.K, p.status, bounds + ci, ci * p.K, AdamArgs{});
 }
 
 cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, const float* bn,
