@@ -60,6 +60,28 @@ def _cfg_json(cfg):
             "input_dtype": cfg.dtype, "value_dtype": cfg.vdtype, "l2": "flushed before every timed step (256 MiB write)"}
 
 
+# ---------------------------------------------------------------- ranks
+def rank_batch(cfg, rank: int, world: int, with_dy: bool = True) -> dict:
+    """One replica's inputs: the same tables on every rank (seed 0), and with more than one
+    rank each its own tokens (and upstream gradient) from seed 1000 + rank."""
+    inp = make_inputs(cfg, seed=0, with_dy=with_dy)
+    if world > 1:
+        other = make_inputs(cfg, seed=1000 + rank, with_dy=with_dy)
+        inp["x"] = other["x"]
+        if with_dy:
+            inp["dy"] = other["dy"]
+    return inp
+
+
+def max_over_ranks(values, dist, device) -> list:
+    """Each timing as the maximum over the ranks (the slowest replica sets the step)."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -161,10 +183,7 @@ def run_b200(args, cfg, rank, world, dist):
     st = torch.cuda.current_stream()
 
     t_gen = time.perf_counter()
-    inp = make_inputs(cfg, seed=0)
-    if world > 1:   # each rank its own batch of tokens; the tables are the same
-        other = make_inputs(cfg.with_(N=cfg.N), seed=1000 + rank)
-        inp["x"], inp["dy"] = other["x"], other["dy"]
+    inp = rank_batch(cfg, rank, world)
     bf = torch.bfloat16
     x = torch.from_numpy(inp["x"]).to(bf).to(dev)
     Wq = torch.from_numpy(inp["Wq"]).to(bf).to(dev)
@@ -295,11 +314,8 @@ def run_b200(args, cfg, rank, world, dist):
     clk = clocks.stop()
 
     # max over ranks
-    vals = torch.tensor([step_ms, fwd_ms, e2e["ms"] if e2e else 0.0], device=dev,
-                        dtype=torch.float64)
-    if dist is not None:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    step_ms, fwd_ms, e2e_ms = (float(v) for v in vals.tolist())
+    step_ms, fwd_ms, e2e_ms = max_over_ranks([step_ms, fwd_ms, e2e["ms"] if e2e else 0.0], dist,
+                                             dev)
     if rank != 0:
         return None
 
@@ -395,11 +411,8 @@ def run_fastweight(args, cfg, rank, world, dist):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     t_gen = time.perf_counter()
-    inp = make_inputs(cfg, seed=0, with_dy=False)
-    tg_np = make_targets(cfg, seed=0)
-    if world > 1:   # each rank its own sequence; the same initial tables
-        inp["x"] = make_inputs(cfg, seed=1000 + rank, with_dy=False)["x"]
-        tg_np = make_targets(cfg, seed=1000 + rank)
+    inp = rank_batch(cfg, rank, world, with_dy=False)   # each rank its own sequence
+    tg_np = make_targets(cfg, seed=1000 + rank if world > 1 else 0)
     f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev)
     sto = (lambda a: f32(a).to(torch.bfloat16)) if cfg.dtype == "bf16" else f32
     x, Wq, bn, sub, V, tg = (sto(inp["x"]), sto(inp["Wq"]), f32(inp["bn"]), sto(inp["subkeys"]),
@@ -493,10 +506,7 @@ def run_fastweight(args, cfg, rank, world, dist):
                                                                workspace=bws, stream=side))
         stage_ms /= args.steps
     clk = clocks.stop()
-    vals = torch.tensor([graph_ms, eager_ms], device=dev, dtype=torch.float64)
-    if dist is not None:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    graph_ms, eager_ms = (float(v) for v in vals.tolist())
+    graph_ms, eager_ms = max_over_ranks([graph_ms, eager_ms], dist, dev)
     if rank != 0:
         return None
 

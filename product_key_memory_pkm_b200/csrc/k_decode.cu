@@ -25,6 +25,7 @@ namespace {
 namespace cg = cooperative_groups;
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kTokGroup = 16, kWarps = 8, kSplit = 8;
+constexpr int kPerLane = 8;  // sub-keys per lane in a slice's selection (slices <= 256)
 
 // 16-byte global -> shared copies that stay in flight together (completion waited for
 // with cp_async_wait_all before the block barrier).
@@ -218,17 +219,47 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kWarps * 32)
     sc[t * per_max + c] = idw ? -0.5f * logf(fmaxf(qn + cn - 2.f * acc, 0.f) + 1e-12f) : acc;
   }
   __syncthreads();
-  // 3. each token's top-KM of the slice: a candidate's place is the number of the slice's
-  //    candidates that rank before it
-  for (int i = tid; i < nt * nct; i += nthr) {
-    const int t = i / nct, c = i % nct;
+  // 3. each token's top-KM of the slice, best first: one warp per token holds the slice's
+  //    candidates (kPerLane per lane) and extracts the best one KM times
+  const int lane = tid & 31, wid = tid >> 5;
+  for (int t = wid; t < nt; t += kWarps) {
     const float* st = sc + t * per_max;
-    const float v = st[c];
-    int r = 0;
-    for (int c2 = 0; c2 < nct; ++c2) r += before(st[c2], c0 + c2, v, c0 + c) ? 1 : 0;
-    if (r < KM) {
-      ls[t * KM + r] = v;
-      li[t * KM + r] = c0 + c;
+    float cv[kPerLane];
+    int ci[kPerLane];
+#pragma unroll
+    for (int m = 0; m < kPerLane; ++m) {
+      const int c = lane + 32 * m;
+      cv[m] = c < nct ? st[c] : -INFINITY;
+      ci[m] = c < nct ? c0 + c : 0x7fffffff;
+    }
+    for (int j = 0; j < KM; ++j) {
+      float bs = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int m = 0; m < kPerLane; ++m)
+        if (before(cv[m], ci[m], bs, bi)) {
+          bs = cv[m];
+          bi = ci[m];
+        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float os = __shfl_xor_sync(kFull, bs, o);
+        const int oi = __shfl_xor_sync(kFull, bi, o);
+        if (before(os, oi, bs, bi)) {
+          bs = os;
+          bi = oi;
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < kPerLane; ++m)
+        if (ci[m] == bi) {  // indices are unique: only the owner matches (padding never wins
+          cv[m] = -INFINITY;  // while a real candidate is left)
+          ci[m] = 0x7fffffff;
+        }
+      if (lane == 0) {
+        ls[t * KM + j] = bs;
+        li[t * KM + j] = bi;
+      }
     }
   }
   cluster.sync();
@@ -260,30 +291,36 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kWarps * 32)
   cluster.sync();  // the other CTAs' lists may be released now
   if (rank != 0) return;
   __syncthreads();
-  // 5. ... and places each element by merge rank: its position in its own list plus, for
-  //    every other list, how many of that list's elements rank before it (binary search)
-  for (int i = tid; i < nt * kSplit * KM; i += nthr) {
-    const int t = i / (kSplit * KM), r = (i / KM) % kSplit, j = i % KM;
-    const float v = ms[i];
-    const int vi = mi[i];
-    if (vi == 0x7fffffff) continue;  // padding
-    int place = j;
-    for (int r2 = 0; r2 < kSplit; ++r2) {
-      if (r2 == r) continue;
-      const float* lv = ms + (t * kSplit + r2) * KM;
-      const int* lx = mi + (t * kSplit + r2) * KM;
-      int lo = 0, hi = KM;  // first element of list r2 that does not rank before (v, vi)
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (before(lv[mid], lx[mid], v, vi)) lo = mid + 1;
-        else hi = mid;
+  // 5. ... and merges them, one warp per token: lane r < kSplit walks list r; each of the k
+  //    steps emits the best head and advances its list
+  for (int t = wid; t < nt; t += kWarps) {
+    const float* lv = ms + (t * kSplit + (lane & (kSplit - 1))) * KM;
+    const int* lx = mi + (t * kSplit + (lane & (kSplit - 1))) * KM;
+    int pos = 0;
+    const int64_t o = (((t0 + t) * h + hh) * 2 + s) * (int64_t)k;
+    for (int j = 0; j < k; ++j) {
+      float hs = -INFINITY;
+      int hx = 0x7fffffff;
+      if (lane < kSplit && pos < KM) {
+        hs = lv[pos];
+        hx = lx[pos];
       }
-      place += lo;
-    }
-    if (place < k) {
-      const int64_t o = (((t0 + t) * h + hh) * 2 + s) * (int64_t)k + place;
-      sub_s[o] = v;
-      sub_i[o] = vi;
+      float bs = hs;
+      int bi = hx;
+#pragma unroll
+      for (int m = 16; m > 0; m >>= 1) {
+        const float os = __shfl_xor_sync(kFull, bs, m);
+        const int oi = __shfl_xor_sync(kFull, bi, m);
+        if (before(os, oi, bs, bi)) {
+          bs = os;
+          bi = oi;
+        }
+      }
+      if (lane < kSplit && hx == bi) ++pos;  // unique indices: one list advances
+      if (lane == 0) {
+        sub_s[o + j] = bs;
+        sub_i[o + j] = bi;
+      }
     }
   }
 }
@@ -297,6 +334,7 @@ size_t scores_small_smem(const Plan& p, int KM) {
 
 bool small_n_supported(const Plan& p) {
   return !p.fp32 && p.N <= kSmallTokens && p.d_in % 8 == 0 && (p.dk / 2) % 8 == 0 &&
+         (std::max(p.C1, p.C2) + kSplit - 1) / kSplit <= 32 * kPerLane &&
          (size_t)kTokGroup * p.d_in * 2 <= 160 * 1024 && scores_small_smem(p, 32) <= 200 * 1024;
 }
 
