@@ -26,6 +26,7 @@ namespace cg = cooperative_groups;
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kTokGroup = 16, kWarps = 8, kSplit = 8;
 constexpr int kPerLane = 8;  // sub-keys per lane in a slice's selection (slices <= 256)
+constexpr int kRankTokens = 2;  // up to this many tokens, selection and merge by rank
 
 // 16-byte global -> shared copies that stay in flight together (completion waited for
 // with cp_async_wait_all before the block barrier).
@@ -219,10 +220,26 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kWarps * 32)
     sc[t * per_max + c] = idw ? -0.5f * logf(fmaxf(qn + cn - 2.f * acc, 0.f) + 1e-12f) : acc;
   }
   __syncthreads();
-  // 3. each token's top-KM of the slice, best first: one warp per token holds the slice's
-  //    candidates (kPerLane per lane) and extracts the best one KM times
+  // 3. each token's top-KM of the slice, best first.  With at most kRankTokens tokens every
+  //    thread places one candidate: its place is the number of the slice's candidates that
+  //    rank before it.  With more, one warp per token holds the slice's candidates
+  //    (kPerLane per lane) and extracts the best one KM times.
   const int lane = tid & 31, wid = tid >> 5;
-  for (int t = wid; t < nt; t += kWarps) {
+  const bool by_rank = nt <= kRankTokens;  // uniform over the cluster
+  if (by_rank) {
+    for (int i = tid; i < nt * nct; i += nthr) {
+      const int t = i / nct, c = i % nct;
+      const float* st = sc + t * per_max;
+      const float v = st[c];
+      int r = 0;
+      for (int c2 = 0; c2 < nct; ++c2) r += before(st[c2], c0 + c2, v, c0 + c) ? 1 : 0;
+      if (r < KM) {
+        ls[t * KM + r] = v;
+        li[t * KM + r] = c0 + c;
+      }
+    }
+  }
+  for (int t = wid; t < nt && !by_rank; t += kWarps) {
     const float* st = sc + t * per_max;
     float cv[kPerLane];
     int ci[kPerLane];
@@ -291,8 +308,37 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kWarps * 32)
   cluster.sync();  // the other CTAs' lists may be released now
   if (rank != 0) return;
   __syncthreads();
-  // 5. ... and merges them, one warp per token: lane r < kSplit walks list r; each of the k
-  //    steps emits the best head and advances its list
+  // 5. ... and merges them.  Few tokens: every element is placed by merge rank -- its
+  //    position in its own list plus, for every other list, how many of that list's elements
+  //    rank before it (binary search).  More: one warp per token, lane r < kSplit walking list
+  //    r; each of the k steps emits the best head and advances its list.
+  if (by_rank) {
+    for (int i = tid; i < nt * kSplit * KM; i += nthr) {
+      const int t = i / (kSplit * KM), r = (i / KM) % kSplit, j = i % KM;
+      const float v = ms[i];
+      const int vi = mi[i];
+      if (vi == 0x7fffffff) continue;  // padding
+      int place = j;
+      for (int r2 = 0; r2 < kSplit; ++r2) {
+        if (r2 == r) continue;
+        const float* lv = ms + (t * kSplit + r2) * KM;
+        const int* lx = mi + (t * kSplit + r2) * KM;
+        int lo = 0, hi = KM;  // first element of list r2 that does not rank before (v, vi)
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (before(lv[mid], lx[mid], v, vi)) lo = mid + 1;
+          else hi = mid;
+        }
+        place += lo;
+      }
+      if (place < k) {
+        const int64_t o = (((t0 + t) * h + hh) * 2 + s) * (int64_t)k + place;
+        sub_s[o] = v;
+        sub_i[o] = vi;
+      }
+    }
+    return;
+  }
   for (int t = wid; t < nt; t += kWarps) {
     const float* lv = ms + (t * kSplit + (lane & (kSplit - 1))) * KM;
     const int* lx = mi + (t * kSplit + (lane & (kSplit - 1))) * KM;

@@ -40,6 +40,7 @@ CASES = {
     "few_tokens_unequal_C_k8": _cfg(N=13, h=2, dk=64, C1=96, C2=40, k=8),
     "few_tokens_k32_small_C": _cfg(N=16, h=3, k=32, C1=40, C2=33, d_v=72),
     "split_bag_37_tokens": _cfg(N=37, h=2, dk=64, C1=96, C2=40, k=8),
+    "two_tokens_k16": _cfg(N=2, h=3, dk=64, C1=96, C2=40, k=16),
 }
 
 
