@@ -288,6 +288,79 @@ pkm_status pkm_fastweight_chunks(const pkm_dims* d, int64_t chunk, float lr, uin
                                  float* y, void* workspace, size_t workspace_bytes,
                                  void* stream);
 
+/* ---------------------------------------------------------------- row-sharded table
+ * "Meta AI 可扩展内存层", 9.1: the value matrix is split by rows of the product-key
+ * index over G ranks, each rank reads only its own rows, and the ranks exchange the
+ * candidate indices and partial weighted sums; 4.5: row i*|C'| + j, so a range of
+ * leading sub-key indices is a contiguous range of rows.  Shard g holds rows
+ * [g*R, min((g+1)*R, C1*C2)) (R = ceil(C1/G)*C2 splits by leading sub-key; any
+ * R >= 1 with G*R >= C1*C2 is accepted), as its own [rows][d_v] table.
+ *
+ * The rank that owns a batch of N tokens (its source) runs pkm_query,
+ * pkm_subkey_scores and pkm_candidate_topk, then pkm_shard_route; the caller's
+ * collective moves, per destination g, counts[g], then the triples, to the owner of
+ * shard g.  The owner runs pkm_shard_bag over what it received (triples of every
+ * source, concatenated in source order) and returns partial row j of each source's
+ * segments to it; the source sums them with pkm_shard_combine.  Backward: the source
+ * sends dy once per segment (pkm_shard_gather_dy), the owner runs
+ * pkm_shard_value_grad (its dV += and dL/dw of every received triple), the source
+ * puts the returned dL/dw in place with pkm_shard_scatter_dw and continues with
+ * pkm_query_grad.  The library moves no data between ranks. */
+#define PKM_MAX_SHARDS 1024
+typedef struct {
+  int32_t seg;  /* the triple's segment: its token's run for this destination, from 0 */
+  int32_t row;  /* row within the destination's shard */
+  float w;      /* softmax weight */
+} pkm_triple;
+/* which: PKM_SHARD_ROUTE (source side; n_triples ignored) or PKM_SHARD_OWNER (owner side,
+ * for up to n_triples received triples; includes the value pass's scratch). */
+#define PKM_SHARD_ROUTE 1
+#define PKM_SHARD_OWNER 2
+size_t pkm_shard_workspace_bytes(const pkm_dims* d, int32_t G, int which, int64_t n_triples);
+/* Source side.  idx, w: [N][h][k] (as pkm_forward's saved idx and w: flat rows).
+ * counts: device [G][2] int32 = {triples, segments} bound for shard g.  segpos: device
+ * [G][N] int32, the row of the combined receive buffer (all partial rows sent back,
+ * shard 0's first) that holds token t's partial from shard g, or -1 when t sent g
+ * nothing.  send: [N*h*k] triples grouped by destination (shard 0's first), within it
+ * by token, within a token in selection order.  perm: [N*h*k], perm[pos] = the flat
+ * selection index t*h*k + s of send[pos].  A row outside the table records
+ * PKM_ERR_DEVICE_INDEX and is routed as row 0.  1 <= G <= PKM_MAX_SHARDS,
+ * G*N < 2^31. */
+pkm_status pkm_shard_route(const pkm_dims* d, int32_t G, int64_t rows_per_shard,
+                           const int32_t* idx, const float* w, int32_t* counts, int32_t* segpos,
+                           pkm_triple* send, int32_t* perm, void* workspace,
+                           size_t workspace_bytes, void* stream);
+/* Owner side.  recv_counts: device [G][2] int32, the counts each source sent this shard;
+ * n_triples, n_segments: their sums (host).  recv: the received triples, source 0's
+ * first.  values: this shard's [shard_rows][d_v] table (bf16, or fp32 with
+ * PKM_F_FP32 / PKM_F_VALUES_FP32).  partial: [n_segments][d_v] fp32, row j = sum over
+ * segment j's triples of w * V[row] (segments numbered across sources in source order).
+ * Out-of-range segments or rows record PKM_ERR_DEVICE_INDEX and are clamped. */
+pkm_status pkm_shard_bag(const pkm_dims* d, int32_t G, int64_t shard_rows,
+                         const int32_t* recv_counts, int64_t n_triples, int64_t n_segments,
+                         const pkm_triple* recv, const void* values, float* partial,
+                         void* workspace, size_t workspace_bytes, void* stream);
+/* Source side.  partial_recv: [n_rows][d_v] fp32, the partial rows every shard sent back
+ * (shard 0's first); y[t] (overwritten) = their sum over shards in ascending order. */
+pkm_status pkm_shard_combine(const pkm_dims* d, int32_t G, const int32_t* segpos,
+                             const float* partial_recv, int64_t n_rows, float* y, void* stream);
+/* Source side.  dy_send[segpos[g][t]] = dy[t] for every segment (n_rows rows). */
+pkm_status pkm_shard_gather_dy(const pkm_dims* d, int32_t G, const int32_t* segpos,
+                               const float* dy, float* dy_send, int64_t n_rows, void* stream);
+/* Owner side, backward.  dy_recv: [n_segments][d_v] fp32 in the received segment order.
+ * dvalues: this shard's dense fp32 [shard_rows][d_v] gradient (+=, one writer per row,
+ * deterministic).  dw_recv: [n_triples] fp32 (overwritten), dL/dw of every received
+ * triple = dy of its segment . V[row]. */
+pkm_status pkm_shard_value_grad(const pkm_dims* d, int32_t G, int64_t shard_rows,
+                                const int32_t* recv_counts, int64_t n_triples,
+                                int64_t n_segments, const pkm_triple* recv, const void* values,
+                                const float* dy_recv, float* dvalues, float* dw_recv,
+                                void* workspace, size_t workspace_bytes, void* stream);
+/* Source side.  dw[perm[i]] = dw_ret[i] for the N*h*k triples this rank sent (dw_ret in
+ * the send order). */
+pkm_status pkm_shard_scatter_dw(const pkm_dims* d, const int32_t* perm, const float* dw_ret,
+                                float* dw, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device status word of the
  * current device.  Returns PKM_OK, PKM_ERR_DEVICE_TIMEOUT, PKM_ERR_DEVICE_INDEX or
  * PKM_ERR_CUDA (when the synchronisation itself failed). */

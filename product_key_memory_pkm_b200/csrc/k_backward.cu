@@ -504,7 +504,8 @@ static BwdCtx bwd_ctx(const Plan& p, void* ws, float* dw_out) {
 
 cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved& s,
                               const float* dy, float* dV, float* dw_out, void* ws,
-                              cudaStream_t st, float* dVc, int32_t* rows_out, int* U_out) {
+                              cudaStream_t st, float* dVc, int32_t* rows_out, int* U_out,
+                              const int32_t* ent_tok) {
   const int64_t E1 = p.N * p.h * p.ksel;
   BwdCtx c = bwd_ctx(p, ws, dw_out);
   sort::RadixBuffers& rb = c.rb;
@@ -539,7 +540,7 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
       return e;                                                                              \
     value_rows_kernel<TV, CHV><<<blocks, kB3Threads, smem, st>>>(                            \
         seg, U, seg_row, ents_sorted, static_cast<const TV*>(values), w_sorted, dy, dV, dw,  \
-        hk, p.d_v, p.K, p.status, dVc, rows_out, U_out);                                     \
+        hk, p.d_v, p.K, p.status, dVc, rows_out, U_out, ent_tok);                            \
   } while (0)
     if (p.vfp32) {
       if (nvec <= kB3Threads) PKM_B3(float, 1);

@@ -126,7 +126,8 @@ __device__ __forceinline__ void prefetch_l1(const void* p) {
 }
 
 // ws_sorted[p] = w[ents[p]]: the selection weights in row order, so staging a batch
-// needs two independent loads.
+// needs two independent loads.  A selection's upstream-gradient row is ent_tok[ent] when
+// that map is given (entries received from other ranks), else ent / hk (its token).
 template <typename TV, int CH>
 // resident CTAs per SM the pass is compiled and launched for (a tuning value)
 #ifndef PKM_B3_MIN_BLOCKS
@@ -138,7 +139,7 @@ __global__ void __launch_bounds__(kB3Threads, PKM_B3_MIN_BLOCKS) value_rows_kern
     const int32_t* __restrict__ ents, const TV* __restrict__ V, const float* __restrict__ ws_sorted,
     const float* __restrict__ dy, float* __restrict__ dV, float* __restrict__ dw, int hk, int d_v,
     int64_t K, int* status, float* __restrict__ dVc, int32_t* __restrict__ rows_out,
-    int* __restrict__ U_out) {
+    int* __restrict__ U_out, const int32_t* __restrict__ ent_tok) {
   constexpr int E = VecT<TV>::E;
   extern __shared__ __align__(16) unsigned char b3_smem[];
   __shared__ int s_t[2][kB3Batch];
@@ -190,7 +191,7 @@ __global__ void __launch_bounds__(kB3Threads, PKM_B3_MIN_BLOCKS) value_rows_kern
     if (tid < min(kB3Batch, q1 - q0)) {
       const int32_t ent = ents[q0 + tid];
       s_e[0][tid] = ent;
-      s_t[0][tid] = ent / hk;
+      s_t[0][tid] = ent_tok ? ent_tok[ent] : ent / hk;
       s_w[0][tid] = ws_sorted[q0 + tid];
     }
   }
@@ -222,7 +223,7 @@ __global__ void __launch_bounds__(kB3Threads, PKM_B3_MIN_BLOCKS) value_rows_kern
     __syncthreads();
     if (abort_flag || !got) break;  // uniform: abort_flag is read after the barrier
     if (tid < nbn) {  // publish the next row's batch and pull its dy lines into L1
-      const int64_t tn = nent / hk;
+      const int64_t tn = ent_tok ? ent_tok[nent] : nent / hk;
       s_e[b ^ 1][tid] = nent;
       s_t[b ^ 1][tid] = (int)tn;
       s_w[b ^ 1][tid] = nw;
@@ -274,7 +275,7 @@ __global__ void __launch_bounds__(kB3Threads, PKM_B3_MIN_BLOCKS) value_rows_kern
           if (tid < nb) {
             const int32_t ent = ents[pb + tid];
             s_e[b][tid] = ent;
-            s_t[b][tid] = ent / hk;
+            s_t[b][tid] = ent_tok ? ent_tok[ent] : ent / hk;
             s_w[b][tid] = ws_sorted[pb + tid];
           }
           __syncthreads();

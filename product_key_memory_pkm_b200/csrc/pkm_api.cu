@@ -691,3 +691,161 @@ extern "C" pkm_status pkm_value_grad_noalloc(const pkm_dims* d, const void* valu
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return cuda_status(launch_value_grad(p, values, *saved, dy, dvalues, dw, scratch, st));
 }
+
+// ------------------------------------------------------------------ row-sharded table
+namespace pkm {
+namespace {
+
+pkm_status validate_shard(const pkm_dims* d, int32_t G) {
+  PKM_TRY(validate_dims(d));
+  if (G < 1 || G > PKM_MAX_SHARDS) return PKM_ERR_INVALID_ARG;
+  if ((int64_t)G * d->N >= ((int64_t)1 << 31)) return PKM_ERR_UNSUPPORTED;
+  return PKM_OK;
+}
+
+pkm_status validate_owner(int64_t shard_rows, int64_t n_tri, int64_t n_seg) {
+  if (shard_rows < 1 || shard_rows >= ((int64_t)1 << 31)) return PKM_ERR_INVALID_ARG;
+  if (n_tri < 0 || n_seg < 0 || n_seg > n_tri || (n_tri > 0 && n_seg == 0))
+    return PKM_ERR_INVALID_ARG;
+  if (n_tri >= ((int64_t)1 << 30)) return PKM_ERR_UNSUPPORTED;
+  return PKM_OK;
+}
+
+// The owner's value pass sees every received triple as one selection of its own
+// one-head, one-key "token" over the shard's rows.
+Plan owner_plan(Plan p, int64_t n_tri, int64_t shard_rows) {
+  p.N = n_tri;
+  p.h = 1;
+  p.k = 1;
+  p.ksel = 1;
+  p.K = shard_rows;
+  return p;
+}
+
+size_t owner_bytes(const pkm_dims* d, int32_t G, int64_t n_tri) {
+  Plan q{};
+  q.d_v = d->d_v;
+  q.dk = d->dk;
+  q.hq = d->dk;
+  q.C1 = d->C1;
+  q.C2 = d->C2;
+  q.fp32 = d->flags & PKM_F_FP32;
+  q = owner_plan(q, n_tri > 0 ? n_tri : 1, 1);
+  return shard_owner_layout(G, n_tri).total + value_stage_scratch_bytes(q);
+}
+
+}  // namespace
+}  // namespace pkm
+
+extern "C" {
+
+size_t pkm_shard_workspace_bytes(const pkm_dims* d, int32_t G, int which, int64_t n_triples) {
+  if (validate_shard(d, G) != PKM_OK) return 0;
+  if (which == PKM_SHARD_ROUTE) return shard_route_layout(d->N > 0 ? d->N : 1, G).total;
+  if (which == PKM_SHARD_OWNER && n_triples >= 0) return owner_bytes(d, G, n_triples);
+  return 0;
+}
+
+pkm_status pkm_shard_route(const pkm_dims* d, int32_t G, int64_t rows_per_shard,
+                           const int32_t* idx, const float* w, int32_t* counts, int32_t* segpos,
+                           pkm_triple* send, int32_t* perm, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  PKM_TRY(validate_shard(d, G));
+  const int64_t K = (int64_t)d->C1 * d->C2;
+  if (rows_per_shard < 1 || (K + rows_per_shard - 1) / rows_per_shard > G)
+    return PKM_ERR_INVALID_ARG;
+  PKM_NEED(counts);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d->N == 0)  // nothing to send: zero counts, so the caller's exchange still runs
+    return cuda_status(cudaMemsetAsync(counts, 0, sizeof(int32_t) * 2 * (size_t)G, st));
+  PKM_NEED(idx); PKM_NEED(w); PKM_NEED(segpos); PKM_NEED(send); PKM_NEED(perm);
+  PKM_TRY(check_workspace(shard_route_layout(d->N, G).total, workspace, workspace_bytes));
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  return cuda_status(
+      launch_shard_route(p, G, rows_per_shard, idx, w, counts, segpos, send, perm, workspace, st));
+}
+
+pkm_status pkm_shard_bag(const pkm_dims* d, int32_t G, int64_t shard_rows,
+                         const int32_t* recv_counts, int64_t n_triples, int64_t n_segments,
+                         const pkm_triple* recv, const void* values, float* partial,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  PKM_TRY(validate_shard(d, G));
+  PKM_TRY(validate_owner(shard_rows, n_triples, n_segments));
+  if (n_segments == 0) return PKM_OK;
+  PKM_NEED(recv_counts); PKM_NEED(recv); PKM_NEED(values); PKM_NEED(partial);
+  PKM_TRY(check_workspace(owner_bytes(d, G, n_triples), workspace, workspace_bytes));
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_shard_owner_index(p, G, recv_counts, n_triples, n_segments, recv,
+                                           shard_rows, workspace, false, st);
+  if (e != cudaSuccess) return PKM_ERR_CUDA;
+  return cuda_status(launch_shard_bag(p, G, n_segments, recv, values, shard_rows, partial,
+                                      workspace, n_triples, st));
+}
+
+pkm_status pkm_shard_combine(const pkm_dims* d, int32_t G, const int32_t* segpos,
+                             const float* partial_recv, int64_t n_rows, float* y, void* stream) {
+  PKM_TRY(validate_shard(d, G));
+  if (n_rows < 0) return PKM_ERR_INVALID_ARG;
+  if (d->N == 0) return PKM_OK;
+  PKM_NEED(segpos); PKM_NEED(y);
+  if (n_rows > 0) PKM_NEED(partial_recv);
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  return cuda_status(launch_shard_combine(p, G, segpos, partial_recv, n_rows, y,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+pkm_status pkm_shard_gather_dy(const pkm_dims* d, int32_t G, const int32_t* segpos,
+                               const float* dy, float* dy_send, int64_t n_rows, void* stream) {
+  PKM_TRY(validate_shard(d, G));
+  if (n_rows < 0) return PKM_ERR_INVALID_ARG;
+  if (d->N == 0 || n_rows == 0) return PKM_OK;
+  PKM_NEED(segpos); PKM_NEED(dy); PKM_NEED(dy_send);
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  return cuda_status(launch_shard_gather_dy(p, G, segpos, dy, n_rows, dy_send,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+pkm_status pkm_shard_value_grad(const pkm_dims* d, int32_t G, int64_t shard_rows,
+                                const int32_t* recv_counts, int64_t n_triples,
+                                int64_t n_segments, const pkm_triple* recv, const void* values,
+                                const float* dy_recv, float* dvalues, float* dw_recv,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  PKM_TRY(validate_shard(d, G));
+  PKM_TRY(validate_owner(shard_rows, n_triples, n_segments));
+  if (n_triples == 0) return PKM_OK;
+  PKM_NEED(recv_counts); PKM_NEED(recv); PKM_NEED(values); PKM_NEED(dy_recv);
+  PKM_NEED(dvalues); PKM_NEED(dw_recv);
+  PKM_TRY(check_workspace(owner_bytes(d, G, n_triples), workspace, workspace_bytes));
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_shard_owner_index(p, G, recv_counts, n_triples, n_segments, recv,
+                                           shard_rows, workspace, true, st);
+  if (e != cudaSuccess) return PKM_ERR_CUDA;
+  const ShardOwnerLayout L = shard_owner_layout(G, n_triples);
+  char* base = static_cast<char*>(workspace);
+  pkm_saved s{};
+  s.idx = reinterpret_cast<int32_t*>(base + L.rows);
+  s.w = reinterpret_cast<float*>(base + L.wv);
+  const int32_t* tok = reinterpret_cast<const int32_t*>(base + L.tok);
+  return cuda_status(launch_value_grad(owner_plan(p, n_triples, shard_rows), values, s, dy_recv,
+                                       dvalues, dw_recv, base + L.total, st, nullptr, nullptr,
+                                       nullptr, tok));
+}
+
+pkm_status pkm_shard_scatter_dw(const pkm_dims* d, const int32_t* perm, const float* dw_ret,
+                                float* dw, void* stream) {
+  PKM_TRY(validate_dims(d));
+  if (d->N == 0) return PKM_OK;
+  PKM_NEED(perm); PKM_NEED(dw_ret); PKM_NEED(dw);
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  return cuda_status(launch_shard_scatter_dw(p, perm, dw_ret, dw, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -167,10 +167,12 @@ cudaError_t launch_fw_write(const Plan& p, int64_t chunk, int64_t ci, const int*
                             const float* dy, float* values, float lr, void* ws, cudaStream_t st);
 // dV (dense table, +=) or, when dVc is given, the compact form: dVc[u] = the gradient of
 // the u-th distinct selected row (ascending), rows_out[u] = that row, *U_out = U.
+// ent_tok, when given, maps every selection to its upstream-gradient row (else
+// selection / (h * ksel)).
 cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved& s,
                               const float* dy, float* dV, float* dw_out, void* ws,
                               cudaStream_t st, float* dVc = nullptr, int32_t* rows_out = nullptr,
-                              int* U_out = nullptr);
+                              int* U_out = nullptr, const int32_t* ent_tok = nullptr);
 cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, const float* bn,
                               const void* subkeys, const pkm_saved& s, float* dx, float* dWq,
                               float* dbn, float* dsub, float* dw_out, void* ws, cudaStream_t st);
@@ -188,6 +190,35 @@ cudaError_t launch_subgrad_tc(const Plan& p, const float* gsub, const int32_t* s
                               const float* qhat, __nv_bfloat16* G, float* dqf,
                               __nv_bfloat16* dq_planes, float* bn_part, float* dsub_part,
                               float* dsub, bool want_dq, cudaStream_t st);
+
+// ---------------------------------------------------------------- row-sharded table
+// Workspace layouts (byte offsets) of the source-side routing and the owner-side index.
+struct ShardRouteLayout {
+  size_t cnt, tri_off, seg_scan, bsum, total;
+};
+struct ShardOwnerLayout {
+  size_t pre, start, rows, wv, tok, total;
+};
+ShardRouteLayout shard_route_layout(int64_t N, int G);
+ShardOwnerLayout shard_owner_layout(int G, int64_t n_tri);
+cudaError_t launch_shard_route(const Plan& p, int G, int64_t R, const int32_t* idx, const float* w,
+                               int32_t* counts, int32_t* segpos, pkm_triple* send, int32_t* perm,
+                               void* ws, cudaStream_t st);
+// Prefix sums and segment starts of the received triples (and, when want_arrays, their
+// rows, weights and global segments for the value pass) in the owner workspace.
+cudaError_t launch_shard_owner_index(const Plan& p, int G, const int32_t* recv_counts,
+                                     int64_t n_tri, int64_t n_seg, const pkm_triple* recv,
+                                     int64_t shard_rows, void* ws, bool want_arrays,
+                                     cudaStream_t st);
+cudaError_t launch_shard_bag(const Plan& p, int G, int64_t n_seg, const pkm_triple* recv,
+                             const void* values, int64_t shard_rows, float* partial, void* ws,
+                             int64_t n_tri, cudaStream_t st);
+cudaError_t launch_shard_combine(const Plan& p, int G, const int32_t* segpos, const float* part,
+                                 int64_t n_rows, float* y, cudaStream_t st);
+cudaError_t launch_shard_gather_dy(const Plan& p, int G, const int32_t* segpos, const float* dy,
+                                   int64_t n_rows, float* out, cudaStream_t st);
+cudaError_t launch_shard_scatter_dw(const Plan& p, const int32_t* perm, const float* dw_ret,
+                                    float* dw, cudaStream_t st);
 
 // ---------------------------------------------------------------- self-test
 cudaError_t launch_wait_timeout_probe(long long budget_cycles, int* status, cudaStream_t st);

@@ -39,6 +39,8 @@ PKM_FW_LOOKAHEAD = 0x1
 PKM_FW_SORT_GLOBAL = 0x2
 PKM_FW_PER_CHUNK = 0x4
 SAVED_FIELDS = ("q", "qhat", "sub_s", "sub_i", "idx", "w", "bn_batch")
+PKM_MAX_SHARDS = 1024
+PKM_SHARD_ROUTE, PKM_SHARD_OWNER = 1, 2
 
 # every symbol include/pkm.h declares
 EXPORTED = ("pkm_saved_bytes", "pkm_workspace_bytes", "pkm_forward", "pkm_backward", "pkm_query",
@@ -46,7 +48,9 @@ EXPORTED = ("pkm_saved_bytes", "pkm_workspace_bytes", "pkm_forward", "pkm_backwa
             "pkm_status_string", "pkm_build_info", "pkm_value_grad", "pkm_query_grad",
             "pkm_launch_count", "pkm_selftest_wait_timeout", "pkm_value_grad_noalloc",
             "pkm_fastweight_workspace_bytes", "pkm_fastweight_chunks", "pkm_value_sgd",
-            "pkm_value_grad_rows", "pkm_value_adam", "pkm_hit_counts", "pkm_bn_running_update")
+            "pkm_value_grad_rows", "pkm_value_adam", "pkm_hit_counts", "pkm_bn_running_update",
+            "pkm_shard_workspace_bytes", "pkm_shard_route", "pkm_shard_bag", "pkm_shard_combine",
+            "pkm_shard_gather_dy", "pkm_shard_value_grad", "pkm_shard_scatter_dw")
 
 
 class PKMError(RuntimeError):
@@ -107,6 +111,15 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "pkm_fastweight_workspace_bytes": (S, [D, ctypes.c_int64, ctypes.c_uint32]),
         "pkm_fastweight_chunks": (I, [D, ctypes.c_int64, ctypes.c_float, ctypes.c_uint32, P, P, P,
                                       P, P, P, P, P, S, P]),
+        "pkm_shard_workspace_bytes": (S, [D, ctypes.c_int32, I, ctypes.c_int64]),
+        "pkm_shard_route": (I, [D, ctypes.c_int32, ctypes.c_int64, P, P, P, P, P, P, P, S, P]),
+        "pkm_shard_bag": (I, [D, ctypes.c_int32, ctypes.c_int64, P, ctypes.c_int64, ctypes.c_int64,
+                              P, P, P, P, S, P]),
+        "pkm_shard_combine": (I, [D, ctypes.c_int32, P, P, ctypes.c_int64, P, P]),
+        "pkm_shard_gather_dy": (I, [D, ctypes.c_int32, P, P, P, ctypes.c_int64, P]),
+        "pkm_shard_value_grad": (I, [D, ctypes.c_int32, ctypes.c_int64, P, ctypes.c_int64,
+                                     ctypes.c_int64, P, P, P, P, P, P, S, P]),
+        "pkm_shard_scatter_dw": (I, [D, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -378,3 +391,60 @@ def alloc_workspace(dims: Dims, which: int, device="cuda"):
     import torch
     n = pkm_workspace_bytes(dims, which)
     return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------- row-sharded table
+# Triples travel as int32 tensors of shape [n, 3] (segment, row, bits of the fp32 weight),
+# the layout of pkm_triple.
+
+def pkm_shard_workspace_bytes(dims: Dims, G: int, which: int, n_triples: int = 0) -> int:
+    return int(load().pkm_shard_workspace_bytes(ctypes.byref(dims.c()), int(G), int(which),
+                                                int(n_triples)))
+
+
+def pkm_shard_route(dims: Dims, G: int, rows_per_shard: int, idx, w, counts, segpos, send, perm,
+                    workspace=None, workspace_bytes: int = 0, stream=None) -> None:
+    _check(load().pkm_shard_route(ctypes.byref(dims.c()), int(G), int(rows_per_shard), _ptr(idx),
+                                  _ptr(w), _ptr(counts), _ptr(segpos), _ptr(send), _ptr(perm),
+                                  _ptr(workspace), _ws(workspace, workspace_bytes),
+                                  _stream(stream)), "pkm_shard_route")
+
+
+def pkm_shard_bag(dims: Dims, G: int, shard_rows: int, recv_counts, n_triples: int,
+                  n_segments: int, recv, values, partial, workspace=None,
+                  workspace_bytes: int = 0, stream=None) -> None:
+    _check(load().pkm_shard_bag(ctypes.byref(dims.c()), int(G), int(shard_rows),
+                                _ptr(recv_counts), int(n_triples), int(n_segments), _ptr(recv),
+                                _ptr(values), _ptr(partial), _ptr(workspace),
+                                _ws(workspace, workspace_bytes), _stream(stream)),
+           "pkm_shard_bag")
+
+
+def pkm_shard_combine(dims: Dims, G: int, segpos, partial_recv, n_rows: int, y,
+                      stream=None) -> None:
+    _check(load().pkm_shard_combine(ctypes.byref(dims.c()), int(G), _ptr(segpos),
+                                    _ptr(partial_recv), int(n_rows), _ptr(y), _stream(stream)),
+           "pkm_shard_combine")
+
+
+def pkm_shard_gather_dy(dims: Dims, G: int, segpos, dy, dy_send, n_rows: int,
+                        stream=None) -> None:
+    _check(load().pkm_shard_gather_dy(ctypes.byref(dims.c()), int(G), _ptr(segpos), _ptr(dy),
+                                      _ptr(dy_send), int(n_rows), _stream(stream)),
+           "pkm_shard_gather_dy")
+
+
+def pkm_shard_value_grad(dims: Dims, G: int, shard_rows: int, recv_counts, n_triples: int,
+                         n_segments: int, recv, values, dy_recv, dvalues, dw_recv,
+                         workspace=None, workspace_bytes: int = 0, stream=None) -> None:
+    _check(load().pkm_shard_value_grad(ctypes.byref(dims.c()), int(G), int(shard_rows),
+                                       _ptr(recv_counts), int(n_triples), int(n_segments),
+                                       _ptr(recv), _ptr(values), _ptr(dy_recv), _ptr(dvalues),
+                                       _ptr(dw_recv), _ptr(workspace),
+                                       _ws(workspace, workspace_bytes), _stream(stream)),
+           "pkm_shard_value_grad")
+
+
+def pkm_shard_scatter_dw(dims: Dims, perm, dw_ret, dw, stream=None) -> None:
+    _check(load().pkm_shard_scatter_dw(ctypes.byref(dims.c()), _ptr(perm), _ptr(dw_ret), _ptr(dw),
+                                       _stream(stream)), "pkm_shard_scatter_dw")

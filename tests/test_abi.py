@@ -253,3 +253,50 @@ def test_all_k2_sizes(lib):
     assert P.pkm_workspace_bytes(d2, P.PKM_BWD) > P.pkm_workspace_bytes(d, P.PKM_BWD)
     big = _dims(N=1 << 18, k=32, h=4, flags=P.PKM_F_ALL_K2)       # 2^18*4*1024*2 = 2^31
     assert _fwd(big) == P.PKM_ERR_UNSUPPORTED
+
+
+def test_shard_validation(lib):
+    """Row-sharded entry points: shard count, shard size, sizes of what was received and
+    the workspace are checked on the host."""
+    L = P.load()
+    d = _dims()                                    # 32 x 32 = 1024 rows
+    c = ctypes.byref(d.c())
+    nb = P.pkm_shard_workspace_bytes(d, 4, P.PKM_SHARD_ROUTE)
+    assert nb >= 3 * 4 * 4 * d.N                   # three [G][N] int32 tables
+    assert P.pkm_shard_workspace_bytes(d, 0, P.PKM_SHARD_ROUTE) == 0
+    assert P.pkm_shard_workspace_bytes(d, P.PKM_MAX_SHARDS + 1, P.PKM_SHARD_ROUTE) == 0
+    assert P.pkm_shard_workspace_bytes(d, 4, 7) == 0
+    own = P.pkm_shard_workspace_bytes(d, 4, P.PKM_SHARD_OWNER, 10)
+    assert P.pkm_shard_workspace_bytes(d, 4, P.PKM_SHARD_OWNER, 1000) > own > 0
+    route = lambda **kw: L.pkm_shard_route(
+        ctypes.byref(kw.get("d", d).c()), kw.get("G", 4), kw.get("R", 256), FAKE, FAKE,
+        kw.get("counts", FAKE), FAKE, kw.get("send", FAKE), FAKE, FAKE, kw.get("nb", nb), None)
+    assert route(G=0) == P.PKM_ERR_INVALID_ARG
+    assert route(G=P.PKM_MAX_SHARDS + 1) == P.PKM_ERR_INVALID_ARG
+    assert route(R=255) == P.PKM_ERR_INVALID_ARG   # 4 shards of 255 rows miss the last rows
+    assert route(R=0) == P.PKM_ERR_INVALID_ARG
+    assert route(counts=None) == P.PKM_ERR_INVALID_ARG
+    assert route(send=FAKE + 4) == P.PKM_ERR_INVALID_ARG
+    assert route(nb=nb - 1) == P.PKM_ERR_WORKSPACE
+    assert route(d=_dims(N=1 << 28), G=8, nb=1 << 40) == P.PKM_ERR_UNSUPPORTED   # G*N >= 2^31
+    bag = lambda **kw: L.pkm_shard_bag(c, 4, kw.get("rows", 256), FAKE, kw.get("nt", 10),
+                                       kw.get("ns", 4), FAKE, FAKE, kw.get("part", FAKE), FAKE,
+                                       kw.get("nb", own), None)
+    assert bag(ns=11) == P.PKM_ERR_INVALID_ARG     # more segments than triples
+    assert bag(ns=0) == P.PKM_ERR_INVALID_ARG      # triples without a segment
+    assert bag(rows=0) == P.PKM_ERR_INVALID_ARG
+    assert bag(part=None) == P.PKM_ERR_INVALID_ARG
+    assert bag(nb=own - 1) == P.PKM_ERR_WORKSPACE
+    assert bag(nt=0, ns=0) == P.PKM_OK             # nothing received
+    vg = lambda **kw: L.pkm_shard_value_grad(c, 4, 256, FAKE, kw.get("nt", 10), kw.get("ns", 4),
+                                             FAKE, FAKE, FAKE, kw.get("dv", FAKE), FAKE, FAKE,
+                                             kw.get("nb", own), None)
+    assert vg(ns=11) == P.PKM_ERR_INVALID_ARG
+    assert vg(dv=None) == P.PKM_ERR_INVALID_ARG
+    assert vg(nb=own - 1) == P.PKM_ERR_WORKSPACE
+    assert vg(nt=0, ns=0) == P.PKM_OK
+    assert L.pkm_shard_combine(c, 4, FAKE, FAKE, -1, FAKE, None) == P.PKM_ERR_INVALID_ARG
+    assert L.pkm_shard_combine(c, 4, None, FAKE, 10, FAKE, None) == P.PKM_ERR_INVALID_ARG
+    assert L.pkm_shard_gather_dy(c, 4, FAKE, None, FAKE, 10, None) == P.PKM_ERR_INVALID_ARG
+    assert L.pkm_shard_gather_dy(c, 4, None, None, None, 0, None) == P.PKM_OK
+    assert L.pkm_shard_scatter_dw(c, None, FAKE, FAKE, None) == P.PKM_ERR_INVALID_ARG
