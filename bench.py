@@ -593,6 +593,7 @@ def run_fastweight(args, cfg, rank, world, dist):
 
 # ---------------------------------------------------------------- decode latency
 DECODE_METRIC = "PKM decode forward latency (us/call) at |K|=1024², h=4, k=32, d=1600"
+SHARD_METRIC = "row-sharded PKM layer tokens/s (fwd+bwd), value rows split over the ranks"
 
 
 def run_decode(args, cfg, rank, world, dist):
@@ -711,6 +712,125 @@ def run_decode(args, cfg, rank, world, dist):
         "clocks": clk, "gpu_launches": int(launches),
         **({"cpu_baseline": cpu} if cpu else {}),
     }
+
+
+def run_sharded(args, cfg, rank, world, dist):
+    """The row-sharded layer, fwd + bwd: every rank its own tokens and 1/world of the value
+    table's rows (whole leading sub-key ranges); the exchanges between the library's calls
+    go through torch.distributed (NCCL), with one rank through nothing.  Also the owner's
+    partial-bag kernel alone, against the HBM roofline."""
+    import torch
+
+    from product_key_memory_pkm_b200 import build as B
+    from product_key_memory_pkm_b200 import pkm as P
+    from product_key_memory_pkm_b200 import sharded as S
+
+    if not os.path.exists(B.LIB):
+        B.build()
+    P.load()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    st = torch.cuda.current_stream()
+    inp = rank_batch(cfg, rank, world)
+    bf = torch.bfloat16
+    r0, r1 = S.shard_range(rank, world, cfg.C1, cfg.C2)
+    x = torch.from_numpy(inp["x"]).to(bf).to(dev)
+    Wq = torch.from_numpy(inp["Wq"]).to(bf).to(dev)
+    bn = torch.from_numpy(inp["bn"]).to(dev)
+    sub = torch.from_numpy(inp["subkeys"]).to(bf).to(dev)
+    Vs = torch.from_numpy(inp["values"][r0:r1]).to(bf).to(dev)
+    dy = torch.from_numpy(inp["dy"]).to(dev)
+    ex = S.TorchExchange() if world > 1 else S.LocalExchange()
+    dims = P.Dims.from_config(cfg)
+    dVs = torch.zeros(max(r1 - r0, 1), cfg.d_v, device=dev)
+    dx = torch.empty(cfg.N, cfg.d_in, device=dev)
+    dWq = torch.zeros(cfg.h * cfg.dk, cfg.d_in, device=dev)
+    dbn = torch.zeros(2, cfg.h * cfg.dk, device=dev)
+    dsub = torch.zeros(cfg.h, cfg.C1 + cfg.C2, cfg.dk // 2, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(st)
+        y, ctx = S.sharded_forward(dims, world, rank, x, Wq, bn, sub, Vs, ex, stream=st)
+        if ev is not None:
+            ev[1].record(st)
+        S.sharded_backward(ctx, dy, ex, Vs, dVs, x, Wq, bn, sub, dx, dWq, dbn, dsub, stream=st)
+        if ev is not None:
+            ev[2].record(st)
+        return ctx
+
+    clocks = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    clocks.start()
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if P.pkm_check_status(st) != P.PKM_OK:
+        raise RuntimeError("device status after warm-up is not OK")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = P.pkm_launch_count()
+    for s_ in range(args.steps):
+        flush.zero_()
+        ctx = step(evs[s_])
+    torch.cuda.synchronize()
+    launches = P.pkm_launch_count() - launches0
+    fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    # the owner's partial bag alone (the shard's HBM-bound kernel), L2 flushed before each
+    n_tri, n_seg = sum(ctx.recv_tri), sum(ctx.recv_seg)
+    part = torch.empty(max(n_seg, 1), cfg.d_v, device=dev)
+    bag_ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        P.pkm_shard_bag(dims, world, ctx.shard_rows, ctx.recv_counts, n_tri, n_seg, ctx.recv,
+                        Vs, part, ctx.owner_ws, stream=st)
+        b.record(st)
+        b.synchronize()
+        bag_ms.append(a.elapsed_time(b))
+    launches += 2 * args.steps   # the bag call above: segment starts, bag
+    if P.pkm_check_status(st) != P.PKM_OK:
+        raise RuntimeError("device status after the timed steps is not OK")
+    clk = clocks.stop()
+    step_ms, fwd_ms, bwd_ms, bag = max_over_ranks(
+        [fwd_ms + bwd_ms, fwd_ms, bwd_ms, float(np.mean(bag_ms))], dist, dev)
+    if dist is not None:
+        dist.barrier()
+    if rank != 0:
+        return None
+    pk = _peaks()
+    bag_bytes = n_tri * cfg.d_v * 2 + n_seg * cfg.d_v * 4 + n_tri * 12
+    ach = bag_bytes / (bag * 1e-3) / 1e9
+    out = {
+        "metric": SHARD_METRIC,
+        "value": round(cfg.N * world / (step_ms * 1e-3), 1),
+        "unit": "tokens/s (fwd+bwd)",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; tables random-init, no trained weights)",
+        "config": dict(_cfg_json(cfg), parallelism=f"rowshard{world}", shard_rows=r1 - r0,
+                       l2="flushed before every timed step (256 MiB write)"),
+        "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
+        "roofline": {"kernel": "shard_bag (owner partial bags)", "bound": "hbm",
+                     "achieved": round(ach, 1), "peak": pk["hbm"], "unit": "GB/s",
+                     "frac": round(ach / pk["hbm"], 4), "traffic": None,
+                     "algorithmic_bytes": int(bag_bytes), "ms": round(bag, 4),
+                     "peak_source": pk["src"]},
+        "clocks": clk, "gpu_launches": int(launches),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        v, n, thr = time_oracle(cfg, inp, args.cpu_seconds)
+        out["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s (fwd+bwd)", "cores": thr,
+                               "kind": "oracle",
+                               "sample": f"{n} tokens of the same batch, fp64 numpy oracle of the "
+                                         f"whole layer (the sharding does not change the result)"}
+    return out
 
 
 def run_stage(args, cfg, dims, saved, P, st, step, flush, names, env):
@@ -869,6 +989,9 @@ def main():
                          "training-mode BatchNorm, or the all-k^2 softmax")
     ap.add_argument("--decode", action="store_true",
                     help="decode-shaped forward latency (N = 1, 8, 64) on the workload's table")
+    ap.add_argument("--sharded", action="store_true",
+                    help="row-sharded value table: each rank 1/N of the rows, exchanges over "
+                         "torch.distributed")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -890,7 +1013,7 @@ def main():
             tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
             dist = tdist
         try:
-            run = (run_decode if args.decode else
+            run = (run_decode if args.decode else run_sharded if args.sharded else
                    run_fastweight if cfg.name == FASTWEIGHT.name else run_b200)
             out = run(args, cfg, rank, world, dist)
         finally:

@@ -19,7 +19,8 @@
 //                       segment (source offset added); segment_start_kernel the first
 //                       triple of every segment (binary search: segment ids ascend inside a
 //                       source's run).
-//   shard_bag_kernel    partial[j] = sum over segment j's triples of w * V[row], fp32.
+//   shard_bag_kernel    partial[j] = sum over segment j's triples of w * V[row], fp32
+//                       (the segment's triples staged in shared memory, 8 rows in flight).
 // and the backward's value pass on its rows reuses the value-row kernel with a per-entry
 // token map (the entry's segment selects its upstream-gradient row).
 #include <algorithm>
@@ -204,67 +205,82 @@ __global__ void segment_start_kernel(const pkm_triple* __restrict__ recv,
   }
 }
 
-template <typename TV>
-struct Vec16;
-template <>
-struct Vec16<__nv_bfloat16> {
-  static constexpr int E = 8;
-  __device__ static void load(const __nv_bfloat16* p, float* f) {
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(p)), f);
-  }
-};
-template <>
-struct Vec16<float> {
-  static constexpr int E = 4;
-  __device__ static void load(const float* p, float* f) {
-    const float4 u = __ldg(reinterpret_cast<const float4*>(p));
-    f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
-  }
-};
+// 16 bytes of a value row, streamed (no L1 allocation: every row is read once here)
+__device__ __forceinline__ uint4 ld_row16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ void to_f32(const uint4& u, __nv_bfloat16, float* f) { bf16x8_to_f32(u, f); }
+__device__ __forceinline__ void to_f32(const uint4& u, float, float* f) {
+  f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+  f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+}
 
-// One CTA per segment; thread = 16-byte column slice; four rows in flight.
+constexpr int kBagChunk = 256, kBagAhead = 8;
+
+// One CTA per segment.  The segment's triples are staged in shared memory (chunks of
+// 256), then thread j accumulates 16-byte column slice j (j + blockDim.x, ...) over them
+// with eight rows in flight; fp32 sums in triple order.
 template <typename TV>
 __global__ void __launch_bounds__(256) shard_bag_kernel(
     const pkm_triple* __restrict__ recv, const int32_t* __restrict__ start, const TV* __restrict__ V,
     int64_t shard_rows, int d_v, float* __restrict__ partial, int* status) {
-  constexpr int E = Vec16<TV>::E;
+  constexpr int E = 16 / sizeof(TV);
+  __shared__ int32_t s_row[kBagChunk];
+  __shared__ float s_w[kBagChunk];
   const int64_t j = blockIdx.x;
   const int i0 = start[j], i1 = start[j + 1];
-  const int nvec = d_v / E;
-  for (int vec = threadIdx.x; vec < nvec; vec += blockDim.x) {
+  const int nvec = d_v / E, tid = threadIdx.x;
+  for (int vb = 0; vb < nvec; vb += blockDim.x) {  // uniform over the CTA
+    const int vec = vb + tid;
+    const bool live = vec < nvec;
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    for (int i = i0; i < i1; i += 4) {
-      float f[4][E];
-      float wt[4];
+    for (int base = i0; base < i1; base += kBagChunk) {
+      const int n = min(kBagChunk, i1 - base);
+      __syncthreads();  // the previous chunk is consumed
+      for (int i = tid; i < n; i += blockDim.x) {
+        const pkm_triple tr = recv[base + i];
+        const bool ok = tr.row >= 0 && tr.row < shard_rows;
+        if (!ok) set_status(status, kDevIndex);
+        s_row[i] = ok ? tr.row : 0;
+        s_w[i] = ok ? tr.w : 0.f;
+      }
+      __syncthreads();
+      if (!live) continue;
+      const TV* col = V + (int64_t)vec * E;
+      int i = 0;
+      for (; i + kBagAhead <= n; i += kBagAhead) {
+        uint4 u[kBagAhead];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        wt[u] = 0.f;
-        if (i + u < i1) {
-          const pkm_triple tr = recv[i + u];
-          if (tr.row >= 0 && tr.row < shard_rows) {
-            wt[u] = tr.w;
-            Vec16<TV>::load(V + (int64_t)tr.row * d_v + (int64_t)vec * E, f[u]);
-          } else if (vec == threadIdx.x) {
-            set_status(status, kDevIndex);
-          }
-        }
-        if (wt[u] == 0.f) {
+        for (int q = 0; q < kBagAhead; ++q) u[q] = ld_row16(col + (int64_t)s_row[i + q] * d_v);
 #pragma unroll
-          for (int e = 0; e < E; ++e) f[u][e] = 0.f;
+        for (int q = 0; q < kBagAhead; ++q) {
+          float f[E];
+          to_f32(u[q], TV(), f);
+          const float wq = s_w[i + q];
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[e] = fmaf(wq, f[e], acc[e]);
         }
       }
+      for (; i < n; ++i) {
+        float f[E];
+        to_f32(ld_row16(col + (int64_t)s_row[i] * d_v), TV(), f);
+        const float wq = s_w[i];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] = fmaf(wt[u], f[u][e], acc[e]);
+        for (int e = 0; e < E; ++e) acc[e] = fmaf(wq, f[e], acc[e]);
       }
     }
-    float4* out = reinterpret_cast<float4*>(partial + j * d_v + (int64_t)vec * E);
+    if (live) {
+      float4* out = reinterpret_cast<float4*>(partial + j * d_v + (int64_t)vec * E);
 #pragma unroll
-    for (int e4 = 0; e4 < E / 4; ++e4)
-      out[e4] = make_float4(acc[4 * e4], acc[4 * e4 + 1], acc[4 * e4 + 2], acc[4 * e4 + 3]);
+      for (int e4 = 0; e4 < E / 4; ++e4)
+        out[e4] = make_float4(acc[4 * e4], acc[4 * e4 + 1], acc[4 * e4 + 2], acc[4 * e4 + 3]);
+    }
   }
 }
 

@@ -9,7 +9,8 @@ module holds only the order of the calls and the exchanges between ranks, made b
 exchange object:
 
 * ``TorchExchange``: ``torch.distributed.all_to_all_single`` on a process group (NCCL
-  on GPUs, gloo on CPUs).
+  on GPUs, gloo on CPUs);
+* ``LocalExchange``: one rank, nothing to move.
 
 Forward on every rank: F1-F3 for its tokens (``pkm_query``, ``pkm_subkey_scores``,
 ``pkm_candidate_topk``; the query network and sub-keys are replicated), then
@@ -39,6 +40,15 @@ def shard_range(g: int, G: int, C1: int, C2: int) -> tuple[int, int]:
     R = rows_per_shard(C1, C2, G)
     K = C1 * C2
     return min(g * R, K), min((g + 1) * R, K)
+
+
+class LocalExchange:
+    """One rank: every all-to-all returns what the rank sent itself."""
+
+    def all_to_all(self, x: torch.Tensor, send_splits: list[int],
+                   recv_splits: list[int]) -> torch.Tensor:
+        assert list(send_splits) == list(recv_splits) and len(send_splits) == 1
+        return x
 
 
 class TorchExchange:
