@@ -886,7 +886,7 @@ def run_sharded(args, cfg, rank, world, dist):
         "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
         "roofline": {"kernel": "shard_bag (owner partial bags)", "bound": "hbm",
                      "achieved": round(ach, 1), "peak": pk["hbm"], "unit": "GB/s",
-                     "frac": round(ach / pk["hbm"], 4), "traffic": None,
+                     "frac": round(ach / pk["hbm"], 4), "traffic": _ncu_traffic("shard_bag"),
                      "algorithmic_bytes": int(bag_bytes), "ms": round(bag, 4),
                      "peak_source": pk["src"]},
         "clocks": clk, "gpu_launches": int(launches),

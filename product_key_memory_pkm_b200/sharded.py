@@ -23,7 +23,7 @@ data-parallel reduction; dV stays on the rank that owns the rows.
 """
 from __future__ import annotations
 
-from dataclasses import dataclass, field
+from dataclasses import dataclass
 
 import torch
 
@@ -81,7 +81,6 @@ class ShardedContext:
     recv_tri: list[int]
     recv_seg: list[int]
     owner_ws: torch.Tensor
-    extra: dict = field(default_factory=dict)
 
 
 def _bytes(n: int, device) -> torch.Tensor:
