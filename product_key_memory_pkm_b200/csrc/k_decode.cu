@@ -12,9 +12,9 @@
 //                        bf16 hi + lo planes (and q-hat), as the tensor-core kernel does.
 //   scores_small_kernel  one 8-CTA cluster per (16-token group, head, half): CTA r scores
 //                        its 1/8 of the sub-keys against every token of the group and keeps
-//                        each token's top-k of its slice; CTA 0 then merges the 8 sorted
-//                        lists per token through distributed shared memory.  Order: (score
-//                        desc, sub-key index asc), as everywhere.
+//                        each token's top-k of its slice; then CTA r merges the 8 sorted
+//                        lists of tokens r and r + 8 through distributed shared memory.
+//                        Order: (score desc, sub-key index asc), as everywhere.
 #include <cooperative_groups.h>
 
 #include "pkm_internal.cuh"
@@ -26,7 +26,7 @@ namespace cg = cooperative_groups;
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kTokGroup = 16, kWarps = 8, kSplit = 8;
 constexpr int kPerLane = 8;  // sub-keys per lane in a slice's selection (slices <= 256)
-constexpr int kRankTokens = 2;  // up to this many tokens, selection and merge by rank
+constexpr int kRankTokens = 2;  // up to this many tokens, selection by rank
 
 // 16-byte global -> shared copies that stay in flight together (completion waited for
 // with cp_async_wait_all before the block barrier).
@@ -280,93 +280,60 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kWarps * 32)
     }
   }
   cluster.sync();
-  // 4. CTA 0 gathers the kSplit sorted lists of every token of the group ...
-  if (rank == 0) {  // eight remote elements per thread and step, loads first
-    const int n_el = nt * kSplit * KM;
-    for (int i0 = tid; i0 < n_el; i0 += 8 * nthr) {
-      float v[8];
-      int x[8];
+  // 4. CTA r gathers the kSplit sorted lists of the group's tokens t = r, r + kSplit, ...
+  //    (at most two per CTA), eight remote elements per thread and step, loads first ...
+  const int my_nt = nt > rank ? (nt - rank + kSplit - 1) / kSplit : 0;
+  const int n_el = my_nt * kSplit * KM;
+  for (int i0 = tid; i0 < n_el; i0 += 8 * nthr) {
+    float v[8];
+    int x[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * nthr;
-        if (i < n_el) {
-          const int t = i / (kSplit * KM), r = (i / KM) % kSplit, j = i % KM;
-          v[u] = cluster.map_shared_rank(ls, r)[t * KM + j];
-          x[u] = cluster.map_shared_rank(li, r)[t * KM + j];
-        }
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * nthr;
+      if (i < n_el) {
+        const int t = rank + (i / (kSplit * KM)) * kSplit, r = (i / KM) % kSplit, j = i % KM;
+        v[u] = cluster.map_shared_rank(ls, r)[t * KM + j];
+        x[u] = cluster.map_shared_rank(li, r)[t * KM + j];
       }
+    }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * nthr;
-        if (i < n_el) {
-          ms[i] = v[u];
-          mi[i] = x[u];
-        }
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * nthr;
+      if (i < n_el) {
+        ms[i] = v[u];
+        mi[i] = x[u];
       }
     }
   }
-  cluster.sync();  // the other CTAs' lists may be released now
-  if (rank != 0) return;
+  cluster.sync();  // the lists may be released now
+  if (my_nt == 0) return;
   __syncthreads();
-  // 5. ... and merges them.  Few tokens: every element is placed by merge rank -- its
-  //    position in its own list plus, for every other list, how many of that list's elements
-  //    rank before it (binary search).  More: one warp per token, lane r < kSplit walking list
-  //    r; each of the k steps emits the best head and advances its list.
-  if (by_rank) {
-    for (int i = tid; i < nt * kSplit * KM; i += nthr) {
-      const int t = i / (kSplit * KM), r = (i / KM) % kSplit, j = i % KM;
-      const float v = ms[i];
-      const int vi = mi[i];
-      if (vi == 0x7fffffff) continue;  // padding
-      int place = j;
-      for (int r2 = 0; r2 < kSplit; ++r2) {
-        if (r2 == r) continue;
-        const float* lv = ms + (t * kSplit + r2) * KM;
-        const int* lx = mi + (t * kSplit + r2) * KM;
-        int lo = 0, hi = KM;  // first element of list r2 that does not rank before (v, vi)
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (before(lv[mid], lx[mid], v, vi)) lo = mid + 1;
-          else hi = mid;
-        }
-        place += lo;
+  // 5. ... and merges them: every element is placed by merge rank -- its position in its
+  //    own list plus, for every other list, how many of that list's elements rank before
+  //    it (binary search).
+  for (int i = tid; i < n_el; i += nthr) {
+    const int lt = i / (kSplit * KM), r = (i / KM) % kSplit, j = i % KM;
+    const int t = rank + lt * kSplit;
+    const float v = ms[i];
+    const int vi = mi[i];
+    if (vi == 0x7fffffff) continue;  // padding
+    int place = j;
+    for (int r2 = 0; r2 < kSplit; ++r2) {
+      if (r2 == r) continue;
+      const float* lv = ms + (lt * kSplit + r2) * KM;
+      const int* lx = mi + (lt * kSplit + r2) * KM;
+      int lo = 0, hi = KM;  // first element of list r2 that does not rank before (v, vi)
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (before(lv[mid], lx[mid], v, vi)) lo = mid + 1;
+        else hi = mid;
       }
-      if (place < k) {
-        const int64_t o = (((t0 + t) * h + hh) * 2 + s) * (int64_t)k + place;
-        sub_s[o] = v;
-        sub_i[o] = vi;
-      }
+      place += lo;
     }
-    return;
-  }
-  for (int t = wid; t < nt; t += kWarps) {
-    const float* lv = ms + (t * kSplit + (lane & (kSplit - 1))) * KM;
-    const int* lx = mi + (t * kSplit + (lane & (kSplit - 1))) * KM;
-    int pos = 0;
-    const int64_t o = (((t0 + t) * h + hh) * 2 + s) * (int64_t)k;
-    for (int j = 0; j < k; ++j) {
-      float hs = -INFINITY;
-      int hx = 0x7fffffff;
-      if (lane < kSplit && pos < KM) {
-        hs = lv[pos];
-        hx = lx[pos];
-      }
-      float bs = hs;
-      int bi = hx;
-#pragma unroll
-      for (int m = 16; m > 0; m >>= 1) {
-        const float os = __shfl_xor_sync(kFull, bs, m);
-        const int oi = __shfl_xor_sync(kFull, bi, m);
-        if (before(os, oi, bs, bi)) {
-          bs = os;
-          bi = oi;
-        }
-      }
-      if (lane < kSplit && hx == bi) ++pos;  // unique indices: one list advances
-      if (lane == 0) {
-        sub_s[o + j] = bs;
-        sub_i[o + j] = bi;
-      }
+    if (place < k) {
+      const int64_t o = (((t0 + t) * h + hh) * 2 + s) * (int64_t)k + place;
+      sub_s[o] = v;
+      sub_i[o] = vi;
     }
   }
 }
