@@ -25,8 +25,7 @@ namespace {
 namespace cg = cooperative_groups;
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kTokGroup = 16, kWarps = 8, kSplit = 8;
-constexpr int kPerLane = 8;  // sub-keys per lane in a slice's selection (slices <= 256)
-constexpr int kRankTokens = 2;  // up to this many tokens, selection by rank
+constexpr int kMaxSlice = 256;  // sub-keys per CTA (a cluster scores up to 8 * 256 per half)
 
 // 16-byte global -> shared copies that stay in flight together (completion waited for
 // with cp_async_wait_all before the block barrier).
@@ -220,63 +219,17 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kWarps * 32)
     sc[t * per_max + c] = idw ? -0.5f * logf(fmaxf(qn + cn - 2.f * acc, 0.f) + 1e-12f) : acc;
   }
   __syncthreads();
-  // 3. each token's top-KM of the slice, best first.  With at most kRankTokens tokens every
-  //    thread places one candidate: its place is the number of the slice's candidates that
-  //    rank before it.  With more, one warp per token holds the slice's candidates
-  //    (kPerLane per lane) and extracts the best one KM times.
-  const int lane = tid & 31, wid = tid >> 5;
-  const bool by_rank = nt <= kRankTokens;  // uniform over the cluster
-  if (by_rank) {
-    for (int i = tid; i < nt * nct; i += nthr) {
-      const int t = i / nct, c = i % nct;
-      const float* st = sc + t * per_max;
-      const float v = st[c];
-      int r = 0;
-      for (int c2 = 0; c2 < nct; ++c2) r += before(st[c2], c0 + c2, v, c0 + c) ? 1 : 0;
-      if (r < KM) {
-        ls[t * KM + r] = v;
-        li[t * KM + r] = c0 + c;
-      }
-    }
-  }
-  for (int t = wid; t < nt && !by_rank; t += kWarps) {
+  // 3. each token's top-KM of the slice, best first: every thread places candidates, each
+  //    at the number of the slice's candidates that rank before it.
+  for (int i = tid; i < nt * nct; i += nthr) {
+    const int t = i / nct, c = i % nct;
     const float* st = sc + t * per_max;
-    float cv[kPerLane];
-    int ci[kPerLane];
-#pragma unroll
-    for (int m = 0; m < kPerLane; ++m) {
-      const int c = lane + 32 * m;
-      cv[m] = c < nct ? st[c] : -INFINITY;
-      ci[m] = c < nct ? c0 + c : 0x7fffffff;
-    }
-    for (int j = 0; j < KM; ++j) {
-      float bs = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int m = 0; m < kPerLane; ++m)
-        if (before(cv[m], ci[m], bs, bi)) {
-          bs = cv[m];
-          bi = ci[m];
-        }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float os = __shfl_xor_sync(kFull, bs, o);
-        const int oi = __shfl_xor_sync(kFull, bi, o);
-        if (before(os, oi, bs, bi)) {
-          bs = os;
-          bi = oi;
-        }
-      }
-#pragma unroll
-      for (int m = 0; m < kPerLane; ++m)
-        if (ci[m] == bi) {  // indices are unique: only the owner matches (padding never wins
-          cv[m] = -INFINITY;  // while a real candidate is left)
-          ci[m] = 0x7fffffff;
-        }
-      if (lane == 0) {
-        ls[t * KM + j] = bs;
-        li[t * KM + j] = bi;
-      }
+    const float v = st[c];
+    int r = 0;
+    for (int c2 = 0; c2 < nct; ++c2) r += before(st[c2], c0 + c2, v, c0 + c) ? 1 : 0;
+    if (r < KM) {
+      ls[t * KM + r] = v;
+      li[t * KM + r] = c0 + c;
     }
   }
   cluster.sync();
@@ -347,7 +300,7 @@ size_t scores_small_smem(const Plan& p, int KM) {
 
 bool small_n_supported(const Plan& p) {
   return !p.fp32 && p.N <= kSmallTokens && p.d_in % 8 == 0 && (p.dk / 2) % 8 == 0 &&
-         (std::max(p.C1, p.C2) + kSplit - 1) / kSplit <= 32 * kPerLane &&
+         (std::max(p.C1, p.C2) + kSplit - 1) / kSplit <= kMaxSlice &&
          (size_t)kTokGroup * p.d_in * 2 <= 160 * 1024 && scores_small_smem(p, 32) <= 200 * 1024;
 }
 
