@@ -136,7 +136,8 @@ class CpuOps:
 
     # -- the exchange steps
     def pkm_shard_route(self, dims, G, R, idx, w, counts, segpos, send, perm, ws, stream=None):
-        c, sp, snd, pm = route(idx.reshape(dims.N, -1).numpy(), w.reshape(dims.N, -1).numpy(),
+        hk = idx.shape[1] * idx.shape[2]
+        c, sp, snd, pm = route(idx.reshape(dims.N, hk).numpy(), w.reshape(dims.N, hk).numpy(),
                                G, R)
         counts[:] = torch.from_numpy(c)
         segpos[:, :dims.N] = torch.from_numpy(sp)

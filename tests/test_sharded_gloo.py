@@ -21,14 +21,14 @@ from tests.shard_ref import CpuOps
 CFG = PKMConfig("sharded", N=24, d_in=16, h=2, dk=8, C1=7, C2=5, k=3, d_v=8, dtype="f32")
 
 
-def _worker(rank, world, port, out):
+def _worker(rank, world, port, out, bounds):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         inp = make_inputs(CFG, seed=3, random_bn=True)
         of = O.forward(inp, CFG)
-        n = CFG.N // world
-        t0 = rank * n
+        t0 = bounds[rank]
+        n = bounds[rank + 1] - t0
         dims = P.Dims.from_config(CFG, N=n)
         ops = CpuOps(of, t0)
         r0, r1 = S.shard_range(rank, world, CFG.C1, CFG.C2)
@@ -45,12 +45,16 @@ def _worker(rank, world, port, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_row_sharded_layer_over_gloo_ranks_matches_the_oracle(world):
-    port = 29700 + world * 10 + (os.getpid() % 500)
+@pytest.mark.parametrize("world,bounds", [
+    (2, (0, 12, 24)),
+    (3, (0, 8, 16, 24)),
+    (2, (0, 24, 24)),          # rank 1 has no tokens; it still owns rows and serves rank 0
+])
+def test_row_sharded_layer_over_gloo_ranks_matches_the_oracle(world, bounds):
+    port = 29700 + world * 10 + bounds[1] + (os.getpid() % 500)
     with mp.Manager() as mgr:
         out = mgr.dict()
-        mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+        mp.spawn(_worker, args=(world, port, out, bounds), nprocs=world, join=True)
         res = [out[r] for r in range(world)]
     inp = make_inputs(CFG, seed=3, random_bn=True)
     of = O.forward(inp, CFG)
