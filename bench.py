@@ -28,6 +28,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -91,7 +92,7 @@ class ClockSampler:
     def __init__(self, gpu_uuid: str | None):
         self.uuid = gpu_uuid
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"pkm_clocks_{os.getpid()}.csv")
 
     def start(self):
         try:
