@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       Prob::epi_begin(P, u, row, epi_smem, es);
       const int nc = Prob::num_chunks(P, u);
       for (int c = 0; c < nc; ++c) {
-        // warp-uniform wait: lane 0 waits, the verdict is broadcast, so the warp reaches
+        // warp-uniform wait: lane 0 waits, the result is broadcast, so the warp reaches
         // the .sync.aligned TMEM loads together or not at all
         int got = 0;
         if (lane == 0) got = mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag, status) ? 1 : 0;
