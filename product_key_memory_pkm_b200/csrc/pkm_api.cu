@@ -752,7 +752,8 @@ pkm_status pkm_shard_route(const pkm_dims* d, int32_t G, int64_t rows_per_shard,
                            size_t workspace_bytes, void* stream) {
   PKM_TRY(validate_shard(d, G));
   const int64_t K = (int64_t)d->C1 * d->C2;
-  if (rows_per_shard < 1 || (K + rows_per_shard - 1) / rows_per_shard > G)
+  // G shards of rows_per_shard rows must cover the table (no overflow for large shards)
+  if (rows_per_shard < 1 || (rows_per_shard < K && (K + rows_per_shard - 1) / rows_per_shard > G))
     return PKM_ERR_INVALID_ARG;
   PKM_NEED(counts);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
