@@ -370,22 +370,24 @@ pkm_status pkm_check_status(void* stream);
 const char* pkm_status_string(pkm_status s);
 
 /* Value-gradient stage (as pkm_value_grad) for callers that cannot allocate device
- * memory, so cannot pass a workspace: for instance code that runs while a stream is
- * being captured into a CUDA graph (a cudaMalloc there is refused or breaks the
- * capture), or a plugin inside a host framework that owns all device memory through
- * its own allocator and gives the plugin no way to reserve more.  This entry point
- * allocates nothing: its scratch is a fixed 64 MiB device array built into the
- * library, which every GPU that loads the library holds until the process exits.
+ * memory, so cannot pass a workspace.  One example is a plugin inside a host framework
+ * that owns all device memory through its own allocator and gives the plugin no way to
+ * reserve more.  Another is a latency-bound loop that must not call cudaMalloc, which
+ * can synchronise the whole device.  This entry point allocates nothing: its scratch
+ * is a fixed 64 MiB device array built into the library, which every GPU that loads
+ * the library holds until the process exits.
  * The pages have no counterpart to this entry point.
- *   - Limit: the scratch must hold the value stage's sort and segment buffers, about
- *     60 bytes per selection (N*h*k selections; e.g. up to N = 8192 tokens at h = 4,
- *     k = 32).  Larger problems return PKM_ERR_WORKSPACE before any device work.
+ *   - Limit: the scratch holds the value stage's sort and segment buffers, about 60
+ *     bytes per selection (N*h*k selections; e.g. up to N = 8192 tokens at h = 4,
+ *     k = 32).  A larger problem returns PKM_ERR_WORKSPACE from a host-side check,
+ *     before any CUDA call.
  *   - The first call on a device fetches the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call before
- *     any stream capture begins.
- *   - Every call shares the one array and each call fully rewrites what it reads, so
- *     nothing needs clearing between calls; but calls whose work overlaps on the GPU
- *     (other streams, other host threads) race on the array and must be serialised.
+ *     (cudaGetSymbolAddress) with that device current.  Make that first call before
+ *     any stream capture begins.  A failed lookup is not cached: the next call retries.
+ *   - Every call shares the one array.  Each call clears or fully rewrites the parts
+ *     it reads, so nothing needs clearing between calls.  Calls whose work overlaps on
+ *     the GPU (other streams, other host threads) race on the array and must be
+ *     serialised by the caller.
  *   - Same arguments and results as pkm_value_grad otherwise. */
 pkm_status pkm_value_grad_noalloc(const pkm_dims* d, const void* values, const pkm_saved* saved,
                                   const float* dy, float* dvalues, float* dw, void* stream);

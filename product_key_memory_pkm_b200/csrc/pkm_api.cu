@@ -71,7 +71,10 @@ pkm_status validate_dims(const pkm_dims* d) {
   return PKM_OK;
 }
 
-Plan make_plan(const pkm_dims* d, int dev) {
+// The shape of a call (everything but the device fields).  make_plan, the workspace
+// queries and the fixed-scratch size check all derive their Plan from this one function,
+// so a buffer layout computed on the host matches the one the launches use.
+Plan shape_plan(const pkm_dims* d) {
   Plan p{};
   p.N = d->N;
   p.d_in = d->d_in;
@@ -93,6 +96,11 @@ Plan make_plan(const pkm_dims* d, int dev) {
   p.bn_train = d->flags & PKM_F_BN_TRAIN;
   p.ksel = (d->flags & PKM_F_ALL_K2) ? d->k * d->k : d->k;
   p.idw = d->flags & PKM_F_IDW;
+  return p;
+}
+
+Plan make_plan(const pkm_dims* d, int dev) {
+  Plan p = shape_plan(d);
   p.sm_count = g_sm_count[dev];
   p.status = g_status_ptr[dev];
   return p;
@@ -200,12 +208,7 @@ size_t pkm_workspace_bytes(const pkm_dims* d, int which) {
   if (validate_dims(d) != PKM_OK) return 0;
   if (which == PKM_FWD) return 0;
   if (which != PKM_BWD || d->N == 0) return 0;
-  Plan p{};
-  p.N = d->N; p.d_in = d->d_in; p.h = d->h; p.dk = d->dk; p.half = d->dk / 2;
-  p.C1 = d->C1; p.C2 = d->C2; p.k = d->k; p.d_v = d->d_v; p.hq = d->h * d->dk;
-  p.K = (int64_t)d->C1 * d->C2; p.fp32 = d->flags & PKM_F_FP32;
-  p.vfp32 = p.fp32 || (d->flags & PKM_F_VALUES_FP32);
-  p.ksel = (d->flags & PKM_F_ALL_K2) ? d->k * d->k : d->k;
+  const Plan p = shape_plan(d);
   return backward_workspace_bytes(p);
 }
 
@@ -648,18 +651,24 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-void* g_noalloc_ptr[kMaxDevices];
-cudaError_t g_noalloc_err[kMaxDevices];
-std::once_flag g_noalloc_once[kMaxDevices];
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
 
-// Device address of the scratch on the current device (nullptr after a failure).
+// Device address of the scratch on the current device, or nullptr if the lookup failed.
+// Only a successful lookup is kept: a failed one (say, made while the stream was being
+// captured) is retried by the next call, and its non-sticky error is cleared.
 void* noalloc_scratch(int dev) {
-  std::call_once(g_noalloc_once[dev], [dev]() {
-    void* ptr = nullptr;
-    g_noalloc_err[dev] = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    g_noalloc_ptr[dev] = g_noalloc_err[dev] == cudaSuccess ? ptr : nullptr;
-  });
-  return g_noalloc_ptr[dev];
+  void* ptr = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (ptr) return ptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  ptr = g_noalloc_ptr[dev].load(std::memory_order_relaxed);
+  if (ptr) return ptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  g_noalloc_ptr[dev].store(ptr, std::memory_order_release);
+  return ptr;
 }
 
 }  // namespace
@@ -673,15 +682,9 @@ extern "C" pkm_status pkm_value_grad_noalloc(const pkm_dims* d, const void* valu
   PKM_NEED(values); PKM_NEED(dy); PKM_NEED(dw); PKM_OPT(dvalues);
   if (!saved) return PKM_ERR_INVALID_ARG;
   PKM_NEED(saved->idx); PKM_NEED(saved->w);
-  {
-    // size check on the host, before any device work
-    Plan q{};
-    q.N = d->N; q.d_in = d->d_in; q.h = d->h; q.dk = d->dk; q.half = d->dk / 2;
-    q.C1 = d->C1; q.C2 = d->C2; q.k = d->k; q.d_v = d->d_v; q.hq = d->h * d->dk;
-    q.K = (int64_t)d->C1 * d->C2; q.fp32 = d->flags & PKM_F_FP32;
-    q.ksel = (d->flags & PKM_F_ALL_K2) ? d->k * d->k : d->k;
-    if (value_stage_scratch_bytes(q) > kNoAllocScratchBytes) return PKM_ERR_WORKSPACE;
-  }
+  // size check on the host, before any CUDA call; shape_plan is the plan make_plan
+  // extends, so the layout checked here is the one the launch uses
+  if (value_stage_scratch_bytes(shape_plan(d)) > kNoAllocScratchBytes) return PKM_ERR_WORKSPACE;
   Plan p;
   PKM_TRY(prepare(d, &p));
   int dev = 0;

@@ -7,11 +7,12 @@ compare with the CPU oracle under the agreement rules of the layer:
   such a gap must agree as a set.  Otherwise several sets are correct: every GPU key
   must then score (in the oracle) at least S_k - tol.
 * outputs and gradients: max relative error 2e-3 per row,
-  max_e |got - want| / max(max_e |want|, 1e-3 * max |want over the tensor|, 1e-30).
-  The floor makes rows that cancel to (near) zero analytically compare in absolute
-  terms at the tensor's scale: e.g. a sub-key shared by every winner of a head has a
-  gradient that is exactly zero (the softmax gradient sums to zero), which fp32 leaves
-  as a ~1e-8 residue.
+  max_e |got - want| / max(max_e |want|, 1e-6).
+  Only the sub-key and BatchNorm gradients (dsub, dbn) take a wider floor,
+  1e-3 * max |want over the tensor|, because they have rows that cancel to zero
+  analytically: a sub-key shared by every winner of a head collects the sum of the
+  softmax gradient over the head, which is exactly zero and which fp32 leaves as a
+  ~1e-8 residue.  Every other tensor (y, w, dw, dV, dx, dWq, ...) has no such rows.
 Tokens with a near-tie head (decided from the oracle alone) are left out of the direct
 output comparison and have their upstream gradient masked to zero, so every compared
 value is unique.
@@ -108,19 +109,28 @@ def check_indices(idx_gpu: np.ndarray, of: dict, cfg, ranked: np.ndarray):
     return clean_tok
 
 
-def row_rel_err(got: np.ndarray, want: np.ndarray) -> float:
+ABS_FLOOR = 1e-6
+ZERO_ROW_FLOOR = 1e-3
+
+
+def row_rel_err(got: np.ndarray, want: np.ndarray, zero_rows: bool = False) -> float:
+    """Max over rows of max_e |got - want| / max(max_e |want|, floor).  The floor is
+    ABS_FLOOR, or ZERO_ROW_FLOOR times the tensor's max |want| for a tensor with rows
+    that are analytically zero (``zero_rows``)."""
     if np.asarray(want).size == 0:
         return 0.0
     got = np.asarray(got, dtype=np.float64).reshape(want.shape[0], -1)
     want = np.asarray(want, dtype=np.float64).reshape(want.shape[0], -1)
     err = np.abs(got - want).max(axis=1)
-    floor = max(1e-3 * float(np.abs(want).max()) if want.size else 0.0, 1e-30)
+    floor = ABS_FLOOR
+    if zero_rows:
+        floor = max(floor, ZERO_ROW_FLOOR * float(np.abs(want).max()))
     den = np.maximum(np.abs(want).max(axis=1), floor)
     return float((err / den).max()) if want.shape[0] else 0.0
 
 
-def assert_rows(got, want, name: str, tol: float = ROW_REL):
-    e = row_rel_err(got, want)
+def assert_rows(got, want, name: str, tol: float = ROW_REL, zero_rows: bool = False):
+    e = row_rel_err(got, want, zero_rows=zero_rows)
     assert e <= tol, f"{name}: max row relative error {e:.3e} > {tol}"
     return e
 

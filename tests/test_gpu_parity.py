@@ -68,9 +68,10 @@ def _full_check(cfg, seed=0, flags=0, inp=None, q_bf16=False, bn_train=False, id
     ob = O.backward(inp, cfg, of, dy)
     H.assert_rows(g["dx"].cpu().numpy(), ob["dx"], "dx")
     H.assert_rows(g["dWq"].cpu().numpy(), ob["dWq"], "dWq")
-    H.assert_rows(g["dbn"].cpu().numpy(), np.stack([ob["dgamma"], ob["dbeta"]]), "dbn")
+    H.assert_rows(g["dbn"].cpu().numpy(), np.stack([ob["dgamma"], ob["dbeta"]]), "dbn",
+                  zero_rows=True)
     H.assert_rows(g["dsub"].cpu().numpy().reshape(-1, cfg.dk // 2),
-                  ob["dsub"].reshape(-1, cfg.dk // 2), "dsub")
+                  ob["dsub"].reshape(-1, cfg.dk // 2), "dsub", zero_rows=True)
     dV = g["dV"].cpu().numpy()
     H.assert_rows(dV[ob["dV_rows"]], ob["dV_vals"], "dV")
     untouched = np.ones(cfg.K, dtype=bool)
@@ -287,8 +288,10 @@ def _sampled_full_size(cfg, n_sample, seed=0, backward=True):
     sample = np.sort(rng.choice(cfg.N, size=n_sample, replace=False))
     sample[0], sample[-1] = 0, cfg.N - 1
     sub_inp = dict(inp, x=inp["x"][sample], dy=inp["dy"][sample])
-    of = O.forward(sub_inp, cfg)
-    ranked = H.oracle_gaps(of, cfg)
+    # the product-key search selects exactly what brute force does (pinned on the CPU)
+    # at a fraction of its cost over a million keys per head
+    of = O.forward(sub_inp, cfg, select="product")
+    ranked = H.oracle_gaps(of, cfg, select="product")
     idx = saved["idx"][torch.from_numpy(sample).cuda()].cpu().numpy()
     clean = H.check_indices(idx, of, cfg, ranked)
     yg = y[torch.from_numpy(sample).cuda()].cpu().numpy()
@@ -308,19 +311,20 @@ def _sampled_full_size(cfg, n_sample, seed=0, backward=True):
     assert not torch.any(dx[mask])
     H.assert_rows(g["dWq"].cpu().numpy(), ob["dWq"], "dWq")
     H.assert_rows(g["dsub"].cpu().numpy().reshape(-1, cfg.dk // 2),
-                  ob["dsub"].reshape(-1, cfg.dk // 2), "dsub")
-    H.assert_rows(g["dbn"].cpu().numpy(), np.stack([ob["dgamma"], ob["dbeta"]]), "dbn")
+                  ob["dsub"].reshape(-1, cfg.dk // 2), "dsub", zero_rows=True)
+    H.assert_rows(g["dbn"].cpu().numpy(), np.stack([ob["dgamma"], ob["dbeta"]]), "dbn",
+                  zero_rows=True)
     rows = torch.from_numpy(ob["dV_rows"]).cuda()
     H.assert_rows(g["dV"][rows].cpu().numpy(), ob["dV_vals"], "dV")
     assert int((g["dV"].abs().sum(1) > 0).sum()) <= len(ob["dV_rows"])
 
 
 def test_forward_K512_full_size_sampled():
-    _sampled_full_size(FWD_K512, 48, backward=False)
+    _sampled_full_size(FWD_K512, 256, backward=False)
 
 
 def test_fwd_bwd_K1024_full_size_sampled():
-    _sampled_full_size(FULL_K1024, 24)
+    _sampled_full_size(FULL_K1024, 128)
 
 
 def test_bounded_wait_expires_with_status_and_context_survives():
@@ -400,9 +404,10 @@ def test_all_k2_variant(n):
     ob = O.backward(inp, cfg, of, dy)
     H.assert_rows(g["dx"].cpu().numpy(), ob["dx"], "dx")
     H.assert_rows(g["dWq"].cpu().numpy(), ob["dWq"], "dWq")
-    H.assert_rows(g["dbn"].cpu().numpy(), np.stack([ob["dgamma"], ob["dbeta"]]), "dbn")
+    H.assert_rows(g["dbn"].cpu().numpy(), np.stack([ob["dgamma"], ob["dbeta"]]), "dbn",
+                  zero_rows=True)
     H.assert_rows(g["dsub"].cpu().numpy().reshape(-1, cfg.dk // 2),
-                  ob["dsub"].reshape(-1, cfg.dk // 2), "dsub")
+                  ob["dsub"].reshape(-1, cfg.dk // 2), "dsub", zero_rows=True)
     H.assert_rows(g["dV"].cpu().numpy()[ob["dV_rows"]], ob["dV_vals"], "dV")
     dwg = H.align_to(idx[clean], of["idx"][clean], g["dw"].cpu().numpy()[clean])
     H.assert_rows(dwg.reshape(-1, kk), ob["dw"][clean].reshape(-1, kk), "dw")
