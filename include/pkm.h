@@ -37,7 +37,7 @@
  *     without touching the device.  Device-side problems (a bounded wait that
  *     expired, an out-of-range index) set a status word that pkm_check_status
  *     reports; kernels never trap.
- *   - Limits: 1 <= k <= 32, k <= min(C1, C2), h <= 64, dk/2 <= 1024 (bf16) or 512 (fp32), dk % 32 == 0 (bf16) or dk % 8 == 0
+ *   - Limits: 1 <= k <= 64, k <= min(C1, C2), h <= 64, dk/2 <= 1024 (bf16) or 512 (fp32), dk % 32 == 0 (bf16) or dk % 8 == 0
  *     (fp32), d_in % 8 == 0, d_v % 8 == 0, C1*C2 < 2^31, pointers 16-byte aligned.
  *     N == 0 is a no-op returning PKM_OK.
  */
@@ -54,7 +54,7 @@ extern "C" {
 typedef enum {
   PKM_OK = 0,
   PKM_ERR_INVALID_ARG = 1,     /* null/misaligned pointer, bad size, k > C, ... */
-  PKM_ERR_UNSUPPORTED = 2,     /* legal but outside this build's limits (k > 32, ...) */
+  PKM_ERR_UNSUPPORTED = 2,     /* legal but outside this build's limits (k > 64, ...) */
   PKM_ERR_WORKSPACE = 3,       /* workspace pointer NULL or smaller than pkm_workspace_bytes */
   PKM_ERR_CUDA = 4,            /* a CUDA runtime call failed (launch, attribute, ...) */
   PKM_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait expired */

@@ -17,6 +17,7 @@
 
 #include "k_sort.cuh"
 #include "k_value_rows.cuh"
+#include "k_value_warp.cuh"
 #include "tc_common.cuh"
 
 namespace pkm {
@@ -140,19 +141,23 @@ __global__ void __launch_bounds__(256) softmax_bwd_all_kernel(
   float s = 0.f;
   for (int c = lane; c < kk; c += 32) s = fmaf(wg[c], dg[c], s);
   s = warp_sum(s);
-  if (lane < k) {
+  for (int a = lane; a < k; a += 32) {
     float g1 = 0.f, g2 = 0.f;
     for (int j = 0; j < k; ++j) {
-      const int ca = lane * k + j, cb = j * k + lane;
+      const int ca = a * k + j, cb = j * k + a;
       g1 += scale * wg[ca] * (dg[ca] - s);
       g2 += scale * wg[cb] * (dg[cb] - s);
     }
-    gsub[g * 2 * k + lane] = g1;
-    gsub[g * 2 * k + k + lane] = g2;
+    gsub[g * 2 * k + a] = g1;
+    gsub[g * 2 * k + k + a] = g2;
   }
 }
 
 // ------------------------------------------------------------------ B4
+// One warp per (token, head); lane j holds winners j and j + 32 (R = 2, for k > 32).
+// dS_j = scale w_j (dw_j - sum w dw); the first half's a-th sub-key collects dS_j of the
+// winners that use it (and likewise the second half's b-th), summed in winner order.
+template <int R>
 __global__ void __launch_bounds__(256) softmax_bwd_kernel(
     const float* __restrict__ w, const float* __restrict__ dw, const int32_t* __restrict__ idx,
     const int32_t* __restrict__ sub_i, float* __restrict__ gsub, int64_t NH, int k, int C2,
@@ -160,25 +165,47 @@ __global__ void __launch_bounds__(256) softmax_bwd_kernel(
   const int lane = threadIdx.x & 31;
   const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (g >= NH) return;
-  const bool live = lane < k;
-  const float wj = live ? w[g * k + lane] : 0.f;
-  const float dwj = live ? dw[g * k + lane] : 0.f;
-  const int32_t ij = live ? idx[g * k + lane] : 0;
-  const float s = warp_sum(wj * dwj);
-  const float dsum = scale * wj * (dwj - s);
-  const int32_t ia = live ? sub_i[g * 2 * k + lane] : -1;
-  const int32_t jb = live ? sub_i[g * 2 * k + k + lane] : -1;
-  float g1 = 0.f, g2 = 0.f;
-  for (int j = 0; j < k; ++j) {
-    const int32_t I = __shfl_sync(kFull, ij / C2, j);
-    const int32_t J = __shfl_sync(kFull, ij % C2, j);
-    const float D = __shfl_sync(kFull, dsum, j);
-    if (ia == I) g1 += D;
-    if (jb == J) g2 += D;
+  bool live[R];
+  float wj[R], dwj[R], dsum[R], g1[R], g2[R];
+  int32_t I[R], J[R], ia[R], jb[R];
+  float part = 0.f;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int j = lane + 32 * r;
+    live[r] = j < k;
+    wj[r] = live[r] ? w[g * k + j] : 0.f;
+    dwj[r] = live[r] ? dw[g * k + j] : 0.f;
+    const int32_t ij = live[r] ? idx[g * k + j] : 0;
+    I[r] = ij / C2;
+    J[r] = ij % C2;
+    ia[r] = live[r] ? sub_i[g * 2 * k + j] : -1;
+    jb[r] = live[r] ? sub_i[g * 2 * k + k + j] : -1;
+    part = fmaf(wj[r], dwj[r], part);
+    g1[r] = g2[r] = 0.f;
   }
-  if (live) {
-    gsub[g * 2 * k + lane] = g1;
-    gsub[g * 2 * k + k + lane] = g2;
+  const float s = warp_sum(part);
+#pragma unroll
+  for (int r = 0; r < R; ++r) dsum[r] = scale * wj[r] * (dwj[r] - s);
+#pragma unroll
+  for (int rs = 0; rs < R; ++rs) {  // winners 32 rs ... 32 rs + 31, in order
+    const int n = min(32, k - 32 * rs);
+    for (int j = 0; j < n; ++j) {
+      const int32_t Ij = __shfl_sync(kFull, I[rs], j);
+      const int32_t Jj = __shfl_sync(kFull, J[rs], j);
+      const float D = __shfl_sync(kFull, dsum[rs], j);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        if (ia[r] == Ij) g1[r] += D;
+        if (jb[r] == Jj) g2[r] += D;
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (live[r]) {
+      gsub[g * 2 * k + lane + 32 * r] = g1[r];
+      gsub[g * 2 * k + k + lane + 32 * r] = g2[r];
+    }
   }
 }
 
@@ -525,7 +552,50 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
   e = sort::segments(rows_sorted, E1, seg, U, rb.bsum, st, seg_row, ents_sorted, s.w, w_sorted);
   if (e != cudaSuccess) return e;
 
-  // B3: value rows
+  // B3: value rows, one warp per row (rows up to 2048 columns with two or more slots per
+  // warp in shared memory), else one CTA per row
+  {
+    const int vbytes_el = p.vfp32 ? 4 : 2;
+    const bool dense = dV != nullptr;
+    const size_t slot = vw_slot_bytes(p.d_v, vbytes_el, dense);
+    const size_t avail = 220 * 1024;
+    const int depth = (int)std::min<size_t>(kVwMaxDepth, avail / ((size_t)kVwWarps * slot));
+    const int nv4 = p.d_v / 4;
+    const int maxj = (nv4 + 31) / 32;
+#ifndef PKM_B3_WARP
+#define PKM_B3_WARP 0
+#endif
+    if (PKM_B3_WARP && maxj <= 16 && depth >= 2) {
+      const size_t smem = (size_t)kVwWarps * depth * slot;
+#ifndef PKM_VW_CONTIGUOUS
+#define PKM_VW_CONTIGUOUS 0
+#endif
+#define PKM_VW(TV, MJ)                                                                        \
+  do {                                                                                        \
+    if ((e = cudaFuncSetAttribute(value_warp_kernel<TV, MJ>,                                  \
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != \
+        cudaSuccess)                                                                          \
+      return e;                                                                               \
+    value_warp_kernel<TV, MJ><<<p.sm_count, kVwWarps * 32, smem, st>>>(                       \
+        seg, U, seg_row, ents_sorted, static_cast<const TV*>(values), w_sorted, dy, dV, dw,   \
+        hk, p.d_v, p.K, p.status, dVc, rows_out, U_out, ent_tok, depth, PKM_VW_CONTIGUOUS);   \
+  } while (0)
+#define PKM_VW_J(TV)                 \
+  do {                               \
+    if (maxj <= 2) PKM_VW(TV, 2);    \
+    else if (maxj <= 4) PKM_VW(TV, 4);   \
+    else if (maxj <= 8) PKM_VW(TV, 8);   \
+    else if (maxj <= 13) PKM_VW(TV, 13); \
+    else PKM_VW(TV, 16);             \
+  } while (0)
+      if (p.vfp32) PKM_VW_J(float);
+      else PKM_VW_J(__nv_bfloat16);
+#undef PKM_VW_J
+#undef PKM_VW
+      PKM_COUNT(1);
+      return cudaGetLastError();
+    }
+  }
   {
     const int E = p.vfp32 ? 4 : 8;
     const int nvec = p.d_v / E;
@@ -907,9 +977,14 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
     if (p.ksel != p.k)
       softmax_bwd_all_kernel<<<(unsigned)((NH + 7) / 8), 256, 0, st>>>(s.w, dw, gsub, NH, p.k,
                                                                        p.scale);
+    else if (p.k <= 32)
+      softmax_bwd_kernel<1><<<(unsigned)((NH + 7) / 8), 256, 0, st>>>(s.w, dw, s.idx, s.sub_i,
+                                                                       gsub, NH, p.k, p.C2,
+                                                                       p.scale);
     else
-      softmax_bwd_kernel<<<(unsigned)((NH + 7) / 8), 256, 0, st>>>(s.w, dw, s.idx, s.sub_i, gsub,
-                                                                    NH, p.k, p.C2, p.scale);
+      softmax_bwd_kernel<2><<<(unsigned)((NH + 7) / 8), 256, 0, st>>>(s.w, dw, s.idx, s.sub_i,
+                                                                       gsub, NH, p.k, p.C2,
+                                                                       p.scale);
     PKM_COUNT(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

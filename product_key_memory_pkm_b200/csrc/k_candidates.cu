@@ -4,12 +4,13 @@
 // similar keys; "Meta AI 可扩展内存层" 4.3 and 5.3; value row i*|C'| + j from 4.5).
 //
 // One warp per (token, head).  Lane a holds the a-th best sub-key of the first half
-// and walks its row of candidates (a, 0), (a, 1), ... whose sums s1[a] + s2[b] are
-// non-increasing in b, so each row is a sorted list.  A k-way merge of the k rows
-// takes k steps: each step reduces the heads with one redux.sync max over the
-// order key of the fp32 sum, resolves rare exact ties by s1, then s2, then the flat
-// row index, emits the winner and advances the winning row.  This visits exactly
-// the order (s1+s2 desc, s1 desc, s2 desc, flat asc) over all k*k candidates.
+// (and, for k > 32, the (a+32)-th as its second row) and walks its row of candidates
+// (a, 0), (a, 1), ... whose sums s1[a] + s2[b] are non-increasing in b, so each row is a
+// sorted list.  A k-way merge of the k rows takes k steps: each step reduces the rows'
+// heads with one redux.sync max over the order key of the fp32 sum, resolves rare exact
+// ties by s1, then s2, then the flat row index, emits the winner and advances the
+// winning row.  This visits exactly the order (s1+s2 desc, s1 desc, s2 desc, flat asc)
+// over all k*k candidates.
 #include "pkm_internal.cuh"
 
 namespace pkm {
@@ -17,6 +18,25 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 
+// Among the rows still in the running (in[r]), keep those whose key equals the warp-wide
+// maximum of their keys.  Returns the number of rows left in the warp.
+template <int R>
+__device__ __forceinline__ int keep_max(bool (&in)[R], const uint32_t (&key)[R]) {
+  uint32_t loc = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r) loc = in[r] ? max(loc, key[r]) : loc;
+  const uint32_t m = __reduce_max_sync(kFull, loc);
+  int n = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    in[r] = in[r] && key[r] == m;
+    n += __popc(__ballot_sync(kFull, in[r]));
+  }
+  return n;
+}
+
+// R = rows of the k x k grid per lane (1 for k <= 32, 2 for k <= 64).
+template <int R>
 __global__ void __launch_bounds__(256) candidate_topk_kernel(
     const float* __restrict__ sub_s, const int32_t* __restrict__ sub_i, int32_t* __restrict__ idx,
     float* __restrict__ w_out, int64_t NH, int k, int C2, float scale) {
@@ -27,60 +47,97 @@ __global__ void __launch_bounds__(256) candidate_topk_kernel(
   if (g >= NH) return;  // warp-uniform
   const float* ss = sub_s + g * 2 * k;
   const int32_t* si = sub_i + g * 2 * k;
-  const bool live = lane < k;
-  const float s1 = live ? ss[lane] : -INFINITY;
-  const float s2 = live ? ss[k + lane] : -INFINITY;
-  const int32_t i1 = live ? si[lane] : 0;
-  const int32_t j2 = live ? si[k + lane] : 0;
-
-  int ptr = 0;            // this lane's (row a = lane) next column b
-  float outS = 0.f;       // lane j ends up holding the j-th winner
-  int32_t outIdx = 0;
+  bool live[R];
+  float s1[R], s2[R];
+  int32_t i1[R], j2[R];
+  int ptr[R];  // row (lane + 32 r)'s next column b
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int a = lane + 32 * r;
+    live[r] = a < k;
+    s1[r] = live[r] ? ss[a] : -INFINITY;
+    s2[r] = live[r] ? ss[k + a] : -INFINITY;
+    i1[r] = live[r] ? si[a] : 0;
+    j2[r] = live[r] ? si[k + a] : 0;
+    ptr[r] = 0;
+  }
+  float outS[R];  // lane j, register r ends up holding winner j + 32 r
+  int32_t outIdx[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    outS[r] = 0.f;
+    outIdx[r] = 0;
+  }
   for (int step = 0; step < k; ++step) {
-    const bool valid = live && ptr < k;
-    const int b = valid ? ptr : 0;
-    const float s2b = __shfl_sync(kFull, s2, b);
-    const int32_t j2b = __shfl_sync(kFull, j2, b);
-    const float S = s1 + s2b;
-    const uint32_t key = valid ? order_key(S) : 0u;
-    const uint32_t m = __reduce_max_sync(kFull, key);
-    unsigned cand = __ballot_sync(kFull, valid && key == m);
-    if (__popc(cand) > 1) {  // exact fp32 tie of the sums: s1 desc, s2 desc, flat asc
-      const bool in = (cand >> lane) & 1u;
-      const uint32_t k1 = in ? order_key(s1) : 0u;
-      const uint32_t m1 = __reduce_max_sync(kFull, k1);
-      cand = __ballot_sync(kFull, in && k1 == m1);
-      if (__popc(cand) > 1) {
-        const bool in2 = (cand >> lane) & 1u;
-        const uint32_t k2 = in2 ? order_key(s2b) : 0u;
-        const uint32_t m2 = __reduce_max_sync(kFull, k2);
-        cand = __ballot_sync(kFull, in2 && k2 == m2);
-        if (__popc(cand) > 1) {
-          const bool in3 = (cand >> lane) & 1u;
-          const uint32_t f = in3 ? (uint32_t)(i1 * C2 + j2b) : 0xffffffffu;
-          const uint32_t mf = __reduce_min_sync(kFull, f);
-          cand = __ballot_sync(kFull, in3 && f == mf);
+    bool in[R];
+    float S[R], s2b[R];
+    int32_t flat[R];
+    uint32_t key[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      in[r] = live[r] && ptr[r] < k;
+      const int b = in[r] ? ptr[r] : 0;
+      // s2[b] and j2[b] live in lane b & 31, register b >> 5
+      float x = __shfl_sync(kFull, s2[0], b & 31);
+      int32_t jx = __shfl_sync(kFull, j2[0], b & 31);
+      if (R > 1) {
+        const float x1 = __shfl_sync(kFull, s2[R - 1], b & 31);
+        const int32_t j1 = __shfl_sync(kFull, j2[R - 1], b & 31);
+        if (b >= 32) {
+          x = x1;
+          jx = j1;
         }
       }
+      s2b[r] = x;
+      S[r] = s1[r] + x;
+      flat[r] = i1[r] * C2 + jx;
+      key[r] = in[r] ? order_key(S[r]) : 0u;
     }
-    const int win = __ffs(cand) - 1;
-    const float wS = __shfl_sync(kFull, S, win);
-    const int32_t wIdx = __shfl_sync(kFull, i1 * C2 + j2b, win);
-    if (lane == step) {
-      outS = wS;
-      outIdx = wIdx;
+    if (keep_max<R>(in, key) > 1) {  // exact fp32 tie of the sums: s1 desc, s2 desc, flat asc
+      uint32_t k1[R], k2[R], kf[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        k1[r] = order_key(s1[r]);
+        k2[r] = order_key(s2b[r]);
+        kf[r] = ~(uint32_t)flat[r];  // the smallest flat index has the largest key
+      }
+      if (keep_max<R>(in, k1) > 1 && keep_max<R>(in, k2) > 1) keep_max<R>(in, kf);
     }
-    if (lane == win) ++ptr;
+    // the winner: the one row left (flat indices are distinct)
+    int wr = 0;
+    unsigned bal = __ballot_sync(kFull, in[0]);
+    if (R > 1 && !bal) {
+      wr = R - 1;
+      bal = __ballot_sync(kFull, in[R - 1]);
+    }
+    const int win = __ffs(bal) - 1;
+    const float wS = __shfl_sync(kFull, wr ? S[R - 1] : S[0], win);
+    const int32_t wIdx = __shfl_sync(kFull, wr ? flat[R - 1] : flat[0], win);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (lane + 32 * r == step) {
+        outS[r] = wS;
+        outIdx[r] = wIdx;
+      }
+      if (lane == win && wr == r) ++ptr[r];
+    }
   }
   // softmax over the k winners of scale * S (winner 0 holds the maximum)
-  const float S0 = __shfl_sync(kFull, outS, 0);
-  float e = live ? expf(scale * (outS - S0)) : 0.f;
-  float sum = e;
+  const float S0 = __shfl_sync(kFull, outS[0], 0);
+  float e[R], sum = 0.f;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    e[r] = live[r] ? expf(scale * (outS[r] - S0)) : 0.f;
+    sum += e[r];
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
-  if (live) {
-    idx[g * k + lane] = outIdx;
-    w_out[g * k + lane] = e / sum;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (live[r]) {
+      idx[g * k + lane + 32 * r] = outIdx[r];
+      w_out[g * k + lane + 32 * r] = e[r] / sum;
+    }
   }
 }
 
@@ -130,8 +187,13 @@ cudaError_t launch_candidates(const Plan& p, const float* sub_s, const int32_t* 
     PKM_COUNT(1);
     return e;
   }
-  cudaError_t e = launch_dependent(candidate_topk_kernel, dim3((unsigned)blocks), dim3(warps * 32),
-                                   0, st, sub_s, sub_i, idx, w, NH, p.k, p.C2, p.scale);
+  cudaError_t e =
+      p.k <= 32 ? launch_dependent(candidate_topk_kernel<1>, dim3((unsigned)blocks),
+                                   dim3(warps * 32), 0, st, sub_s, sub_i, idx, w, NH, p.k, p.C2,
+                                   p.scale)
+                : launch_dependent(candidate_topk_kernel<2>, dim3((unsigned)blocks),
+                                   dim3(warps * 32), 0, st, sub_s, sub_i, idx, w, NH, p.k, p.C2,
+                                   p.scale);
   PKM_COUNT(1);
   return e;
 }

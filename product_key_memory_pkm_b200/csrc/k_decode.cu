@@ -301,7 +301,8 @@ size_t scores_small_smem(const Plan& p, int KM) {
 bool small_n_supported(const Plan& p) {
   return !p.fp32 && p.N <= kSmallTokens && p.d_in % 8 == 0 && (p.dk / 2) % 8 == 0 &&
          (std::max(p.C1, p.C2) + kSplit - 1) / kSplit <= kMaxSlice &&
-         (size_t)kTokGroup * p.d_in * 2 <= 160 * 1024 && scores_small_smem(p, 32) <= 200 * 1024;
+         (size_t)kTokGroup * p.d_in * 2 <= 160 * 1024 &&
+         scores_small_smem(p, p.k <= 32 ? 32 : 64) <= 200 * 1024;
 }
 
 cudaError_t launch_query_small(const Plan& p, const void* x, const void* Wq, const float* bn,
@@ -344,8 +345,10 @@ cudaError_t launch_scores_small(const Plan& p, const void* subkeys, const void* 
     PKM_SS(8);
   else if (p.k <= 16)
     PKM_SS(16);
-  else
+  else if (p.k <= 32)
     PKM_SS(32);
+  else
+    PKM_SS(64);
 #undef PKM_SS
   PKM_COUNT(1);
   return cudaGetLastError();

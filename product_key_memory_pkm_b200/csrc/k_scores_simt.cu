@@ -14,6 +14,9 @@ namespace pkm {
 namespace {
 
 constexpr int TT = 64, TC = 64, BK = 16, TPB = 256;
+constexpr int kQsBytes = BK * (TT + 4) * 4, kCsBytes = BK * (TC + 4) * 4;
+constexpr int kTileBytes = kQsBytes + kCsBytes + TT * (TC + 1) * 4;
+constexpr int simt_smem_bytes(int KM) { return kTileBytes + KM * TT * 8; }
 
 // lo_scale = 0 drops the lo plane: q rounded to bf16 (single-pass scoring)
 template <bool kSplitQ>
@@ -38,11 +41,13 @@ __global__ void __launch_bounds__(TPB) scores_topk_simt(const void* __restrict__
                                                         int32_t* __restrict__ sub_i, int64_t N,
                                                         int h, int dk, int C1, int C2, int k,
                                                         float lo_scale) {
-  __shared__ __align__(16) float Qs[BK][TT + 4];
-  __shared__ __align__(16) float Cs[BK][TC + 4];
-  __shared__ float Ssc[TT][TC + 1];
-  __shared__ float Ls[KM][TT];
-  __shared__ int Li[KM][TT];
+  // shared memory (dynamic: 25 KB of tiles plus KM * 512 bytes of lists)
+  extern __shared__ __align__(16) unsigned char simt_smem[];
+  auto& Qs = *reinterpret_cast<float(*)[BK][TT + 4]>(simt_smem);
+  auto& Cs = *reinterpret_cast<float(*)[BK][TC + 4]>(simt_smem + kQsBytes);
+  auto& Ssc = *reinterpret_cast<float(*)[TT][TC + 1]>(simt_smem + kQsBytes + kCsBytes);
+  auto& Ls = *reinterpret_cast<float(*)[KM][TT]>(simt_smem + kTileBytes);
+  auto& Li = *reinterpret_cast<int(*)[KM][TT]>(simt_smem + kTileBytes + KM * TT * 4);
 
   const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
   const int64_t t0 = (int64_t)blockIdx.x * TT;
@@ -145,15 +150,26 @@ cudaError_t dispatch_km(const Plan& p, const void* subkeys, const void* q, float
                         int32_t* sub_i, cudaStream_t st) {
   dim3 grid((unsigned)((p.N + TT - 1) / TT), (unsigned)(p.h * 2));
   const TS* sub = static_cast<const TS*>(subkeys);
+  cudaError_t e = cudaSuccess;
 #define PKM_LAUNCH(KMV)                                                                      \
-  scores_topk_simt<kSplitQ, TS, KMV, kIdw><<<grid, TPB, 0, st>>>(                          \
-      q, sub, sub_s, sub_i, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.bf16q ? 0.f : 1.f)
+  do {                                                                                       \
+    constexpr int smem = simt_smem_bytes(KMV);                                               \
+    if (smem > 48 * 1024 &&                                                                  \
+        (e = cudaFuncSetAttribute(scores_topk_simt<kSplitQ, TS, KMV, kIdw>,                  \
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=     \
+            cudaSuccess)                                                                     \
+      return e;                                                                              \
+    scores_topk_simt<kSplitQ, TS, KMV, kIdw><<<grid, TPB, smem, st>>>(                       \
+        q, sub, sub_s, sub_i, p.N, p.h, p.dk, p.C1, p.C2, p.k, p.bf16q ? 0.f : 1.f);         \
+  } while (0)
   if (p.k <= 8)
     PKM_LAUNCH(8);
   else if (p.k <= 16)
     PKM_LAUNCH(16);
-  else
+  else if (p.k <= 32)
     PKM_LAUNCH(32);
+  else
+    PKM_LAUNCH(64);
 #undef PKM_LAUNCH
   PKM_COUNT(1);
   return cudaGetLastError();

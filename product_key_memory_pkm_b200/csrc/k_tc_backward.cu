@@ -80,7 +80,7 @@ struct DxProb {
       if (n0 >= P.d_in) break;  // warp-uniform
       uint32_t r[32];
       tmem_ld32(taddr + (uint32_t)(piece * 32), r);
-      tmem_wait_ld();
+      tmem_wait_ld(r);
       if (t < P.N) store_piece(P.dx + t * P.d_in + n0, n0, P.d_in, r, false);
     }
   }
@@ -126,7 +126,7 @@ struct DwqProb {
       if (n0 >= P.d_in) break;  // warp-uniform
       uint32_t r[32];
       tmem_ld32(taddr + (uint32_t)(piece * 32), r);
-      tmem_wait_ld();
+      tmem_wait_ld(r);
       if (o < P.hq) store_piece(P.dWq + (int64_t)o * P.d_in + n0, n0, P.d_in, r, true);
     }
   }

@@ -120,7 +120,7 @@ struct QueryProb {
       if (n0 >= hq) break;  // warp-uniform
       uint32_t r[32];
       tmem_ld32(taddr + (uint32_t)(piece * 32), r);
-      tmem_wait_ld();
+      tmem_wait_ld(r);
       if (t >= P.N) continue;
       uint32_t hi2[16], lo2[16];
       float qh[32];
@@ -292,7 +292,7 @@ struct ScoresProb {
       if (col0 >= C) break;  // warp-uniform
       uint32_t r[32];
       tmem_ld32(taddr + (uint32_t)(piece * 32), r);
-      tmem_wait_ld();
+      tmem_wait_ld(r);
       int first = 0;
       if (es.root_leaf < 0) {  // first piece of the unit (uniform across the warp)
         build(ts, tp, row, r, col0, C, es);

@@ -29,7 +29,8 @@ constexpr int kBnTokens = 64;        // tokens per BatchNorm-backward block (par
 
 // ------------------------------------------------------------------ dense G planes
 // One warp per (padded token t, head-half hs): zero the row in both planes, then
-// write the k selected entries (distinct within a half, so no accumulation).
+// write the k selected entries (distinct within a half, so no accumulation; lanes
+// stride over them for k > 32).
 __global__ void __launch_bounds__(256) g_dense_kernel(const float* __restrict__ gsub,
                                                       const int32_t* __restrict__ sub_i,
                                                       __nv_bfloat16* __restrict__ G, int64_t N,
@@ -48,14 +49,16 @@ __global__ void __launch_bounds__(256) g_dense_kernel(const float* __restrict__ 
     reinterpret_cast<uint4*>(lo)[c] = z;
   }
   __syncwarp();
-  if (t < N && lane < k) {
+  if (t < N) {
     const int hh = hs >> 1, s = hs & 1;
-    const int64_t o = ((t * h + hh) * 2 + s) * k + lane;
-    const float g = gsub[o];
-    const int32_t i = sub_i[o];
-    const __nv_bfloat16 gh = __float2bfloat16_rn(g);
-    hi[i] = gh;
-    lo[i] = __float2bfloat16_rn(g - __bfloat162float(gh));
+    for (int j = lane; j < k; j += 32) {
+      const int64_t o = ((t * h + hh) * 2 + s) * k + j;
+      const float g = gsub[o];
+      const int32_t i = sub_i[o];
+      const __nv_bfloat16 gh = __float2bfloat16_rn(g);
+      hi[i] = gh;
+      lo[i] = __float2bfloat16_rn(g - __bfloat162float(gh));
+    }
   }
 }
 
@@ -122,7 +125,7 @@ struct DqProb {
       if (n0 >= P.half) break;  // warp-uniform
       uint32_t r[32];
       tmem_ld32(taddr + (uint32_t)(piece * 32), r);
-      tmem_wait_ld();
+      tmem_wait_ld(r);
       if (t < P.N) store_piece(P.dqf + t * P.hq + hh * P.dk + s * P.half + n0, n0, P.half, r);
     }
   }
@@ -192,7 +195,7 @@ struct DsubProb {
       if (n0 >= P.half) break;  // warp-uniform
       uint32_t r[32];
       tmem_ld32(taddr + (uint32_t)(piece * 32), r);
-      tmem_wait_ld();
+      tmem_wait_ld(r);
       if (c < C)
         store_piece(P.part + (((int64_t)sp * 2 * P.h + hs) * P.Cp + c) * P.half + n0, n0, P.half,
                     r);

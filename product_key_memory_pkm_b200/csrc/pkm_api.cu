@@ -62,7 +62,7 @@ pkm_status validate_dims(const pkm_dims* d) {
   if (d->dk % 2) return PKM_ERR_INVALID_ARG;
   if (d->d_in % 8 || d->d_v % 8) return PKM_ERR_INVALID_ARG;
   if (fp32 ? (d->dk % 8) : (d->dk % 32)) return PKM_ERR_INVALID_ARG;
-  if (d->k > 32 || d->h > 64) return PKM_ERR_UNSUPPORTED;
+  if (d->k > 64 || d->h > 64) return PKM_ERR_UNSUPPORTED;
   const int half = d->dk / 2;
   if (fp32 ? (half / 4 > 128) : (half / 8 > 128)) return PKM_ERR_UNSUPPORTED;
   const int64_t ksel = (d->flags & PKM_F_ALL_K2) ? (int64_t)d->k * d->k : d->k;
@@ -152,7 +152,8 @@ cudaError_t run_query(const Plan& p, const void* x, const void* Wq, const float*
 cudaError_t run_scores(const Plan& p, const void* subkeys, const void* q, float* sub_s,
                        int32_t* sub_i, cudaStream_t st) {
   if (small_n_supported(p)) return launch_scores_small(p, subkeys, q, sub_s, sub_i, st);
-  if (tc_forward_supported(p) && !p.idw) return launch_scores_tc(p, subkeys, q, sub_s, sub_i, st);
+  if (tc_forward_supported(p) && !p.idw && p.k <= kScoresTcMaxK)
+    return launch_scores_tc(p, subkeys, q, sub_s, sub_i, st);
   return launch_scores_simt(p, subkeys, q, sub_s, sub_i, st);
 }
 

@@ -96,7 +96,9 @@ cudaError_t launch_query_simt(const Plan& p, const void* x, const void* Wq, cons
                               void* q, float* qhat, cudaStream_t st);
 cudaError_t launch_scores_simt(const Plan& p, const void* subkeys, const void* q, float* sub_s,
                                int32_t* sub_i, cudaStream_t st);
-// tcgen05 forward GEMMs (bf16 storage, dk/2 % 64 == 0)
+// tcgen05 forward GEMMs (bf16 storage, dk/2 % 64 == 0); the tensor-core scorer keeps
+// at most kScoresTcMaxK keys per token and half (larger k runs on CUDA cores)
+constexpr int kScoresTcMaxK = 32;
 bool tc_forward_supported(const Plan& p);
 cudaError_t launch_query_tc(const Plan& p, const void* x, const void* Wq, const float* bn,
                             void* q, float* qhat, cudaStream_t st);

@@ -81,7 +81,7 @@ def _fwd(d, **over):
 
 
 @pytest.mark.parametrize("over,code", [
-    (dict(k=33, C1=64, C2=64), P.PKM_ERR_UNSUPPORTED),
+    (dict(k=65, C1=80, C2=80), P.PKM_ERR_UNSUPPORTED),
     (dict(k=9, C1=8), P.PKM_ERR_INVALID_ARG),
     (dict(dk=48), P.PKM_ERR_INVALID_ARG),            # bf16 needs dk % 32 == 0
     (dict(d_in=60), P.PKM_ERR_INVALID_ARG),
@@ -95,6 +95,17 @@ def _fwd(d, **over):
 ])
 def test_forward_rejects_bad_dims(lib, over, code):
     assert _fwd(_dims(**over)) == code
+
+
+def test_k_up_to_64_passes_validation(lib):
+    """k from 33 to 64 is within the boundary's limits (the host-side size queries
+    accept it); k = 65 is outside them."""
+    for k in (33, 48, 64):
+        d = _dims(k=k, C1=64, C2=80)
+        assert P.pkm_saved_bytes(d, "idx") == 4 * 64 * 2 * k
+        assert P.pkm_saved_bytes(d, "sub_s") == 4 * 64 * 2 * 2 * k
+        assert P.pkm_workspace_bytes(d, P.PKM_BWD) > 0
+    assert P.pkm_saved_bytes(_dims(k=65, C1=80, C2=80), "idx") == 0
 
 
 def test_forward_rejects_null_and_misaligned_pointers(lib):

@@ -41,6 +41,11 @@ CASES = {
     "few_tokens_k32_small_C": _cfg(N=16, h=3, k=32, C1=40, C2=33, d_v=72),
     "split_bag_37_tokens": _cfg(N=37, h=2, dk=64, C1=96, C2=40, k=8),
     "two_tokens_k16": _cfg(N=2, h=3, dk=64, C1=96, C2=40, k=16),
+    # k above 32: two candidate rows per lane, 64-key scoring lists
+    "k48": _cfg(N=150, h=2, C1=96, C2=72, k=48),
+    "k64": _cfg(N=150, h=2, C1=128, C2=64, k=64, d_v=136),
+    "k64_fp32": _cfg(name="k64f", N=90, h=2, dtype="f32", dk=40, C1=80, C2=64, k=64),
+    "few_tokens_k64": _cfg(N=5, h=2, dk=64, C1=96, C2=70, k=64),
 }
 
 
@@ -151,10 +156,11 @@ def test_training_mode_batch_norm(case):
     H.assert_rows(bn.cpu().numpy(), want, "running statistics")
 
 
-def test_stagewise_scores_given_oracle_query():
+@pytest.mark.parametrize("k", [16, 32, 48, 64])
+def test_stagewise_scores_given_oracle_query(k):
     """F2 alone: fed the oracle's q (as its hi/lo split), the per-half lists match the
     oracle's per-half top-k computed from the same q."""
-    cfg = _cfg(N=257)
+    cfg = _cfg(N=257, C1=96, C2=72, k=k)
     inp = make_inputs(cfg, seed=3, random_bn=True)
     of = O.forward(inp, cfg)
     q32 = torch.from_numpy(of["q"].astype(np.float32))
@@ -181,10 +187,11 @@ def test_stagewise_scores_given_oracle_query():
                                            atol=1e-5)
 
 
-def test_stagewise_candidates_given_oracle_lists():
+@pytest.mark.parametrize("k", [32, 48, 64])
+def test_stagewise_candidates_given_oracle_lists(k):
     """F3 alone: fed per-half lists (fp32), the winners and weights match the oracle's
     product-key combine of the same lists."""
-    cfg = _cfg(N=500, k=32, C1=64, C2=64)
+    cfg = _cfg(N=500 if k == 32 else 200, k=k, C1=80, C2=64)
     rng = np.random.default_rng(5)
     N, h, k = cfg.N, cfg.h, cfg.k
     s1 = rng.standard_normal((N, h, cfg.C1)).astype(np.float32)
