@@ -6,8 +6,8 @@
 // F2 pkm_subkey_scores: for each (128-token block, head, half) the scores
 //   s[c] = q_half . C_half[c] over all c, as hi and lo K-blocks accumulated into one
 //   fp32 accumulator (q_hi C + q_lo C), 256 sub-keys per chunk.  The epilogue keeps a
-//   running top-k per token in a shared-memory min-heap (root = worst kept key by
-//   (score desc, index asc)); sub-keys arrive in increasing index order, so a
+//   running top-k per token in a shared-memory tournament tree (root = worst kept key
+//   by (score desc, index asc)); sub-keys arrive in increasing index order, so a
 //   strict '>' against the root keeps equal scores in index order.  Scores never
 //   reach HBM.  ("Large Memory Layers with Product Keys", method details: q split
 //   in two, each half searched in its own sub-key set; "Meta AI 可扩展内存层" 4.3-4.4.)
@@ -160,19 +160,30 @@ struct QueryProb {
 
 // ================================================================== F2 sub-key scores
 // Per-token running top-KM over one half's sub-keys, one epilogue thread per token.
-// The kept keys live in a tournament tree in shared memory: KM leaves hold (score,
-// key) and every node holds the worst key of its subtree, so the root is the current
-// threshold and names the leaf to replace.  A key is packed as (sub-key index << 5 |
-// leaf), so comparing packed keys compares sub-key indices (lower index ranks higher
-// at equal score).  Replacing a leaf rewrites its path to the root; the siblings on
-// that path are known before any comparison, so their loads issue together.
+// The kept keys live in a tournament tree in shared memory: KM leaves and, in every
+// internal node, the worst key of its subtree, so the root is the current threshold and
+// names the leaf to replace.  A key is one 64-bit word ordered like the ranking: the
+// high half is the order key of the score, the low half (kColMask - sub-key index) << 5
+// | leaf, so a larger word ranks higher (higher score, then lower index) and the root
+// word carries its leaf.  Sub-keys arrive in increasing index order, so a new score
+// equal to the threshold ranks below every kept key and a strict '>' test is exact.
+//
+// Per 32-column piece each thread marks the columns above its threshold; the warp then
+// runs a uniform loop whose trip count is the largest number of marked columns of any
+// lane.  Every iteration takes the lane's next marked column (its score staged in shared
+// memory and fetched one iteration ahead) and, if it still beats the threshold,
+// replaces the root's leaf: the siblings along the leaf-to-root path are loaded together
+// and the path is rewritten with running minima.  Lanes without a candidate in an
+// iteration do the same work with their stores predicated off, so the loop never
+// diverges.
 template <int KM>
 struct ScoresProb {
   static constexpr int kAMN = 0, kBMN = 0;
   static constexpr int kStages = 3;
   static constexpr int kLog = KM == 32 ? 5 : (KM == 16 ? 4 : 3);
   static constexpr int kNodes = 2 * KM;  // nodes 1 .. 2*KM-1; leaves KM .. 2*KM-1
-  // tree: kNodes (score, packed) per row; staging: one 32-column piece per row
+  static constexpr uint32_t kColMask = (1u << 27) - 1u;
+  // tree: kNodes 64-bit keys per row; staging: one 32-column piece per row
   static constexpr int kEpiSmem = kNodes * kBM * 8 + 32 * kBM * 4;
   struct Params {
     int* status;
@@ -183,8 +194,9 @@ struct ScoresProb {
     int planes;  // 2: q_hi and q_lo K-blocks; 1: q_hi only (q rounded to bf16)
   };
   struct EpiState {
-    float thr;
-    int root_leaf;
+    uint64_t root;  // worst kept key
+    float thr;      // its score (-inf while a leaf is still empty)
+    bool built;
   };
 
   __device__ static int num_units(const Params& P) { return P.m_tiles * P.h * 2; }
@@ -205,87 +217,53 @@ struct ScoresProb {
     tma_load_2d(sb, B, kk * kBK, hh * (P.C1 + P.C2) + s * P.C1 + c * kBN, bar);
   }
 
-  __device__ static float* ts_(unsigned char* sm) { return reinterpret_cast<float*>(sm); }
-  __device__ static int* tp_(unsigned char* sm) {
-    return reinterpret_cast<int*>(sm + kNodes * kBM * 4);
-  }
+  __device__ static uint64_t* tree_(unsigned char* sm) { return reinterpret_cast<uint64_t*>(sm); }
   __device__ static float* stage_(unsigned char* sm) {
     return reinterpret_cast<float*>(sm + kNodes * kBM * 8);
   }
 
-  // a ranks below b in (score desc, sub-key index asc)
-  __device__ static bool worse(float sa, int pa, float sb, int pb) {
-    return sa < sb || (sa == sb && pa > pb);
+  __device__ static uint64_t make_key(float v, int col, int leaf) {
+    return ((uint64_t)order_key(v) << 32) | (((kColMask - (uint32_t)col) << 5) | (uint32_t)leaf);
   }
+  // an empty leaf: below every real key (the order key of any score is nonzero)
+  __device__ static uint64_t empty_key(int leaf) { return (uint64_t)(uint32_t)leaf; }
+  __device__ static float key_score(uint64_t key) {
+    const uint32_t b = (uint32_t)(key >> 32);
+    if (b == 0u) return -INFINITY;
+    return __uint_as_float((b & 0x80000000u) ? (b & 0x7fffffffu) : ~b);
+  }
+  __device__ static int key_col(uint64_t key) {
+    return (int)(kColMask - (((uint32_t)key >> 5) & kColMask));
+  }
+  __device__ static uint64_t kmin(uint64_t a, uint64_t b) { return a < b ? a : b; }
 
   __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState& es) {
+    es.root = 0;
     es.thr = -INFINITY;
-    es.root_leaf = -1;  // tree not built yet
+    es.built = false;
   }
 
   // Build the tree from the first KM columns held in registers (columns col0 + j).
-  __device__ static void build(float* ts, int* tp, int row, const uint32_t (&r)[32], int col0,
-                               int C, EpiState& es) {
-    float s[kNodes];
-    int p[kNodes];
+  __device__ static void build(uint64_t* tr, int row, const uint32_t (&r)[32], int col0, int C,
+                               EpiState& es) {
+    uint64_t nd[kNodes];
 #pragma unroll
-    for (int j = 0; j < KM; ++j) {
-      const bool ok = col0 + j < C;
-      s[KM + j] = ok ? __uint_as_float(r[j]) : -INFINITY;
-      p[KM + j] = ((ok ? col0 + j : 0x3FFFFFF) << 5) | j;
-    }
+    for (int j = 0; j < KM; ++j)
+      nd[KM + j] = col0 + j < C ? make_key(__uint_as_float(r[j]), col0 + j, j) : empty_key(j);
 #pragma unroll
-    for (int n = KM - 1; n >= 1; --n) {
-      const bool rw = worse(s[2 * n + 1], p[2 * n + 1], s[2 * n], p[2 * n]);
-      s[n] = rw ? s[2 * n + 1] : s[2 * n];
-      p[n] = rw ? p[2 * n + 1] : p[2 * n];
-    }
+    for (int n = KM - 1; n >= 1; --n) nd[n] = kmin(nd[2 * n], nd[2 * n + 1]);
 #pragma unroll
-    for (int n = 1; n < kNodes; ++n) {
-      ts[n * kBM + row] = s[n];
-      tp[n * kBM + row] = p[n];
-    }
-    es.thr = s[1];
-    es.root_leaf = p[1] & 31;
-  }
-
-  // Replace the worst kept key (the root's leaf) with (v, col).
-  __device__ static void replace_root(float* ts, int* tp, int row, float v, int col,
-                                      EpiState& es) {
-    const int leaf = es.root_leaf;
-    int node = KM + leaf;
-    float sib_s[kLog];
-    int sib_p[kLog];
-#pragma unroll
-    for (int l = 0; l < kLog; ++l) {  // siblings along the fixed path, loaded together
-      const int sib = (node >> l) ^ 1;
-      sib_s[l] = ts[sib * kBM + row];
-      sib_p[l] = tp[sib * kBM + row];
-    }
-    float cs = v;
-    int cp = (col << 5) | leaf;
-    ts[node * kBM + row] = cs;
-    tp[node * kBM + row] = cp;
-#pragma unroll
-    for (int l = 0; l < kLog; ++l) {
-      if (worse(sib_s[l], sib_p[l], cs, cp)) {
-        cs = sib_s[l];
-        cp = sib_p[l];
-      }
-      node >>= 1;
-      ts[node * kBM + row] = cs;
-      tp[node * kBM + row] = cp;
-    }
-    es.thr = cs;
-    es.root_leaf = cp & 31;
+    for (int n = 1; n < kNodes; ++n) tr[n * kBM + row] = nd[n];
+    es.root = nd[1];
+    es.thr = key_score(nd[1]);
+    es.built = true;
   }
 
   __device__ static void epi_chunk(const Params& P, int u, int c, int row, uint32_t taddr,
                                    unsigned char* sm, EpiState& es) {
     const int hs_idx = u / P.m_tiles;
     const int C = (hs_idx & 1) ? P.C2 : P.C1;
-    float* ts = ts_(sm);
-    int* tp = tp_(sm);
+    uint64_t* tr = tree_(sm);
     float* stg = stage_(sm);
     for (int piece = 0; piece < kBN / 32; ++piece) {
       const int col0 = c * kBN + piece * 32;
@@ -293,25 +271,48 @@ struct ScoresProb {
       uint32_t r[32];
       tmem_ld32(taddr + (uint32_t)(piece * 32), r);
       tmem_wait_ld(r);
-      int first = 0;
-      if (es.root_leaf < 0) {  // first piece of the unit (uniform across the warp)
-        build(ts, tp, row, r, col0, C, es);
-        first = KM;
+      uint32_t skip = 0u;  // columns already placed by the build
+      if (!es.built) {     // first piece of the unit (uniform across the warp)
+        build(tr, row, r, col0, C, es);
+        skip = KM >= 32 ? 0xffffffffu : ((1u << KM) - 1u);
       }
       // candidates of this piece against the threshold at its start
       uint32_t mask = 0;
 #pragma unroll
       for (int j = 0; j < 32; ++j) mask |= (__uint_as_float(r[j]) > es.thr ? 1u : 0u) << j;
-      if (first) mask &= first >= 32 ? 0u : ~((1u << first) - 1u);
+      mask &= ~skip;
       if (C - col0 < 32) mask &= (1u << (C - col0)) - 1u;
+      const int trips = __reduce_max_sync(0xffffffffu, __popc(mask));
+      if (trips == 0) continue;  // warp-uniform
       if (mask) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) stg[j * kBM + row] = __uint_as_float(r[j]);
-        while (mask) {
-          const int j = __ffs(mask) - 1;
-          mask &= mask - 1u;
-          const float v = stg[j * kBM + row];
-          if (v > es.thr) replace_root(ts, tp, row, v, col0 + j, es);
+      }
+      int j = mask ? __ffs(mask) - 1 : 0;
+      float v = mask ? stg[j * kBM + row] : -INFINITY;
+      for (int it = 0; it < trips; ++it) {
+        // this iteration's candidate (v, j); fetch the next one early
+        const int jc = j;
+        const float vc = v;
+        mask &= mask - 1u;
+        j = mask ? __ffs(mask) - 1 : 0;
+        v = mask ? stg[j * kBM + row] : -INFINITY;
+        const bool act = vc > es.thr;
+        const int leaf = (int)((uint32_t)es.root & (uint32_t)(KM - 1));
+        const int node0 = KM + leaf;
+        uint64_t sib[kLog];
+#pragma unroll
+        for (int l = 0; l < kLog; ++l) sib[l] = tr[(((node0 >> l) ^ 1)) * kBM + row];
+        uint64_t cur = make_key(vc, col0 + jc, leaf);
+        if (act) tr[node0 * kBM + row] = cur;
+#pragma unroll
+        for (int l = 0; l < kLog; ++l) {
+          cur = kmin(cur, sib[l]);
+          if (act) tr[(node0 >> (l + 1)) * kBM + row] = cur;
+        }
+        if (act) {
+          es.root = cur;
+          es.thr = key_score(cur);
         }
       }
     }
@@ -322,45 +323,46 @@ struct ScoresProb {
     const int hh = hs_idx >> 1, s = hs_idx & 1;
     const int64_t t = (int64_t)mt * kBM + row;
     if (t >= P.N) return;
-    const float* ts = ts_(sm);
-    const int* tp = tp_(sm);
-    float v[KM];
-    int q[KM];
+    const uint64_t* tr = tree_(sm);
+    uint64_t key[KM];
 #pragma unroll
-    for (int j = 0; j < KM; ++j) {
-      v[j] = ts[(KM + j) * kBM + row];
-      q[j] = tp[(KM + j) * kBM + row] >> 5;
-    }
-    // bitonic sort, best first: (score desc, index asc)
+    for (int j = 0; j < KM; ++j) key[j] = tr[(KM + j) * kBM + row];
+    // bitonic sort, best (largest key) first
 #pragma unroll
     for (int size = 2; size <= KM; size <<= 1) {
 #pragma unroll
       for (int stride = size >> 1; stride > 0; stride >>= 1) {
 #pragma unroll
         for (int i = 0; i < KM; ++i) {
-          const int j = i ^ stride;
-          if (j > i) {
+          const int jx = i ^ stride;
+          if (jx > i) {
             const bool desc = (i & size) == 0;
-            // in a "desc" run the better key goes first
-            const bool jbetter = worse(v[i], q[i], v[j], q[j]);
-            if (jbetter == desc) {
-              const float tv = v[i];
-              v[i] = v[j];
-              v[j] = tv;
-              const int tq = q[i];
-              q[i] = q[j];
-              q[j] = tq;
-            }
+            const uint64_t a = key[i], b = key[jx];
+            const bool swap = desc ? (a < b) : (a > b);
+            key[i] = swap ? b : a;
+            key[jx] = swap ? a : b;
           }
         }
       }
     }
     const int64_t o = ((t * P.h + hh) * 2 + s) * P.k;
+    if ((P.k & 3) == 0 && P.k == KM) {  // whole list, 16-byte stores
 #pragma unroll
-    for (int j = 0; j < KM; ++j) {
-      if (j < P.k) {
-        P.sub_s[o + j] = v[j];
-        P.sub_i[o + j] = q[j];
+      for (int j = 0; j < KM; j += 4) {
+        *reinterpret_cast<float4*>(P.sub_s + o + j) =
+            make_float4(key_score(key[j]), key_score(key[j + 1]), key_score(key[j + 2]),
+                        key_score(key[j + 3]));
+        *reinterpret_cast<int4*>(P.sub_i + o + j) =
+            make_int4(key_col(key[j]), key_col(key[j + 1]), key_col(key[j + 2]),
+                      key_col(key[j + 3]));
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < KM; ++j) {
+        if (j < P.k) {
+          P.sub_s[o + j] = key_score(key[j]);
+          P.sub_i[o + j] = key_col(key[j]);
+        }
       }
     }
   }

@@ -191,7 +191,7 @@ def test_stagewise_scores_given_oracle_query(k):
 def test_stagewise_candidates_given_oracle_lists(k):
     """F3 alone: fed per-half lists (fp32), the winners and weights match the oracle's
     product-key combine of the same lists."""
-    cfg = _cfg(N=500 if k == 32 else 200, k=k, C1=80, C2=64)
+    cfg = _cfg(N=500 if k == 32 else 200, k=k, C1=80, C2=72)   # k + 1 <= C for the gaps
     rng = np.random.default_rng(5)
     N, h, k = cfg.N, cfg.h, cfg.k
     s1 = rng.standard_normal((N, h, cfg.C1)).astype(np.float32)
