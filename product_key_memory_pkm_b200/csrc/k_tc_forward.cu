@@ -170,8 +170,8 @@ struct QueryProb {
 //
 // Per 32-column piece each thread marks the columns above its threshold; the warp then
 // runs a uniform loop whose trip count is the largest number of marked columns of any
-// lane.  Every iteration takes the lane's next marked column (its score staged in shared
-// memory and fetched one iteration ahead) and, if it still beats the threshold,
+// lane.  Every iteration takes the lane's next marked column (its score picked from the
+// piece's registers one iteration ahead) and, if it still beats the threshold,
 // replaces the root's leaf: the siblings along the leaf-to-root path are loaded together
 // and the path is rewritten with running minima.  Lanes without a candidate in an
 // iteration do the same work with their stores predicated off, so the loop never
@@ -179,12 +179,15 @@ struct QueryProb {
 template <int KM>
 struct ScoresProb {
   static constexpr int kAMN = 0, kBMN = 0;
-  static constexpr int kStages = 3;
+  // two epilogue sets (two units in flight, two epilogue warps per SM sub-partition);
+  // their trees leave room for two operand stages
+  static constexpr int kSets = 2;
+  static constexpr int kStages = 2;
   static constexpr int kLog = KM == 32 ? 5 : (KM == 16 ? 4 : 3);
   static constexpr int kNodes = 2 * KM;  // nodes 1 .. 2*KM-1; leaves KM .. 2*KM-1
   static constexpr uint32_t kColMask = (1u << 27) - 1u;
-  // tree: kNodes 64-bit keys per row; staging: one 32-column piece per row
-  static constexpr int kEpiSmem = kNodes * kBM * 8 + 32 * kBM * 4;
+  // tree: kNodes 64-bit keys per row (node 0 is a dump for predicated-off stores)
+  static constexpr int kEpiSmem = kNodes * kBM * 8;
   struct Params {
     int* status;
     float* sub_s;
@@ -218,8 +221,19 @@ struct ScoresProb {
   }
 
   __device__ static uint64_t* tree_(unsigned char* sm) { return reinterpret_cast<uint64_t*>(sm); }
-  __device__ static float* stage_(unsigned char* sm) {
-    return reinterpret_cast<float*>(sm + kNodes * kBM * 8);
+
+  // r[j] for a per-lane column j: a five-level tree of selects on the bits of j
+  __device__ static float pick(const uint32_t (&r)[32], int j) {
+    float a[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a[i] = __uint_as_float((j & 16) ? r[i + 16] : r[i]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = (j & 8) ? a[i + 8] : a[i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = (j & 4) ? a[i + 4] : a[i];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) a[i] = (j & 2) ? a[i + 2] : a[i];
+    return (j & 1) ? a[1] : a[0];
   }
 
   __device__ static uint64_t make_key(float v, int col, int leaf) {
@@ -229,8 +243,8 @@ struct ScoresProb {
   __device__ static uint64_t empty_key(int leaf) { return (uint64_t)(uint32_t)leaf; }
   __device__ static float key_score(uint64_t key) {
     const uint32_t b = (uint32_t)(key >> 32);
-    if (b == 0u) return -INFINITY;
-    return __uint_as_float((b & 0x80000000u) ? (b & 0x7fffffffu) : ~b);
+    const float f = __uint_as_float((b & 0x80000000u) ? (b & 0x7fffffffu) : ~b);
+    return b == 0u ? -INFINITY : f;
   }
   __device__ static int key_col(uint64_t key) {
     return (int)(kColMask - (((uint32_t)key >> 5) & kColMask));
@@ -264,7 +278,6 @@ struct ScoresProb {
     const int hs_idx = u / P.m_tiles;
     const int C = (hs_idx & 1) ? P.C2 : P.C1;
     uint64_t* tr = tree_(sm);
-    float* stg = stage_(sm);
     for (int piece = 0; piece < kBN / 32; ++piece) {
       const int col0 = c * kBN + piece * 32;
       if (col0 >= C) break;  // warp-uniform
@@ -284,36 +297,43 @@ struct ScoresProb {
       if (C - col0 < 32) mask &= (1u << (C - col0)) - 1u;
       const int trips = __reduce_max_sync(0xffffffffu, __popc(mask));
       if (trips == 0) continue;  // warp-uniform
-      if (mask) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) stg[j * kBM + row] = __uint_as_float(r[j]);
-      }
+      // Branch-free: every lane runs every trip.  A lane without a candidate (or whose
+      // candidate no longer beats its threshold) writes its keys into node 0, which the
+      // tree does not use, and keeps its root.
       int j = mask ? __ffs(mask) - 1 : 0;
-      float v = mask ? stg[j * kBM + row] : -INFINITY;
+      float v = pick(r, j);
+      v = mask ? v : -INFINITY;
       for (int it = 0; it < trips; ++it) {
-        // this iteration's candidate (v, j); fetch the next one early
+        // this trip's candidate (v, j); fetch the next one early
         const int jc = j;
         const float vc = v;
         mask &= mask - 1u;
         j = mask ? __ffs(mask) - 1 : 0;
-        v = mask ? stg[j * kBM + row] : -INFINITY;
+        v = pick(r, j);
+        v = mask ? v : -INFINITY;
         const bool act = vc > es.thr;
         const int leaf = (int)((uint32_t)es.root & (uint32_t)(KM - 1));
         const int node0 = KM + leaf;
         uint64_t sib[kLog];
 #pragma unroll
-        for (int l = 0; l < kLog; ++l) sib[l] = tr[(((node0 >> l) ^ 1)) * kBM + row];
-        uint64_t cur = make_key(vc, col0 + jc, leaf);
-        if (act) tr[node0 * kBM + row] = cur;
+        for (int l = 0; l < kLog; ++l) sib[l] = tr[((node0 >> l) ^ 1) * kBM + row];
+        const uint64_t nk = make_key(vc, col0 + jc, leaf);
+        // the new root: the least of the new key and the siblings (a balanced tree of minima)
+        const uint64_t m01 = kmin(nk, sib[0]);
+        uint64_t root = m01;
+#pragma unroll
+        for (int l = 1; l < kLog; l += 2)
+          root = kmin(root, l + 1 < kLog ? kmin(sib[l], sib[l + 1]) : sib[l]);
+        // the path, leaf to root: running minima
+        tr[(act ? node0 : 0) * kBM + row] = nk;
+        uint64_t cur = m01;
 #pragma unroll
         for (int l = 0; l < kLog; ++l) {
-          cur = kmin(cur, sib[l]);
-          if (act) tr[(node0 >> (l + 1)) * kBM + row] = cur;
+          if (l > 0) cur = kmin(cur, sib[l]);
+          tr[(act ? (node0 >> (l + 1)) : 0) * kBM + row] = cur;
         }
-        if (act) {
-          es.root = cur;
-          es.thr = key_score(cur);
-        }
+        es.root = act ? root : es.root;
+        es.thr = act ? key_score(root) : es.thr;
       }
     }
   }

@@ -6,9 +6,12 @@
 //   warp 1     MMA issuer: allocates 512 TMEM columns (two 256-column fp32
 //              accumulators), one lane issues tcgen05.mma K=16 steps, commits each
 //              stage back to the producer and each finished chunk to the epilogue
-//   warps 2-5  epilogue: 128 threads, thread r owns accumulator row r (TMEM lane
-//              r), reads 32-column pieces with tcgen05.ld and hands them to the
-//              problem's epilogue; releases the accumulator with an mbarrier
+//   warps 2..  epilogue: one or two sets of 128 threads; thread r of a set owns
+//              accumulator row r (TMEM lane r), reads 32-column pieces with tcgen05.ld
+//              and hands them to the problem's epilogue; releases the accumulator with
+//              an mbarrier.  One set alternates between the two accumulators chunk by
+//              chunk; with two sets (Prob::kSets = 2) set s owns accumulator s and every
+//              other unit, and the MMA issuer interleaves the two units' chunks.
 //
 // A "unit" is a 128-row block of the output that the problem walks in chunks of
 // 256 columns (the scoring problem keeps a running top-k across the chunks of a
@@ -22,6 +25,8 @@
 //            box per MN block.  A K=16 step advances 16 rows = 2 KiB.
 #pragma once
 
+#include <type_traits>
+
 #include "tc_common.cuh"
 
 namespace pkm {
@@ -31,21 +36,59 @@ constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kStageA = kBM * kBK * 2;  // 16 KiB
 constexpr int kStageB = kBN * kBK * 2;  // 32 KiB
 constexpr int kStageBytes = kStageA + kStageB;
-constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 
+// Epilogue sets of a problem (Prob::kSets, default 1).  With one set, the 128 epilogue
+// threads alternate between the two 256-column accumulators chunk by chunk.  With two
+// sets, each set of 128 threads owns one accumulator and every other unit of the CTA:
+// the MMA issuer interleaves the two units' chunks, so two epilogue warps share each
+// SM sub-partition and hide each other's latency.
+template <class P, class = void>
+struct SetsOf {
+  static constexpr int value = 1;
+};
+template <class P>
+struct SetsOf<P, std::void_t<decltype(P::kSets)>> {
+  static constexpr int value = P::kSets;
+};
+
 template <class Prob>
-constexpr size_t smem_bytes() {
-  return 1024 + (size_t)Prob::kStages * kStageBytes + Prob::kEpiSmem;
+constexpr int threads_of() {
+  return 64 + 128 * SetsOf<Prob>::value;
 }
 
 template <class Prob>
-__global__ void __launch_bounds__(kThreads, 1)
+constexpr size_t smem_bytes() {
+  return 1024 + (size_t)Prob::kStages * kStageBytes + (size_t)SetsOf<Prob>::value * Prob::kEpiSmem;
+}
+
+// The CTA's chunk schedule, walked identically by the producer, the MMA issuer and each
+// epilogue set: rounds of kSets consecutive units of the CTA (unit i of the CTA is
+// blockIdx.x + i * gridDim.x); within a round chunk c of every unit of the round, unit
+// by unit, before chunk c + 1.  set_chunks(r, s) is the number of chunks of the round's
+// s-th unit (0 past the end).
+template <class Prob>
+struct Schedule {
+  static constexpr int S = SetsOf<Prob>::value;
+  const typename Prob::Params& P;
+  int nunits;
+  __device__ int unit(int r, int s) const {
+    return (int)blockIdx.x + (r * S + s) * (int)gridDim.x;
+  }
+  __device__ int set_chunks(int r, int s) const {
+    const int u = unit(r, s);
+    return u < nunits ? Prob::num_chunks(P, u) : 0;
+  }
+};
+
+template <class Prob>
+__global__ void __launch_bounds__(threads_of<Prob>(), 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
                    const __grid_constant__ CUtensorMap tmA1,
                    const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB1, const typename Prob::Params P) {
   constexpr int S = Prob::kStages;
+  constexpr int NS = SetsOf<Prob>::value;
   extern __shared__ unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], tfull_bar[2], tempty_bar[2],
       drain_bar;
@@ -85,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
   int* status = P.status;
-  const int nunits = Prob::num_units(P);
+  const Schedule<Prob> sch{P, Prob::num_units(P)};
   const int nk = Prob::num_kblocks(P);
 
   if (warp == 0) {
@@ -96,23 +139,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t issued_mask = 0;  // stages that received at least one load
       uint32_t parity_mask = 0;  // bit s: full-barrier parity the last load on s completes
       bool ok = true;
-      for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
-        const int nc = Prob::num_chunks(P, u);
-        for (int c = 0; c < nc && ok; ++c) {
-          for (int kb = 0; kb < nk; ++kb) {
-            if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, status)) {
-              ok = false;
-              break;
-            }
-            unsigned char* sa = smem + (size_t)stage * kStageBytes;
-            mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
-            Prob::load(P, &tmA0, &tmA1, &tmB, &tmB1, u, c, kb, sa, sa + kStageA,
-                       &full_bar[stage]);
-            issued_mask |= 1u << stage;
-            parity_mask = (parity_mask & ~(1u << stage)) | (phase << stage);
-            if (++stage == S) {
-              stage = 0;
-              phase ^= 1u;
+      for (int r = 0; ok; ++r) {
+        int nc[NS], maxc = 0;
+#pragma unroll
+        for (int s = 0; s < NS; ++s) {
+          nc[s] = sch.set_chunks(r, s);
+          maxc = nc[s] > maxc ? nc[s] : maxc;
+        }
+        if (maxc == 0) break;
+        for (int c = 0; c < maxc && ok; ++c) {
+#pragma unroll
+          for (int s = 0; s < NS; ++s) {
+            if (c >= nc[s] || !ok) continue;
+            const int u = sch.unit(r, s);
+            for (int kb = 0; kb < nk; ++kb) {
+              if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag, status)) {
+                ok = false;
+                break;
+              }
+              unsigned char* sa = smem + (size_t)stage * kStageBytes;
+              mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
+              Prob::load(P, &tmA0, &tmA1, &tmB, &tmB1, u, c, kb, sa, sa + kStageA,
+                         &full_bar[stage]);
+              issued_mask |= 1u << stage;
+              parity_mask = (parity_mask & ~(1u << stage)) | (phase << stage);
+              if (++stage == S) {
+                stage = 0;
+                phase ^= 1u;
+              }
             }
           }
         }
@@ -135,47 +189,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = idesc_bf16(kBM, kBN, Prob::kAMN, Prob::kBMN);
       int stage = 0;
       uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
+      int alt = 0;                // one set: the accumulator of the next chunk
+      uint32_t acc_phase = 0u;    // bit a: parity of accumulator a's next phase
       bool ok = true;
       bool issued = false;
-      for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
-        const int nc = Prob::num_chunks(P, u);
-        for (int c = 0; c < nc && ok; ++c) {
-          if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_flag, status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t dt = tmem_base + (uint32_t)acc * kBN;
-          for (int kb = 0; kb < nk; ++kb) {
-            if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status)) {
+      for (int r = 0; ok; ++r) {
+        int nc[NS], maxc = 0;
+#pragma unroll
+        for (int s = 0; s < NS; ++s) {
+          nc[s] = sch.set_chunks(r, s);
+          maxc = nc[s] > maxc ? nc[s] : maxc;
+        }
+        if (maxc == 0) break;
+        for (int c = 0; c < maxc && ok; ++c) {
+#pragma unroll
+          for (int s = 0; s < NS; ++s) {
+            if (c >= nc[s] || !ok) continue;
+            const int acc = NS == 1 ? alt : s;
+            if (!mbar_wait(&tempty_bar[acc], ((acc_phase >> acc) & 1u) ^ 1u, &abort_flag, status)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t sa = smem_u32(smem + (size_t)stage * kStageBytes);
-            const uint32_t sb = sa + kStageA;
+            const uint32_t dt = tmem_base + (uint32_t)acc * kBN;
+            for (int kb = 0; kb < nk; ++kb) {
+              if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t sa = smem_u32(smem + (size_t)stage * kStageBytes);
+              const uint32_t sb = sa + kStageA;
 #pragma unroll
-            for (int k = 0; k < kBK / 16; ++k) {
-              const uint64_t da = Prob::kAMN ? desc_mnmajor_sw128(sa + 2048u * k, 8192u, 1024u)
-                                             : desc_kmajor_sw128(sa) + (uint64_t)(2 * k);
-              const uint64_t db = Prob::kBMN ? desc_mnmajor_sw128(sb + 2048u * k, 8192u, 1024u)
-                                             : desc_kmajor_sw128(sb) + (uint64_t)(2 * k);
-              mma_bf16(dt, da, db, idesc, (kb | k) != 0 ? 1u : 0u);
+              for (int k = 0; k < kBK / 16; ++k) {
+                const uint64_t da = Prob::kAMN ? desc_mnmajor_sw128(sa + 2048u * k, 8192u, 1024u)
+                                               : desc_kmajor_sw128(sa) + (uint64_t)(2 * k);
+                const uint64_t db = Prob::kBMN ? desc_mnmajor_sw128(sb + 2048u * k, 8192u, 1024u)
+                                               : desc_kmajor_sw128(sb) + (uint64_t)(2 * k);
+                mma_bf16(dt, da, db, idesc, (kb | k) != 0 ? 1u : 0u);
+              }
+              issued = true;
+              umma_commit(&empty_bar[stage]);
+              if (++stage == S) {
+                stage = 0;
+                phase ^= 1u;
+              }
             }
-            issued = true;
-            umma_commit(&empty_bar[stage]);
-            if (++stage == S) {
-              stage = 0;
-              phase ^= 1u;
-            }
-          }
-          if (!ok) break;
-          umma_commit(&tfull_bar[acc]);
-          if (++acc == 2) {
-            acc = 0;
-            acc_phase ^= 1u;
+            if (!ok) break;
+            umma_commit(&tfull_bar[acc]);
+            acc_phase ^= 1u << acc;
+            alt ^= 1;
           }
         }
       }
@@ -189,37 +252,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    const int set = NS == 1 ? 0 : (warp - 2) >> 2;
     const int quarter = warp & 3;            // TMEM lanes [32*quarter, 32*quarter + 32)
     const int row = quarter * 32 + lane;     // accumulator row owned by this thread
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    int acc = 0;
-    uint32_t acc_phase = 0;
+    unsigned char* my_smem = epi_smem + (size_t)set * Prob::kEpiSmem;
+    int alt = 0;
+    uint32_t acc_phase = 0u;  // bit a: parity of accumulator a's next phase
     bool ok = true;
-    for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+    for (int r = 0; ok; ++r) {
+      const int nc = sch.set_chunks(r, set);
+      if (nc == 0) {
+        // past this set's last unit: with one set that is the end; with two sets the
+        // round may still have a unit for the other set, and later rounds none for this
+        if (NS == 1 || sch.set_chunks(r, 0) == 0) break;
+        continue;
+      }
+      const int u = sch.unit(r, set);
       typename Prob::EpiState es;
-      Prob::epi_begin(P, u, row, epi_smem, es);
-      const int nc = Prob::num_chunks(P, u);
+      Prob::epi_begin(P, u, row, my_smem, es);
       for (int c = 0; c < nc; ++c) {
+        const int acc = NS == 1 ? alt : set;
         // warp-uniform wait: lane 0 waits, the result is broadcast, so the warp reaches
         // the .sync.aligned TMEM loads together or not at all
         int got = 0;
-        if (lane == 0) got = mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag, status) ? 1 : 0;
+        if (lane == 0)
+          got = mbar_wait(&tfull_bar[acc], (acc_phase >> acc) & 1u, &abort_flag, status) ? 1 : 0;
         got = __shfl_sync(0xffffffffu, got, 0);
         if (!got) {
           ok = false;
           break;
         }
         tc_fence_after();
-        Prob::epi_chunk(P, u, c, row, tmem_base + lane_addr + (uint32_t)acc * kBN, epi_smem, es);
+        Prob::epi_chunk(P, u, c, row, tmem_base + lane_addr + (uint32_t)acc * kBN, my_smem, es);
         tc_fence_before();
         mbar_arrive(&tempty_bar[acc]);
-        if (++acc == 2) {
-          acc = 0;
-          acc_phase ^= 1u;
-        }
+        acc_phase ^= 1u << acc;
+        alt ^= 1;
       }
       if (!ok) break;
-      Prob::epi_end(P, u, row, epi_smem, es);
+      Prob::epi_end(P, u, row, my_smem, es);
     }
   }
   tc_fence_before();

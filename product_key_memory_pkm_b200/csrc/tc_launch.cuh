@@ -22,7 +22,7 @@ cudaError_t launch_tc(const CUtensorMap& A0, const CUtensorMap& A1, const CUtens
   if (attr_err != cudaSuccess) return attr_err;
   const int grid = nunits < sm_count ? nunits : sm_count;
   if (grid <= 0) return cudaSuccess;
-  tc_gemm_kernel<Prob><<<grid, kThreads, smem, st>>>(A0, A1, B, B1 ? *B1 : B, P);
+  tc_gemm_kernel<Prob><<<grid, threads_of<Prob>(), smem, st>>>(A0, A1, B, B1 ? *B1 : B, P);
   PKM_COUNT(1);
   return cudaGetLastError();
 }
