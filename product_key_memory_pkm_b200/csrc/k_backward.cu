@@ -435,7 +435,7 @@ inline int bits_for(int64_t maxkey) {
 // ------------------------------------------------------------------ workspace
 struct Layout {
   size_t keysA, valsA, keysB, valsB, hist, bsum, seg, segrow, wsorted, U, dw, gsub, dq, part,
-      G, dqf, dspart, bneff, bntot, total;
+      G, dspart, bneff, bntot, total;
 };
 
 inline size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -466,11 +466,13 @@ Layout layout(const Plan& p) {
   L.dw = take(4 * E1);
   L.gsub = take(4 * E2);
   L.dq = take(4 * p.N * p.hq);
-  const int64_t nblk = (p.N + kDqTokensPerBlock - 1) / kDqTokensPerBlock;
+  // BatchNorm partial sums: 64-token blocks (CUDA-core path) or 32-token blocks (fused
+  // into the tensor-core dq GEMM)
+  const int64_t nblk = std::max((p.N + kDqTokensPerBlock - 1) / kDqTokensPerBlock,
+                                subgrad_part_blocks(p.N));
   L.part = take(4 * nblk * 2 * p.hq);
-  if (!p.fp32) {  // tensor-core sub-key gradients: dense G planes, fp32 dq, split partials
+  if (!p.fp32) {  // tensor-core sub-key gradients: dense G planes, split partials
     L.G = take(2 * (size_t)(2 * p.h) * 2 * subgrad_pad_tokens(p.N) * subgrad_pad_keys(p.C1, p.C2));
-    L.dqf = take(4 * (size_t)p.N * p.hq);
     L.dspart = take(4 * subgrad_partial_floats(p));
   }
   L.bneff = take(4 * 4 * (size_t)p.hq);  // training-mode BatchNorm: (mean, var, gamma, beta)
@@ -501,7 +503,6 @@ struct BwdCtx {
   float* dq_pre;
   float* part;
   __nv_bfloat16* G;
-  float* dqf;
   float* dspart;
   float* bneff;
   float* bntot;
@@ -522,7 +523,6 @@ static BwdCtx bwd_ctx(const Plan& p, void* ws, float* dw_out) {
   c.dq_pre = at<float>(ws, L.dq);
   c.part = at<float>(ws, L.part);
   c.G = at<__nv_bfloat16>(ws, L.G);
-  c.dqf = at<float>(ws, L.dqf);
   c.dspart = at<float>(ws, L.dspart);
   c.bneff = at<float>(ws, L.bneff);
   c.bntot = at<float>(ws, L.bntot);
@@ -1002,11 +1002,11 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
   if (tc_subgrad) {
     const bool want_dq = dx || dWq || dbn;
     e = launch_subgrad_tc(p, gsub, s.sub_i, subkeys, s.q, bn, dbn_acc ? s.qhat : nullptr,
-                          c.G, c.dqf, reinterpret_cast<__nv_bfloat16*>(dq_pre),
+                          c.G, reinterpret_cast<__nv_bfloat16*>(dq_pre),
                           dbn_acc ? part : nullptr, c.dspart, dsub, want_dq, st);
     if (e != cudaSuccess) return e;
     if (dbn_acc) {
-      const int64_t nblk = (p.N + kDqTokensPerBlock - 1) / kDqTokensPerBlock;
+      const int64_t nblk = subgrad_part_blocks(p.N);
       if (train && (e = cudaMemsetAsync(c.bntot, 0, 2 * sizeof(float) * p.hq, st)) != cudaSuccess)
         return e;
       dbn_reduce_kernel<<<(2 * p.hq + 255) / 256, 256, 0, st>>>(part, (int)nblk, p.hq, dbn_acc);
@@ -1052,7 +1052,8 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
                                 st);
     if (e != cudaSuccess) return e;
     if (dbn) {  // the caller's (d gamma, d beta) += the column sums
-      const int64_t nblk = (p.N + kDqTokensPerBlock - 1) / kDqTokensPerBlock;
+      const int64_t nblk = tc_subgrad ? subgrad_part_blocks(p.N)
+                                      : (p.N + kDqTokensPerBlock - 1) / kDqTokensPerBlock;
       dbn_reduce_kernel<<<(2 * p.hq + 255) / 256, 256, 0, st>>>(part, (int)nblk, p.hq, dbn);
       PKM_COUNT(1);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;

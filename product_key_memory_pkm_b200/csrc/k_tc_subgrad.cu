@@ -78,13 +78,43 @@ __device__ __forceinline__ void store_piece(float* dst, int n0, int n_lim,
 }
 
 // ------------------------------------------------------------------ dq_half = G C_half
+// The epilogue also runs the BatchNorm eval backward on its tile: dq_pre = dq gamma /
+// sqrt(var + eps) is written straight to the bf16 hi/lo planes the dense query GEMMs
+// read, and the per-column partial sums of dq * qhat (d gamma) and dq (d beta) over each
+// warp's 32 tokens are reduced across the warp and written as one partial row per
+// 32-token block (summed in block order afterwards).
+constexpr int kPartTokens = 32;
+
+// x[j] summed over the 32 lanes; lane l ends with the sum of x[l] (butterfly with
+// halving, 31 shuffles).
+__device__ __forceinline__ float warp_transpose_sum(float (&x)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const bool up = (lane & off) != 0;
+      const float send = up ? x[i] : x[i + off];
+      const float keep = up ? x[i + off] : x[i];
+      x[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return x[0];
+}
+
 struct DqProb {
   static constexpr int kAMN = 0, kBMN = 1;
   static constexpr int kStages = 4;
-  static constexpr int kEpiSmem = 0;
+  // per-tile BatchNorm scales gamma / sqrt(var + eps) of the 256 columns, one private
+  // copy per epilogue warp
+  static constexpr int kEpiSmem = 4 * kBN * 4;
   struct Params {
     int* status;
-    float* dqf;  // [N][hq]
+    __nv_bfloat16* planes;  // [2][N][hq] dq_pre hi, lo
+    const float* bn;        // [4][hq]
+    const float* qhat;      // [N][hq] or null
+    float* part;            // [ceil(N / 32)][2][hq] or null
+    float eps;
     int64_t N, Np;
     int h, dk, half, C1, C2, Cp, hq, m_tiles, n_tiles, nkc;  // nkc = Cp / 64
   };
@@ -112,21 +142,90 @@ struct DqProb {
       tma_load_2d(b + j * kMNBoxBytes, B, nt * kBN + j * kMNBox,
                   hh * (P.C1 + P.C2) + s * P.C1 + kk * kBK, bar);
   }
-  __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState&) {}
+  __device__ static float* scales(unsigned char* sm, int row) {
+    return reinterpret_cast<float*>(sm) + (row >> 5) * kBN;
+  }
+  __device__ static void epi_begin(const Params& P, int u, int row, unsigned char* sm,
+                                   EpiState&) {
+    int hs, mt, nt;
+    decode(P, u, hs, mt, nt);
+    const int base = (hs >> 1) * P.dk + (hs & 1) * P.half + nt * kBN;
+    float* sc = scales(sm, row);
+    __syncwarp();  // this warp's reads of the previous tile's scales are done
+    for (int j = row & 31; j < kBN; j += 32) {
+      const int n = nt * kBN + j;
+      sc[j] = n < P.half ? P.bn[2 * P.hq + base + j] / sqrtf(P.bn[P.hq + base + j] + P.eps)
+                         : 0.f;
+    }
+    __syncwarp();
+  }
   __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&) {}
   __device__ static void epi_chunk(const Params& P, int u, int, int row, uint32_t taddr,
-                                   unsigned char*, EpiState&) {
+                                   unsigned char* sm, EpiState&) {
     int hs, mt, nt;
     decode(P, u, hs, mt, nt);
     const int hh = hs >> 1, s = hs & 1;
     const int64_t t = (int64_t)mt * kBM + row;
+    const int64_t tb = ((int64_t)mt * kBM + (row & ~31)) / kPartTokens;  // this warp's block
+    const float* sc = scales(sm, row);
     for (int piece = 0; piece < kBN / 32; ++piece) {
       const int n0 = nt * kBN + piece * 32;
       if (n0 >= P.half) break;  // warp-uniform
       uint32_t r[32];
       tmem_ld32(taddr + (uint32_t)(piece * 32), r);
       tmem_wait_ld(r);
-      if (t < P.N) store_piece(P.dqf + t * P.hq + hh * P.dk + s * P.half + n0, n0, P.half, r);
+      const int64_t col = (int64_t)hh * P.dk + s * P.half + n0;
+      float pg[32], pb[32];
+      if (t < P.N) {
+        uint32_t hi2[16], lo2[16];
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float v0 = __uint_as_float(r[j]) * sc[piece * 32 + j];
+          const float v1 = __uint_as_float(r[j + 1]) * sc[piece * 32 + j + 1];
+          const __nv_bfloat162 hb = __floats2bfloat162_rn(v0, v1);
+          const float2 hf = __bfloat1622float2(hb);
+          const __nv_bfloat162 lb = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
+          hi2[j / 2] = *reinterpret_cast<const uint32_t*>(&hb);
+          lo2[j / 2] = *reinterpret_cast<const uint32_t*>(&lb);
+        }
+        uint4* ph = reinterpret_cast<uint4*>(P.planes + t * P.hq + col);
+        uint4* pl = reinterpret_cast<uint4*>(P.planes + P.N * P.hq + t * P.hq + col);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          ph[v] = make_uint4(hi2[4 * v], hi2[4 * v + 1], hi2[4 * v + 2], hi2[4 * v + 3]);
+          pl[v] = make_uint4(lo2[4 * v], lo2[4 * v + 1], lo2[4 * v + 2], lo2[4 * v + 3]);
+        }
+        if (P.part) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) pb[j] = __uint_as_float(r[j]);
+          if (P.qhat) {
+            const float4* qh = reinterpret_cast<const float4*>(P.qhat + t * P.hq + col);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const float4 q4 = qh[v];
+              pg[4 * v] = pb[4 * v] * q4.x;
+              pg[4 * v + 1] = pb[4 * v + 1] * q4.y;
+              pg[4 * v + 2] = pb[4 * v + 2] * q4.z;
+              pg[4 * v + 3] = pb[4 * v + 3] * q4.w;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) pg[j] = 0.f;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) pg[j] = pb[j] = 0.f;
+      }
+      if (P.part) {  // warp-uniform
+        const float sg = warp_transpose_sum(pg);
+        const float sb = warp_transpose_sum(pb);
+        if (tb * kPartTokens < P.N) {
+          const int lane = row & 31;
+          P.part[(tb * 2 + 0) * P.hq + col + lane] = sg;
+          P.part[(tb * 2 + 1) * P.hq + col + lane] = sb;
+        }
+      }
     }
   }
 };
@@ -223,39 +322,6 @@ __global__ void dsub_reduce_kernel(const float* __restrict__ part, float* __rest
   dsub[i] += acc;
 }
 
-// BatchNorm eval backward: dq_pre = dq gamma / sqrt(var + eps), written as bf16 hi/lo
-// planes for the dense query GEMMs, plus per-64-token partial sums of dq * qhat and
-// dq (the same partial layout the fp32 path produces for dbn_reduce).
-__global__ void __launch_bounds__(256) bn_bwd_kernel(const float* __restrict__ dqf,
-                                                     const float* __restrict__ bn,
-                                                     const float* __restrict__ qhat,
-                                                     __nv_bfloat16* __restrict__ planes,
-                                                     float* __restrict__ part, int64_t N, int hq,
-                                                     float eps) {
-  const int col = blockIdx.y * 256 + threadIdx.x;
-  if (col >= hq) return;
-  const float scale = bn[2 * hq + col] / sqrtf(bn[hq + col] + eps);
-  const int64_t t0 = (int64_t)blockIdx.x * kBnTokens;
-  float pg = 0.f, pb = 0.f;
-  for (int tt = 0; tt < kBnTokens; ++tt) {
-    const int64_t t = t0 + tt;
-    if (t >= N) break;
-    const float dq = dqf[t * hq + col];
-    const float v = dq * scale;
-    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-    planes[t * hq + col] = hi;
-    planes[N * hq + t * hq + col] = __float2bfloat16_rn(v - __bfloat162float(hi));
-    if (part) {
-      pg = fmaf(dq, qhat[t * hq + col], pg);
-      pb += dq;
-    }
-  }
-  if (part) {
-    part[((int64_t)blockIdx.x * 2 + 0) * hq + col] = pg;
-    part[((int64_t)blockIdx.x * 2 + 1) * hq + col] = pb;
-  }
-}
-
 }  // namespace
 
 int64_t subgrad_pad_tokens(int64_t N) { return (N + 63) / 64 * 64; }
@@ -264,11 +330,13 @@ size_t subgrad_partial_floats(const Plan& p) {
   return (size_t)kSplits * 2 * p.h * subgrad_pad_keys(p.C1, p.C2) * p.half;
 }
 
+int64_t subgrad_part_blocks(int64_t N) { return (N + kPartTokens - 1) / kPartTokens; }
+
 cudaError_t launch_subgrad_tc(const Plan& p, const float* gsub, const int32_t* sub_i,
                               const void* subkeys, const void* q_planes, const float* bn,
-                              const float* qhat, __nv_bfloat16* G, float* dqf,
-                              __nv_bfloat16* dq_planes, float* bn_part, float* dsub_part,
-                              float* dsub, bool want_dq, cudaStream_t st) {
+                              const float* qhat, __nv_bfloat16* G, __nv_bfloat16* dq_planes,
+                              float* bn_part, float* dsub_part, float* dsub, bool want_dq,
+                              cudaStream_t st) {
   const int64_t Np = subgrad_pad_tokens(p.N);
   const int Cp = subgrad_pad_keys(p.C1, p.C2);
   const int hs2 = 2 * p.h;
@@ -288,7 +356,11 @@ cudaError_t launch_subgrad_tc(const Plan& p, const float* gsub, const int32_t* s
       return cudaErrorInvalidValue;
     DqProb::Params P{};
     P.status = p.status;
-    P.dqf = dqf;
+    P.planes = dq_planes;
+    P.bn = bn;
+    P.qhat = qhat;
+    P.part = bn_part;
+    P.eps = p.eps;
     P.N = p.N;
     P.Np = Np;
     P.h = p.h;
@@ -304,10 +376,6 @@ cudaError_t launch_subgrad_tc(const Plan& p, const float* gsub, const int32_t* s
     if ((e = launch_tc<DqProb>(ta, ta, tb, P, hs2 * P.m_tiles * P.n_tiles, p.sm_count, st)) !=
         cudaSuccess)
       return e;
-    const dim3 grid((unsigned)((p.N + kBnTokens - 1) / kBnTokens), (unsigned)((p.hq + 255) / 256));
-    bn_bwd_kernel<<<grid, 256, 0, st>>>(dqf, bn, qhat, dq_planes, bn_part, p.N, p.hq, p.eps);
-    PKM_COUNT(1);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (dsub) {
     const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q_planes);

@@ -185,11 +185,13 @@ cudaError_t launch_backward(const Plan& p, const void* x, const void* Wq, const 
 
 // tcgen05 sub-key / query-half gradients and BatchNorm backward (bf16 storage)
 int64_t subgrad_pad_tokens(int64_t N);
+// Partial-sum blocks (32 tokens each) of the BatchNorm backward fused into dq = G C.
+int64_t subgrad_part_blocks(int64_t N);
 int subgrad_pad_keys(int C1, int C2);
 size_t subgrad_partial_floats(const Plan& p);
 cudaError_t launch_subgrad_tc(const Plan& p, const float* gsub, const int32_t* sub_i,
                               const void* subkeys, const void* q_planes, const float* bn,
-                              const float* qhat, __nv_bfloat16* G, float* dqf,
+                              const float* qhat, __nv_bfloat16* G,
                               __nv_bfloat16* dq_planes, float* bn_part, float* dsub_part,
                               float* dsub, bool want_dq, cudaStream_t st);
 
