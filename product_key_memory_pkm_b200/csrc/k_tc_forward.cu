@@ -249,7 +249,11 @@ struct ScoresProb {
   __device__ static int key_col(uint64_t key) {
     return (int)(kColMask - (((uint32_t)key >> 5) & kColMask));
   }
-  __device__ static uint64_t kmin(uint64_t a, uint64_t b) { return a < b ? a : b; }
+  __device__ static uint64_t kmin(uint64_t a, uint64_t b) {
+    uint64_t m;
+    asm("min.u64 %0, %1, %2;" : "=l"(m) : "l"(a), "l"(b));
+    return m;
+  }
 
   __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState& es) {
     es.root = 0;
@@ -303,6 +307,7 @@ struct ScoresProb {
       int j = mask ? __ffs(mask) - 1 : 0;
       float v = pick(r, j);
       v = mask ? v : -INFINITY;
+      uint64_t* trow = tr + row;  // node n of this row's tree: trow[n * kBM]
       for (int it = 0; it < trips; ++it) {
         // this trip's candidate (v, j); fetch the next one early
         const int jc = j;
@@ -316,24 +321,19 @@ struct ScoresProb {
         const int node0 = KM + leaf;
         uint64_t sib[kLog];
 #pragma unroll
-        for (int l = 0; l < kLog; ++l) sib[l] = tr[((node0 >> l) ^ 1) * kBM + row];
-        const uint64_t nk = make_key(vc, col0 + jc, leaf);
-        // the new root: the least of the new key and the siblings (a balanced tree of minima)
-        const uint64_t m01 = kmin(nk, sib[0]);
-        uint64_t root = m01;
-#pragma unroll
-        for (int l = 1; l < kLog; l += 2)
-          root = kmin(root, l + 1 < kLog ? kmin(sib[l], sib[l + 1]) : sib[l]);
-        // the path, leaf to root: running minima
-        tr[(act ? node0 : 0) * kBM + row] = nk;
-        uint64_t cur = m01;
+        for (int l = 0; l < kLog; ++l) sib[l] = trow[((node0 >> l) ^ 1) * kBM];
+        // the path, leaf to root, with running minima; the root itself lives in registers
+        // (it is never a sibling), so its node is not stored
+        uint64_t cur = make_key(vc, col0 + jc, leaf);
+        const int dump = act ? 1 : 0;  // 0: aim the stores at node 0, which is unused
+        trow[(node0 & -dump) * kBM] = cur;
 #pragma unroll
         for (int l = 0; l < kLog; ++l) {
-          if (l > 0) cur = kmin(cur, sib[l]);
-          tr[(act ? (node0 >> (l + 1)) : 0) * kBM + row] = cur;
+          cur = kmin(cur, sib[l]);
+          if (l + 1 < kLog) trow[((node0 >> (l + 1)) & -dump) * kBM] = cur;
         }
-        es.root = act ? root : es.root;
-        es.thr = act ? key_score(root) : es.thr;
+        es.root = act ? cur : es.root;
+        es.thr = act ? key_score(cur) : es.thr;
       }
     }
   }
