@@ -17,7 +17,6 @@
 
 #include "k_sort.cuh"
 #include "k_value_rows.cuh"
-#include "k_value_warp.cuh"
 #include "tc_common.cuh"
 
 namespace pkm {
@@ -552,50 +551,7 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
   e = sort::segments(rows_sorted, E1, seg, U, rb.bsum, st, seg_row, ents_sorted, s.w, w_sorted);
   if (e != cudaSuccess) return e;
 
-  // B3: value rows, one warp per row (rows up to 2048 columns with two or more slots per
-  // warp in shared memory), else one CTA per row
-  {
-    const int vbytes_el = p.vfp32 ? 4 : 2;
-    const bool dense = dV != nullptr;
-    const size_t slot = vw_slot_bytes(p.d_v, vbytes_el, dense);
-    const size_t avail = 220 * 1024;
-    const int depth = (int)std::min<size_t>(kVwMaxDepth, avail / ((size_t)kVwWarps * slot));
-    const int nv4 = p.d_v / 4;
-    const int maxj = (nv4 + 31) / 32;
-#ifndef PKM_B3_WARP
-#define PKM_B3_WARP 0
-#endif
-    if (PKM_B3_WARP && maxj <= 16 && depth >= 2) {
-      const size_t smem = (size_t)kVwWarps * depth * slot;
-#ifndef PKM_VW_CONTIGUOUS
-#define PKM_VW_CONTIGUOUS 0
-#endif
-#define PKM_VW(TV, MJ)                                                                        \
-  do {                                                                                        \
-    if ((e = cudaFuncSetAttribute(value_warp_kernel<TV, MJ>,                                  \
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != \
-        cudaSuccess)                                                                          \
-      return e;                                                                               \
-    value_warp_kernel<TV, MJ><<<p.sm_count, kVwWarps * 32, smem, st>>>(                       \
-        seg, U, seg_row, ents_sorted, static_cast<const TV*>(values), w_sorted, dy, dV, dw,   \
-        hk, p.d_v, p.K, p.status, dVc, rows_out, U_out, ent_tok, depth, PKM_VW_CONTIGUOUS);   \
-  } while (0)
-#define PKM_VW_J(TV)                 \
-  do {                               \
-    if (maxj <= 2) PKM_VW(TV, 2);    \
-    else if (maxj <= 4) PKM_VW(TV, 4);   \
-    else if (maxj <= 8) PKM_VW(TV, 8);   \
-    else if (maxj <= 13) PKM_VW(TV, 13); \
-    else PKM_VW(TV, 16);             \
-  } while (0)
-      if (p.vfp32) PKM_VW_J(float);
-      else PKM_VW_J(__nv_bfloat16);
-#undef PKM_VW_J
-#undef PKM_VW
-      PKM_COUNT(1);
-      return cudaGetLastError();
-    }
-  }
+  // B3: value rows
   {
     const int E = p.vfp32 ? 4 : 8;
     const int nvec = p.d_v / E;
