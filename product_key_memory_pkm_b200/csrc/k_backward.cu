@@ -323,14 +323,28 @@ __global__ void __launch_bounds__(256) dq_kernel(
   }
 }
 
-__global__ void dbn_reduce_kernel(const float* __restrict__ part, int nblk, int hq,
-                                  float* __restrict__ dbn) {
-  const int col = blockIdx.x * blockDim.x + threadIdx.x;
-  if (col >= 2 * hq) return;
-  const int which = col / hq, c = col % hq;
+// dbn[which][c] += sum over the nblk partial rows, in a fixed order: 32 columns per
+// block (lane = column), warp w sums the rows b = w, w + 8, ..., then the 8 warp sums
+// are added in warp order.
+__global__ void __launch_bounds__(256) dbn_reduce_kernel(const float* __restrict__ part,
+                                                         int nblk, int hq,
+                                                         float* __restrict__ dbn) {
+  __shared__ float red[8][32];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int col = blockIdx.x * 32 + lane;
+  const bool live = col < 2 * hq;
+  const int which = live ? col / hq : 0, c = live ? col % hq : 0;
   float s = 0.f;
-  for (int b = 0; b < nblk; ++b) s += part[((int64_t)b * 2 + which) * hq + c];
-  dbn[which * hq + c] += s;
+  if (live)
+    for (int b = wid; b < nblk; b += 8) s += part[((int64_t)b * 2 + which) * hq + c];
+  red[wid][lane] = s;
+  __syncthreads();
+  if (wid == 0 && live) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += red[w][lane];
+    dbn[which * hq + c] += t;
+  }
 }
 
 // ------------------------------------------------------------------ B5b keys
@@ -965,7 +979,7 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
       const int64_t nblk = subgrad_part_blocks(p.N);
       if (train && (e = cudaMemsetAsync(c.bntot, 0, 2 * sizeof(float) * p.hq, st)) != cudaSuccess)
         return e;
-      dbn_reduce_kernel<<<(2 * p.hq + 255) / 256, 256, 0, st>>>(part, (int)nblk, p.hq, dbn_acc);
+      dbn_reduce_kernel<<<(2 * p.hq + 31) / 32, 256, 0, st>>>(part, (int)nblk, p.hq, dbn_acc);
       PKM_COUNT(1);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -998,7 +1012,7 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
     if (dbn_acc) {
       if (train && (e = cudaMemsetAsync(c.bntot, 0, 2 * sizeof(float) * p.hq, st)) != cudaSuccess)
         return e;
-      dbn_reduce_kernel<<<(2 * p.hq + 255) / 256, 256, 0, st>>>(part, (int)nblk, p.hq, dbn_acc); PKM_COUNT(1);
+      dbn_reduce_kernel<<<(2 * p.hq + 31) / 32, 256, 0, st>>>(part, (int)nblk, p.hq, dbn_acc); PKM_COUNT(1);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
   }
@@ -1010,7 +1024,7 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
     if (dbn) {  // the caller's (d gamma, d beta) += the column sums
       const int64_t nblk = tc_subgrad ? subgrad_part_blocks(p.N)
                                       : (p.N + kDqTokensPerBlock - 1) / kDqTokensPerBlock;
-      dbn_reduce_kernel<<<(2 * p.hq + 255) / 256, 256, 0, st>>>(part, (int)nblk, p.hq, dbn);
+      dbn_reduce_kernel<<<(2 * p.hq + 31) / 32, 256, 0, st>>>(part, (int)nblk, p.hq, dbn);
       PKM_COUNT(1);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
