@@ -724,8 +724,14 @@ def run_decode(args, cfg, rank, world, dist):
             saved = P.alloc_saved(dims, with_qhat=False)
             x = x_all[:n].contiguous()
             y = torch.empty(n, cfg.d_v, device=dev)
+            # few tokens: the optional workspace runs the forward as one fused kernel
+            fused_ws = (P.alloc_workspace(dims, P.PKM_FWD_FUSED)
+                        if P.pkm_workspace_bytes(dims, P.PKM_FWD_FUSED) > 0 else None)
 
-            def call():
+            def call(ws=fused_ws):
+                P.pkm_forward(dims, x, Wq, bn, sub, V, y, saved, workspace=ws, stream=side)
+
+            def call_separate():
                 P.pkm_forward(dims, x, Wq, bn, sub, V, y, saved, stream=side)
             for _ in range(args.warmup):
                 call()
@@ -764,6 +770,19 @@ def run_decode(args, cfg, rank, world, dist):
             graph_warm = burst(g.replay)
             graph_cold = cold(g.replay)
             eager_cold = cold(call)
+            sep = None
+            if fused_ws is not None:  # the four separate kernels, for comparison
+                l1 = P.pkm_launch_count()
+                call_separate()
+                side.synchronize()
+                launches += (P.pkm_launch_count() - l1) * (reps + args.steps * 5)
+                g2 = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g2, stream=side):
+                    call_separate()
+                g2.replay()
+                sep = {"graph_us_l2_warm": round(burst(g2.replay), 2),
+                       "graph_us_l2_flushed": round(cold(g2.replay), 2)}
+                del g2
             launches += per_call * (reps + args.steps * 5) * 2
             assert P.pkm_check_status(side) == P.PKM_OK
             # bytes a call must move: Wq and the sub-keys once, then n*h*k value rows
@@ -773,7 +792,8 @@ def run_decode(args, cfg, rank, world, dist):
                       "graph_us_l2_flushed": round(graph_cold, 2),
                       "eager_us_l2_warm": round(eager_warm, 2),
                       "eager_us_l2_flushed": round(eager_cold, 2),
-                      "kernels_per_call": int(per_call), "algorithmic_bytes": int(alg)}
+                      "kernels_per_call": int(per_call), "algorithmic_bytes": int(alg),
+                      **({"separate_kernels": sep} if sep else {})}
             del g
     clk = clocks.stop()
     if rank != 0:

@@ -134,13 +134,21 @@ typedef struct {
 
 #define PKM_FWD 0
 #define PKM_BWD 1
+#define PKM_FWD_FUSED 2
 
 /* Bytes of one pkm_saved field (PKM_SAVED_*) for these dims; 0 for bad input. */
 size_t pkm_saved_bytes(const pkm_dims* d, int field);
 
 /* Bytes of device workspace pkm_forward (which = PKM_FWD) or pkm_backward
  * (PKM_BWD) needs.  The workspace is scratch: its contents on entry are ignored
- * and on return are unspecified.  256-byte alignment is required. */
+ * and on return are unspecified.  256-byte alignment is required.
+ * which = PKM_FWD_FUSED: the optional forward workspace of few-token calls (0 when it
+ * does not apply).  When pkm_forward gets at least this many bytes (N <= 16, bf16
+ * storage, eval-mode BatchNorm, dot-product scores, 1 <= k <= 32, dk/2 <= 512, C1 and C2
+ * <= 4096), it runs the four steps as one cooperative kernel with grid-wide barriers
+ * (one launch instead of four; the results are those of the separate kernels).  Every
+ * barrier wait is bounded and reports PKM_ERR_DEVICE_TIMEOUT through pkm_check_status.
+ * Without it, or when the device cannot hold one CTA per SM, the separate kernels run. */
 size_t pkm_workspace_bytes(const pkm_dims* d, int which);
 
 /* Forward F1..F4 ("Large Memory Layers with Product Keys", method details).

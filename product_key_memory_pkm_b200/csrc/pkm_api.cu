@@ -208,6 +208,7 @@ size_t pkm_saved_bytes(const pkm_dims* d, int field) {
 size_t pkm_workspace_bytes(const pkm_dims* d, int which) {
   if (validate_dims(d) != PKM_OK) return 0;
   if (which == PKM_FWD) return 0;
+  if (which == PKM_FWD_FUSED) return d->N == 0 ? 0 : fused_decode_bytes(shape_plan(d));
   if (which != PKM_BWD || d->N == 0) return 0;
   const Plan p = shape_plan(d);
   return backward_workspace_bytes(p);
@@ -275,6 +276,19 @@ pkm_status pkm_forward(const pkm_dims* d, const void* x, const void* Wq, const f
   Plan p;
   PKM_TRY(prepare(d, &p));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // few tokens with enough workspace: the whole forward as one kernel
+  const size_t fused = fused_decode_bytes(p);
+  if (fused && workspace && workspace_bytes >= fused &&
+      !(reinterpret_cast<uintptr_t>(workspace) & 255u)) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PKM_ERR_CUDA;
+    const cudaError_t e = launch_fused_decode(p, dev, x, Wq, bn, subkeys, values, y, *saved,
+                                              workspace, st);
+    if (e == cudaSuccess) return PKM_OK;
+    // the CTAs could not all be resident: run the separate kernels instead
+    if (e != cudaErrorCooperativeLaunchTooLarge) return PKM_ERR_CUDA;
+    (void)cudaGetLastError();
+  }
   PKM_TRY(cuda_status(run_query(p, x, Wq, bn, saved->q, saved->qhat, st, saved->bn_batch)));
   PKM_TRY(cuda_status(run_scores(p, subkeys, saved->q, saved->sub_s, saved->sub_i, st)));
   PKM_TRY(cuda_status(launch_candidates(p, saved->sub_s, saved->sub_i, saved->idx, saved->w, st)));

@@ -130,6 +130,12 @@ cudaError_t launch_scores_small(const Plan& p, const void* subkeys, const void* 
                                 int32_t* sub_i, cudaStream_t st);
 cudaError_t launch_gather(const Plan& p, const void* values, const int32_t* idx, const float* w,
                           float* y, cudaStream_t st);
+// The whole few-token forward as one cooperative kernel (workspace: fused_decode_bytes).
+bool fused_decode_supported(const Plan& p);
+size_t fused_decode_bytes(const Plan& p);
+cudaError_t launch_fused_decode(const Plan& p, int dev, const void* x, const void* Wq,
+                                const float* bn, const void* subkeys, const void* values,
+                                float* y, const pkm_saved& s, void* ws, cudaStream_t st);
 
 // ---------------------------------------------------------------- backward launches
 struct BwdWs;  // workspace layout, defined in k_backward.cu

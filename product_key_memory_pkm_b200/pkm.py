@@ -34,7 +34,7 @@ PKM_F_BF16_Q = 0x8
 PKM_F_BN_TRAIN = 0x10
 PKM_F_ALL_K2 = 0x20
 PKM_F_IDW = 0x40
-PKM_FWD, PKM_BWD = 0, 1
+PKM_FWD, PKM_BWD, PKM_FWD_FUSED = 0, 1, 2
 PKM_FW_LOOKAHEAD = 0x1
 PKM_FW_SORT_GLOBAL = 0x2
 PKM_FW_PER_CHUNK = 0x4
