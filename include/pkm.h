@@ -146,9 +146,13 @@ size_t pkm_saved_bytes(const pkm_dims* d, int field);
  * does not apply).  When pkm_forward gets at least this many bytes (N <= 16, bf16
  * storage, eval-mode BatchNorm, dot-product scores, 1 <= k <= 32, dk/2 <= 512, C1 and C2
  * <= 4096), it runs the four steps as one cooperative kernel with grid-wide barriers
- * (one launch instead of four; the results are those of the separate kernels).  Every
- * barrier wait is bounded and reports PKM_ERR_DEVICE_TIMEOUT through pkm_check_status.
- * Without it, or when the device cannot hold one CTA per SM, the separate kernels run. */
+ * (one launch instead of four).  Its results agree with the separate kernels' to fp32
+ * rounding: the dot products are summed in another order, so keys whose scores tie to
+ * within that rounding may be kept or ordered differently.  Every barrier wait is
+ * bounded and reports PKM_ERR_DEVICE_TIMEOUT through pkm_check_status; after an expired
+ * wait every later fused call on that device reports the timeout and computes nothing.
+ * Without the workspace, or when the device cannot hold one CTA per SM, the separate
+ * kernels run. */
 size_t pkm_workspace_bytes(const pkm_dims* d, int which);
 
 /* Forward F1..F4 ("Large Memory Layers with Product Keys", method details).
