@@ -53,9 +53,14 @@ using namespace tc;
 struct QueryProb {
   static constexpr int kAMN = 0, kBMN = 0;
   static constexpr int kStages = 4;
-  // per-tile BatchNorm constants (mean, 1/sqrt(var + eps), gamma, beta) for the 256
-  // columns, one private copy per epilogue warp so no barrier spans warps
-  static constexpr int kEpiSmem = 4 * 4 * kBN * 4;
+  // two epilogue sets (eight epilogue warps): the BatchNorm, the hi/lo split and three
+  // output streams of a tile take about as long as its mainloop, so each set gets two
+  // units' MMA time to finish one
+  static constexpr int kSets = 2;
+  // per-tile BatchNorm constants {mean, 1/sqrt(var + eps), gamma, beta} of the 256
+  // columns as one float4 each, one private copy per epilogue warp so no barrier spans
+  // warps
+  static constexpr int kEpiSmem = 4 * kBN * 16;
   struct Params {
     int* status;
     const float* bn;
@@ -79,14 +84,14 @@ struct QueryProb {
     tma_load_2d(sb, B, kb * kBK, nt * kBN, bar);
   }
 
-  __device__ static float* consts(unsigned char* sm, int row) {
-    return reinterpret_cast<float*>(sm) + (row >> 5) * 4 * kBN;
+  __device__ static float4* consts(unsigned char* sm, int row) {
+    return reinterpret_cast<float4*>(sm) + (row >> 5) * kBN;
   }
 
   __device__ static void epi_begin(const Params& P, int u, int row, unsigned char* sm,
                                    EpiState&) {
     const int nt = u % P.n_tiles;
-    float* c = consts(sm, row);
+    float4* c = consts(sm, row);
     __syncwarp();  // this warp's reads of the previous tile's constants are done
     for (int j = row & 31; j < kBN; j += 32) {
       const int n = nt * kBN + j;
@@ -100,10 +105,7 @@ struct QueryProb {
         gamma = P.bn[2 * P.hq + n];
         beta = P.bn[3 * P.hq + n];
       }
-      c[j] = mean;
-      c[kBN + j] = inv;
-      c[2 * kBN + j] = gamma;
-      c[3 * kBN + j] = beta;
+      c[j] = make_float4(mean, inv, gamma, beta);
     }
     __syncwarp();
   }
@@ -114,7 +116,7 @@ struct QueryProb {
     const int mt = u / P.n_tiles, nt = u % P.n_tiles;
     const int64_t t = (int64_t)mt * kBM + row;
     const int hq = P.hq;
-    const float* cst = consts(sm, row);
+    const float4* cst = consts(sm, row);
     for (int piece = 0; piece < kBN / 32; ++piece) {
       const int n0 = nt * kBN + piece * 32;
       if (n0 >= hq) break;  // warp-uniform
@@ -129,10 +131,10 @@ struct QueryProb {
         float qq[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int jj = piece * 32 + j + e;
-          const float h = (__uint_as_float(r[j + e]) - cst[jj]) * cst[kBN + jj];
+          const float4 c4 = cst[piece * 32 + j + e];  // mean, inv, gamma, beta
+          const float h = (__uint_as_float(r[j + e]) - c4.x) * c4.y;
           qh[j + e] = h;
-          qq[e] = fmaf(cst[2 * kBN + jj], h, cst[3 * kBN + jj]);
+          qq[e] = fmaf(c4.z, h, c4.w);
         }
         const __nv_bfloat162 hb = __floats2bfloat162_rn(qq[0], qq[1]);
         const float2 hf = __bfloat1622float2(hb);
