@@ -999,6 +999,16 @@ def run_stage(args, cfg, dims, saved, P, st, step, flush, names, env):
             calls[prev]()
         torch.cuda.synchronize()
         fn = calls[args.stage]
+        if args.stage in ("gather_bag", "value_grad"):
+            # the same algorithmic bytes as the full step's roofline
+            sel = cfg.N * cfg.h * cfg.k
+            if args.stage == "gather_bag":
+                alg = sel * cfg.d_v * 2 + cfg.N * cfg.d_v * 4 + sel * 8
+                extra = {"algorithmic_bytes": int(alg)}
+            else:
+                U = int(torch.unique(saved["idx"]).numel())
+                alg = U * cfg.d_v * (2 + 8) + cfg.N * cfg.d_v * 4 + sel * 12
+                extra = {"distinct_rows": U, "algorithmic_bytes": int(alg)}
     for _ in range(args.warmup):
         flush.zero_()
         fn()
