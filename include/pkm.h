@@ -394,8 +394,8 @@ const char* pkm_status_string(pkm_status s);
  *     k = 32).  A larger problem returns PKM_ERR_WORKSPACE from a host-side check,
  *     before any CUDA call.
  *   - The first call on a device fetches the array's device address
- *     (cudaGetSymbolAddress) with that device current.  Make that first call before
- *     any stream capture begins.  A failed lookup is not cached: the next call retries.
+ *     (cudaGetSymbolAddress) with that device current.  A failed lookup returns
+ *     PKM_ERR_CUDA and is not cached: the next call retries.
  *   - Every call shares the one array.  Each call clears or fully rewrites the parts
  *     it reads, so nothing needs clearing between calls.  Calls whose work overlaps on
  *     the GPU (other streams, other host threads) race on the array and must be

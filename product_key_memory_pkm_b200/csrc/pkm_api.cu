@@ -670,8 +670,8 @@ std::atomic<void*> g_noalloc_ptr[kMaxDevices];
 std::mutex g_noalloc_mu;
 
 // Device address of the scratch on the current device, or nullptr if the lookup failed.
-// Only a successful lookup is kept: a failed one (say, made while the stream was being
-// captured) is retried by the next call, and its non-sticky error is cleared.
+// Only a successful lookup is kept: a failed one is retried by the next call, and its
+// non-sticky error is cleared.
 void* noalloc_scratch(int dev) {
   void* ptr = g_noalloc_ptr[dev].load(std::memory_order_acquire);
   if (ptr) return ptr;
@@ -704,6 +704,7 @@ extern "C" pkm_status pkm_value_grad_noalloc(const pkm_dims* d, const void* valu
   PKM_TRY(prepare(d, &p));
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PKM_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return PKM_ERR_UNSUPPORTED;
   void* scratch = noalloc_scratch(dev);
   if (!scratch) return PKM_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
