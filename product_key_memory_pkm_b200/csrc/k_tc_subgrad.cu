@@ -105,6 +105,9 @@ __device__ __forceinline__ float warp_transpose_sum(float (&x)[32]) {
 struct DqProb {
   static constexpr int kAMN = 0, kBMN = 1;
   static constexpr int kStages = 4;
+  // two epilogue sets: the BatchNorm backward makes the epilogue as long as a unit's
+  // mainloop, so each set gets two units' MMA time to finish one
+  static constexpr int kSets = 2;
   // per-tile BatchNorm scales gamma / sqrt(var + eps) of the 256 columns, one private
   // copy per epilogue warp
   static constexpr int kEpiSmem = 4 * kBN * 4;
