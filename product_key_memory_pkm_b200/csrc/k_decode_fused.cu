@@ -11,10 +11,11 @@
 //      hi/lo planes (and q-hat) the other entry points use ("Large Memory Layers with
 //      Product Keys", method details: the query network).
 //   B  sub-key scores: one item per (head, half, block of 64 sub-keys); the block's rows
-//      copied into shared memory (asynchronous copies, the rows asked of L2 at kernel
-//      start), every token's scores against them as four partial dot products per key,
-//      and each token's best k of the block by rank (score desc, index asc) written to
-//      the workspace.
+//      copied into shared memory by asynchronous copies (a CTA's first block at kernel
+//      start, since it does not depend on q; the others asked of L2 then), every
+//      token's scores against them as eight partial dot products per key (each thread
+//      accumulating all tokens), and each token's best k of the block by rank (score
+//      desc, index asc) written to the workspace.
 //   C  one item per (token, head): each half's block lists merged pairwise in shared
 //      memory (log2 of the block count levels, every entry placed by its merge rank),
 //      then the top k of the k x k candidate combine, found by ranking only the pairs
@@ -74,6 +75,7 @@ struct FusedArgs {
   int* status;
   int64_t K;
   int N, d_in, h, dk, half, C1, C2, k, d_v, hq, nb1, nb2, nblk;
+  int b_off;  // byte offset of phase B's shared memory; > 0: its first block is copied at start
   float eps, scale, lo_scale;
 };
 
@@ -249,11 +251,24 @@ __device__ void prefetch_blocks(const FusedArgs& a) {
   }
 }
 
+// The block rows of scoring item `it` into the padded rows of kc (asynchronous copies).
+__device__ void issue_block_rows(const FusedArgs& a, int it, __nv_bfloat16* kc) {
+  const BlockItem b = block_item(a, it);
+  const int ks = a.half + 8, npc = a.half / 8;
+  const uint4* src = reinterpret_cast<const uint4*>(block_rows(a, b));
+  for (int i = threadIdx.x; i < b.nc * npc; i += kFT) {
+    const int c = i / npc, pc = i % npc;
+    cp_async16(kc + (size_t)c * ks + pc * 8, src + i);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
 template <int TB>
 __device__ void phase_scores(const FusedArgs& a, unsigned char* sm) {
   const int tid = threadIdx.x;
   const int ks = a.half + 8;  // bf16 row stride (16-byte pad: conflict-free rows)
   const int NT = a.N * kBlkKeys;
+  sm += a.b_off;
   __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(sm);
   float* qs = reinterpret_cast<float*>(sm + (size_t)kBlkKeys * ks * 2);
   float* scp = qs + (size_t)a.N * a.half;  // [kParts][N][64]
@@ -262,11 +277,8 @@ __device__ void phase_scores(const FusedArgs& a, unsigned char* sm) {
   const int items = a.h * (a.nb1 + a.nb2);
   for (int it = blockIdx.x; it < items; it += gridDim.x) {
     const BlockItem b = block_item(a, it);
-    const uint4* src = reinterpret_cast<const uint4*>(block_rows(a, b));
-    for (int i = tid; i < b.nc * npc; i += kFT) {
-      const int c = i / npc, pc = i % npc;
-      cp_async16(kc + (size_t)c * ks + pc * 8, src + i);
-    }
+    // the first block's rows were copied at kernel start when there was room
+    if (a.b_off == 0 || it != (int)blockIdx.x) issue_block_rows(a, it, kc);
     // q = hi + lo_scale * lo of this head-half, written by phase A (read through L2)
     for (int i = tid; i < a.N * npc; i += kFT) {
       const int t = i / npc, pc = i % npc;
@@ -523,6 +535,13 @@ __device__ void phase_select(const FusedArgs& a, unsigned char* sm) {
       }
     }
     __syncthreads();
+    if (warp == 1 && lane < k) {  // the bag reads the winners' rows next: ask L2 for them
+      const int32_t row = oI[lane];
+      if (row >= 0 && row < a.K)
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.V + (int64_t)row * a.d_v),
+                     "r"((uint32_t)(a.d_v * 2))
+                     : "memory");
+    }
     if (warp == 0) {
       const bool live = lane < k;
       const float outS = live ? oS[lane] : 0.f;
@@ -536,10 +555,6 @@ __device__ void phase_select(const FusedArgs& a, unsigned char* sm) {
         const int32_t row = oI[lane];
         a.idx[wo + lane] = row;
         a.w[wo + lane] = ex / sum;
-        if (row >= 0 && row < a.K)  // the bag reads this row next: ask L2 for it now
-          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.V + (int64_t)row * a.d_v),
-                       "r"((uint32_t)(a.d_v * 2))
-                       : "memory");
       }
     }
     __syncthreads();  // the next item reuses the lists
@@ -611,6 +626,10 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(const FusedArgs a)
     if (threadIdx.x == 0) set_status(a.status, kDevTimeout);
     return;
   }
+  // phase B's first block does not depend on q: when its shared memory lies past phase
+  // A's, its rows come in while the query network runs
+  if (a.b_off > 0 && (int)blockIdx.x < a.h * (a.nb1 + a.nb2))
+    issue_block_rows(a, blockIdx.x, reinterpret_cast<__nv_bfloat16*>(fsm + a.b_off));
   prefetch_blocks(a);
   phase_query<TB>(a, fsm);
   if (!grid_sync(a, 1, &s_ok)) return;
@@ -624,13 +643,23 @@ __global__ void __launch_bounds__(kFT, 1) decode_fused_kernel(const FusedArgs a)
 
 int nblk_of(int C) { return (C + kBlkKeys - 1) / kBlkKeys; }
 
+constexpr size_t kFusedSmemMax = 200 * 1024;  // dynamic shared memory the layout may take
+
+// Phase B's shared-memory offset: past phase A's staged tokens when both fit.
+size_t fused_b_off(const Plan& p) {
+  const size_t qa = ((size_t)p.N * p.d_in * 2 + 127) & ~size_t(127);
+  const size_t sb = (size_t)kBlkKeys * (p.half + 8) * 2 + (size_t)p.N * p.half * 4 +
+                    (kParts + 1) * (size_t)p.N * kBlkKeys * 4;
+  return qa + sb <= kFusedSmemMax ? qa : 0;
+}
+
 size_t fused_smem(const Plan& p) {
   const size_t qa = (size_t)p.N * p.d_in * 2;
   const size_t sb = (size_t)kBlkKeys * (p.half + 8) * 2 + (size_t)p.N * p.half * 4 +
                     (kParts + 1) * (size_t)p.N * kBlkKeys * 4;
   const size_t sc = (size_t)2 * 2 * nblk_of(std::max(p.C1, p.C2)) * p.k * 8 + kMaxPairs * 24 +
                     96 * 4;
-  return std::max(std::max(qa, sb), sc);
+  return std::max(std::max(qa, fused_b_off(p) + sb), sc);
 }
 
 constexpr int kMaxFusedDevices = 64;
@@ -737,6 +766,7 @@ cudaError_t launch_fused_decode(const Plan& p, int dev, const void* x, const voi
   a.eps = p.eps;
   a.scale = p.scale;
   a.lo_scale = p.bf16q ? 0.f : 1.f;
+  a.b_off = (int)fused_b_off(p);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.sm_count);
   cfg.blockDim = dim3(kFT);
