@@ -360,6 +360,11 @@ FUSED_CASES = {
     "sixteen_tokens_k32": _cfg(N=16, h=2, C1=200, C2=130, k=32, d_v=264),
     "k_equals_C": _cfg(N=3, h=2, C1=32, C2=32, k=32, d_v=64),
     "k1_single_pass_q": _cfg(N=7, h=2, k=1),
+    # 64 block lists in the first half (the most the merge takes: six levels), a ragged last
+    # block, and an odd list count in the second half
+    "C4096_six_merge_levels": _cfg(N=2, h=1, dk=64, C1=4096, C2=200, k=8, d_v=16),
+    "sixteen_tokens_wide_input": _cfg(N=16, d_in=2048, h=2, dk=256, C1=130, C2=96, k=16,
+                                      d_v=40),
 }
 
 
