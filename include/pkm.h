@@ -186,6 +186,18 @@ pkm_status pkm_backward(const pkm_dims* d, const void* x, const void* Wq, const 
 pkm_status pkm_value_grad(const pkm_dims* d, const void* values, const pkm_saved* saved,
                           const float* dy, float* dvalues, float* dw, void* workspace,
                           size_t workspace_bytes, void* stream);
+/* The value stage in its two parts (pkm_value_grad runs both, with the same results):
+ * pkm_value_sort sorts saved->idx by value row and leaves the sorted selections, the
+ * distinct rows and the weights in row order (gathered from saved->w) in the workspace;
+ * pkm_value_rows then runs the pass per distinct row from that workspace.  Between the
+ * two calls the workspace belongs to them: nothing else may write it, and the dims must
+ * be the same.  pkm_value_sort needs only the forward's selection, so a caller can run it
+ * before the upstream gradient exists (e.g. beside the forward's bag on another stream). */
+pkm_status pkm_value_sort(const pkm_dims* d, const pkm_saved* saved, void* workspace,
+                          size_t workspace_bytes, void* stream);
+pkm_status pkm_value_rows(const pkm_dims* d, const void* values, const float* dy,
+                          float* dvalues, float* dw, void* workspace, size_t workspace_bytes,
+                          void* stream);
 pkm_status pkm_query_grad(const pkm_dims* d, const void* x, const void* Wq, const float* bn,
                           const void* subkeys, const pkm_saved* saved, const float* dw, float* dx,
                           float* dWq, float* dbn, float* dsubkeys, void* workspace,

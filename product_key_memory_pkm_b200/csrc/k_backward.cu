@@ -542,35 +542,31 @@ static BwdCtx bwd_ctx(const Plan& p, void* ws, float* dw_out) {
   return c;
 }
 
-cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved& s,
-                              const float* dy, float* dV, float* dw_out, void* ws,
-                              cudaStream_t st, float* dVc, int32_t* rows_out, int* U_out,
-                              const int32_t* ent_tok) {
+// B1-B2: the selections sorted by value row (stable radix sort), the segment table of
+// the distinct rows and the weights in row order, all in the workspace.
+cudaError_t launch_value_sort(const Plan& p, const pkm_saved& s, void* ws, cudaStream_t st) {
   const int64_t E1 = p.N * p.h * p.ksel;
-  BwdCtx c = bwd_ctx(p, ws, dw_out);
-  sort::RadixBuffers& rb = c.rb;
-  int* seg = c.seg;
-  int32_t* seg_row = c.seg_row;
-  int* U = c.U;
-  float* dw = c.dw;
-  cudaError_t e;
-  const int hk = p.h * p.ksel;
-  const int persist_blocks = p.sm_count * 8;
-
-  // B1-B2: selections sorted by value row
+  BwdCtx c = bwd_ctx(p, ws, nullptr);
   const int32_t *rows_sorted, *ents_sorted;
-  e = sort::radix_sort(s.idx, E1, bits_for(p.K - 1), rb, &rows_sorted, &ents_sorted, st);
+  cudaError_t e =
+      sort::radix_sort(s.idx, E1, bits_for(p.K - 1), c.rb, &rows_sorted, &ents_sorted, st);
   if (e != cudaSuccess) return e;
-  float* w_sorted = c.w_sorted;
-  e = sort::segments(rows_sorted, E1, seg, U, rb.bsum, st, seg_row, ents_sorted, s.w, w_sorted);
-  if (e != cudaSuccess) return e;
+  return sort::segments(rows_sorted, E1, c.seg, c.U, c.rb.bsum, st, c.seg_row, ents_sorted, s.w,
+                        c.w_sorted);
+}
 
-  // B3: value rows
-  {
-    const int E = p.vfp32 ? 4 : 8;
-    const int nvec = p.d_v / E;
-    const int blocks = p.sm_count * PKM_B3_MIN_BLOCKS;
-    const size_t smem = value_rows_smem(p);
+// B3: one pass per distinct value row over what launch_value_sort left in the workspace.
+cudaError_t launch_value_rows(const Plan& p, const void* values, const float* dy, float* dV,
+                              float* dw_out, void* ws, cudaStream_t st, float* dVc,
+                              int32_t* rows_out, int* U_out, const int32_t* ent_tok) {
+  BwdCtx c = bwd_ctx(p, ws, dw_out);
+  const int32_t* ents_sorted = sort::radix_sorted_vals(c.rb, bits_for(p.K - 1));
+  const int hk = p.h * p.ksel;
+  cudaError_t e;
+  const int E = p.vfp32 ? 4 : 8;
+  const int nvec = p.d_v / E;
+  const int blocks = p.sm_count * PKM_B3_MIN_BLOCKS;
+  const size_t smem = value_rows_smem(p);
 #define PKM_B3(TV, CHV)                                                                      \
   do {                                                                                       \
     if (smem > 48 * 1024 &&                                                                  \
@@ -579,23 +575,28 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
             cudaSuccess)                                                                     \
       return e;                                                                              \
     value_rows_kernel<TV, CHV><<<blocks, kB3Threads, smem, st>>>(                            \
-        seg, U, seg_row, ents_sorted, static_cast<const TV*>(values), w_sorted, dy, dV, dw,  \
-        hk, p.d_v, p.K, p.status, dVc, rows_out, U_out, ent_tok);                            \
+        c.seg, c.U, c.seg_row, ents_sorted, static_cast<const TV*>(values), c.w_sorted, dy,  \
+        dV, c.dw, hk, p.d_v, p.K, p.status, dVc, rows_out, U_out, ent_tok);                  \
   } while (0)
-    if (p.vfp32) {
-      if (nvec <= kB3Threads) PKM_B3(float, 1);
-      else PKM_B3(float, 2);
-    } else {
-      if (nvec <= kB3Threads) PKM_B3(__nv_bfloat16, 1);
-      else PKM_B3(__nv_bfloat16, 2);
-    }
-#undef PKM_B3
-    PKM_COUNT(1);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    (void)persist_blocks;
+  if (p.vfp32) {
+    if (nvec <= kB3Threads) PKM_B3(float, 1);
+    else PKM_B3(float, 2);
+  } else {
+    if (nvec <= kB3Threads) PKM_B3(__nv_bfloat16, 1);
+    else PKM_B3(__nv_bfloat16, 2);
   }
+#undef PKM_B3
+  PKM_COUNT(1);
+  return cudaGetLastError();
+}
 
-  return cudaSuccess;
+cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved& s,
+                              const float* dy, float* dV, float* dw_out, void* ws,
+                              cudaStream_t st, float* dVc, int32_t* rows_out, int* U_out,
+                              const int32_t* ent_tok) {
+  cudaError_t e = launch_value_sort(p, s, ws, st);
+  if (e != cudaSuccess) return e;
+  return launch_value_rows(p, values, dy, dV, dw_out, ws, st, dVc, rows_out, U_out, ent_tok);
 }
 
 cudaError_t launch_value_sgd(const Plan& p, float* values, const pkm_saved& s, const float* dy,

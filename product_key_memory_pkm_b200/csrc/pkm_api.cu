@@ -315,6 +315,31 @@ pkm_status pkm_backward(const pkm_dims* d, const void* x, const void* Wq, const 
                                      dsubkeys, dvalues, dw_out, workspace, st));
 }
 
+pkm_status pkm_value_sort(const pkm_dims* d, const pkm_saved* saved, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  PKM_TRY(validate_dims(d));
+  if (d->N == 0) return PKM_OK;
+  if (!saved) return PKM_ERR_INVALID_ARG;
+  PKM_NEED(saved->idx); PKM_NEED(saved->w);
+  PKM_TRY(check_workspace(pkm_workspace_bytes(d, PKM_BWD), workspace, workspace_bytes));
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  return cuda_status(launch_value_sort(p, *saved, workspace, static_cast<cudaStream_t>(stream)));
+}
+
+pkm_status pkm_value_rows(const pkm_dims* d, const void* values, const float* dy,
+                          float* dvalues, float* dw, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  PKM_TRY(validate_dims(d));
+  if (d->N == 0) return PKM_OK;
+  PKM_NEED(values); PKM_NEED(dy); PKM_NEED(dw); PKM_OPT(dvalues);
+  PKM_TRY(check_workspace(pkm_workspace_bytes(d, PKM_BWD), workspace, workspace_bytes));
+  Plan p;
+  PKM_TRY(prepare(d, &p));
+  return cuda_status(launch_value_rows(p, values, dy, dvalues, dw, workspace,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 pkm_status pkm_value_grad(const pkm_dims* d, const void* values, const pkm_saved* saved,
                           const float* dy, float* dvalues, float* dw, void* workspace,
                           size_t workspace_bytes, void* stream) {

@@ -181,6 +181,11 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
                               const float* dy, float* dV, float* dw_out, void* ws,
                               cudaStream_t st, float* dVc = nullptr, int32_t* rows_out = nullptr,
                               int* U_out = nullptr, const int32_t* ent_tok = nullptr);
+cudaError_t launch_value_sort(const Plan& p, const pkm_saved& s, void* ws, cudaStream_t st);
+cudaError_t launch_value_rows(const Plan& p, const void* values, const float* dy, float* dV,
+                              float* dw_out, void* ws, cudaStream_t st, float* dVc = nullptr,
+                              int32_t* rows_out = nullptr, int* U_out = nullptr,
+                              const int32_t* ent_tok = nullptr);
 cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, const float* bn,
                               const void* subkeys, const pkm_saved& s, float* dx, float* dWq,
                               float* dbn, float* dsub, float* dw_out, void* ws, cudaStream_t st);

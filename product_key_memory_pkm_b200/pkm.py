@@ -45,7 +45,8 @@ PKM_SHARD_ROUTE, PKM_SHARD_OWNER = 1, 2
 # every symbol include/pkm.h declares
 EXPORTED = ("pkm_saved_bytes", "pkm_workspace_bytes", "pkm_forward", "pkm_backward", "pkm_query",
             "pkm_subkey_scores", "pkm_candidate_topk", "pkm_gather_bag", "pkm_check_status",
-            "pkm_status_string", "pkm_build_info", "pkm_value_grad", "pkm_query_grad",
+            "pkm_status_string", "pkm_build_info", "pkm_value_grad", "pkm_value_sort",
+            "pkm_value_rows", "pkm_query_grad",
             "pkm_launch_count", "pkm_selftest_wait_timeout", "pkm_value_grad_noalloc",
             "pkm_fastweight_workspace_bytes", "pkm_fastweight_chunks", "pkm_value_sgd",
             "pkm_value_grad_rows", "pkm_value_adam", "pkm_hit_counts", "pkm_bn_running_update",
@@ -98,6 +99,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "pkm_status_string": (ctypes.c_char_p, [I]),
         "pkm_build_info": (ctypes.c_char_p, []),
         "pkm_value_grad": (I, [D, P, SV, P, P, P, P, S, P]),
+        "pkm_value_sort": (I, [D, SV, P, S, P]),
+        "pkm_value_rows": (I, [D, P, P, P, P, P, S, P]),
         "pkm_query_grad": (I, [D, P, P, P, P, SV, P, P, P, P, P, P, S, P]),
         "pkm_launch_count": (ctypes.c_ulonglong, []),
         "pkm_selftest_wait_timeout": (I, [ctypes.c_uint32, P]),
@@ -234,6 +237,25 @@ def pkm_value_grad(dims: Dims, values, saved: dict, dy, dw, dvalues=None, worksp
                                  _ptr(dvalues), _ptr(dw), _ptr(workspace),
                                  _ws(workspace, workspace_bytes), _stream(stream)),
            "pkm_value_grad")
+
+
+def pkm_value_sort(dims: Dims, saved: dict, workspace=None, workspace_bytes: int = 0,
+                   stream=None) -> None:
+    """First half of pkm_value_grad: the selections sorted by value row, into the workspace."""
+    s = _saved_c(saved)
+    _check(load().pkm_value_sort(ctypes.byref(dims.c()), ctypes.byref(s), _ptr(workspace),
+                                 _ws(workspace, workspace_bytes), _stream(stream)),
+           "pkm_value_sort")
+
+
+def pkm_value_rows(dims: Dims, values, dy, dw, dvalues=None, workspace=None,
+                   workspace_bytes: int = 0, stream=None) -> None:
+    """Second half of pkm_value_grad: the per-row pass over what pkm_value_sort left in the
+    same workspace."""
+    _check(load().pkm_value_rows(ctypes.byref(dims.c()), _ptr(values), _ptr(dy), _ptr(dvalues),
+                                 _ptr(dw), _ptr(workspace), _ws(workspace, workspace_bytes),
+                                 _stream(stream)),
+           "pkm_value_rows")
 
 
 def pkm_value_grad_noalloc(dims: Dims, values, saved: dict, dy, dw, dvalues=None,

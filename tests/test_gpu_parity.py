@@ -259,6 +259,31 @@ def test_value_gradient_is_deterministic_under_duplicates():
         assert torch.equal(g1[k], g2[k]), k
 
 
+@pytest.mark.parametrize("case", ["duplicate_heavy", "ragged_multihead_bf16"])
+def test_value_stage_in_two_parts_equals_the_whole(case):
+    """pkm_value_sort then pkm_value_rows (another stream's work in between, the workspace
+    left alone) gives pkm_value_grad's dV and dw bit for bit."""
+    cfg = CASES[case]
+    inp = make_inputs(cfg, seed=4)
+    dev = H.to_dev(inp, cfg)
+    dims, saved, _ = H.gpu_forward(cfg, dev)
+    dy = torch.from_numpy(inp["dy"]).cuda()
+    V = dev["values"]
+    ws = P.alloc_workspace(dims, P.PKM_BWD)
+    dV1 = torch.zeros(cfg.K, cfg.d_v, device="cuda")
+    dw1 = torch.empty(cfg.N, cfg.h, cfg.k, device="cuda")
+    P.pkm_value_grad(dims, V, saved, dy, dw1, dvalues=dV1, workspace=ws)
+    dV2 = torch.zeros_like(dV1)
+    dw2 = torch.full_like(dw1, float("nan"))
+    ws.fill_(0xA5)  # stale contents must not matter to the sort
+    P.pkm_value_sort(dims, saved, workspace=ws)
+    torch.cuda.synchronize()
+    P.pkm_value_rows(dims, V, dy, dw2, dvalues=dV2, workspace=ws)
+    assert P.pkm_check_status() == P.PKM_OK
+    assert torch.equal(dV1, dV2)
+    assert torch.equal(dw1, dw2)
+
+
 def test_gradients_accumulate_into_caller_buffers():
     cfg = CASES["tiny_bf16"]
     inp = make_inputs(cfg, seed=1)
