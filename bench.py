@@ -225,6 +225,9 @@ def run_b200(args, cfg, rank, world, dist):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
     names = ["query", "subkey_scores", "candidate_topk", "gather_bag", "value_grad", "query_grad"]
+    # high priority: the sort's short kernels are scheduled ahead of the bag's waiting CTAs
+    side = torch.cuda.Stream(device=dev, priority=-1)
+    fork_ev, join_ev = torch.cuda.Event(), torch.cuda.Event()
 
     def step(ev=None):
         def mark(i):
@@ -237,10 +240,16 @@ def run_b200(args, cfg, rank, world, dist):
         mark(2)
         P.pkm_candidate_topk(dims, saved, stream=st)
         mark(3)
+        # the value stage (pkm_value_grad) in its two parts: the sort needs only the
+        # selection, so it runs on a second stream beside the bag; the row pass is timed
+        # alone (any wait for the sort is in the value stage's time)
+        fork_ev.record(st)
+        side.wait_event(fork_ev)
+        P.pkm_value_sort(dims, saved, workspace=ws, stream=side)
+        join_ev.record(side)
         P.pkm_gather_bag(dims, V, saved["idx"], saved["w"], y, stream=st)
         mark(4)
-        # the value stage (pkm_value_grad) in its two parts, so the row pass is timed alone
-        P.pkm_value_sort(dims, saved, workspace=ws, stream=st)
+        st.wait_event(join_ev)
         mark(5)
         P.pkm_value_rows(dims, V, dy, dw, dvalues=dV, workspace=ws, stream=st)
         mark(6)
@@ -395,12 +404,16 @@ def run_b200(args, cfg, rank, world, dist):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded; tables random-init, no trained weights)",
         "config": dict(_cfg_json(cfg), parallelism=f"replicas{world}" if world > 1 else "single",
-                       variant=args.variant),
+                       variant=args.variant,
+                       streams="value sort on a second stream beside the bag"),
         "fwd": {"value": round(cfg.N * world / (fwd_ms * 1e-3), 1), "unit": "tokens/s (fwd)",
                 "ms": round(fwd_ms, 4)},
         "stage_ms": {n: round(float(v), 4) for n, v in zip(names, st_mean)},
         "roofline": roof(dom),
-        "roofline_other": [roof(n) for n in rl if n != dom],
+        "roofline_other": [dict(roof(n), note="the value stage's sort runs beside this kernel "
+                                              "on a high-priority second stream; this interval "
+                                              "includes its share")
+                           if n == "gather_bag" else roof(n) for n in rl if n != dom],
         "clocks": clk,
         "gpu_launches": int(launches),
         "input_gen_s": round(gen_s, 1),
