@@ -290,7 +290,19 @@ def run_b200(args, cfg, rank, world, dist):
                          for s in range(args.steps)])
     rows_ms = float(np.mean([evs[s][5].elapsed_time(evs[s][6]) for s in range(args.steps)]))
     step_ms = float(stage_ms.sum(1).mean())
-    fwd_ms = float(stage_ms[:, :4].sum(1).mean())
+    # the forward alone (F1-F4), timed in its own steps: in the full step the bag's interval
+    # also holds the backward's sort, which runs beside it
+    fwd_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for s_ in range(args.steps):
+        flush.zero_()
+        fwd_ev[s_][0].record(st)
+        P.pkm_query(dims, x, Wq, bn, saved, stream=st)
+        P.pkm_subkey_scores(dims, sub, saved, stream=st)
+        P.pkm_candidate_topk(dims, saved, stream=st)
+        P.pkm_gather_bag(dims, V, saved["idx"], saved["w"], y, stream=st)
+        fwd_ev[s_][1].record(st)
+    torch.cuda.synchronize()
+    fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in fwd_ev]))
     if P.pkm_check_status(st) != P.PKM_OK:
         raise RuntimeError("device status after the timed steps is not OK")
 
