@@ -178,6 +178,9 @@ pkm_status pkm_backward(const pkm_dims* d, const void* x, const void* Wq, const 
                         size_t workspace_bytes, void* stream);
 
 /* ---- the backward's two stages; pkm_backward runs both ----
+ * (The gradient reaches only the selected value rows and sub-keys: "Meta AI 可扩展内存层"
+ * sections 6.1 and 9.2; the query-side chain follows "Large Memory Layers with Product
+ * Keys", method details.)
  * Value stage (sort of the selections by value row, then one pass per distinct row):
  *   dw [N][h][k] fp32 out (required), dvalues += (NULL: skip).
  * Query stage (softmax backward onto the selected sub-keys, query-half and sub-key
