@@ -416,8 +416,8 @@ def run_b200(args, cfg, rank, world, dist):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded; tables random-init, no trained weights)",
         "config": dict(_cfg_json(cfg), parallelism=f"replicas{world}" if world > 1 else "single",
-                       variant=args.variant,
-                       streams="value sort on a second stream beside the bag"),
+                       variant=args.variant),
+        "schedule": "the value stage's sort on a high-priority second stream beside the bag",
         "fwd": {"value": round(cfg.N * world / (fwd_ms * 1e-3), 1), "unit": "tokens/s (fwd)",
                 "ms": round(fwd_ms, 4)},
         "stage_ms": {n: round(float(v), 4) for n, v in zip(names, st_mean)},
