@@ -31,34 +31,65 @@ constexpr int kBnTokens = 64;        // tokens per BatchNorm-backward block (par
 // One warp per (padded token t, head-half hs): zero the row in both planes, then
 // write the k selected entries (distinct within a half, so no accumulation; lanes
 // stride over them for k > 32).
+constexpr int kGWin = 1024;  // columns of a G row built in shared memory at a time
+
+// One warp per (token row, head-half): the row of both planes is built in shared memory
+// window by window (zeros, then the row's selected sub-keys), then written out with
+// 16-byte stores, so every byte of the planes is written once.
 __global__ void __launch_bounds__(256) g_dense_kernel(const float* __restrict__ gsub,
                                                       const int32_t* __restrict__ sub_i,
                                                       __nv_bfloat16* __restrict__ G, int64_t N,
                                                       int64_t Np, int h, int k, int Cp) {
-  const int lane = threadIdx.x & 31;
-  const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  __shared__ __align__(16) __nv_bfloat16 srow[8][2][kGWin];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t w = (int64_t)blockIdx.x * 8 + wid;
   const int hs2 = 2 * h;
-  if (w >= Np * hs2) return;
+  if (w >= Np * hs2) return;  // warp-uniform
   const int64_t t = w / hs2;
   const int hs = (int)(w % hs2);
-  __nv_bfloat16* hi = G + ((int64_t)(hs * 2 + 0) * Np + t) * Cp;
-  __nv_bfloat16* lo = G + ((int64_t)(hs * 2 + 1) * Np + t) * Cp;
-  const uint4 z = make_uint4(0, 0, 0, 0);
-  for (int c = lane; c < Cp / 8; c += 32) {
-    reinterpret_cast<uint4*>(hi)[c] = z;
-    reinterpret_cast<uint4*>(lo)[c] = z;
-  }
-  __syncwarp();
+  uint4* hi = reinterpret_cast<uint4*>(G + ((int64_t)(hs * 2 + 0) * Np + t) * Cp);
+  uint4* lo = reinterpret_cast<uint4*>(G + ((int64_t)(hs * 2 + 1) * Np + t) * Cp);
+  // this lane's selections of the row (k <= 64: two per lane at most)
+  int32_t ci[2] = {-1, -1};
+  __nv_bfloat16 ch[2], cl[2];
   if (t < N) {
     const int hh = hs >> 1, s = hs & 1;
-    for (int j = lane; j < k; j += 32) {
-      const int64_t o = ((t * h + hh) * 2 + s) * k + j;
-      const float g = gsub[o];
-      const int32_t i = sub_i[o];
-      const __nv_bfloat16 gh = __float2bfloat16_rn(g);
-      hi[i] = gh;
-      lo[i] = __float2bfloat16_rn(g - __bfloat162float(gh));
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int j = lane + 32 * r;
+      if (j < k) {
+        const int64_t o = ((t * h + hh) * 2 + s) * k + j;
+        const float g = gsub[o];
+        ci[r] = sub_i[o];
+        ch[r] = __float2bfloat16_rn(g);
+        cl[r] = __float2bfloat16_rn(g - __bfloat162float(ch[r]));
+      }
     }
+  }
+  uint4* sh = reinterpret_cast<uint4*>(srow[wid][0]);
+  uint4* sl = reinterpret_cast<uint4*>(srow[wid][1]);
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  for (int c0 = 0; c0 < Cp; c0 += kGWin) {
+    const int wn = min(kGWin, Cp - c0) / 8;  // 16-byte pieces of this window
+    for (int c = lane; c < wn; c += 32) {
+      sh[c] = z;
+      sl[c] = z;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int i = ci[r] - c0;
+      if (i >= 0 && i < wn * 8) {
+        srow[wid][0][i] = ch[r];
+        srow[wid][1][i] = cl[r];
+      }
+    }
+    __syncwarp();
+    for (int c = lane; c < wn; c += 32) {
+      hi[c0 / 8 + c] = sh[c];
+      lo[c0 / 8 + c] = sl[c];
+    }
+    __syncwarp();  // the window's shared memory is reused
   }
 }
 
