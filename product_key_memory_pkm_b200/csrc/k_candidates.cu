@@ -17,6 +17,7 @@ namespace pkm {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
+constexpr int kCandWarps = 8;  // warps per block of the candidate kernels
 
 // Among the rows still in the running (in[r]), keep those whose key equals the warp-wide
 // maximum of their keys.  Returns the number of rows left in the warp.
@@ -42,8 +43,11 @@ __global__ void __launch_bounds__(256) candidate_topk_kernel(
     float* __restrict__ w_out, int64_t NH, int k, int C2, float scale) {
   grid_dependency_wait();  // the per-half lists come from the previous kernel
   allow_dependent_launch();
-  const int lane = threadIdx.x & 31;
-  const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  // the winners in order, written by the winning lane of each step
+  __shared__ float wS_s[kCandWarps][32 * R];
+  __shared__ int32_t wI_s[kCandWarps][32 * R];
+  const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + wid;
   if (g >= NH) return;  // warp-uniform
   const float* ss = sub_s + g * 2 * k;
   const int32_t* si = sub_i + g * 2 * k;
@@ -60,13 +64,6 @@ __global__ void __launch_bounds__(256) candidate_topk_kernel(
     i1[r] = live[r] ? si[a] : 0;
     j2[r] = live[r] ? si[k + a] : 0;
     ptr[r] = 0;
-  }
-  float outS[R];  // lane j, register r ends up holding winner j + 32 r
-  int32_t outIdx[R];
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    outS[r] = 0.f;
-    outIdx[r] = 0;
   }
   for (int step = 0; step < k; ++step) {
     bool in[R];
@@ -111,19 +108,25 @@ __global__ void __launch_bounds__(256) candidate_topk_kernel(
       bal = __ballot_sync(kFull, in[R - 1]);
     }
     const int win = __ffs(bal) - 1;
-    const float wS = __shfl_sync(kFull, wr ? S[R - 1] : S[0], win);
-    const int32_t wIdx = __shfl_sync(kFull, wr ? flat[R - 1] : flat[0], win);
+    if (lane == win) {
+      wS_s[wid][step] = wr ? S[R - 1] : S[0];
+      wI_s[wid][step] = wr ? flat[R - 1] : flat[0];
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      if (lane + 32 * r == step) {
-        outS[r] = wS;
-        outIdx[r] = wIdx;
-      }
-      if (lane == win && wr == r) ++ptr[r];
+      for (int r = 0; r < R; ++r)
+        if (wr == r) ++ptr[r];
     }
   }
+  __syncwarp();
+  // lane j, register r: winner j + 32 r
+  float outS[R];
+  int32_t outIdx[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    outS[r] = live[r] ? wS_s[wid][lane + 32 * r] : 0.f;
+    outIdx[r] = live[r] ? wI_s[wid][lane + 32 * r] : 0;
+  }
   // softmax over the k winners of scale * S (winner 0 holds the maximum)
-  const float S0 = __shfl_sync(kFull, outS[0], 0);
+  const float S0 = wS_s[wid][0];
   float e[R], sum = 0.f;
 #pragma unroll
   for (int r = 0; r < R; ++r) {
@@ -179,7 +182,7 @@ __global__ void __launch_bounds__(256) candidate_all_kernel(
 cudaError_t launch_candidates(const Plan& p, const float* sub_s, const int32_t* sub_i,
                               int32_t* idx, float* w, cudaStream_t st) {
   const int64_t NH = p.N * p.h;
-  const int warps = 8;
+  const int warps = kCandWarps;
   const int64_t blocks = (NH + warps - 1) / warps;
   if (p.ksel != p.k) {
     cudaError_t e = launch_dependent(candidate_all_kernel, dim3((unsigned)blocks), dim3(warps * 32),
