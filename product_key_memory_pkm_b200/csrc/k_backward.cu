@@ -942,8 +942,14 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
   }
   float* dbn_acc = train ? c.bntot : dbn;  // where the partial column sums are reduced
 
+  // B5 + B6 run on tensor cores (dense G planes) unless the storage or the scorer needs the
+  // CUDA-core path; there, with k winners per head, the G row build also computes the
+  // softmax backward (B4)
+  const bool tc_subgrad = tc_backward_supported(p) && p.half % 64 == 0 && !p.idw;
+  const bool fold_b4 = tc_subgrad && p.ksel == p.k;
+
   // B4: softmax backward onto the selected sub-keys
-  {
+  if (!fold_b4) {
     const int64_t NH = p.N * p.h;
     if (p.ksel != p.k)
       softmax_bwd_all_kernel<<<(unsigned)((NH + 7) / 8), 256, 0, st>>>(s.w, dw, gsub, NH, p.k,
@@ -969,12 +975,13 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
 
   // B5 + B6 on tensor cores: dense G planes, dq = G C, BatchNorm backward, dC = G^T Q
   // (the inverse-distance variant's corrections run on the CUDA-core path)
-  const bool tc_subgrad = tc_backward_supported(p) && p.half % 64 == 0 && !p.idw;
   if (tc_subgrad) {
     const bool want_dq = dx || dWq || dbn;
     e = launch_subgrad_tc(p, gsub, s.sub_i, subkeys, s.q, bn, dbn_acc ? s.qhat : nullptr,
                           c.G, reinterpret_cast<__nv_bfloat16*>(dq_pre),
-                          dbn_acc ? part : nullptr, c.dspart, dsub, want_dq, st);
+                          dbn_acc ? part : nullptr, c.dspart, dsub, want_dq, st,
+                          fold_b4 ? s.w : nullptr, fold_b4 ? dw : nullptr,
+                          fold_b4 ? s.idx : nullptr);
     if (e != cudaSuccess) return e;
     if (dbn_acc) {
       const int64_t nblk = subgrad_part_blocks(p.N);

@@ -204,7 +204,8 @@ cudaError_t launch_subgrad_tc(const Plan& p, const float* gsub, const int32_t* s
                               const void* subkeys, const void* q_planes, const float* bn,
                               const float* qhat, __nv_bfloat16* G,
                               __nv_bfloat16* dq_planes, float* bn_part, float* dsub_part,
-                              float* dsub, bool want_dq, cudaStream_t st);
+                              float* dsub, bool want_dq, cudaStream_t st, const float* w = nullptr,
+                              const float* dw = nullptr, const int32_t* idx = nullptr);
 
 // ---------------------------------------------------------------- row-sharded table
 // Workspace layouts (byte offsets) of the source-side routing and the owner-side index.
