@@ -121,10 +121,6 @@ __device__ __forceinline__ void smem_vals<float>(const float* p, float* f) {
   f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
 }
 
-__device__ __forceinline__ void prefetch_l1(const void* p) {
-  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
-}
-
 // ws_sorted[p] = w[ents[p]]: the selection weights in row order, so staging a batch
 // needs two independent loads.  A selection's upstream-gradient row is ent_tok[ent] when
 // that map is given (entries received from other ranks), else ent / hk (its token).
@@ -222,18 +218,11 @@ __global__ void __launch_bounds__(kB3Threads, PKM_B3_MIN_BLOCKS) value_rows_kern
     pending_bits &= ~(1u << b);
     __syncthreads();
     if (abort_flag || !got) break;  // uniform: abort_flag is read after the barrier
-    if (tid < nbn) {  // publish the next row's batch and pull its dy lines into L1
+    if (tid < nbn) {  // publish the next row's batch
       const int64_t tn = ent_tok ? ent_tok[nent] : nent / hk;
       s_e[b ^ 1][tid] = nent;
       s_t[b ^ 1][tid] = (int)tn;
       s_w[b ^ 1][tid] = nw;
-#ifndef PKM_B3_DY_PREFETCH
-#define PKM_B3_DY_PREFETCH 0
-#endif
-      if (PKM_B3_DY_PREFETCH) {
-        const char* row = reinterpret_cast<const char*>(dy + tn * d_v);
-        for (int off = 0; off < d_v * 4; off += 128) prefetch_l1(row + off);
-      }
     }
     if (r < 0 || r >= K) {  // status already recorded by the issuing thread
       __syncthreads();
