@@ -334,10 +334,18 @@ __global__ void __launch_bounds__(256) dbn_reduce_kernel(const float* __restrict
   const int col = blockIdx.x * 32 + lane;
   const bool live = col < 2 * hq;
   const int which = live ? col / hq : 0, c = live ? col % hq : 0;
-  float s = 0.f;
-  if (live)
-    for (int b = wid; b < nblk; b += 8) s += part[((int64_t)b * 2 + which) * hq + c];
-  red[wid][lane] = s;
+  // four running sums (blocks wid + 8 (4 m + i)), combined in a fixed order
+  float s4[4] = {0.f, 0.f, 0.f, 0.f};
+  if (live) {
+    for (int b0 = wid; b0 < nblk; b0 += 32) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int b = b0 + 8 * i;
+        if (b < nblk) s4[i] += part[((int64_t)b * 2 + which) * hq + c];
+      }
+    }
+  }
+  red[wid][lane] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
   __syncthreads();
   if (wid == 0 && live) {
     float t = 0.f;
