@@ -69,10 +69,10 @@ struct DxProb {
     for (int j = 0; j < kBN / kMNBox; ++j)
       tma_load_2d(b + j * kMNBoxBytes, B, nt * kBN + j * kMNBox, kk * kBK, bar);
   }
-  __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState&) {}
-  __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&) {}
+  __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState&, const EpiCtx&) {}
+  __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&, const EpiCtx&) {}
   __device__ static void epi_chunk(const Params& P, int u, int, int row, uint32_t taddr,
-                                   unsigned char*, EpiState&) {
+                                   unsigned char*, EpiState&, const EpiCtx&) {
     const int mt = u / P.n_tiles, nt = u % P.n_tiles;
     const int64_t t = (int64_t)mt * kBM + row;
     for (int piece = 0; piece < kBN / 32; ++piece) {
@@ -115,10 +115,10 @@ struct DwqProb {
     for (int j = 0; j < kBN / kMNBox; ++j)
       tma_load_2d(b + j * kMNBoxBytes, B, nt * kBN + j * kMNBox, kk * kBK, bar);
   }
-  __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState&) {}
-  __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&) {}
+  __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState&, const EpiCtx&) {}
+  __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&, const EpiCtx&) {}
   __device__ static void epi_chunk(const Params& P, int u, int, int row, uint32_t taddr,
-                                   unsigned char*, EpiState&) {
+                                   unsigned char*, EpiState&, const EpiCtx&) {
     const int mt = u / P.n_tiles, nt = u % P.n_tiles;
     const int o = mt * kBM + row;
     for (int piece = 0; piece < kBN / 32; ++piece) {

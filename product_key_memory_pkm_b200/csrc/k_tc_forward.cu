@@ -21,8 +21,7 @@
 namespace pkm {
 
 // ------------------------------------------------------------------ host: tensor maps
-bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                       uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+static PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   static std::once_flag once;
   std::call_once(once, []() {
@@ -33,6 +32,32 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint6
         q == cudaDriverEntryPointSuccess)
       encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   });
+  return encode;
+}
+
+bool make_tmap_store(CUtensorMap* map, bool fp32, int rank, const void* base,
+                     const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                     CUtensorMapSwizzle swizzle) {
+  const PFN_cuTensorMapEncodeTiled_v12000 encode = tmap_encoder();
+  if (!encode || rank < 2 || rank > 3) return false;
+  cuuint64_t d[3], str[2];
+  cuuint32_t bx[3], estr[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) str[i] = strides_bytes[i];
+  CUresult r = encode(map,
+                      fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                      (cuuint32_t)rank, const_cast<void*>(base), d, str, bx, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                       uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+  const PFN_cuTensorMapEncodeTiled_v12000 encode = tmap_encoder();
   if (!encode) return false;
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_pitch_bytes};
@@ -50,25 +75,32 @@ namespace {
 using namespace tc;
 
 // ================================================================== F1 query network
+// The epilogue stages each warp's 32 x 32 piece (32 tokens, 32 columns) in shared memory
+// and writes it with TMA tile stores: q_hi and q_lo as one 3-D store each into the
+// [2][N][hq] planes, qhat as one 2-D store.  A store covers whole 64- and 128-byte row
+// segments; stores of a thread's own row touched 32 cache lines per warp instruction and
+// bounded the kernel.
 struct QueryProb {
   static constexpr int kAMN = 0, kBMN = 0;
-  static constexpr int kStages = 4;
+  static constexpr int kStages = 3;
   // two epilogue sets (eight epilogue warps): the BatchNorm, the hi/lo split and three
   // output streams of a tile take about as long as its mainloop, so each set gets two
   // units' MMA time to finish one
   static constexpr int kSets = 2;
-  // per-tile BatchNorm constants {mean, 1/sqrt(var + eps), gamma, beta} of the 256
-  // columns as one float4 each, one private copy per epilogue warp so no barrier spans
-  // warps
-  static constexpr int kEpiSmem = 4 * kBN * 16;
+  // per set: four 8 KiB warp staging tiles (qhat 4 KiB with 128-byte swizzle, q_hi and
+  // q_lo 2 KiB each with 64-byte swizzle), then two buffers of the tile's BatchNorm
+  // constants {mean, 1/sqrt(var + eps), gamma, beta} (one float4 per column), written by
+  // the set's first warp and published through the set's two mbarriers
+  static constexpr int kWarpStage = 8192;
+  static constexpr int kConstOff = 4 * kWarpStage;
+  static constexpr int kEpiSmem = kConstOff + 2 * kBN * 16;
   struct Params {
     int* status;
     const float* bn;
-    __nv_bfloat16* q;  // [2][N][hq]
-    float* qhat;       // optional
     int64_t N;
     int hq, m_tiles, n_tiles, nk;
     float eps;
+    int has_qhat;  // out1 maps qhat [N][hq] fp32
   };
   struct EpiState {};
 
@@ -84,16 +116,21 @@ struct QueryProb {
     tma_load_2d(sb, B, kb * kBK, nt * kBN, bar);
   }
 
-  __device__ static float4* consts(unsigned char* sm, int row) {
-    return reinterpret_cast<float4*>(sm) + (row >> 5) * kBN;
+  // constants buffer of the set's seq-th unit
+  __device__ static float4* consts(unsigned char* sm, int seq) {
+    return reinterpret_cast<float4*>(sm + kConstOff) + (seq & 1) * kBN;
   }
 
-  __device__ static void epi_begin(const Params& P, int u, int row, unsigned char* sm,
-                                   EpiState&) {
+  // The set's first warp fills the unit's constants buffer and publishes it.  Buffer
+  // seq & 1 was last read in the epilogue of unit seq - 2, which ended before this warp
+  // could start unit seq - 1 (the accumulator of seq - 1 is filled only after every
+  // thread of the set released seq - 2).
+  __device__ static void epi_begin(const Params& P, int u, int, unsigned char* sm, EpiState&,
+                                   const EpiCtx& cx) {
+    if (cx.quarter != 0) return;
     const int nt = u % P.n_tiles;
-    float4* c = consts(sm, row);
-    __syncwarp();  // this warp's reads of the previous tile's constants are done
-    for (int j = row & 31; j < kBN; j += 32) {
+    float4* c = consts(sm, cx.seq);
+    for (int j = cx.lane; j < kBN; j += 32) {
       const int n = nt * kBN + j;
       float mean = 0.f, inv = 0.f, gamma = 0.f, beta = 0.f;
       if (n < P.hq && !P.bn) {  // identity: q = x Wq^T (training-mode BatchNorm follows)
@@ -108,22 +145,31 @@ struct QueryProb {
       c[j] = make_float4(mean, inv, gamma, beta);
     }
     __syncwarp();
+    if (cx.lane == 0) mbar_arrive(&cx.bar[cx.seq & 1]);
   }
-  __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&) {}
+  __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&,
+                                 const EpiCtx&) {}
 
-  __device__ static void epi_chunk(const Params& P, int u, int, int row, uint32_t taddr,
-                                   unsigned char* sm, EpiState&) {
+  __device__ static void epi_chunk(const Params& P, int u, int, int, uint32_t taddr,
+                                   unsigned char* sm, EpiState&, const EpiCtx& cx) {
     const int mt = u / P.n_tiles, nt = u % P.n_tiles;
-    const int64_t t = (int64_t)mt * kBM + row;
-    const int hq = P.hq;
-    const float4* cst = consts(sm, row);
+    const int hq = P.hq, lane = cx.lane;
+    int got = 0;
+    if (lane == 0)
+      got = mbar_wait(&cx.bar[cx.seq & 1], (cx.seq >> 1) & 1, cx.abort, cx.status) ? 1 : 0;
+    if (!__shfl_sync(0xffffffffu, got, 0)) return;
+    const float4* cst = consts(sm, cx.seq);
+    unsigned char* stg = sm + cx.quarter * kWarpStage;
+    float4* s_qh = reinterpret_cast<float4*>(stg);
+    uint4* s_hi = reinterpret_cast<uint4*>(stg + 4096);
+    uint4* s_lo = reinterpret_cast<uint4*>(stg + 6144);
+    const int y0 = mt * kBM + cx.quarter * 32;  // token of the warp's first row
     for (int piece = 0; piece < kBN / 32; ++piece) {
       const int n0 = nt * kBN + piece * 32;
       if (n0 >= hq) break;  // warp-uniform
       uint32_t r[32];
       tmem_ld32(taddr + (uint32_t)(piece * 32), r);
       tmem_wait_ld(r);
-      if (t >= P.N) continue;
       uint32_t hi2[16], lo2[16];
       float qh[32];
 #pragma unroll
@@ -142,19 +188,30 @@ struct QueryProb {
         hi2[j / 2] = *reinterpret_cast<const uint32_t*>(&hb);
         lo2[j / 2] = *reinterpret_cast<const uint32_t*>(&lb);
       }
-      const int64_t o = t * hq + n0;
-      uint4* ph = reinterpret_cast<uint4*>(P.q + o);
-      uint4* pl = reinterpret_cast<uint4*>(P.q + P.N * hq + o);
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        ph[v] = make_uint4(hi2[4 * v], hi2[4 * v + 1], hi2[4 * v + 2], hi2[4 * v + 3]);
-        pl[v] = make_uint4(lo2[4 * v], lo2[4 * v + 1], lo2[4 * v + 2], lo2[4 * v + 3]);
-      }
-      if (P.qhat) {
-        float4* pq = reinterpret_cast<float4*>(P.qhat + o);
+      // the stores of the previous piece have read the staging tile
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
+      // row = lane; 16-byte chunk v of the row sits at chunk v ^ (address bits 7..9 of the
+      // row) for the 128-byte swizzle, v ^ (bits 7..8) for the 64-byte one
+      if (P.has_qhat) {
 #pragma unroll
         for (int v = 0; v < 8; ++v)
-          pq[v] = make_float4(qh[4 * v], qh[4 * v + 1], qh[4 * v + 2], qh[4 * v + 3]);
+          s_qh[lane * 8 + (v ^ (lane & 7))] =
+              make_float4(qh[4 * v], qh[4 * v + 1], qh[4 * v + 2], qh[4 * v + 3]);
+      }
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int o = lane * 4 + (v ^ ((lane >> 1) & 3));
+        s_hi[o] = make_uint4(hi2[4 * v], hi2[4 * v + 1], hi2[4 * v + 2], hi2[4 * v + 3]);
+        s_lo[o] = make_uint4(lo2[4 * v], lo2[4 * v + 1], lo2[4 * v + 2], lo2[4 * v + 3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(cx.out0, s_hi, n0, y0, 0);
+        tma_store_3d(cx.out0, s_lo, n0, y0, 1);
+        if (P.has_qhat) tma_store_2d(cx.out1, s_qh, n0, y0);
+        bulk_commit();
       }
     }
   }
@@ -257,7 +314,8 @@ struct ScoresProb {
     return m;
   }
 
-  __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState& es) {
+  __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState& es,
+                                   const EpiCtx&) {
     es.root = 0;
     es.thr = -INFINITY;
     es.built = false;
@@ -280,7 +338,7 @@ struct ScoresProb {
   }
 
   __device__ static void epi_chunk(const Params& P, int u, int c, int row, uint32_t taddr,
-                                   unsigned char* sm, EpiState& es) {
+                                   unsigned char* sm, EpiState& es, const EpiCtx&) {
     const int hs_idx = u / P.m_tiles;
     const int C = (hs_idx & 1) ? P.C2 : P.C1;
     uint64_t* tr = tree_(sm);
@@ -340,7 +398,8 @@ struct ScoresProb {
     }
   }
 
-  __device__ static void epi_end(const Params& P, int u, int row, unsigned char* sm, EpiState&) {
+  __device__ static void epi_end(const Params& P, int u, int row, unsigned char* sm, EpiState&,
+                                 const EpiCtx&) {
     const int hs_idx = u / P.m_tiles, mt = u % P.m_tiles;
     const int hh = hs_idx >> 1, s = hs_idx & 1;
     const int64_t t = (int64_t)mt * kBM + row;
@@ -402,18 +461,34 @@ cudaError_t launch_query_tc(const Plan& p, const void* x, const void* Wq, const 
   if (!make_tmap_bf16_2d(&ta, x, p.d_in, p.N, (uint64_t)p.d_in * 2, kBK, kBM) ||
       !make_tmap_bf16_2d(&tb, Wq, p.d_in, p.hq, (uint64_t)p.d_in * 2, kBK, kBN))
     return cudaErrorInvalidValue;
+  // q planes [2][N][hq] bf16 and qhat [N][hq] fp32, stored in 32 x 32 tiles
+  CUtensorMap tq, tqh;
+  {
+    const uint64_t dims[3] = {(uint64_t)p.hq, (uint64_t)p.N, 2};
+    const uint64_t strides[2] = {(uint64_t)p.hq * 2, (uint64_t)p.N * p.hq * 2};
+    const uint32_t box[3] = {32, 32, 1};
+    if (!make_tmap_store(&tq, false, 3, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B))
+      return cudaErrorInvalidValue;
+  }
+  if (qhat) {
+    const uint64_t dims[2] = {(uint64_t)p.hq, (uint64_t)p.N};
+    const uint64_t strides[1] = {(uint64_t)p.hq * 4};
+    const uint32_t box[2] = {32, 32};
+    if (!make_tmap_store(&tqh, true, 2, qhat, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
   QueryProb::Params P{};
   P.status = p.status;
   P.bn = bn;
-  P.q = static_cast<__nv_bfloat16*>(q);
-  P.qhat = qhat;
+  P.has_qhat = qhat != nullptr;
   P.N = p.N;
   P.hq = p.hq;
   P.m_tiles = (int)((p.N + kBM - 1) / kBM);
   P.n_tiles = (p.hq + kBN - 1) / kBN;
   P.nk = (p.d_in + kBK - 1) / kBK;
   P.eps = p.eps;
-  return launch_tc<QueryProb>(ta, ta, tb, P, P.m_tiles * P.n_tiles, p.sm_count, st);
+  return launch_tc<QueryProb>(ta, ta, tb, P, P.m_tiles * P.n_tiles, p.sm_count, st, nullptr, &tq,
+                             qhat ? &tqh : nullptr);
 }
 
 cudaError_t launch_scores_tc(const Plan& p, const void* subkeys, const void* q, float* sub_s,

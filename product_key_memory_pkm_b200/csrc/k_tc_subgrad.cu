@@ -279,7 +279,7 @@ struct DqProb {
     return reinterpret_cast<float*>(sm) + (row >> 5) * kBN;
   }
   __device__ static void epi_begin(const Params& P, int u, int row, unsigned char* sm,
-                                   EpiState&) {
+                                   EpiState&, const EpiCtx&) {
     int hs, mt, nt;
     decode(P, u, hs, mt, nt);
     const int base = (hs >> 1) * P.dk + (hs & 1) * P.half + nt * kBN;
@@ -292,9 +292,9 @@ struct DqProb {
     }
     __syncwarp();
   }
-  __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&) {}
+  __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&, const EpiCtx&) {}
   __device__ static void epi_chunk(const Params& P, int u, int, int row, uint32_t taddr,
-                                   unsigned char* sm, EpiState&) {
+                                   unsigned char* sm, EpiState&, const EpiCtx&) {
     int hs, mt, nt;
     decode(P, u, hs, mt, nt);
     const int hh = hs >> 1, s = hs & 1;
@@ -414,10 +414,10 @@ struct DsubProb {
       tma_load_2d(b + j * kMNBoxBytes, B, hh * P.dk + s * P.half + nt * kBN + j * kMNBox, qy,
                   bar);
   }
-  __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState&) {}
-  __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&) {}
+  __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState&, const EpiCtx&) {}
+  __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&, const EpiCtx&) {}
   __device__ static void epi_chunk(const Params& P, int u, int, int row, uint32_t taddr,
-                                   unsigned char*, EpiState&) {
+                                   unsigned char*, EpiState&, const EpiCtx&) {
     int sp, hs, mt, nt;
     decode(P, u, sp, hs, mt, nt);
     const int C = (hs & 1) ? P.C2 : P.C1;

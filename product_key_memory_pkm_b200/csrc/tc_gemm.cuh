@@ -38,6 +38,21 @@ constexpr int kStageB = kBN * kBK * 2;  // 32 KiB
 constexpr int kStageBytes = kStageA + kStageB;
 constexpr uint32_t kTmemCols = 512;
 
+// What the engine hands every epilogue hook besides the problem's parameters: the two
+// output tensor maps (for problems that store tiles through TMA), two mbarriers of
+// count 1 private to the epilogue set, the CTA's abort flag and the status word, the
+// index of the current unit among the set's units, and the thread's warp quarter
+// (TMEM lanes [32 * quarter, 32 * quarter + 32)) and lane.
+struct EpiCtx {
+  const CUtensorMap* out0;
+  const CUtensorMap* out1;
+  uint64_t* bar;
+  volatile int* abort;
+  int* status;
+  int seq;
+  int quarter, lane;
+};
+
 // Epilogue sets of a problem (Prob::kSets, default 1).  With one set, the 128 epilogue
 // threads alternate between the two 256-column accumulators chunk by chunk.  With two
 // sets, each set of 128 threads owns one accumulator and every other unit of the CTA:
@@ -86,12 +101,14 @@ __global__ void __launch_bounds__(threads_of<Prob>(), 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
                    const __grid_constant__ CUtensorMap tmA1,
                    const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmB1, const typename Prob::Params P) {
+                   const __grid_constant__ CUtensorMap tmB1,
+                   const __grid_constant__ CUtensorMap tmO0,
+                   const __grid_constant__ CUtensorMap tmO1, const typename Prob::Params P) {
   constexpr int S = Prob::kStages;
   constexpr int NS = SetsOf<Prob>::value;
   extern __shared__ unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], tfull_bar[2], tempty_bar[2],
-      drain_bar;
+      drain_bar, epi_bar[2][2];
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
 
@@ -110,6 +127,7 @@ __global__ void __launch_bounds__(threads_of<Prob>(), 1)
       mbar_init(&tempty_bar[b], 128);
     }
     mbar_init(&drain_bar, 1);
+    for (int b = 0; b < 4; ++b) mbar_init(&epi_bar[b >> 1][b & 1], 1);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -257,6 +275,7 @@ __global__ void __launch_bounds__(threads_of<Prob>(), 1)
     const int row = quarter * 32 + lane;     // accumulator row owned by this thread
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     unsigned char* my_smem = epi_smem + (size_t)set * Prob::kEpiSmem;
+    EpiCtx cx{&tmO0, &tmO1, epi_bar[set], &abort_flag, status, 0, quarter, lane};
     int alt = 0;
     uint32_t acc_phase = 0u;  // bit a: parity of accumulator a's next phase
     bool ok = true;
@@ -270,7 +289,7 @@ __global__ void __launch_bounds__(threads_of<Prob>(), 1)
       }
       const int u = sch.unit(r, set);
       typename Prob::EpiState es;
-      Prob::epi_begin(P, u, row, my_smem, es);
+      Prob::epi_begin(P, u, row, my_smem, es, cx);
       for (int c = 0; c < nc; ++c) {
         const int acc = NS == 1 ? alt : set;
         // warp-uniform wait: lane 0 waits, the result is broadcast, so the warp reaches
@@ -284,15 +303,19 @@ __global__ void __launch_bounds__(threads_of<Prob>(), 1)
           break;
         }
         tc_fence_after();
-        Prob::epi_chunk(P, u, c, row, tmem_base + lane_addr + (uint32_t)acc * kBN, my_smem, es);
+        Prob::epi_chunk(P, u, c, row, tmem_base + lane_addr + (uint32_t)acc * kBN, my_smem, es,
+                        cx);
         tc_fence_before();
         mbar_arrive(&tempty_bar[acc]);
         acc_phase ^= 1u << acc;
         alt ^= 1;
       }
       if (!ok) break;
-      Prob::epi_end(P, u, row, my_smem, es);
+      Prob::epi_end(P, u, row, my_smem, es, cx);
+      ++cx.seq;
     }
+    // tile stores issued by the epilogue complete before the CTA exits
+    if (lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
