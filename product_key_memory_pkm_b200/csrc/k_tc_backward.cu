@@ -46,8 +46,11 @@ __device__ __forceinline__ void store_piece(float* dst, int64_t n0, int64_t n_li
 // ------------------------------------------------------------------ dx = dq_pre Wq
 struct DxProb {
   static constexpr int kAMN = 0, kBMN = 1;
-  static constexpr int kStages = 4;
-  static constexpr int kEpiSmem = 0;
+  // a stage holds one k-block of dq_hi, dq_lo and Wq (64 KiB); two products per k-block
+  static constexpr int kStages = 3;
+  static constexpr int kAPlanes = 2, kBPlanes = 1;
+  // per epilogue warp a 32 x 32 fp32 staging tile for the TMA stores of dx
+  static constexpr int kEpiSmem = 4 * 4096;
   struct Params {
     int* status;
     float* dx;
@@ -57,13 +60,17 @@ struct DxProb {
   struct EpiState {};
   __device__ static int num_units(const Params& P) { return P.m_tiles * P.n_tiles; }
   __device__ static int num_chunks(const Params&, int) { return 1; }
-  __device__ static int num_kblocks(const Params& P) { return 2 * P.nkh; }
+  __device__ static int num_kblocks(const Params& P) { return P.nkh; }
+  __device__ static int num_pairs(const Params&) { return 2; }
+  __device__ static int pair_a(const Params&, int i) { return i; }
+  __device__ static int pair_b(const Params&, int) { return 0; }
+  __device__ static uint32_t tx_bytes(const Params&) { return 2 * kStageA + kStageB; }
   __device__ static void load(const Params& P, const CUtensorMap* A0, const CUtensorMap* A1,
-                              const CUtensorMap* B, const CUtensorMap*, int u, int, int kb, void* sa, void* sb,
+                              const CUtensorMap* B, const CUtensorMap*, int u, int, int kk, void* sa, void* sb,
                               uint64_t* bar) {
     const int mt = u / P.n_tiles, nt = u % P.n_tiles;
-    const int plane = kb / P.nkh, kk = kb % P.nkh;
-    tma_load_2d(sa, plane ? A1 : A0, kk * kBK, mt * kBM, bar);
+    tma_load_2d(sa, A0, kk * kBK, mt * kBM, bar);
+    tma_load_2d(static_cast<unsigned char*>(sa) + kStageA, A1, kk * kBK, mt * kBM, bar);
     unsigned char* b = static_cast<unsigned char*>(sb);
 #pragma unroll
     for (int j = 0; j < kBN / kMNBox; ++j)
@@ -71,17 +78,20 @@ struct DxProb {
   }
   __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState&, const EpiCtx&) {}
   __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&, const EpiCtx&) {}
-  __device__ static void epi_chunk(const Params& P, int u, int, int row, uint32_t taddr,
-                                   unsigned char*, EpiState&, const EpiCtx&) {
+  // dx pieces leave through the warp's staging tile as TMA stores (out0 maps dx); rows
+  // past N and columns past d_in are not written
+  __device__ static void epi_chunk(const Params& P, int u, int, int, uint32_t taddr,
+                                   unsigned char* sm, EpiState&, const EpiCtx& cx) {
     const int mt = u / P.n_tiles, nt = u % P.n_tiles;
-    const int64_t t = (int64_t)mt * kBM + row;
+    const int y0 = mt * kBM + cx.quarter * 32;
+    unsigned char* stg = sm + cx.quarter * 4096;
     for (int piece = 0; piece < kBN / 32; ++piece) {
       const int n0 = nt * kBN + piece * 32;
       if (n0 >= P.d_in) break;  // warp-uniform
       uint32_t r[32];
       tmem_ld32(taddr + (uint32_t)(piece * 32), r);
       tmem_wait_ld(r);
-      if (t < P.N) store_piece(P.dx + t * P.d_in + n0, n0, P.d_in, r, false);
+      store_piece_tma(cx.out0, stg, cx.lane, r, n0, y0);
     }
   }
 };
@@ -89,7 +99,10 @@ struct DxProb {
 // ------------------------------------------------------------------ dWq += dq_pre^T x
 struct DwqProb {
   static constexpr int kAMN = 1, kBMN = 1;
-  static constexpr int kStages = 4;
+  // a stage holds one 64-token block of dq_hi, dq_lo and x (64 KiB); two products per
+  // k-block
+  static constexpr int kStages = 3;
+  static constexpr int kAPlanes = 2, kBPlanes = 1;
   static constexpr int kEpiSmem = 0;
   struct Params {
     int* status;
@@ -100,17 +113,22 @@ struct DwqProb {
   struct EpiState {};
   __device__ static int num_units(const Params& P) { return P.m_tiles * P.n_tiles; }
   __device__ static int num_chunks(const Params&, int) { return 1; }
-  __device__ static int num_kblocks(const Params& P) { return 2 * P.nkt; }
+  __device__ static int num_kblocks(const Params& P) { return P.nkt; }
+  __device__ static int num_pairs(const Params&) { return 2; }
+  __device__ static int pair_a(const Params&, int i) { return i; }
+  __device__ static int pair_b(const Params&, int) { return 0; }
+  __device__ static uint32_t tx_bytes(const Params&) { return 2 * kStageA + kStageB; }
   __device__ static void load(const Params& P, const CUtensorMap* A0, const CUtensorMap* A1,
-                              const CUtensorMap* B, const CUtensorMap*, int u, int, int kb, void* sa, void* sb,
+                              const CUtensorMap* B, const CUtensorMap*, int u, int, int kk, void* sa, void* sb,
                               uint64_t* bar) {
     const int mt = u / P.n_tiles, nt = u % P.n_tiles;
-    const int plane = kb / P.nkt, kk = kb % P.nkt;
     unsigned char* a = static_cast<unsigned char*>(sa);
     unsigned char* b = static_cast<unsigned char*>(sb);
 #pragma unroll
-    for (int j = 0; j < kBM / kMNBox; ++j)
-      tma_load_2d(a + j * kMNBoxBytes, plane ? A1 : A0, mt * kBM + j * kMNBox, kk * kBK, bar);
+    for (int j = 0; j < kBM / kMNBox; ++j) {
+      tma_load_2d(a + j * kMNBoxBytes, A0, mt * kBM + j * kMNBox, kk * kBK, bar);
+      tma_load_2d(a + kStageA + j * kMNBoxBytes, A1, mt * kBM + j * kMNBox, kk * kBK, bar);
+    }
 #pragma unroll
     for (int j = 0; j < kBN / kMNBox; ++j)
       tma_load_2d(b + j * kMNBoxBytes, B, nt * kBN + j * kMNBox, kk * kBK, bar);
@@ -153,7 +171,15 @@ cudaError_t launch_dx_tc(const Plan& p, const void* dq_planes, const void* Wq, f
   P.m_tiles = (int)((p.N + kBM - 1) / kBM);
   P.n_tiles = (p.d_in + kBN - 1) / kBN;
   P.nkh = (p.hq + kBK - 1) / kBK;
-  return launch_tc<DxProb>(a0, a1, b, P, P.m_tiles * P.n_tiles, p.sm_count, st);
+  CUtensorMap tdx;
+  {
+    const uint64_t dims[2] = {(uint64_t)p.d_in, (uint64_t)p.N};
+    const uint64_t strides[1] = {(uint64_t)p.d_in * 4};
+    const uint32_t box[2] = {32, 32};
+    if (!make_tmap_store(&tdx, true, 2, dx, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  return launch_tc<DxProb>(a0, a1, b, P, P.m_tiles * P.n_tiles, p.sm_count, st, nullptr, &tdx);
 }
 
 cudaError_t launch_dwq_tc(const Plan& p, const void* dq_planes, const void* x, float* dWq,

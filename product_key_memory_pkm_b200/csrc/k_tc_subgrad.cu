@@ -234,7 +234,9 @@ __device__ __forceinline__ float warp_transpose_sum(float (&x)[32]) {
 
 struct DqProb {
   static constexpr int kAMN = 0, kBMN = 1;
-  static constexpr int kStages = 4;
+  // a stage holds one k-block of G_hi, G_lo and C_half (64 KiB); two products per k-block
+  static constexpr int kStages = 3;
+  static constexpr int kAPlanes = 2, kBPlanes = 1;
   // two epilogue sets: the BatchNorm backward makes the epilogue as long as a unit's
   // mainloop, so each set gets two units' MMA time to finish one
   static constexpr int kSets = 2;
@@ -254,7 +256,11 @@ struct DqProb {
   struct EpiState {};
   __device__ static int num_units(const Params& P) { return 2 * P.h * P.m_tiles * P.n_tiles; }
   __device__ static int num_chunks(const Params&, int) { return 1; }
-  __device__ static int num_kblocks(const Params& P) { return 2 * P.nkc; }
+  __device__ static int num_kblocks(const Params& P) { return P.nkc; }
+  __device__ static int num_pairs(const Params&) { return 2; }
+  __device__ static int pair_a(const Params&, int i) { return i; }
+  __device__ static int pair_b(const Params&, int) { return 0; }
+  __device__ static uint32_t tx_bytes(const Params&) { return 2 * kStageA + kStageB; }
   __device__ static void decode(const Params& P, int u, int& hs, int& mt, int& nt) {
     const int per = P.m_tiles * P.n_tiles;
     hs = u / per;
@@ -267,8 +273,10 @@ struct DqProb {
     int hs, mt, nt;
     decode(P, u, hs, mt, nt);
     const int hh = hs >> 1, s = hs & 1;
-    const int plane = kb / P.nkc, kk = kb % P.nkc;
-    tma_load_2d(sa, A0, kk * kBK, (int)((int64_t)(hs * 2 + plane) * P.Np + mt * kBM), bar);
+    const int kk = kb;
+    for (int plane = 0; plane < 2; ++plane)
+      tma_load_2d(static_cast<unsigned char*>(sa) + plane * kStageA, A0, kk * kBK,
+                  (int)((int64_t)(hs * 2 + plane) * P.Np + mt * kBM), bar);
     unsigned char* b = static_cast<unsigned char*>(sb);
 #pragma unroll
     for (int j = 0; j < kBN / kMNBox; ++j)
@@ -366,7 +374,10 @@ struct DqProb {
 // ------------------------------------------------------------------ dC_half = G^T Q_half
 struct DsubProb {
   static constexpr int kAMN = 1, kBMN = 1;
-  static constexpr int kStages = 4;
+  // a stage holds one 64-token block of G_hi, G_lo, Q_hi and Q_lo (96 KiB) and the
+  // k-block issues the two or three products on it, so each plane is read once per tile
+  static constexpr int kStages = 2;
+  static constexpr int kAPlanes = 2, kBPlanes = 2;
   static constexpr int kEpiSmem = 0;
   struct Params {
     int* status;
@@ -380,7 +391,14 @@ struct DsubProb {
     return kSplits * 2 * P.h * P.m_tiles * P.n_tiles;
   }
   __device__ static int num_chunks(const Params&, int) { return 1; }
-  __device__ static int num_kblocks(const Params& P) { return P.npass * P.kper; }
+  __device__ static int num_kblocks(const Params& P) { return P.kper; }
+  // npass 3: (G_hi, Q_hi), (G_hi, Q_lo), (G_lo, Q_hi); npass 2: (G_hi, Q_hi), (G_lo, Q_hi)
+  __device__ static int num_pairs(const Params& P) { return P.npass; }
+  __device__ static int pair_a(const Params& P, int i) { return P.npass == 3 ? (i == 2) : i; }
+  __device__ static int pair_b(const Params& P, int i) { return P.npass == 3 ? (i == 1) : 0; }
+  __device__ static uint32_t tx_bytes(const Params& P) {
+    return 2 * kStageA + (P.npass == 3 ? 2 : 1) * kStageB;
+  }
   __device__ static void decode(const Params& P, int u, int& sp, int& hs, int& mt, int& nt) {
     const int per = P.m_tiles * P.n_tiles;
     sp = u / (2 * P.h * per);
@@ -395,24 +413,25 @@ struct DsubProb {
     int sp, hs, mt, nt;
     decode(P, u, sp, hs, mt, nt);
     const int hh = hs >> 1, s = hs & 1;
-    const int pass = (P.npass == 2 && kb >= P.kper) ? 2 : kb / P.kper;
-    const int kk = sp * P.kper + kb % P.kper;  // 64-token block
-    const int gplane = pass == 2 ? 1 : 0;    // G_hi Q_hi, G_hi Q_lo, G_lo Q_hi
-    const int qplane = pass == 1 ? 1 : 0;
+    const int kk = sp * P.kper + kb;  // 64-token block
     // token blocks past the padded range read beyond both tensors: zero fill
     const bool live = kk < P.nkt;
-    const int gy = live ? (int)((int64_t)(hs * 2 + gplane) * P.Np + kk * kBK)
-                        : (int)(4 * (int64_t)P.h * P.Np);
-    const int qy = live ? (int)((int64_t)qplane * P.N + kk * kBK) : (int)(2 * P.N);
-    unsigned char* a = static_cast<unsigned char*>(sa);
-    unsigned char* b = static_cast<unsigned char*>(sb);
+    for (int plane = 0; plane < 2; ++plane) {
+      const int gy = live ? (int)((int64_t)(hs * 2 + plane) * P.Np + kk * kBK)
+                          : (int)(4 * (int64_t)P.h * P.Np);
+      unsigned char* a = static_cast<unsigned char*>(sa) + plane * kStageA;
 #pragma unroll
-    for (int j = 0; j < kBM / kMNBox; ++j)
-      tma_load_2d(a + j * kMNBoxBytes, A0, mt * kBM + j * kMNBox, gy, bar);
+      for (int j = 0; j < kBM / kMNBox; ++j)
+        tma_load_2d(a + j * kMNBoxBytes, A0, mt * kBM + j * kMNBox, gy, bar);
+    }
+    for (int plane = 0; plane < (P.npass == 3 ? 2 : 1); ++plane) {
+      const int qy = live ? (int)((int64_t)plane * P.N + kk * kBK) : (int)(2 * P.N);
+      unsigned char* b = static_cast<unsigned char*>(sb) + plane * kStageB;
 #pragma unroll
-    for (int j = 0; j < kBN / kMNBox; ++j)
-      tma_load_2d(b + j * kMNBoxBytes, B, hh * P.dk + s * P.half + nt * kBN + j * kMNBox, qy,
-                  bar);
+      for (int j = 0; j < kBN / kMNBox; ++j)
+        tma_load_2d(b + j * kMNBoxBytes, B, hh * P.dk + s * P.half + nt * kBN + j * kMNBox, qy,
+                    bar);
+    }
   }
   __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState&, const EpiCtx&) {}
   __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&, const EpiCtx&) {}

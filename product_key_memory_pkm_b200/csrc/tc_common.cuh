@@ -129,6 +129,30 @@ __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// Writes a warp's 32 x 32 fp32 piece (row = lane, r = the row's 32 columns) to the tile
+// at (x, y) of `map` (fp32, 32 x 32 box, 128-byte swizzle) through the warp's 4 KiB
+// staging tile `stg` (1024-byte aligned).  Waits first until the warp's previous stores
+// have read the staging tile.  Row chunk v (16 bytes) sits at chunk v ^ (lane & 7),
+// where the swizzle expects it.
+__device__ __forceinline__ void store_piece_tma(const CUtensorMap* map, unsigned char* stg,
+                                                int lane, const uint32_t (&r)[32], int x,
+                                                int y) {
+  if (lane == 0) bulk_wait_read_all();
+  __syncwarp();
+  float4* s = reinterpret_cast<float4*>(stg);
+#pragma unroll
+  for (int v = 0; v < 8; ++v)
+    s[lane * 8 + (v ^ (lane & 7))] =
+        make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                    __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(map, stg, x, y);
+    bulk_commit();
+  }
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

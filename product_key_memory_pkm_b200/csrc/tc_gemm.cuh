@@ -67,6 +67,35 @@ struct SetsOf<P, std::void_t<decltype(P::kSets)>> {
   static constexpr int value = P::kSets;
 };
 
+// Operand planes of a problem's stage.  By default a stage holds one A tile (128 x 64)
+// and one B tile (256 x 64) and a k-block is one product of the two.  A problem with
+// kAPlanes / kBPlanes > 1 (e.g. the hi and lo bf16 planes of an fp32 operand) loads all
+// planes of a k-block into one stage, A planes first, each 16 KiB, then the B planes, each
+// 32 KiB, and issues num_pairs(P) products per k-block: pair i multiplies A plane
+// pair_a(P, i) with B plane pair_b(P, i), all into the one accumulator.  tx_bytes(P) is
+// what the stage's loads deliver (planes a problem does not need are not loaded).
+template <class P, class = void>
+struct PlanesOf {
+  static constexpr int a = 1, b = 1;
+  __device__ static int pairs(const typename P::Params&) { return 1; }
+  __device__ static int pair_a(const typename P::Params&, int) { return 0; }
+  __device__ static int pair_b(const typename P::Params&, int) { return 0; }
+  __device__ static uint32_t tx(const typename P::Params&) { return kStageA + kStageB; }
+};
+template <class P>
+struct PlanesOf<P, std::void_t<decltype(P::kAPlanes)>> {
+  static constexpr int a = P::kAPlanes, b = P::kBPlanes;
+  __device__ static int pairs(const typename P::Params& p) { return P::num_pairs(p); }
+  __device__ static int pair_a(const typename P::Params& p, int i) { return P::pair_a(p, i); }
+  __device__ static int pair_b(const typename P::Params& p, int i) { return P::pair_b(p, i); }
+  __device__ static uint32_t tx(const typename P::Params& p) { return P::tx_bytes(p); }
+};
+
+template <class Prob>
+constexpr int stage_bytes_of() {
+  return PlanesOf<Prob>::a * kStageA + PlanesOf<Prob>::b * kStageB;
+}
+
 template <class Prob>
 constexpr int threads_of() {
   return 64 + 128 * SetsOf<Prob>::value;
@@ -74,7 +103,8 @@ constexpr int threads_of() {
 
 template <class Prob>
 constexpr size_t smem_bytes() {
-  return 1024 + (size_t)Prob::kStages * kStageBytes + (size_t)SetsOf<Prob>::value * Prob::kEpiSmem;
+  return 1024 + (size_t)Prob::kStages * stage_bytes_of<Prob>() +
+         (size_t)SetsOf<Prob>::value * Prob::kEpiSmem;
 }
 
 // The CTA's chunk schedule, walked identically by the producer, the MMA issuer and each
@@ -106,6 +136,9 @@ __global__ void __launch_bounds__(threads_of<Prob>(), 1)
                    const __grid_constant__ CUtensorMap tmO1, const typename Prob::Params P) {
   constexpr int S = Prob::kStages;
   constexpr int NS = SetsOf<Prob>::value;
+  using PL = PlanesOf<Prob>;
+  constexpr int SB = stage_bytes_of<Prob>();
+  constexpr int kOffB = PL::a * kStageA;  // first B plane within a stage
   extern __shared__ unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], tfull_bar[2], tempty_bar[2],
       drain_bar, epi_bar[2][2];
@@ -114,7 +147,7 @@ __global__ void __launch_bounds__(threads_of<Prob>(), 1)
 
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* epi_smem = smem + (size_t)S * kStageBytes;
+  unsigned char* epi_smem = smem + (size_t)S * SB;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -175,9 +208,9 @@ __global__ void __launch_bounds__(threads_of<Prob>(), 1)
                 ok = false;
                 break;
               }
-              unsigned char* sa = smem + (size_t)stage * kStageBytes;
-              mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
-              Prob::load(P, &tmA0, &tmA1, &tmB, &tmB1, u, c, kb, sa, sa + kStageA,
+              unsigned char* sa = smem + (size_t)stage * SB;
+              mbar_arrive_expect_tx(&full_bar[stage], PL::tx(P));
+              Prob::load(P, &tmA0, &tmA1, &tmB, &tmB1, u, c, kb, sa, sa + kOffB,
                          &full_bar[stage]);
               issued_mask |= 1u << stage;
               parity_mask = (parity_mask & ~(1u << stage)) | (phase << stage);
@@ -236,15 +269,21 @@ __global__ void __launch_bounds__(threads_of<Prob>(), 1)
                 break;
               }
               tc_fence_after();
-              const uint32_t sa = smem_u32(smem + (size_t)stage * kStageBytes);
-              const uint32_t sb = sa + kStageA;
+              const uint32_t s0 = smem_u32(smem + (size_t)stage * SB);
+              const int np = PL::pairs(P);
+              for (int pi = 0; pi < np; ++pi) {
+                const uint32_t sa = s0 + (uint32_t)PL::pair_a(P, pi) * kStageA;
+                const uint32_t sb = s0 + kOffB + (uint32_t)PL::pair_b(P, pi) * kStageB;
 #pragma unroll
-              for (int k = 0; k < kBK / 16; ++k) {
-                const uint64_t da = Prob::kAMN ? desc_mnmajor_sw128(sa + 2048u * k, 8192u, 1024u)
-                                               : desc_kmajor_sw128(sa) + (uint64_t)(2 * k);
-                const uint64_t db = Prob::kBMN ? desc_mnmajor_sw128(sb + 2048u * k, 8192u, 1024u)
-                                               : desc_kmajor_sw128(sb) + (uint64_t)(2 * k);
-                mma_bf16(dt, da, db, idesc, (kb | k) != 0 ? 1u : 0u);
+                for (int k = 0; k < kBK / 16; ++k) {
+                  const uint64_t da = Prob::kAMN
+                                          ? desc_mnmajor_sw128(sa + 2048u * k, 8192u, 1024u)
+                                          : desc_kmajor_sw128(sa) + (uint64_t)(2 * k);
+                  const uint64_t db = Prob::kBMN
+                                          ? desc_mnmajor_sw128(sb + 2048u * k, 8192u, 1024u)
+                                          : desc_kmajor_sw128(sb) + (uint64_t)(2 * k);
+                  mma_bf16(dt, da, db, idesc, (kb | k | pi) != 0 ? 1u : 0u);
+                }
               }
               issued = true;
               umma_commit(&empty_bar[stage]);
