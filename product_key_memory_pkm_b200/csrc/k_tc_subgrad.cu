@@ -211,41 +211,27 @@ __device__ __forceinline__ void store_piece(float* dst, int n0, int n_lim,
 // The epilogue also runs the BatchNorm eval backward on its tile: dq_pre = dq gamma /
 // sqrt(var + eps) is written straight to the bf16 hi/lo planes the dense query GEMMs
 // read, and the per-column partial sums of dq * qhat (d gamma) and dq (d beta) over each
-// warp's 32 tokens are reduced across the warp and written as one partial row per
-// 32-token block (summed in block order afterwards).
+// warp's 32 tokens are written as one partial row per 32-token block (summed in block
+// order afterwards).
 constexpr int kPartTokens = 32;
-
-// x[j] summed over the 32 lanes; lane l ends with the sum of x[l] (butterfly with
-// halving, 31 shuffles).
-__device__ __forceinline__ float warp_transpose_sum(float (&x)[32]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) {
-#pragma unroll
-    for (int i = 0; i < off; ++i) {
-      const bool up = (lane & off) != 0;
-      const float send = up ? x[i] : x[i + off];
-      const float keep = up ? x[i + off] : x[i];
-      x[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-    }
-  }
-  return x[0];
-}
 
 struct DqProb {
   static constexpr int kAMN = 0, kBMN = 1;
   // a stage holds one k-block of G_hi, G_lo and C_half (64 KiB); two products per k-block
-  static constexpr int kStages = 3;
-  static constexpr int kAPlanes = 2, kBPlanes = 1;
-  // two epilogue sets: the BatchNorm backward makes the epilogue as long as a unit's
-  // mainloop, so each set gets two units' MMA time to finish one
+  static constexpr int kStages = 2;
+  // two epilogue sets: with the BatchNorm backward a tile's epilogue takes about as long
+  // as its mainloop, so each set gets two units' MMA time to finish one (measured: 3
+  // stages with one set was slower)
   static constexpr int kSets = 2;
-  // per-tile BatchNorm scales gamma / sqrt(var + eps) of the 256 columns, one private
-  // copy per epilogue warp
-  static constexpr int kEpiSmem = 4 * kBN * 4;
+  static constexpr int kAPlanes = 2, kBPlanes = 1;
+  // per epilogue warp: a 4 KiB staging tile (first the warp's 32 x 32 accumulator piece
+  // for the BatchNorm partial sums, then the dq_pre hi and lo pieces for the TMA stores)
+  // and the tile's 256 BatchNorm scales gamma / sqrt(var + eps)
+  static constexpr int kWarpStage = 4096;
+  static constexpr int kScaleOff = 4 * kWarpStage;
+  static constexpr int kEpiSmem = kScaleOff + 4 * kBN * 4;
   struct Params {
     int* status;
-    __nv_bfloat16* planes;  // [2][N][hq] dq_pre hi, lo
     const float* bn;        // [4][hq]
     const float* qhat;      // [N][hq] or null
     float* part;            // [ceil(N / 32)][2][hq] or null
@@ -268,12 +254,11 @@ struct DqProb {
     nt = u % P.n_tiles;
   }
   __device__ static void load(const Params& P, const CUtensorMap* A0, const CUtensorMap*,
-                              const CUtensorMap* B, const CUtensorMap*, int u, int, int kb,
+                              const CUtensorMap* B, const CUtensorMap*, int u, int, int kk,
                               void* sa, void* sb, uint64_t* bar) {
     int hs, mt, nt;
     decode(P, u, hs, mt, nt);
     const int hh = hs >> 1, s = hs & 1;
-    const int kk = kb;
     for (int plane = 0; plane < 2; ++plane)
       tma_load_2d(static_cast<unsigned char*>(sa) + plane * kStageA, A0, kk * kBK,
                   (int)((int64_t)(hs * 2 + plane) * P.Np + mt * kBM), bar);
@@ -283,89 +268,113 @@ struct DqProb {
       tma_load_2d(b + j * kMNBoxBytes, B, nt * kBN + j * kMNBox,
                   hh * (P.C1 + P.C2) + s * P.C1 + kk * kBK, bar);
   }
-  __device__ static float* scales(unsigned char* sm, int row) {
-    return reinterpret_cast<float*>(sm) + (row >> 5) * kBN;
+  __device__ static float* scales(unsigned char* sm, int quarter) {
+    return reinterpret_cast<float*>(sm + kScaleOff) + quarter * kBN;
   }
-  __device__ static void epi_begin(const Params& P, int u, int row, unsigned char* sm,
-                                   EpiState&, const EpiCtx&) {
+  __device__ static void epi_begin(const Params& P, int u, int, unsigned char* sm, EpiState&,
+                                   const EpiCtx& cx) {
     int hs, mt, nt;
     decode(P, u, hs, mt, nt);
     const int base = (hs >> 1) * P.dk + (hs & 1) * P.half + nt * kBN;
-    float* sc = scales(sm, row);
+    float* sc = scales(sm, cx.quarter);
     __syncwarp();  // this warp's reads of the previous tile's scales are done
-    for (int j = row & 31; j < kBN; j += 32) {
+    for (int j = cx.lane; j < kBN; j += 32) {
       const int n = nt * kBN + j;
       sc[j] = n < P.half ? P.bn[2 * P.hq + base + j] / sqrtf(P.bn[P.hq + base + j] + P.eps)
                          : 0.f;
     }
     __syncwarp();
   }
-  __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&, const EpiCtx&) {}
-  __device__ static void epi_chunk(const Params& P, int u, int, int row, uint32_t taddr,
-                                   unsigned char* sm, EpiState&, const EpiCtx&) {
+  __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&,
+                                 const EpiCtx&) {}
+  // Per 32 x 32 piece (the warp's 32 tokens, 32 columns): the BatchNorm partial sums
+  // d gamma = sum_t dq * qhat and d beta = sum_t dq over the warp's tokens, lane c
+  // summing column c from the staged piece in token order, then dq_pre = dq * scale as
+  // bf16 hi and lo pieces through TMA stores (out0 maps the [2][N][hq] planes).
+  __device__ static void epi_chunk(const Params& P, int u, int, int, uint32_t taddr,
+                                   unsigned char* sm, EpiState&, const EpiCtx& cx) {
     int hs, mt, nt;
     decode(P, u, hs, mt, nt);
-    const int hh = hs >> 1, s = hs & 1;
-    const int64_t t = (int64_t)mt * kBM + row;
-    const int64_t tb = ((int64_t)mt * kBM + (row & ~31)) / kPartTokens;  // this warp's block
-    const float* sc = scales(sm, row);
+    const int hh = hs >> 1, s = hs & 1, lane = cx.lane;
+    const int64_t y0 = (int64_t)mt * kBM + cx.quarter * 32;  // token of the warp's first row
+    const bool row_live = y0 + lane < P.N;
+    const float* sc = scales(sm, cx.quarter);
+    unsigned char* stg = sm + cx.quarter * kWarpStage;
     for (int piece = 0; piece < kBN / 32; ++piece) {
       const int n0 = nt * kBN + piece * 32;
       if (n0 >= P.half) break;  // warp-uniform
+      const int col = hh * P.dk + s * P.half + n0;
+      // qhat of the piece, lane c on column c (row loads of 128 bytes), requested before the
+      // accumulator is read
+      float qv[32];
+      if (P.part && P.qhat) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          qv[i] = y0 + i < P.N ? P.qhat[(y0 + i) * P.hq + col + lane] : 0.f;
+      }
       uint32_t r[32];
       tmem_ld32(taddr + (uint32_t)(piece * 32), r);
       tmem_wait_ld(r);
-      const int64_t col = (int64_t)hh * P.dk + s * P.half + n0;
-      float pg[32], pb[32];
-      if (t < P.N) {
-        uint32_t hi2[16], lo2[16];
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float v0 = __uint_as_float(r[j]) * sc[piece * 32 + j];
-          const float v1 = __uint_as_float(r[j + 1]) * sc[piece * 32 + j + 1];
-          const __nv_bfloat162 hb = __floats2bfloat162_rn(v0, v1);
-          const float2 hf = __bfloat1622float2(hb);
-          const __nv_bfloat162 lb = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
-          hi2[j / 2] = *reinterpret_cast<const uint32_t*>(&hb);
-          lo2[j / 2] = *reinterpret_cast<const uint32_t*>(&lb);
-        }
-        uint4* ph = reinterpret_cast<uint4*>(P.planes + t * P.hq + col);
-        uint4* pl = reinterpret_cast<uint4*>(P.planes + P.N * P.hq + t * P.hq + col);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          ph[v] = make_uint4(hi2[4 * v], hi2[4 * v + 1], hi2[4 * v + 2], hi2[4 * v + 3]);
-          pl[v] = make_uint4(lo2[4 * v], lo2[4 * v + 1], lo2[4 * v + 2], lo2[4 * v + 3]);
-        }
-        if (P.part) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) pb[j] = __uint_as_float(r[j]);
-          if (P.qhat) {
-            const float4* qh = reinterpret_cast<const float4*>(P.qhat + t * P.hq + col);
-#pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              const float4 q4 = qh[v];
-              pg[4 * v] = pb[4 * v] * q4.x;
-              pg[4 * v + 1] = pb[4 * v + 1] * q4.y;
-              pg[4 * v + 2] = pb[4 * v + 2] * q4.z;
-              pg[4 * v + 3] = pb[4 * v + 3] * q4.w;
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) pg[j] = 0.f;
-          }
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) pg[j] = pb[j] = 0.f;
-      }
+      // the previous piece's stores have read the staging tile
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
       if (P.part) {  // warp-uniform
-        const float sg = warp_transpose_sum(pg);
-        const float sb = warp_transpose_sum(pb);
-        if (tb * kPartTokens < P.N) {
-          const int lane = row & 31;
+        // row = lane, 16-byte chunk v at chunk v ^ (lane & 7): the column reads below
+        // (row i, the 32 lanes on its 32 columns) touch 32 distinct banks
+        float4* sr = reinterpret_cast<float4*>(stg);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          sr[lane * 8 + (v ^ (lane & 7))] =
+              row_live ? make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                     __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        __syncwarp();
+        const float* srf = reinterpret_cast<const float*>(stg);
+        float sg = 0.f, sb = 0.f;
+        if (P.qhat) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float a = srf[i * 32 + ((((lane >> 2) ^ (i & 7))) << 2) + (lane & 3)];
+            sg = fmaf(a, qv[i], sg);
+            sb += a;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sb += srf[i * 32 + ((((lane >> 2) ^ (i & 7))) << 2) + (lane & 3)];
+        }
+        if (y0 < P.N) {
+          const int64_t tb = y0 / kPartTokens;
           P.part[(tb * 2 + 0) * P.hq + col + lane] = sg;
           P.part[(tb * 2 + 1) * P.hq + col + lane] = sb;
         }
+        __syncwarp();  // the staged piece is read before the planes overwrite it
+      }
+      uint32_t hi2[16], lo2[16];
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        const float v0 = __uint_as_float(r[j]) * sc[piece * 32 + j];
+        const float v1 = __uint_as_float(r[j + 1]) * sc[piece * 32 + j + 1];
+        const __nv_bfloat162 hb = __floats2bfloat162_rn(v0, v1);
+        const float2 hf = __bfloat1622float2(hb);
+        const __nv_bfloat162 lb = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
+        hi2[j / 2] = *reinterpret_cast<const uint32_t*>(&hb);
+        lo2[j / 2] = *reinterpret_cast<const uint32_t*>(&lb);
+      }
+      // 64-byte swizzle: row chunk v at chunk v ^ ((lane >> 1) & 3)
+      uint4* s_hi = reinterpret_cast<uint4*>(stg);
+      uint4* s_lo = reinterpret_cast<uint4*>(stg + 2048);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int o = lane * 4 + (v ^ ((lane >> 1) & 3));
+        s_hi[o] = make_uint4(hi2[4 * v], hi2[4 * v + 1], hi2[4 * v + 2], hi2[4 * v + 3]);
+        s_lo[o] = make_uint4(lo2[4 * v], lo2[4 * v + 1], lo2[4 * v + 2], lo2[4 * v + 3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(cx.out0, s_hi, col, (int)y0, 0);
+        tma_store_3d(cx.out0, s_lo, col, (int)y0, 1);
+        bulk_commit();
       }
     }
   }
@@ -514,9 +523,18 @@ cudaError_t launch_subgrad_tc(const Plan& p, const float* gsub, const int32_t* s
         !make_tmap_bf16_2d(&tb, subkeys, p.half, (uint64_t)p.h * (p.C1 + p.C2),
                            (uint64_t)p.half * 2, kMNBox, kBK))
       return cudaErrorInvalidValue;
+    // dq_pre planes [2][N][hq] bf16, stored in 32 x 32 tiles
+    CUtensorMap tq;
+    {
+      const uint64_t dims[3] = {(uint64_t)p.hq, (uint64_t)p.N, 2};
+      const uint64_t strides[2] = {(uint64_t)p.hq * 2, (uint64_t)p.N * p.hq * 2};
+      const uint32_t box[3] = {32, 32, 1};
+      if (!make_tmap_store(&tq, false, 3, dq_planes, dims, strides, box,
+                           CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
+    }
     DqProb::Params P{};
     P.status = p.status;
-    P.planes = dq_planes;
     P.bn = bn;
     P.qhat = qhat;
     P.part = bn_part;
@@ -533,8 +551,8 @@ cudaError_t launch_subgrad_tc(const Plan& p, const float* gsub, const int32_t* s
     P.m_tiles = (int)(Np / kBM + (Np % kBM ? 1 : 0));
     P.n_tiles = (p.half + kBN - 1) / kBN;
     P.nkc = Cp / kBK;
-    if ((e = launch_tc<DqProb>(ta, ta, tb, P, hs2 * P.m_tiles * P.n_tiles, p.sm_count, st)) !=
-        cudaSuccess)
+    if ((e = launch_tc<DqProb>(ta, ta, tb, P, hs2 * P.m_tiles * P.n_tiles, p.sm_count, st,
+                               nullptr, &tq)) != cudaSuccess)
       return e;
   }
   if (dsub) {
