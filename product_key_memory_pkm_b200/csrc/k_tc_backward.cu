@@ -56,7 +56,9 @@ struct DxProb {
     float* dx;
     int64_t N;
     int d_in, hq, m_tiles, n_tiles, nkh;  // nkh = ceil(hq / 64)
+    int nw;                               // output columns per tile (64 .. 256)
   };
+  __device__ static int mma_n(const Params& P) { return P.nw; }
   struct EpiState {};
   __device__ static int num_units(const Params& P) { return P.m_tiles * P.n_tiles; }
   __device__ static int num_chunks(const Params&, int) { return 1; }
@@ -64,7 +66,9 @@ struct DxProb {
   __device__ static int num_pairs(const Params&) { return 2; }
   __device__ static int pair_a(const Params&, int i) { return i; }
   __device__ static int pair_b(const Params&, int) { return 0; }
-  __device__ static uint32_t tx_bytes(const Params&) { return 2 * kStageA + kStageB; }
+  __device__ static uint32_t tx_bytes(const Params& P) {
+    return 2 * kStageA + (P.nw / kMNBox) * kMNBoxBytes;
+  }
   __device__ static void load(const Params& P, const CUtensorMap* A0, const CUtensorMap* A1,
                               const CUtensorMap* B, const CUtensorMap*, int u, int, int kk, void* sa, void* sb,
                               uint64_t* bar) {
@@ -72,9 +76,8 @@ struct DxProb {
     tma_load_2d(sa, A0, kk * kBK, mt * kBM, bar);
     tma_load_2d(static_cast<unsigned char*>(sa) + kStageA, A1, kk * kBK, mt * kBM, bar);
     unsigned char* b = static_cast<unsigned char*>(sb);
-#pragma unroll
-    for (int j = 0; j < kBN / kMNBox; ++j)
-      tma_load_2d(b + j * kMNBoxBytes, B, nt * kBN + j * kMNBox, kk * kBK, bar);
+    for (int j = 0; j < P.nw / kMNBox; ++j)
+      tma_load_2d(b + j * kMNBoxBytes, B, nt * P.nw + j * kMNBox, kk * kBK, bar);
   }
   __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState&, const EpiCtx&) {}
   __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&, const EpiCtx&) {}
@@ -85,8 +88,8 @@ struct DxProb {
     const int mt = u / P.n_tiles, nt = u % P.n_tiles;
     const int y0 = mt * kBM + cx.quarter * 32;
     unsigned char* stg = sm + cx.quarter * 4096;
-    for (int piece = 0; piece < kBN / 32; ++piece) {
-      const int n0 = nt * kBN + piece * 32;
+    for (int piece = 0; piece < P.nw / 32; ++piece) {
+      const int n0 = nt * P.nw + piece * 32;
       if (n0 >= P.d_in) break;  // warp-uniform
       uint32_t r[32];
       tmem_ld32(taddr + (uint32_t)(piece * 32), r);
@@ -109,7 +112,9 @@ struct DwqProb {
     float* dWq;
     int64_t N;
     int d_in, hq, m_tiles, n_tiles, nkt;  // nkt = ceil(N / 64)
+    int nw;                               // output columns per tile (64 .. 256)
   };
+  __device__ static int mma_n(const Params& P) { return P.nw; }
   struct EpiState {};
   __device__ static int num_units(const Params& P) { return P.m_tiles * P.n_tiles; }
   __device__ static int num_chunks(const Params&, int) { return 1; }
@@ -117,7 +122,9 @@ struct DwqProb {
   __device__ static int num_pairs(const Params&) { return 2; }
   __device__ static int pair_a(const Params&, int i) { return i; }
   __device__ static int pair_b(const Params&, int) { return 0; }
-  __device__ static uint32_t tx_bytes(const Params&) { return 2 * kStageA + kStageB; }
+  __device__ static uint32_t tx_bytes(const Params& P) {
+    return 2 * kStageA + (P.nw / kMNBox) * kMNBoxBytes;
+  }
   __device__ static void load(const Params& P, const CUtensorMap* A0, const CUtensorMap* A1,
                               const CUtensorMap* B, const CUtensorMap*, int u, int, int kk, void* sa, void* sb,
                               uint64_t* bar) {
@@ -129,9 +136,8 @@ struct DwqProb {
       tma_load_2d(a + j * kMNBoxBytes, A0, mt * kBM + j * kMNBox, kk * kBK, bar);
       tma_load_2d(a + kStageA + j * kMNBoxBytes, A1, mt * kBM + j * kMNBox, kk * kBK, bar);
     }
-#pragma unroll
-    for (int j = 0; j < kBN / kMNBox; ++j)
-      tma_load_2d(b + j * kMNBoxBytes, B, nt * kBN + j * kMNBox, kk * kBK, bar);
+    for (int j = 0; j < P.nw / kMNBox; ++j)
+      tma_load_2d(b + j * kMNBoxBytes, B, nt * P.nw + j * kMNBox, kk * kBK, bar);
   }
   __device__ static void epi_begin(const Params&, int, int, unsigned char*, EpiState&, const EpiCtx&) {}
   __device__ static void epi_end(const Params&, int, int, unsigned char*, EpiState&, const EpiCtx&) {}
@@ -139,8 +145,8 @@ struct DwqProb {
                                    unsigned char*, EpiState&, const EpiCtx&) {
     const int mt = u / P.n_tiles, nt = u % P.n_tiles;
     const int o = mt * kBM + row;
-    for (int piece = 0; piece < kBN / 32; ++piece) {
-      const int n0 = nt * kBN + piece * 32;
+    for (int piece = 0; piece < P.nw / 32; ++piece) {
+      const int n0 = nt * P.nw + piece * 32;
       if (n0 >= P.d_in) break;  // warp-uniform
       uint32_t r[32];
       tmem_ld32(taddr + (uint32_t)(piece * 32), r);
@@ -149,6 +155,23 @@ struct DwqProb {
     }
   }
 };
+
+// Output-tile width for `cols` columns over `m_tiles` row tiles: the one of 256, 192 and
+// 128 whose round count times width (the per-SM MMA time of the last round) is least;
+// ties go to the wider tile (fewer operand bytes per product).
+int tile_width(int64_t m_tiles, int cols, int sm_count) {
+  int best = kBN;
+  int64_t best_cost = -1;
+  for (int w : {256, 192, 128}) {
+    const int64_t units = m_tiles * ((cols + w - 1) / w);
+    const int64_t cost = ((units + sm_count - 1) / sm_count) * w;
+    if (best_cost < 0 || cost < best_cost) {
+      best = w;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
 
 }  // namespace
 
@@ -169,7 +192,8 @@ cudaError_t launch_dx_tc(const Plan& p, const void* dq_planes, const void* Wq, f
   P.d_in = p.d_in;
   P.hq = p.hq;
   P.m_tiles = (int)((p.N + kBM - 1) / kBM);
-  P.n_tiles = (p.d_in + kBN - 1) / kBN;
+  P.nw = tile_width(P.m_tiles, p.d_in, p.sm_count);
+  P.n_tiles = (p.d_in + P.nw - 1) / P.nw;
   P.nkh = (p.hq + kBK - 1) / kBK;
   CUtensorMap tdx;
   {
@@ -197,7 +221,8 @@ cudaError_t launch_dwq_tc(const Plan& p, const void* dq_planes, const void* x, f
   P.d_in = p.d_in;
   P.hq = p.hq;
   P.m_tiles = (p.hq + kBM - 1) / kBM;
-  P.n_tiles = (p.d_in + kBN - 1) / kBN;
+  P.nw = tile_width(P.m_tiles, p.d_in, p.sm_count);
+  P.n_tiles = (p.d_in + P.nw - 1) / P.nw;
   P.nkt = (int)((p.N + kBK - 1) / kBK);
   return launch_tc<DwqProb>(a0, a1, b, P, P.m_tiles * P.n_tiles, p.sm_count, st);
 }

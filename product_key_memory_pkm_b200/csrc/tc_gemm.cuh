@@ -91,6 +91,18 @@ struct PlanesOf<P, std::void_t<decltype(P::kAPlanes)>> {
   __device__ static uint32_t tx(const typename P::Params& p) { return P::tx_bytes(p); }
 };
 
+// MMA width of a problem's chunks: kBN (256) by default; a problem with mma_n(P) runs
+// narrower chunks (a multiple of 64 up to 256) so that more units fill the SMs.  Its
+// accumulator slots stay 256 columns apart.
+template <class P, class = void>
+struct MmaNOf {
+  __device__ static int get(const typename P::Params&) { return kBN; }
+};
+template <class P>
+struct MmaNOf<P, std::void_t<decltype(&P::mma_n)>> {
+  __device__ static int get(const typename P::Params& p) { return P::mma_n(p); }
+};
+
 template <class Prob>
 constexpr int stage_bytes_of() {
   return PlanesOf<Prob>::a * kStageA + PlanesOf<Prob>::b * kStageB;
@@ -237,7 +249,7 @@ __global__ void __launch_bounds__(threads_of<Prob>(), 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(kBM, kBN, Prob::kAMN, Prob::kBMN);
+      const uint32_t idesc = idesc_bf16(kBM, MmaNOf<Prob>::get(P), Prob::kAMN, Prob::kBMN);
       int stage = 0;
       uint32_t phase = 0;
       int alt = 0;                // one set: the accumulator of the next chunk

@@ -361,6 +361,12 @@ def test_fwd_bwd_K1024_full_size_sampled():
     _sampled_full_size(FULL_K1024, 128)
 
 
+def test_fwd_bwd_K512_sampled():
+    """4096 tokens, |K| = 512^2, d_in = 1024: the backward at the second workload's size,
+    sampled tokens against the oracle."""
+    _sampled_full_size(FWD_K512, 256)
+
+
 def test_bounded_wait_expires_with_status_and_context_survives():
     """A wait on a barrier that nothing completes gives up after its budget, records
     PKM_ERR_DEVICE_TIMEOUT, and the next call on the same context works."""
