@@ -93,10 +93,11 @@ __global__ void __launch_bounds__(256) g_dense_kernel(const float* __restrict__ 
   }
 }
 
-// The same rows built straight from the selection (k <= 32 * R): the softmax backward
-// dS_j = scale w_j (dw_j - sum_l w_l dw_l) of the head's winners, each added to its
-// sub-key's column of this half in winner order (the order the per-half-list sums take),
-// so no per-half gradient list goes through memory.
+// The same rows built straight from the selection (k <= 32 * R), one warp per (token,
+// head) for both halves: the softmax backward dS_j = scale w_j (dw_j - sum_l w_l dw_l)
+// of the head's winners, each added to its sub-key's column of each half in winner order
+// (the order the per-half-list sums take), so no per-half gradient list goes through
+// memory and the head's selection is read once.
 template <int R>
 __global__ void __launch_bounds__(256) g_dense_dw_kernel(
     const float* __restrict__ w, const float* __restrict__ dw, const int32_t* __restrict__ idx,
@@ -105,21 +106,17 @@ __global__ void __launch_bounds__(256) g_dense_dw_kernel(
   __shared__ __align__(16) __nv_bfloat16 srow[8][2][kGWin];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int64_t wi = (int64_t)blockIdx.x * 8 + wid;
-  const int hs2 = 2 * h;
-  if (wi >= Np * hs2) return;  // warp-uniform
-  const int64_t t = wi / hs2;
-  const int hs = (int)(wi % hs2);
-  uint4* hi = reinterpret_cast<uint4*>(G + ((int64_t)(hs * 2 + 0) * Np + t) * Cp);
-  uint4* lo = reinterpret_cast<uint4*>(G + ((int64_t)(hs * 2 + 1) * Np + t) * Cp);
-  int32_t col[R];
+  if (wi >= Np * h) return;  // warp-uniform
+  const int64_t t = wi / h;
+  const int hh = (int)(wi % h);
+  int32_t ij[R];
   float D[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    col[r] = -1;
+    ij[r] = -1;
     D[r] = 0.f;
   }
   if (t < N) {  // warp-uniform
-    const int hh = hs >> 1, s = hs & 1;
     const int64_t o = (t * h + hh) * k;
     float wj[R], dwj[R], part = 0.f;
 #pragma unroll
@@ -128,8 +125,7 @@ __global__ void __launch_bounds__(256) g_dense_dw_kernel(
       const bool live = j < k;
       wj[r] = live ? w[o + j] : 0.f;
       dwj[r] = live ? dw[o + j] : 0.f;
-      const int32_t ij = live ? idx[o + j] : 0;
-      col[r] = live ? (s ? ij % C2 : ij / C2) : -1;
+      ij[r] = live ? idx[o + j] : -1;
       part = fmaf(wj[r], dwj[r], part);
     }
 #pragma unroll
@@ -137,58 +133,66 @@ __global__ void __launch_bounds__(256) g_dense_dw_kernel(
 #pragma unroll
     for (int r = 0; r < R; ++r) D[r] = scale * wj[r] * (dwj[r] - part);
   }
-  // each entry's column total, summed in winner order; the column's first winner writes it
-  float gs[R];
-  bool first[R];
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    gs[r] = 0.f;
-    first[r] = col[r] >= 0;
-  }
-#pragma unroll
-  for (int rs = 0; rs < R; ++rs) {
-    for (int b = 0; b < 32; ++b) {
-      const int32_t cb = __shfl_sync(0xffffffffu, col[rs], b);
-      const float Db = __shfl_sync(0xffffffffu, D[rs], b);
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        if (col[r] >= 0 && cb == col[r]) {
-          gs[r] += Db;
-          if (b + 32 * rs < lane + 32 * r) first[r] = false;
-        }
-      }
-    }
-  }
-  __nv_bfloat16 ch[R], cl[R];
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    ch[r] = __float2bfloat16_rn(gs[r]);
-    cl[r] = __float2bfloat16_rn(gs[r] - __bfloat162float(ch[r]));
-  }
   uint4* sh = reinterpret_cast<uint4*>(srow[wid][0]);
   uint4* sl = reinterpret_cast<uint4*>(srow[wid][1]);
   const uint4 z = make_uint4(0, 0, 0, 0);
-  for (int c0 = 0; c0 < Cp; c0 += kGWin) {
-    const int wn = min(kGWin, Cp - c0) / 8;
-    for (int c = lane; c < wn; c += 32) {
-      sh[c] = z;
-      sl[c] = z;
-    }
-    __syncwarp();
+  for (int s = 0; s < 2; ++s) {
+    const int hs = 2 * hh + s;
+    uint4* hi = reinterpret_cast<uint4*>(G + ((int64_t)(hs * 2 + 0) * Np + t) * Cp);
+    uint4* lo = reinterpret_cast<uint4*>(G + ((int64_t)(hs * 2 + 1) * Np + t) * Cp);
+    int32_t col[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) col[r] = ij[r] < 0 ? -1 : (s ? ij[r] % C2 : ij[r] / C2);
+    // each entry's column total, summed in winner order; the column's first winner writes it
+    float gs[R];
+    bool first[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      const int i = col[r] - c0;
-      if (first[r] && i >= 0 && i < wn * 8) {
-        srow[wid][0][i] = ch[r];
-        srow[wid][1][i] = cl[r];
+      gs[r] = 0.f;
+      first[r] = col[r] >= 0;
+    }
+#pragma unroll
+    for (int rs = 0; rs < R; ++rs) {
+      for (int b = 0; b < 32; ++b) {
+        const int32_t cb = __shfl_sync(0xffffffffu, col[rs], b);
+        const float Db = __shfl_sync(0xffffffffu, D[rs], b);
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          if (col[r] >= 0 && cb == col[r]) {
+            gs[r] += Db;
+            if (b + 32 * rs < lane + 32 * r) first[r] = false;
+          }
+        }
       }
     }
-    __syncwarp();
-    for (int c = lane; c < wn; c += 32) {
-      hi[c0 / 8 + c] = sh[c];
-      lo[c0 / 8 + c] = sl[c];
+    __nv_bfloat16 ch[R], cl[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      ch[r] = __float2bfloat16_rn(gs[r]);
+      cl[r] = __float2bfloat16_rn(gs[r] - __bfloat162float(ch[r]));
     }
-    __syncwarp();
+    for (int c0 = 0; c0 < Cp; c0 += kGWin) {
+      const int wn = min(kGWin, Cp - c0) / 8;
+      for (int c = lane; c < wn; c += 32) {
+        sh[c] = z;
+        sl[c] = z;
+      }
+      __syncwarp();
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int i = col[r] - c0;
+        if (first[r] && i >= 0 && i < wn * 8) {
+          srow[wid][0][i] = ch[r];
+          srow[wid][1][i] = cl[r];
+        }
+      }
+      __syncwarp();
+      for (int c = lane; c < wn; c += 32) {
+        hi[c0 / 8 + c] = sh[c];
+        lo[c0 / 8 + c] = sl[c];
+      }
+      __syncwarp();  // the window's shared memory is reused
+    }
   }
 }
 
@@ -506,12 +510,13 @@ cudaError_t launch_subgrad_tc(const Plan& p, const float* gsub, const int32_t* s
   {
     const int64_t warps = Np * hs2;
     const unsigned blocks = (unsigned)((warps + 7) / 8);
+    const unsigned hblocks = (unsigned)((Np * p.h + 7) / 8);  // one warp per (token, head)
     if (w && p.k <= 32)  // the softmax backward folded into the row build
-      g_dense_dw_kernel<1><<<blocks, 256, 0, st>>>(w, dw, idx, G, p.N, Np, p.h, p.k, p.C2, Cp,
-                                                   p.scale);
+      g_dense_dw_kernel<1><<<hblocks, 256, 0, st>>>(w, dw, idx, G, p.N, Np, p.h, p.k, p.C2, Cp,
+                                                    p.scale);
     else if (w)
-      g_dense_dw_kernel<2><<<blocks, 256, 0, st>>>(w, dw, idx, G, p.N, Np, p.h, p.k, p.C2, Cp,
-                                                   p.scale);
+      g_dense_dw_kernel<2><<<hblocks, 256, 0, st>>>(w, dw, idx, G, p.N, Np, p.h, p.k, p.C2, Cp,
+                                                    p.scale);
     else
       g_dense_kernel<<<blocks, 256, 0, st>>>(gsub, sub_i, G, p.N, Np, p.h, p.k, Cp);
     PKM_COUNT(1);
