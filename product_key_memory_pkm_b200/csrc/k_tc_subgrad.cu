@@ -467,24 +467,40 @@ struct DsubProb {
   }
 };
 
-// dsub[h][row(s, c)][d] += sum over splits, in split order.
-__global__ void dsub_reduce_kernel(const float* __restrict__ part, float* __restrict__ dsub, int h,
-                                   int C1, int C2, int Cp, int half) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t total = (int64_t)h * (C1 + C2) * half;
-  if (i >= total) return;
-  const int d = (int)(i % half);
-  const int64_t rr = i / half;
-  const int hh = (int)(rr / (C1 + C2));
-  const int within = (int)(rr % (C1 + C2));
+// dsub[h][row(s, c)][d] += sum over splits, in split order.  One block per dsub row; a
+// thread takes 4 consecutive d when vec4 (half % 4 == 0 and dsub 16-byte aligned), else one.
+__global__ void __launch_bounds__(128) dsub_reduce_kernel(const float* __restrict__ part,
+                                                          float* __restrict__ dsub, int h,
+                                                          int C1, int C2, int Cp, int half,
+                                                          int vec4) {
+  const int rr = blockIdx.x;  // hh * (C1 + C2) + row within the head
+  const int hh = rr / (C1 + C2), within = rr - hh * (C1 + C2);
   const int s = within >= C1 ? 1 : 0;
   const int c = within - s * C1;
   const int hs = hh * 2 + s;
-  float acc = 0.f;
+  float* drow = dsub + (int64_t)rr * half;
+  const float* prow = part + ((int64_t)hs * Cp + c) * half;
+  const int64_t split = (int64_t)2 * h * Cp * half;  // floats between splits
+  if (vec4) {
+    for (int v = threadIdx.x; v < half / 4; v += blockDim.x) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int sp = 0; sp < kSplits; ++sp)
-    acc += part[(((int64_t)sp * 2 * h + hs) * Cp + c) * half + d];
-  dsub[i] += acc;
+      for (int sp = 0; sp < kSplits; ++sp) {
+        const float4 q = reinterpret_cast<const float4*>(prow + sp * split)[v];
+        acc.x += q.x; acc.y += q.y; acc.z += q.z; acc.w += q.w;
+      }
+      float4 o = reinterpret_cast<float4*>(drow)[v];
+      o.x += acc.x; o.y += acc.y; o.z += acc.z; o.w += acc.w;
+      reinterpret_cast<float4*>(drow)[v] = o;
+    }
+  } else {
+    for (int d = threadIdx.x; d < half; d += blockDim.x) {
+      float acc = 0.f;
+#pragma unroll
+      for (int sp = 0; sp < kSplits; ++sp) acc += prow[sp * split + d];
+      drow[d] += acc;
+    }
+  }
 }
 
 }  // namespace
@@ -584,9 +600,9 @@ cudaError_t launch_subgrad_tc(const Plan& p, const float* gsub, const int32_t* s
     P.npass = p.bf16q ? 2 : 3;
     const int units = kSplits * hs2 * P.m_tiles * P.n_tiles;
     if ((e = launch_tc<DsubProb>(ta, ta, tb, P, units, p.sm_count, st)) != cudaSuccess) return e;
-    const int64_t total = (int64_t)p.h * (p.C1 + p.C2) * p.half;
-    dsub_reduce_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(dsub_part, dsub, p.h,
-                                                                         p.C1, p.C2, Cp, p.half);
+    const int vec4 = p.half % 4 == 0 && (reinterpret_cast<uintptr_t>(dsub) & 15u) == 0;
+    dsub_reduce_kernel<<<(unsigned)(p.h * (p.C1 + p.C2)), 128, 0, st>>>(
+        dsub_part, dsub, p.h, p.C1, p.C2, Cp, p.half, vec4);
     PKM_COUNT(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
