@@ -404,7 +404,7 @@ const char* pkm_status_string(pkm_status s);
  * is a fixed 64 MiB device array built into the library, which every GPU that loads
  * the library holds until the process exits.
  * The pages have no counterpart to this entry point.
- *   - Limit: the scratch holds the value stage's sort and segment buffers, about 60
+ *   - Limit: the scratch holds the value stage's sort and segment buffers, about 53
  *     bytes per selection (N*h*k selections; e.g. up to N = 8192 tokens at h = 4,
  *     k = 32).  A larger problem returns PKM_ERR_WORKSPACE from a host-side check,
  *     before any CUDA call.

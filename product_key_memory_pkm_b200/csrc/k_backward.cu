@@ -552,15 +552,18 @@ static BwdCtx bwd_ctx(const Plan& p, void* ws, float* dw_out) {
 
 // B1-B2: the selections sorted by value row (stable radix sort), the segment table of
 // the distinct rows and the weights in row order, all in the workspace.
-cudaError_t launch_value_sort(const Plan& p, const pkm_saved& s, void* ws, cudaStream_t st) {
+// The weights ride through the sort beside their selections (read in entry order, written
+// in runs), so no pass gathers them at random; wtmp (E1 floats: the caller's dw, which
+// the row pass overwrites, else the workspace's) holds them between passes.
+cudaError_t launch_value_sort(const Plan& p, const pkm_saved& s, void* ws, cudaStream_t st,
+                              float* wtmp) {
   const int64_t E1 = p.N * p.h * p.ksel;
-  BwdCtx c = bwd_ctx(p, ws, nullptr);
+  BwdCtx c = bwd_ctx(p, ws, wtmp);
   const int32_t *rows_sorted, *ents_sorted;
-  cudaError_t e =
-      sort::radix_sort(s.idx, E1, bits_for(p.K - 1), c.rb, &rows_sorted, &ents_sorted, st);
+  cudaError_t e = sort::radix_sort(s.idx, E1, bits_for(p.K - 1), c.rb, &rows_sorted,
+                                   &ents_sorted, st, s.w, c.dw, c.w_sorted);
   if (e != cudaSuccess) return e;
-  return sort::segments(rows_sorted, E1, c.seg, c.U, c.rb.bsum, st, c.seg_row, ents_sorted, s.w,
-                        c.w_sorted);
+  return sort::segments(rows_sorted, E1, c.seg, c.U, c.rb.bsum, st, c.seg_row);
 }
 
 // B3: one pass per distinct value row over what launch_value_sort left in the workspace.
@@ -602,7 +605,7 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
                               const float* dy, float* dV, float* dw_out, void* ws,
                               cudaStream_t st, float* dVc, int32_t* rows_out, int* U_out,
                               const int32_t* ent_tok) {
-  cudaError_t e = launch_value_sort(p, s, ws, st);
+  cudaError_t e = launch_value_sort(p, s, ws, st, dw_out);
   if (e != cudaSuccess) return e;
   return launch_value_rows(p, values, dy, dV, dw_out, ws, st, dVc, rows_out, U_out, ent_tok);
 }

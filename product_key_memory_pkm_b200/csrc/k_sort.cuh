@@ -10,7 +10,10 @@ namespace pkm {
 namespace sort {
 
 constexpr int kScanTPB = 512, kScanItems = 8, kScanTile = kScanTPB * kScanItems;
-constexpr int kRadixTile = 2048, kRadixWarps = 4, kRadixMaxBits = 11;
+// Radix tiles of 4096 keys and digits of at most 10 bits: each pass reorders its tile in
+// shared memory before writing, so the writes leave in runs of the tile's keys per digit
+// instead of one scattered word per key.
+constexpr int kRadixTile = 4096, kRadixWarps = 8, kRadixMaxBits = 10;
 
 // --------------------------------------------------------------- scan
 template <class In>
@@ -110,9 +113,12 @@ inline int64_t radix_hist_len(int64_t n) { return (int64_t)(1 << kRadixMaxBits) 
 
 // Sorts n pairs by key in [0, 2^bits_total) stably.  The first pass reads
 // (keys_src, payload = position); later passes ping-pong between A and B.
-// Returns the buffers holding the result.
+// Returns the buffers holding the result.  When w_src is given, a float per key rides
+// along (w_src[i] with key i) and ends in w_dst; w_tmp (n floats) holds it between passes.
 cudaError_t radix_sort(const int32_t* keys_src, int64_t n, int bits_total, const RadixBuffers& b,
-                       const int32_t** keys_out, const int32_t** vals_out, cudaStream_t st);
+                       const int32_t** keys_out, const int32_t** vals_out, cudaStream_t st,
+                       const float* w_src = nullptr, float* w_tmp = nullptr,
+                       float* w_dst = nullptr);
 
 // Where radix_sort(bits_total) leaves the sorted payloads (*vals_out of that call).
 inline const int32_t* radix_sorted_vals(const RadixBuffers& b, int bits_total) {

@@ -181,7 +181,9 @@ cudaError_t launch_value_grad(const Plan& p, const void* values, const pkm_saved
                               const float* dy, float* dV, float* dw_out, void* ws,
                               cudaStream_t st, float* dVc = nullptr, int32_t* rows_out = nullptr,
                               int* U_out = nullptr, const int32_t* ent_tok = nullptr);
-cudaError_t launch_value_sort(const Plan& p, const pkm_saved& s, void* ws, cudaStream_t st);
+// wtmp: E1 floats the sort may use between passes (null: the workspace's dw region)
+cudaError_t launch_value_sort(const Plan& p, const pkm_saved& s, void* ws, cudaStream_t st,
+                              float* wtmp = nullptr);
 cudaError_t launch_value_rows(const Plan& p, const void* values, const float* dy, float* dV,
                               float* dw_out, void* ws, cudaStream_t st, float* dVc = nullptr,
                               int32_t* rows_out = nullptr, int* U_out = nullptr,

@@ -78,10 +78,10 @@ def test_too_large_for_the_fixed_scratch_is_refused_on_the_host():
     assert _noalloc_rc_with_fake_pointers(d) == P.PKM_ERR_WORKSPACE
 
 
-def test_the_size_limit_is_about_sixty_bytes_per_selection():
+def test_the_size_limit_is_about_53_bytes_per_selection():
     n = _largest_fitting_selections()
-    # the documented limit: about 60 bytes per selection in 64 MiB
-    assert 0.9 * (64 << 20) / 60 < n < 1.1 * (64 << 20) / 60, n
+    # the documented limit: about 53 bytes per selection in 64 MiB
+    assert 0.95 * (64 << 20) / 53 < n < 1.05 * (64 << 20) / 53, n
     assert _noalloc_rc_with_fake_pointers(P.Dims(N=n + 1, **LIMIT_SHAPE)) == P.PKM_ERR_WORKSPACE
 
 
