@@ -25,13 +25,21 @@ __global__ void __launch_bounds__(256) radix_hist(const int32_t* __restrict__ ke
                                                   int64_t ntiles) {
   __shared__ int h[1 << kRadixMaxBits];
   for (int d = threadIdx.x; d < bins; d += blockDim.x) h[d] = 0;
-  __syncthreads();
   const int64_t base = (int64_t)blockIdx.x * kRadixTile;
   const uint32_t mask = (uint32_t)bins - 1u;
-  for (int i = threadIdx.x; i < kRadixTile; i += blockDim.x) {
-    int64_t g = base + i;
-    if (g < n) atomicAdd(&h[((uint32_t)keys[g] >> shift) & mask], 1);
+  // every key of the thread requested before the first count (keys[j] = position
+  // threadIdx.x + 256 j of the tile)
+  constexpr int kPer = kRadixTile / 256;
+  int32_t kv[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int64_t g = base + threadIdx.x + 256 * j;
+    kv[j] = g < n ? keys[g] : -1;
   }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kPer; ++j)
+    if (base + threadIdx.x + 256 * j < n) atomicAdd(&h[((uint32_t)kv[j] >> shift) & mask], 1);
   __syncthreads();
   for (int d = threadIdx.x; d < bins; d += blockDim.x) hist[(int64_t)d * ntiles + blockIdx.x] = h[d];
 }
