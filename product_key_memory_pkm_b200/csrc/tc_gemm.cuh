@@ -17,6 +17,12 @@
 // 256 columns (the scoring problem keeps a running top-k across the chunks of a
 // row; the other problems have one chunk per unit).  No TMA multicast is used.
 //
+// Per problem, optionally: several operand planes per stage with several products per
+// k-block (PlanesOf: the hi and lo bf16 planes of an operand read once per k-block
+// beside the other operand), a narrower MMA (MmaNOf: 192 or 128 columns, to fill the
+// SMs), and two output tensor maps for epilogues that write their pieces with TMA tile
+// stores (EpiCtx).
+//
 // Operand layouts in a stage (both 128-byte swizzled, as TMA writes them):
 //   K-major  (Prob::kAMN / kBMN == 0): rows of 64 k-elements (128 B), 8-row groups
 //            1024 B apart; one TMA box of 64 x rows.
