@@ -324,23 +324,23 @@ __global__ void __launch_bounds__(256) dq_kernel(
 }
 
 // dbn[which][c] += sum over the nblk partial rows, in a fixed order: 32 columns per
-// block (lane = column), warp w sums the rows b = w, w + 8, ..., then the 8 warp sums
-// are added in warp order.
-__global__ void __launch_bounds__(256) dbn_reduce_kernel(const float* __restrict__ part,
-                                                         int nblk, int hq,
-                                                         float* __restrict__ dbn) {
-  __shared__ float red[8][32];
+// block (lane = column), 32 warps; warp w sums the rows b = w, w + 32, ... in four running
+// sums (rows w + 32 (4 m + i) into sum i), then the 32 warp sums are added in warp order.
+constexpr int kDbnWarps = 32;
+__global__ void __launch_bounds__(kDbnWarps * 32) dbn_reduce_kernel(const float* __restrict__ part,
+                                                                    int nblk, int hq,
+                                                                    float* __restrict__ dbn) {
+  __shared__ float red[kDbnWarps][32];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int col = blockIdx.x * 32 + lane;
   const bool live = col < 2 * hq;
   const int which = live ? col / hq : 0, c = live ? col % hq : 0;
-  // four running sums (blocks wid + 8 (4 m + i)), combined in a fixed order
   float s4[4] = {0.f, 0.f, 0.f, 0.f};
   if (live) {
-    for (int b0 = wid; b0 < nblk; b0 += 32) {
+    for (int b0 = wid; b0 < nblk; b0 += 4 * kDbnWarps) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int b = b0 + 8 * i;
+        const int b = b0 + kDbnWarps * i;
         if (b < nblk) s4[i] += part[((int64_t)b * 2 + which) * hq + c];
       }
     }
@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(256) dbn_reduce_kernel(const float* __restrict
   if (wid == 0 && live) {
     float t = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) t += red[w][lane];
+    for (int w = 0; w < kDbnWarps; ++w) t += red[w][lane];
     dbn[which * hq + c] += t;
   }
 }
@@ -998,7 +998,7 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
       const int64_t nblk = subgrad_part_blocks(p.N);
       if (train && (e = cudaMemsetAsync(c.bntot, 0, 2 * sizeof(float) * p.hq, st)) != cudaSuccess)
         return e;
-      dbn_reduce_kernel<<<(2 * p.hq + 31) / 32, 256, 0, st>>>(part, (int)nblk, p.hq, dbn_acc);
+      dbn_reduce_kernel<<<(2 * p.hq + 31) / 32, kDbnWarps * 32, 0, st>>>(part, (int)nblk, p.hq, dbn_acc);
       PKM_COUNT(1);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -1031,7 +1031,7 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
     if (dbn_acc) {
       if (train && (e = cudaMemsetAsync(c.bntot, 0, 2 * sizeof(float) * p.hq, st)) != cudaSuccess)
         return e;
-      dbn_reduce_kernel<<<(2 * p.hq + 31) / 32, 256, 0, st>>>(part, (int)nblk, p.hq, dbn_acc); PKM_COUNT(1);
+      dbn_reduce_kernel<<<(2 * p.hq + 31) / 32, kDbnWarps * 32, 0, st>>>(part, (int)nblk, p.hq, dbn_acc); PKM_COUNT(1);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
   }
@@ -1043,7 +1043,7 @@ cudaError_t launch_query_grad(const Plan& p, const void* x, const void* Wq, cons
     if (dbn) {  // the caller's (d gamma, d beta) += the column sums
       const int64_t nblk = tc_subgrad ? subgrad_part_blocks(p.N)
                                       : (p.N + kDqTokensPerBlock - 1) / kDqTokensPerBlock;
-      dbn_reduce_kernel<<<(2 * p.hq + 31) / 32, 256, 0, st>>>(part, (int)nblk, p.hq, dbn);
+      dbn_reduce_kernel<<<(2 * p.hq + 31) / 32, kDbnWarps * 32, 0, st>>>(part, (int)nblk, p.hq, dbn);
       PKM_COUNT(1);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
